@@ -1,0 +1,271 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle.
+
+Each ``pin_*`` function takes an :class:`oracle.oracle.Oracle` and raises
+``AssertionError`` when the oracle disagrees with the pages or with the
+mathematics.  ``test_oracle_pins.py`` runs them on the real oracle;
+``test_oracle_mutants.py`` runs them on copies of the oracle with a planted
+mistake and requires that some pin fails for every such copy.
+
+What pins what:
+
+* exp / SiLU        -- float64 ``math.exp`` error bound (2 ulp); silu(0) = 0;
+                       silu(x) - silu(-x) = x.
+* bf16 rounding     -- torch's CPU float32 -> bfloat16 cast.
+* quantiser         -- hand-worked fixtures with exact ties (golden
+                       ``quant_hand.json``); absmax element -> +-127;
+                       scale * 127 ~ absmax; round-trip bound; q monotone
+                       in x; bf16 input path == widened fp32 path.
+* INT8 GEMM         -- numpy int64 matmul (brute force); closed forms
+                       (all-127 operands give 16129 K); identity weights;
+                       the int32 bound K * 127^2 < 2^31.
+* epilogues         -- float64 value within the rounding bound of the
+                       left-to-right fp32 chain; exact power-of-two cases;
+                       group mode against a float64 sum of per-group terms.
+* whole chain       -- hand-worked example (golden ``linear_hand.json``).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def ulp32(x: float) -> float:
+    return float(np.spacing(np.float32(abs(x))))
+
+
+# --------------------------------------------------------------------------- exp / silu
+def pin_exp(O) -> None:
+    """qko_exp is within 2 ulp of float64 exp over the clamped range."""
+    grid = np.concatenate([np.linspace(-87.0, 88.0, 40001, dtype=np.float32),
+                           np.float32([0.0, 1.0, -1.0, 0.5, -0.5, 1e-8, -1e-8, 0.34657359, -0.34657359])])
+    got = O.exp_array(grid)
+    worst = 0.0
+    for t, g in zip(grid.tolist(), got.tolist()):
+        ref = math.exp(t)
+        err = abs(g - ref) / ulp32(ref)
+        worst = max(worst, err)
+    assert worst <= 2.0, f"exp error {worst} ulp"
+    assert O.exp(0.0) == 1.0
+
+
+def pin_silu(O) -> None:
+    assert O.silu(0.0) == 0.0
+    rng = np.random.default_rng(7)
+    xs = np.concatenate([rng.standard_normal(2000).astype(np.float32) * 4,
+                         np.float32([1e-3, -1e-3, 10.0, -10.0, 30.0, -30.0])])
+    for x in xs.tolist():
+        s_pos, s_neg = O.silu(x), O.silu(-x)
+        # silu(x) - silu(-x) = x * (sigmoid(x) + sigmoid(-x)) = x
+        assert abs((s_pos - s_neg) - x) <= 4 * ulp32(x) + 4 * ulp32(max(abs(s_pos), abs(s_neg))), x
+        ref = x / (1.0 + math.exp(-x))
+        assert abs(s_pos - ref) <= 4 * ulp32(ref) + 1e-37, (x, s_pos, ref)
+
+
+# --------------------------------------------------------------------------- bf16
+def pin_bf16_rounding(O) -> None:
+    import torch
+
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal(20000).astype(np.float32) * np.float32(100)
+    bits = x.view(np.uint32)
+    # plant exact ties (low 16 bits == 0x8000) with both parities of the kept lsb
+    ties = (bits[:4000] & np.uint32(0xFFFF0000)) | np.uint32(0x8000)
+    x = np.concatenate([x, ties.view(np.float32), np.float32([0.0, -0.0, 1.0, 3.4e38, -3.4e38, 1e-40])])
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = O.f32_to_bf16(x)
+    assert np.array_equal(got, ref), int(np.sum(got != ref))
+
+
+# --------------------------------------------------------------------------- quantiser
+def pin_quant_golden(O) -> None:
+    for case in _golden("quant_hand.json")["cases"]:
+        x = np.float32([case["x"]])
+        q, s = O.quantize_per_token(x)
+        assert q[0].tolist() == case["q"], (case["x"], q[0].tolist(), case["q"])
+        if "scale" in case:
+            assert float(s[0]) == case["scale"]
+        else:
+            target = case["scale_times_127_approx"]
+            assert abs(float(s[0]) * 127.0 - target) <= 1e-6 * target
+
+
+def _check_quant_invariants(x32: np.ndarray, q: np.ndarray, s: np.ndarray) -> None:
+    m, k = x32.shape
+    x64 = x32.astype(np.float64)
+    amax = np.abs(x64).max(axis=1)
+    for r in range(m):
+        sc = float(s[r])
+        floor = max(float(amax[r]), float(np.float32(1e-12)))
+        # scale is the fp32 rounding of max(amax, 1e-12) / 127: within half an ulp (+ the
+        # rounding of 1e-12 itself)
+        assert abs(sc * 127.0 - floor) <= 127.0 * ulp32(sc), (r, sc, floor)
+        # round trip: |x - q * scale| <= scale * (1/2 + 2^-16)
+        err = np.abs(x64[r] - q[r].astype(np.float64) * sc)
+        assert float(err.max()) <= sc * (0.5 + 2.0 ** -16), (r, float(err.max()), sc)
+        # range and the absmax element
+        assert int(np.abs(q[r].astype(np.int32)).max()) <= 127
+        if amax[r] >= 1e-12:
+            i = int(np.argmax(np.abs(x64[r])))
+            assert abs(int(q[r, i])) == 127 and np.sign(q[r, i]) == np.sign(x64[r, i])
+        # monotone: sorting x sorts q
+        order = np.argsort(x64[r], kind="stable")
+        assert np.all(np.diff(q[r][order].astype(np.int32)) >= 0)
+
+
+def pin_quant_invariants(O) -> None:
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((9, 333)).astype(np.float32)
+    x[1] *= 1e-3
+    x[2, 17] = 250.0  # one outlier
+    x[3] = 0.0
+    x[4] = 1e-14
+    x[5] = np.abs(x[5])
+    x[6] = -np.abs(x[6]) * 7
+    q, s = O.quantize_per_token(x)
+    _check_quant_invariants(x, q, s)
+    # zero row -> 0; a constant row below the 1e-12 floor -> round(1e-14 * 127 / 1e-12) = 1
+    assert np.all(q[3] == 0) and np.all(q[4] == 1)
+
+
+def pin_quant_bf16_path(O) -> None:
+    """bf16 input gives the same result as its exact fp32 widening."""
+    import torch
+
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 520)).astype(np.float32) * 3
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    bits = xb.view(torch.int16).numpy().view(np.uint16)
+    wide = xb.to(torch.float32).numpy()
+    q1, s1 = O.quantize_per_token(bits)
+    q2, s2 = O.quantize_per_token(wide)
+    assert np.array_equal(q1, q2) and np.array_equal(s1.view(np.uint32), s2.view(np.uint32))
+    _check_quant_invariants(wide, q1, s1)
+
+
+def pin_silu_quant(O) -> None:
+    """fused path == silu then quantise; packed [T, 2d] == separate tensors."""
+    import torch
+
+    rng = np.random.default_rng(9)
+    g = rng.standard_normal((5, 264)).astype(np.float32)
+    u = rng.standard_normal((5, 264)).astype(np.float32)
+    q, s = O.silu_mul_quant_per_token(g, u)
+    h = np.empty_like(g)
+    for r in range(5):
+        for i in range(264):
+            h[r, i] = np.float32(O.silu(float(g[r, i]))) * u[r, i]
+    _check_quant_invariants(h, q, s)
+    qh, sh = O.quantize_per_token(h)
+    assert np.array_equal(q, qh) and np.array_equal(s, sh)
+    gb = torch.from_numpy(g).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    ub = torch.from_numpy(u).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    q1, s1 = O.silu_mul_quant_per_token(gb, ub)
+    q2, s2 = O.silu_mul_quant_packed(np.concatenate([gb, ub], axis=1))
+    assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
+
+
+# --------------------------------------------------------------------------- GEMM
+def pin_gemm_bruteforce(O) -> None:
+    rng = np.random.default_rng(13)
+    for (m, n, k) in [(1, 1, 1), (3, 5, 7), (2, 9, 33), (16, 256, 512), (7, 13, 200)]:
+        a = rng.integers(-127, 128, (m, k), dtype=np.int8)
+        w = rng.integers(-127, 128, (n, k), dtype=np.int8)
+        ref = a.astype(np.int64) @ w.astype(np.int64).T
+        got = O.gemm_s32(a, w)
+        assert np.array_equal(got.astype(np.int64), ref), (m, n, k)
+
+
+def pin_gemm_closed_forms(O) -> None:
+    for k in (4096, 8192, 14336):
+        a = np.full((2, k), 127, np.int8)
+        w = np.full((3, k), 127, np.int8)
+        assert np.all(O.gemm_s32(a, w) == 16129 * k)
+        assert np.all(O.gemm_s32(a, -w) == -16129 * k)
+    # identity-like weights pick columns of a
+    rng = np.random.default_rng(17)
+    a = rng.integers(-127, 128, (4, 48), dtype=np.int8)
+    w = np.zeros((10, 48), np.int8)
+    for n in range(10):
+        w[n, n] = 1
+    assert np.array_equal(O.gemm_s32(a, w), a[:, :10].astype(np.int32))
+    # the int32 bound: K * 127^2 < 2^31 holds up to K = 133144 and fails after it
+    ok = O.gemm_s32(np.full((1, 133144), 127, np.int8), np.full((1, 133144), 127, np.int8))
+    assert int(ok[0, 0]) == 16129 * 133144 == 2147479576
+    try:
+        O.gemm_s32(np.full((1, 133145), 127, np.int8), np.full((1, 133145), 127, np.int8))
+    except OverflowError:
+        pass
+    else:
+        raise AssertionError("int32 overflow not reported")
+
+
+# --------------------------------------------------------------------------- epilogues
+def pin_epilogue_per_channel(O) -> None:
+    rng = np.random.default_rng(19)
+    m, n = 12, 40
+    acc = rng.integers(-2 ** 31 + 1, 2 ** 31 - 1, (m, n), dtype=np.int64).astype(np.int32)
+    acc[0, :] = rng.integers(-1000, 1000, n)
+    sa = rng.uniform(1e-4, 1.0, m).astype(np.float32)
+    sw = rng.uniform(1e-3, 1e-2, n).astype(np.float32)
+    for alpha in (1.0, 0.37):
+        got = O.epilogue_per_channel(acc, sa, sw, alpha).astype(np.float64)
+        exact = (acc.astype(np.float64) * sa.astype(np.float64)[:, None]
+                 * sw.astype(np.float64)[None, :] * np.float64(np.float32(alpha)))
+        # four binary32 roundings (int->float and three products): relative <= 4 * 2^-24 (+)
+        bound = 4.0001 * 2.0 ** -24 * np.abs(exact)
+        assert np.all(np.abs(got - exact) <= bound)
+    # exact powers of two
+    out = O.epilogue_per_channel(np.int32([[3, -5]]), np.float32([0.5]), np.float32([0.25, 4.0]), 2.0)
+    assert out.tolist() == [[0.75, -20.0]]
+
+
+def pin_group(O) -> None:
+    rng = np.random.default_rng(23)
+    for (m, n, k, grp) in [(3, 5, 256, 128), (4, 6, 384, 128), (2, 3, 192, 64)]:
+        a = rng.integers(-127, 128, (m, k), dtype=np.int8)
+        w = rng.integers(-127, 128, (n, k), dtype=np.int8)
+        ng = k // grp
+        sa = rng.uniform(1e-3, 1.0, m).astype(np.float32)
+        sw = rng.uniform(1e-3, 1e-2, (n, ng)).astype(np.float32)
+        alpha = 1.5
+        out, acc = O.gemm_group(a, w, sa, sw, grp, alpha)
+        parts = np.stack([a[:, g * grp:(g + 1) * grp].astype(np.int64)
+                          @ w[:, g * grp:(g + 1) * grp].astype(np.int64).T for g in range(ng)])
+        assert np.array_equal(acc.astype(np.int64), parts.sum(0))
+        terms = parts.astype(np.float64) * sw.astype(np.float64).T[:, None, :]
+        exact = terms.sum(0) * sa.astype(np.float64)[:, None] * alpha
+        mag = np.abs(terms).sum(0) * sa.astype(np.float64)[:, None] * alpha
+        bound = (ng + 2.0001) * 2.0 ** -24 * mag
+        assert np.all(np.abs(out.astype(np.float64) - exact) <= bound)
+    # one group with power-of-two scales is exact
+    a = np.int8([[1, 2, 3, 4]])
+    w = np.int8([[5, 6, 7, 8], [-1, -1, -1, -1]])
+    out, acc = O.gemm_group(a, w, np.float32([0.5]), np.float32([[0.25], [2.0]]), 4, 1.0)
+    assert acc.tolist() == [[70, -10]] and out.tolist() == [[8.75, -10.0]]
+
+
+# --------------------------------------------------------------------------- whole chain
+def pin_linear_golden(O) -> None:
+    g = _golden("linear_hand.json")
+    x = np.float32(g["x"])
+    w = np.int8(g["w"])
+    res = O.linear(x, w, np.float32(g["sw"]), 0, g["alpha"])
+    assert res["q"].tolist() == g["q"]
+    assert res["sa"].tolist() == g["sa"]
+    assert res["acc"].tolist() == g["acc"]
+    assert res["out_f32"].tolist() == g["out"]
+
+
+ALL_PINS = [pin_exp, pin_silu, pin_bf16_rounding, pin_quant_golden, pin_quant_invariants,
+            pin_quant_bf16_path, pin_silu_quant, pin_gemm_bruteforce, pin_gemm_closed_forms,
+            pin_epilogue_per_channel, pin_group, pin_linear_golden]

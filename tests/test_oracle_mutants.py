@@ -1,0 +1,75 @@
+"""Plant plausible mistakes in a copy of the oracle and require that the pins
+catch every one: a dropped term, a wrong sign, a wrong index, a transposed
+operand, the wrong rounding, the wrong qmax, the epsilon in the wrong place.
+
+The mistakes are planted on the CPU only, in a temporary copy of
+``oracle/qk_oracle.c``; the real oracle is untouched.
+"""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle_pins
+from oracle.oracle import Oracle, load
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle",
+                   "qk_oracle.c")
+
+# (name, original text, planted text) -- the original must occur exactly once.
+MUTANTS = [
+    ("qmax_128", "float s = fmaxf(amax, 1e-12f) / 127.0f;", "float s = fmaxf(amax, 1e-12f) / 128.0f;"),
+    ("eps_after_divide", "float s = fmaxf(amax, 1e-12f) / 127.0f;",
+     "float s = fmaxf(amax / 127.0f, 1e-12f);"),
+    ("round_half_away", "float r = nearbyintf(y);", "float r = roundf(y);"),
+    ("round_truncate", "float r = nearbyintf(y);", "float r = truncf(y);"),
+    ("absmax_signed", "float a = fabsf(x[i]);", "float a = x[i];"),
+    ("gemm_dropped_first_term", "for (int i = 0; i < k; ++i) s += (int64_t)ar[i] * (int64_t)wr[i];",
+     "for (int i = 1; i < k; ++i) s += (int64_t)ar[i] * (int64_t)wr[i];"),
+    ("gemm_transposed_w", "const int8_t* wr = j->w + (int64_t)c * k;",
+     "const int8_t* wr = j->w + (int64_t)(c % (j->m1 > 0 ? j->m1 : 1)) * k;"),
+    ("gemm_int8_wrap", "if (s > INT32_MAX || s < INT32_MIN) j->overflow = 1;", ""),
+    ("epi_wrong_scale_index", "o = o * sw[c];", "o = o * sw[r % n];"),
+    ("epi_wrong_sign", "o = o * sa[r];", "o = o * -sa[r];"),
+    ("epi_dropped_alpha", "      o = o * alpha;\n      out[", "      out["),
+    ("group_scale_transposed", "f = fmaf((float)(int32_t)p, j->sw[(int64_t)c * ng + g], f);",
+     "f = fmaf((float)(int32_t)p, j->sw[(int64_t)g * ng + c % ng], f);"),
+    ("group_dropped_last", "for (int g = 0; g < ng; ++g) {", "for (int g = 0; g < ng - 1; ++g) {"),
+    ("exp_wrong_coeff", "p = fmaf(p, r, (float)(1.0 / 24.0));", "p = fmaf(p, r, (float)(1.0 / 25.0));"),
+    ("exp_wrong_sign", "float e = qko_exp(-g);", "float e = qko_exp(g);"),
+    ("silu_times", "return g / d;", "return g * d;"),
+    ("bf16_round_half_up", "u += 0x7fffu + lsb;", "u += 0x8000u;"),
+    ("bf16_truncate", "u += 0x7fffu + lsb;", "u += 0u * lsb;"),
+    ("bf16_widen_wrong", "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)b) << 15;"),
+    ("silu_ld_ignored", "float u = qko_load(up, dtype, (int64_t)r * ld + i);",
+     "float u = qko_load(up, dtype, (int64_t)r * k + i);"),
+]
+
+
+@pytest.fixture(scope="module")
+def workdir(tmp_path_factory):
+    return tmp_path_factory.mktemp("mutants")
+
+
+@pytest.mark.parametrize("name,orig,planted", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(workdir, name, orig, planted):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc missing")
+    text = open(SRC).read()
+    assert text.count(orig) == 1, f"mutation anchor for {name} not unique"
+    src = os.path.join(workdir, f"{name}.c")
+    lib = os.path.join(workdir, f"lib{name}.so")
+    with open(src, "w") as f:
+        f.write(text.replace(orig, planted))
+    subprocess.run(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
+                    "-o", lib, src, "-lm"], check=True)
+    O = Oracle(load(lib), nthreads=2)
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(O)
+        except (AssertionError, OverflowError, ValueError) as e:  # a pin caught it
+            failed.append(pin.__name__)
+            del e
+    assert failed, f"planted mistake {name} passed every pin"
