@@ -1,0 +1,203 @@
+/*
+ * qk.h -- C ABI of the W8A8 INT8 quantized linear layer for NVIDIA B200
+ * (sm_100a).  Library: libqk.so (built from w8a8_int8_quantized_qk_b200/csrc).
+ *
+ * The layer has three stages, one entry point each:
+ *   1. qk_quantize_per_token / qk_silu_mul_quant_per_token -- dynamic
+ *      per-token symmetric INT8 quantisation of the activation, optionally
+ *      fused with silu(gate) * up;
+ *   2. + 3. qk_w8a8_gemm -- INT8 x INT8 GEMM with INT32 accumulation and a
+ *      fused dequantisation epilogue (per-token x per-output-channel, or
+ *      per-token x per-(channel, 128-wide K group) fp32 scales).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every tensor pointer is DEVICE memory owned by the caller.  The library
+ *   never allocates, frees or retains caller memory, and keeps no state
+ *   between calls except one device status word (qk_device_status) and the
+ *   cached properties (SM count, compute capability) of each device used.
+ * - Matrices are row-major and densely packed: x, q [m, k]; b (weights)
+ *   [n, k] with K contiguous (one output channel per row, nn.Linear layout);
+ *   out, c [m, n].
+ * - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and the call returns without synchronising.  Arguments are
+ *   checked on the host before anything is launched; a rejected call
+ *   launches nothing and writes nothing.
+ * - The return value is a qk_status.  No entry point throws, aborts, traps
+ *   or asserts on the device.
+ * - Values of int8 operands are in [-127, 127] (what the quantisers
+ *   produce); -128 and non-finite floating-point inputs are outside the
+ *   contract and are not checked.
+ */
+#ifndef QK_H_
+#define QK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of the C ABI are the only ones the library exports. */
+#if defined(__GNUC__)
+#define QK_API __attribute__((visibility("default")))
+#else
+#define QK_API
+#endif
+
+/* Version of this ABI.  qk_abi_version() returns the value the library was
+ * built with; a binding must refuse to use a library whose number differs
+ * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
+ * number baked into the binary and checked at import). */
+#define QK_ABI_VERSION 1
+
+typedef enum qk_status {
+  QK_OK = 0,
+  QK_ERR_INVALID_ARG = 1,    /* bad size, dtype, group size or NULL pointer */
+  QK_ERR_MISALIGNED = 2,     /* a pointer or row stride breaks its alignment rule */
+  QK_ERR_UNSUPPORTED = 3,    /* valid request this build does not implement
+                                (e.g. no sm_100 device) */
+  QK_ERR_OVERFLOW_BOUND = 4, /* k * 127^2 >= 2^31: the INT32 sum could overflow */
+  QK_ERR_CUDA = 5,           /* a CUDA runtime/driver call or launch failed */
+  QK_ERR_TIMEOUT = 6,        /* a kernel's bounded wait expired (device status) */
+  QK_ERR_WORKSPACE = 7       /* workspace NULL or smaller than the size query */
+} qk_status;
+
+typedef enum qk_dtype { QK_F32 = 0, QK_BF16 = 1 } qk_dtype;
+
+/* cudaStream_t is `struct CUstream_st *`; this alias keeps the header free of
+ * CUDA includes while staying the same type. */
+typedef struct CUstream_st* qk_stream;
+
+/* ABI number the library was built with (== QK_ABI_VERSION of its header). */
+QK_API int qk_abi_version(void);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+QK_API const char* qk_status_string(int status);
+
+/*
+ * qk_quantize_per_token -- dynamic per-token symmetric INT8 quantisation.
+ *
+ * Defined by: "write-int8-quantized-kernel" (agentmods skill), section
+ * "Inputs the agent should gather first": per-token granularity (one scale per
+ * activation row) and the symmetric range [-127, 127] with zero-point 0; and
+ * the vLLM PR "fused silu_and_mul + dynamic per-token FP8 quantization",
+ * Purpose / Algorithm: the scale of a token is max(absmax, 1e-12) / qmax of its
+ * own row, and values are quantised with the per-token inverse scale.  With
+ * qmax = 127, for every row r:
+ *     amax     = max_i |x[r, i]|                       (exact)
+ *     scale[r] = max(amax, 1e-12f) / 127.0f            (binary32, RN)
+ *     inv      = 1.0f / scale[r]                       (binary32, RN)
+ *     q[r, i]  = clamp(rint_half_even(x[r, i] * inv), -127, 127)
+ * scale is the DEQUANT multiplier: x ~= q * scale.
+ *
+ * m        rows (tokens), >= 0 (m == 0 is a no-op)
+ * k        row length, > 0 and a multiple of 16
+ * x        [m, k] fp32 or bf16 (x_dtype), 16-byte aligned
+ * q        [m, k] int8 output, 16-byte aligned
+ * scale    [m] fp32 output, 4-byte aligned
+ * Errors: QK_ERR_INVALID_ARG (m < 0, k <= 0, k % 16, NULL, bad dtype),
+ *         QK_ERR_MISALIGNED, QK_ERR_CUDA.
+ */
+QK_API qk_status qk_quantize_per_token(int m, int k, const void* x, qk_dtype x_dtype, int8_t* q,
+                                float* scale, qk_stream stream);
+
+/*
+ * qk_silu_mul_quant_per_token -- h = silu(gate) * up, then the per-token
+ * quantisation above applied to h.
+ *
+ * Defined by: the vLLM PR "fused silu_and_mul + dynamic per-token FP8
+ * quantization", Purpose / Algorithm (SiLU gating fused with dynamic
+ * per-token quantisation, scale from the row's own absmax), with qmax = 127.
+ * h is computed in fp32 and is not rounded to bf16 before quantisation:
+ *     e = exp(-g) (the library's fixed binary32 exp: Cody-Waite reduction,
+ *                  degree-7 Taylor polynomial, clamp to [-87, 88]);
+ *     silu = g / (1 + e);   h = silu * u          (binary32, RN)
+ * The kernel keeps h on chip, so gate and up are read from memory once.
+ *
+ * gate, up [m, k] with row stride ld_in ELEMENTS (ld_in >= k).  Pass the
+ * halves of one [m, 2k] buffer as gate = base, up = base + k, ld_in = 2k, or
+ * two separate [m, k] tensors with ld_in = k.  Both 16-byte aligned, and
+ * ld_in * element size a multiple of 16 bytes.
+ * q [m, k] int8, scale [m] fp32 as for qk_quantize_per_token.
+ * Errors: as qk_quantize_per_token, plus QK_ERR_INVALID_ARG if ld_in < k.
+ */
+QK_API qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, const void* up,
+                                      int64_t ld_in, qk_dtype in_dtype, int8_t* q, float* scale,
+                                      qk_stream stream);
+
+/*
+ * qk_w8a8_gemm -- INT8 x INT8 GEMM with INT32 accumulation and a fused
+ * dequantisation epilogue.
+ *
+ * Defined by: "16. Deploying Custom Kernels", section "C++ Kernel
+ * Interface" (GemmConfig: m, n, k, int8 a and b, int32 c, fp32 scale_a and
+ * scale_b, float output_scale, stream; status-returning quantized_gemm);
+ * "write-int8-quantized-kernel", Inputs (INT32 accumulation, FP32/FP16 output
+ * after dequantisation); "KV-cache kernels" (day 26), section 02 (int8
+ * products accumulate in int32 and are scaled by a_scale * b_scale at the
+ * end) and section 03 (per-group scales every 64-128 channels).
+ *
+ *   acc[i, j] = sum_k a[i, k] * b[j, k]                     (int32, exact)
+ *   group_k == 0   (per-token x per-channel):
+ *     out[i, j] = (((float)acc[i, j] * scale_a[i]) * scale_b[j]) * output_scale
+ *   group_k == 128 (per-token x per-(channel, K group)):
+ *     P_g = sum_{k in group g} a[i, k] * b[j, k]            (int32)
+ *     f = 0; for g = 0, 1, ...: f = fmaf((float)P_g, scale_b[j, g], f)
+ *     out[i, j] = (f * scale_a[i]) * output_scale
+ *   Each step is one binary32 RN operation, in the order written; a bf16
+ *   output is the round-to-nearest-even of the fp32 value.
+ *
+ * m, n, k        m >= 0, n >= 0 (either 0: no-op); k > 0, k % 16 == 0,
+ *                n % 8 == 0, and k <= 133144 so that k * 127^2 < 2^31
+ * a              [m, k] int8 activations (e.g. q of the quantiser), 16-B aligned
+ * b              [n, k] int8 weights, K contiguous, 16-B aligned
+ * scale_a        [m] fp32 per-token dequant scales
+ * scale_b        [n] fp32 (group_k == 0) or [n, k / 128] fp32 row-major
+ *                (group_k == 128); scale_a and scale_b 16-byte aligned
+ * group_k        0 or 128 (128 requires k % 128 == 0)
+ * output_scale   extra fp32 multiplier applied last (GemmConfig.output_scale)
+ * c              optional [m, n] int32 output of the full-K sum acc (in group
+ *                mode the sum of the group partials); NULL to skip; 16-B aligned
+ * out            optional [m, n] output in out_dtype (QK_BF16 or QK_F32);
+ *                NULL to skip; 16-B aligned.  At least one of c, out non-NULL.
+ * workspace      device scratch of at least qk_w8a8_gemm_workspace_size()
+ *                bytes, 256-B aligned; may be NULL when that size is 0.  The
+ *                call owns it until the work on `stream` completes.
+ * Errors: QK_ERR_INVALID_ARG, QK_ERR_MISALIGNED, QK_ERR_OVERFLOW_BOUND,
+ *         QK_ERR_WORKSPACE, QK_ERR_UNSUPPORTED, QK_ERR_CUDA.
+ */
+QK_API qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
+                       const float* scale_a, const float* scale_b, int group_k,
+                       float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
+                       void* workspace, size_t workspace_bytes, qk_stream stream);
+
+/* Bytes of workspace qk_w8a8_gemm needs for this problem (0 when none).
+ * Returns 0 for arguments qk_w8a8_gemm would reject. */
+QK_API size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k);
+
+/*
+ * qk_device_status -- read and clear the library's device status word on the
+ * current device.  Kernels that wait on a barrier give up after a bounded
+ * time (about one second) instead of hanging; when that happens they record
+ * QK_ERR_TIMEOUT there, release what they hold and return early, so their
+ * outputs are incomplete.  This call synchronises `stream` first; it returns
+ * QK_OK, QK_ERR_TIMEOUT or QK_ERR_CUDA.
+ */
+QK_API qk_status qk_device_status(qk_stream stream);
+
+/*
+ * qk_selftest_bounded_wait -- diagnostic: launch one block that waits on a
+ * barrier nobody arrives at, with a limit of `timeout_us` microseconds
+ * (1 .. 2,000,000).  When the limit passes the kernel records QK_ERR_TIMEOUT in
+ * the device status word and returns.  Lets a caller check, without any fault,
+ * that the bounded-wait path works on this device.
+ */
+QK_API qk_status qk_selftest_bounded_wait(int timeout_us, qk_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QK_H_ */

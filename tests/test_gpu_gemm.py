@@ -1,0 +1,157 @@
+"""GPU parity of qk_w8a8_gemm against the CPU oracle.
+
+INT32 accumulators bit-exact; fp32/bf16 outputs within the tolerance of
+gpu_util.check_out and, because the kernels keep the oracle's operation
+order, bit-identical as well.  Small shapes span several tiles with ragged
+M, N and K tails, on each kernel (decode GEMV for m <= 8, the tcgen05 kernel
+per channel and per 128-group); the five workloads run at full size with the
+oracle evaluated on sampled rows."""
+import numpy as np
+import pytest
+
+from gpu_util import assert_bits, check_out, dev, host, need_gpu, x_dev
+from oracle.oracle import Oracle
+from w8a8_int8_quantized_qk_b200 import qk, synth
+
+pytestmark = pytest.mark.gpu
+
+import torch  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def O():
+    need_gpu()
+    return Oracle()
+
+
+def _problem(m, n, k, group_k, seed):
+    r = synth.streams(seed, ["a", "w", "sa", "sw"])
+    a = synth.int8_uniform(r["a"], (m, k))
+    w = synth.int8_uniform(r["w"], (n, k))
+    sa = synth.scales_uniform(r["sa"], (m,), 0.001, 0.05)
+    sw = synth.scales_uniform(r["sw"], (n, k // group_k) if group_k else (n,))
+    return a, w, sa, sw
+
+
+def _run(a, w, sa, sw, group_k, alpha, out_dtype=torch.bfloat16, want_c=True):
+    out, c = qk.w8a8_gemm(dev(a), dev(w), dev(sa), dev(sw), group_k, alpha, out_dtype,
+                          want_out=out_dtype is not None, want_c=want_c)
+    torch.cuda.synchronize()
+    assert qk.device_status() == qk.QK_OK
+    return (None if out is None else host(out)), (None if c is None else host(c))
+
+
+SHAPES = [
+    # decode GEMV (m <= 8)
+    (1, 8, 16), (3, 24, 48), (4, 136, 272), (8, 1032, 4112), (5, 64, 1024),
+    # tcgen05 per-channel: one tile, tails in M / N / K, several tiles and waves
+    (9, 256, 128), (128, 256, 128), (130, 264, 272), (257, 520, 1040), (300, 1000, 1552),
+    (1024, 2048, 512), (640, 256, 4096), (17, 8, 16),
+]
+
+
+@pytest.mark.parametrize("m,n,k", SHAPES)
+def test_gemm_per_channel(O, m, n, k):
+    a, w, sa, sw = _problem(m, n, k, 0, seed=m * 131 + n * 7 + k)
+    alpha = 0.75
+    out, c = _run(a, w, sa, sw, 0, alpha)
+    ref = O.linear_from_q(a, sa, w, sw, 0, alpha)
+    assert_bits(c, ref["acc"], "acc")
+    exact = check_out(out, ref["out_f32"], ref["out_bf16"])
+    assert exact == 1.0, exact
+
+
+@pytest.mark.parametrize("m,n,k", [(4, 64, 256), (200, 264, 384)])
+def test_gemm_fp32_out_and_c_only(O, m, n, k):
+    a, w, sa, sw = _problem(m, n, k, 0, seed=77 + m)
+    out, c = _run(a, w, sa, sw, 0, 1.0, out_dtype=torch.float32)
+    ref = O.linear_from_q(a, sa, w, sw, 0, 1.0)
+    assert_bits(c, ref["acc"], "acc")
+    assert_bits(out, ref["out_f32"], "fp32 out")
+    out2, c2 = _run(a, w, sa, sw, 0, 1.0, out_dtype=None, want_c=True)
+    assert out2 is None
+    assert_bits(c2, ref["acc"], "acc (c only)")
+    out3, c3 = _run(a, w, sa, sw, 0, 1.0, want_c=False)
+    assert c3 is None
+    assert_bits(out3, ref["out_bf16"], "bf16 (out only)")
+
+
+GROUP_SHAPES = [(1, 128, 128), (7, 136, 256), (129, 136, 256), (200, 264, 384), (256, 512, 1024),
+                (333, 1032, 2048)]
+
+
+@pytest.mark.parametrize("m,n,k", GROUP_SHAPES)
+def test_gemm_group(O, m, n, k):
+    a, w, sa, sw = _problem(m, n, k, 128, seed=m * 17 + n + k)
+    alpha = 1.25
+    out, c = _run(a, w, sa, sw, 128, alpha)
+    ref = O.linear_from_q(a, sa, w, sw, 128, alpha)
+    assert_bits(c, ref["acc"], "acc")
+    exact = check_out(out, ref["out_f32"], ref["out_bf16"])
+    assert exact == 1.0, exact
+    out_nc, _ = _run(a, w, sa, sw, 128, alpha, want_c=False)
+    assert_bits(out_nc, out, "group out without c")
+
+
+def test_gemm_saturating_closed_form(O):
+    # all operands 127: acc = 16129 k at the largest k the bound allows (multiple of 128)
+    k = 133120
+    a = np.full((3, k), 127, np.int8)
+    w = np.full((16, k), 127, np.int8)
+    sa = np.ones(3, np.float32)
+    sw = np.ones(16, np.float32)
+    _, c = _run(a, w, sa, sw, 0, 1.0, out_dtype=None)
+    assert np.all(c == 16129 * k)
+    a9 = np.full((9, k), 127, np.int8)
+    _, c9 = _run(a9, -w, np.ones(9, np.float32), sw, 0, 1.0, out_dtype=None)
+    assert np.all(c9 == -16129 * k)
+
+
+def test_gemm_empty(O):
+    a = torch.empty((0, 64), dtype=torch.int8, device="cuda")
+    w = torch.zeros((16, 64), dtype=torch.int8, device="cuda")
+    sa = torch.empty((0,), dtype=torch.float32, device="cuda")
+    sw = torch.ones((16,), dtype=torch.float32, device="cuda")
+    out, _ = qk.w8a8_gemm(a, w, sa, sw)
+    assert out.shape == (0, 16)
+
+
+def _sample_rows(m, count, seed):
+    rows = np.unique(np.concatenate([[0, m - 1], np.random.default_rng(seed).choice(m, count)]))
+    return rows
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "mlp_down", "group"])
+def test_workload_full_size(O, name):
+    w = synth.make(name)
+    if name == "tiny":
+        # per-output-channel weight quantisation with the same per-row rule
+        w_q, sw = qk.quantize_per_token(dev(w.w_f32))
+        w_q_ref, sw_ref = O.quantize_per_token(w.w_f32)
+        assert_bits(host(w_q), w_q_ref, "weight q")
+        assert_bits(host(sw), sw_ref, "weight scale")
+        w_q_h, sw_h = w_q_ref, sw_ref
+    else:
+        w_q, sw = dev(w.w_q), dev(w.sw)
+        w_q_h, sw_h = w.w_q, w.sw
+    if name == "mlp_down":
+        q, sa = qk.silu_mul_quant_per_token(x_dev(w.gate), x_dev(w.up))
+        q_ref, sa_ref = O.silu_mul_quant_per_token(w.gate, w.up)
+    else:
+        q, sa = qk.quantize_per_token(x_dev(w.x))
+        q_ref, sa_ref = O.quantize_per_token(w.x)
+    assert_bits(host(q), q_ref, "q")
+    assert_bits(host(sa), sa_ref, "scale")
+    out_dtype = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    out, c = qk.w8a8_gemm(q, w_q, sa, sw, w.group_k, w.alpha, out_dtype, want_c=True)
+    torch.cuda.synchronize()
+    assert qk.device_status() == qk.QK_OK
+    rows = np.arange(w.m) if w.m <= 256 else _sample_rows(w.m, 40, seed=len(name))
+    ref = O.linear_from_q(q_ref[rows], sa_ref[rows], w_q_h, sw_h, w.group_k, w.alpha)
+    out_h, c_h = host(out), host(c)
+    assert_bits(c_h[rows], ref["acc"], "acc")
+    if out_dtype == torch.float32:
+        assert_bits(out_h[rows], ref["out_f32"], "fp32 out")
+    else:
+        exact = check_out(out_h[rows], ref["out_f32"], ref["out_bf16"])
+        assert exact == 1.0, exact

@@ -1,0 +1,539 @@
+// gemm_sm100.cuh -- large-M W8A8 GEMM on the 5th-generation tensor cores.
+//
+// acc = A[m, k] * B[n, k]^T in int32 ("write-int8-quantized-kernel", Inputs:
+// INT32 accumulation is mandatory; "KV-cache kernels" section 02: int8
+// products accumulate in int32 and the scales are applied at the end), then
+// the dequant epilogue in registers.  The pages' kernels (dp4a, a Triton
+// tl.dot loop, cuBLAS/CUTLASS) are prior art; this is the sm_100a form:
+//
+//  - one persistent CTA per SM walks output tiles (tile = blockIdx + i*grid);
+//  - warp 0 / lane 0 is the TMA producer: 128-byte-swizzled K-major tiles of
+//    A (128 x 128 B) and B (BN x 128 B) into a STAGES-deep shared-memory ring,
+//    completion counted in bytes on an mbarrier;
+//  - warp 1 / lane 0 issues tcgen05.mma.kind::i8 (M = 128, N = BN, K = 32,
+//    four per stage) into an int32 accumulator in tensor memory, and frees
+//    ring slots / publishes accumulators with tcgen05.commit;
+//  - epilogue warps read the accumulator with tcgen05.ld (32 lanes x 32
+//    columns per instruction), apply the scales and store the outputs;
+//  - per-channel mode keeps two 128 x 256 accumulators in TMEM (all 512
+//    columns), so the epilogue of tile i overlaps the MMAs of tile i+1;
+//  - per-group mode (group = 128 = one stage of K) keeps four 128 x 128
+//    int32 partial buffers in TMEM: the MMA writes one group's partial per
+//    buffer and moves on while eight epilogue warps convert each partial
+//    exactly to fp32 and fold it in with fmaf(P_g, s[n, g], f), in
+//    ascending group order, in registers.
+//
+// Every wait is bounded (about one second): on expiry the kernel records
+// QK_ERR_TIMEOUT, every role leaves its loop, the producer waits (bounded)
+// for its in-flight copies, the MMA thread waits for its in-flight MMAs, and
+// the TMEM is freed before the CTA exits.
+#pragma once
+
+#include "qk_common.cuh"
+
+namespace qk {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 128;     // K bytes per stage: one 128-byte swizzle row
+constexpr int UMMA_K = 32;  // K of one kind::i8 MMA instruction
+constexpr int kTmemCols = 512;
+
+struct Args {
+  int m, n, k;
+  const float* sa;  // [m]
+  const float* sw;  // [n] or [n, groups]
+  float alpha;
+  int32_t* c;       // [m, n] or null
+  void* out;        // [m, n] or null
+  int out_bf16;
+  int tiles_m, tiles_n, num_kb, groups;
+};
+
+template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
+struct alignas(1024) Storage {
+  uint8_t a[STAGES][BM * BK];
+  uint8_t b[STAGES][BN * BK];
+  float scales[SCALE_FLOATS > 0 ? SCALE_FLOATS : 1];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t acc_full[NACC];
+  uint64_t acc_empty[NACC];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
+// all lanes saw the phase complete.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  const bool all = __all_sync(0xFFFFFFFFu, ok);
+  if (!all) *abort = 1;
+  return all;
+}
+
+// ---------------------------------------------------------------- producer
+template <int BN, int STAGES, class S>
+__device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, const Args& p) {
+  const int ntiles = p.tiles_m * p.tiles_n;
+  const uint32_t bytes = static_cast<uint32_t>((BM + BN) * BK);
+  uint32_t stage = 0, phase = 0, issued = 0;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    for (int kb = 0; kb < p.num_kb; ++kb) {
+      if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, &s.abort)) {
+        ok = false;
+        break;
+      }
+      const uint32_t fb = smem_addr(&s.full[stage]);
+      mbar_arrive_expect_tx(fb, bytes);
+      tma_load_2d(smem_addr(s.a[stage]), tmA, fb, kb * BK, tm * BM);
+      tma_load_2d(smem_addr(s.b[stage]), tmB, fb, kb * BK, tn * BN);
+      ++issued;
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  // No copy may still be landing in shared memory when the CTA exits: wait
+  // (bounded, ignoring the abort flag) for the last STAGES copies issued.
+  const uint32_t first = issued > STAGES ? issued - STAGES : 0u;
+  for (uint32_t i = first; i < issued; ++i)
+    mbar_wait(smem_addr(&s.full[i % STAGES]), (i / STAGES) & 1u, nullptr);
+}
+
+// ---------------------------------------------------------------- MMA issuer
+// GROUP: one accumulator buffer per K block (each K block is one group);
+// otherwise one buffer per tile.
+template <int BN, int STAGES, int NACC, bool GROUP, class S>
+__device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
+  const int ntiles = p.tiles_m * p.tiles_n;
+  constexpr uint32_t idesc = idesc_i8(BM, BN);
+  uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    if (!GROUP) {
+      if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) break;
+      tc_fence_after();
+    }
+    for (int kb = 0; kb < p.num_kb; ++kb) {
+      if (GROUP) {
+        if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (!mbar_wait(smem_addr(&s.full[stage]), phase, &s.abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d = tmem + abuf * BN;
+      const uint32_t a0 = smem_addr(s.a[stage]);
+      const uint32_t b0 = smem_addr(s.b[stage]);
+#pragma unroll
+      for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+        const uint32_t acc = GROUP ? (kk > 0) : (kb > 0 || kk > 0);
+        mma_i8(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc, acc);
+      }
+      mma_commit(smem_addr(&s.empty[stage]));
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      if (GROUP) {
+        mma_commit(smem_addr(&s.acc_full[abuf]));
+        if (++abuf == NACC) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
+      }
+    }
+    if (!GROUP && ok) {
+      mma_commit(smem_addr(&s.acc_full[abuf]));
+      if (++abuf == NACC) {
+        abuf = 0;
+        aphase ^= 1u;
+      }
+    }
+  }
+  // Every MMA issued must be complete before the TMEM can be released.
+  mma_commit(smem_addr(&s.drain));
+  mbar_wait(smem_addr(&s.drain), 0u, nullptr);
+}
+
+// ---------------------------------------------------------------- epilogues
+// 8 consecutive outputs (row, col .. col+7) from 8 int32 accumulators.
+__device__ __forceinline__ void store8_channel(const Args& p, int row, int col, float sa,
+                                               const uint32_t* v) {
+  const int64_t o = static_cast<int64_t>(row) * p.n + col;
+  if (p.c) {
+    int4* dst = reinterpret_cast<int4*>(p.c + o);
+    dst[0] = make_int4(v[0], v[1], v[2], v[3]);
+    dst[1] = make_int4(v[4], v[5], v[6], v[7]);
+  }
+  if (p.out) {
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.sw + col));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.sw + col + 4));
+    const float sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float t = __int2float_rn(static_cast<int>(v[j]));
+      t = __fmul_rn(t, sa);
+      t = __fmul_rn(t, sw[j]);
+      f[j] = __fmul_rn(t, p.alpha);
+    }
+    if (p.out_bf16) {
+      uint4 pk;
+      pk.x = pack_bf16x2(f[0], f[1]);
+      pk.y = pack_bf16x2(f[2], f[3]);
+      pk.z = pack_bf16x2(f[4], f[5]);
+      pk.w = pack_bf16x2(f[6], f[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o) = pk;
+    } else {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
+      dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+      dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+  }
+}
+
+// Per-channel epilogue, 4 warps; warp (w % 4) owns TMEM lanes 32*(w%4) ..
+template <int BN, int NACC, class S>
+__device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p) {
+  const int ntiles = p.tiles_m * p.tiles_n;
+  const int lane = threadIdx.x & 31;
+  const int quad = (threadIdx.x >> 5) & 3;
+  uint32_t abuf = 0, aphase = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    if (!warp_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) break;
+    tc_fence_after();
+    const int row = tm * BM + quad * 32 + lane;
+    const bool rv = row < p.m;
+    const float sa = rv ? __ldg(p.sa + row) : 0.0f;
+    const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN;
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tb + ch * 32, v);
+      tmem_ld_wait();
+      const int col0 = tn * BN + ch * 32;
+      if (rv) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          if (col0 + g * 8 < p.n) store8_channel(p, row, col0 + g * 8, sa, v + g * 8);
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[abuf]));
+    if (++abuf == NACC) {
+      abuf = 0;
+      aphase ^= 1u;
+    }
+  }
+}
+
+// Per-group epilogue, 8 warps: warp w (2..9) owns TMEM lanes 32*(w%4) and
+// columns [64*h, 64*h + 64) of the 128-column tile, h = (w - 2) / 4.  Each
+// warp stages the scales of its 64 columns for SG groups at a time in its own
+// slice of shared memory (only __syncwarp is needed, so an abort can never
+// strand a warp at a CTA-wide barrier).
+constexpr int kGroupCols = 64;
+constexpr int kScaleGroups = 16;
+
+template <int BN, int NACC, bool WITH_C, class S>
+__device__ void epilogue_group(S& s, uint32_t tmem, const Args& p) {
+  const int ntiles = p.tiles_m * p.tiles_n;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int quad = warp & 3;
+  const int half = (warp - 2) >> 2;
+  float* ws = s.scales + (warp - 2) * (kScaleGroups * kGroupCols);  // [SG][64]
+  uint32_t abuf = 0, aphase = 0;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    const int colbase = tn * BN + half * kGroupCols;
+    float f[kGroupCols];
+    int cs[WITH_C ? kGroupCols : 1];
+#pragma unroll
+    for (int j = 0; j < kGroupCols; ++j) f[j] = 0.0f;
+    if constexpr (WITH_C) {
+#pragma unroll
+      for (int j = 0; j < kGroupCols; ++j) cs[j] = 0;
+    }
+    for (int g = 0; g < p.groups; ++g) {
+      const int gs = g % kScaleGroups;
+      if (gs == 0) {
+        __syncwarp();
+        // lane owns columns lane and lane + 32 of this warp's 64
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int col = colbase + lane + 32 * cc;
+          const float* src = p.sw + static_cast<int64_t>(col) * p.groups + g;
+#pragma unroll 4
+          for (int gg = 0; gg < kScaleGroups; ++gg) {
+            const bool in = col < p.n && g + gg < p.groups;
+            ws[gg * kGroupCols + lane + 32 * cc] = in ? __ldg(src + gg) : 0.0f;
+          }
+        }
+        __syncwarp();
+      }
+      if (!warp_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[kGroupCols];
+      const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN +
+                          half * kGroupCols;
+      tmem_ld_32x32b_x32(tb, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld_32x32b_x32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[abuf]));
+      if (++abuf == NACC) {
+        abuf = 0;
+        aphase ^= 1u;
+      }
+      const float4* sc = reinterpret_cast<const float4*>(ws + gs * kGroupCols);
+#pragma unroll
+      for (int j4 = 0; j4 < kGroupCols / 4; ++j4) {
+        const float4 s4 = sc[j4];
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = j4 * 4 + e;
+          // |P| < 2^22: adding P to the bits of 1.5 * 2^23 and subtracting
+          // 1.5 * 2^23 gives (float)P exactly.
+          const float pf = __fsub_rn(__int_as_float(static_cast<int>(v[j]) + 0x4B400000),
+                                     12582912.0f);
+          f[j] = __fmaf_rn(pf, sv[e], f[j]);
+          if constexpr (WITH_C) cs[j] += static_cast<int>(v[j]);
+        }
+      }
+    }
+    if (!ok) break;
+    const int row = tm * BM + quad * 32 + lane;
+    if (row < p.m) {
+      const float sa = __ldg(p.sa + row);
+#pragma unroll
+      for (int g8 = 0; g8 < kGroupCols / 8; ++g8) {
+        const int col = colbase + g8 * 8;
+        if (col >= p.n) break;
+        const int64_t o = static_cast<int64_t>(row) * p.n + col;
+        float r[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = __fmul_rn(__fmul_rn(f[g8 * 8 + e], sa), p.alpha);
+        if (p.out) {
+          if (p.out_bf16) {
+            uint4 pk;
+            pk.x = pack_bf16x2(r[0], r[1]);
+            pk.y = pack_bf16x2(r[2], r[3]);
+            pk.z = pack_bf16x2(r[4], r[5]);
+            pk.w = pack_bf16x2(r[6], r[7]);
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o) = pk;
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
+            dst[0] = make_float4(r[0], r[1], r[2], r[3]);
+            dst[1] = make_float4(r[4], r[5], r[6], r[7]);
+          }
+        }
+        if constexpr (WITH_C) {
+          int4* dst = reinterpret_cast<int4*>(p.c + o);
+          dst[0] = make_int4(cs[g8 * 8 + 0], cs[g8 * 8 + 1], cs[g8 * 8 + 2], cs[g8 * 8 + 3]);
+          dst[1] = make_int4(cs[g8 * 8 + 4], cs[g8 * 8 + 5], cs[g8 * 8 + 6], cs[g8 * 8 + 7]);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- kernels
+template <class S>
+__device__ __forceinline__ S& storage(uint8_t* raw) {
+  return *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+template <class S, int STAGES, int NACC, int EPI_WARPS>
+__device__ __forceinline__ void setup(S& s) {
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(smem_addr(&s.full[i]), 1);
+      mbar_init(smem_addr(&s.empty[i]), 1);
+    }
+    for (int i = 0; i < NACC; ++i) {
+      mbar_init(smem_addr(&s.acc_full[i]), 1);
+      mbar_init(smem_addr(&s.acc_empty[i]), EPI_WARPS);
+    }
+    mbar_init(smem_addr(&s.drain), 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&s.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+template <class S>
+__device__ __forceinline__ void teardown(S& s, uint32_t tmem) {
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if ((threadIdx.x >> 5) == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+constexpr int kChannelBN = 256;
+constexpr int kChannelStages = 4;
+constexpr int kChannelThreads = 64 + 4 * 32;
+using ChannelStorage = Storage<kChannelBN, kChannelStages, 2, 0>;
+
+__global__ void __launch_bounds__(kChannelThreads, 1)
+    gemm_i8_channel_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmB, const Args p) {
+  extern __shared__ uint8_t smem_raw[];
+  ChannelStorage& s = storage<ChannelStorage>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  setup<ChannelStorage, kChannelStages, 2, 4>(s);
+  const uint32_t tmem = s.tmem_base;
+  if (warp == 0) {
+    if (lane == 0) produce<kChannelBN, kChannelStages>(s, &tmA, &tmB, p);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false>(s, tmem, p);
+    __syncwarp();
+  } else {
+    epilogue_channel<kChannelBN, 2>(s, tmem, p);
+  }
+  teardown(s, tmem);
+}
+
+constexpr int kGroupBN = 128;
+constexpr int kGroupStages = 5;
+constexpr int kGroupThreads = 64 + 8 * 32;
+using GroupStorage = Storage<kGroupBN, kGroupStages, 4, 8 * kScaleGroups * kGroupCols>;
+
+template <bool WITH_C>
+__global__ void __launch_bounds__(kGroupThreads, 1)
+    gemm_i8_group_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB, const Args p) {
+  extern __shared__ uint8_t smem_raw[];
+  GroupStorage& s = storage<GroupStorage>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  setup<GroupStorage, kGroupStages, 4, 8>(s);
+  const uint32_t tmem = s.tmem_base;
+  if (warp == 0) {
+    if (lane == 0) produce<kGroupBN, kGroupStages>(s, &tmA, &tmB, p);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) mma_issue<kGroupBN, kGroupStages, 4, true>(s, tmem, p);
+    __syncwarp();
+  } else {
+    epilogue_group<kGroupBN, 4, WITH_C>(s, tmem, p);
+  }
+  teardown(s, tmem);
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// int8 [rows, k] row-major, box = 128 bytes of K x box_rows rows, 128-byte
+// swizzle; out-of-range rows/columns read as zero.
+inline bool make_tmap(CUtensorMap* map, const void* base, int rows, int k, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+inline size_t channel_smem() { return sizeof(ChannelStorage) + 1024; }
+inline size_t group_smem() { return sizeof(GroupStorage) + 1024; }
+
+// 0 ok, 1 tensor-map failure, 2 CUDA error
+inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int num_sms,
+                  cudaStream_t stream, cudaError_t* err) {
+  const int bn = group ? kGroupBN : kChannelBN;
+  a.tiles_m = (a.m + BM - 1) / BM;
+  a.tiles_n = (a.n + bn - 1) / bn;
+  a.num_kb = (a.k + BK - 1) / BK;
+  a.groups = group ? a.k / 128 : 0;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, A, a.m, a.k, BM) || !make_tmap(&tb, B, a.n, a.k, bn)) return 1;
+  const int ntiles = a.tiles_m * a.tiles_n;
+  const int grid = ntiles < num_sms ? ntiles : num_sms;
+  cudaError_t e;
+  if (!group) {
+    const size_t smem = channel_smem();
+    e = cudaFuncSetAttribute(gemm_i8_channel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e == cudaSuccess) {
+      gemm_i8_channel_kernel<<<grid, kChannelThreads, smem, stream>>>(ta, tb, a);
+      e = cudaGetLastError();
+    }
+  } else {
+    const size_t smem = group_smem();
+    if (a.c) {
+      e = cudaFuncSetAttribute(gemm_i8_group_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) {
+        gemm_i8_group_kernel<true><<<grid, kGroupThreads, smem, stream>>>(ta, tb, a);
+        e = cudaGetLastError();
+      }
+    } else {
+      e = cudaFuncSetAttribute(gemm_i8_group_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e == cudaSuccess) {
+        gemm_i8_group_kernel<false><<<grid, kGroupThreads, smem, stream>>>(ta, tb, a);
+        e = cudaGetLastError();
+      }
+    }
+  }
+  *err = e;
+  return e == cudaSuccess ? 0 : 2;
+}
+
+}  // namespace gemm
+}  // namespace qk

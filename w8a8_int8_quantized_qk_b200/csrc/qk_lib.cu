@@ -1,0 +1,236 @@
+// qk_lib.cu -- the C ABI of libqk.so (declared in include/qk.h): argument
+// checks on the host, then one kernel launch per stage on the caller's
+// stream.  All kernels of the library are compiled in this one translation
+// unit, so the device status word is a single symbol.
+//
+// Interface source: "16. Deploying Custom Kernels", C++ Kernel Interface
+// (GemmConfig's m, n, k, int8 a / b, int32 c, scale_a, scale_b,
+// output_scale, stream; a status-returning entry point) and Python Bindings
+// (the same fields passed as plain integers, pointers and a float).
+#include <mutex>
+
+#include "gemm_sm100.cuh"
+#include "gemv.cuh"
+#include "qk_common.cuh"
+#include "quant.cuh"
+
+namespace qk {
+namespace {
+
+struct DeviceInfo {
+  bool valid = false;
+  int sms = 0;
+  int major = 0;
+  int minor = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_devices_mu;
+
+// Properties of the current device (cached); nullptr on a CUDA error.
+const DeviceInfo* current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_devices_mu);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.valid) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return nullptr;
+    d.valid = true;
+  }
+  return &d;
+}
+
+// The kernels are built for sm_100a only, which runs on compute capability
+// 10.0 devices.
+qk_status check_device(const DeviceInfo** out) {
+  const DeviceInfo* d = current_device();
+  if (d == nullptr) return QK_ERR_CUDA;
+  if (d->major != 10 || d->minor != 0) return QK_ERR_UNSUPPORTED;
+  *out = d;
+  return QK_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+// K * 127^2 < 2^31  <=>  K <= 133144
+constexpr int kMaxK = 133144;
+
+qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, qk_dtype dt,
+                       int8_t* q, float* scale, qk_stream stream, bool silu) {
+  if (m < 0 || k <= 0 || (k % 16) != 0) return QK_ERR_INVALID_ARG;
+  if (dt != QK_F32 && dt != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (ld < k) return QK_ERR_INVALID_ARG;
+  if (m == 0) return QK_OK;
+  if (x == nullptr || q == nullptr || scale == nullptr || (silu && up == nullptr))
+    return QK_ERR_INVALID_ARG;
+  const int64_t esize = dt == QK_BF16 ? 2 : 4;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale, 4) || (silu && !aligned(up, 16)) ||
+      (ld * esize) % 16 != 0)
+    return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  quant::Args a;
+  a.m = m;
+  a.k = k;
+  a.x = x;
+  a.up = up;
+  a.ld = ld;
+  a.q = q;
+  a.scale = scale;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = silu ? quant::launch<true>(a, dt == QK_BF16, dev->sms, s)
+                             : quant::launch<false>(a, dt == QK_BF16, dev->sms, s);
+  return e == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+}
+
+// Which kernel runs a GEMM of this shape.
+enum class GemmPath { kGemv, kTensorChannel, kTensorGroup };
+
+GemmPath gemm_path(int m, int group_k) {
+  if (group_k != 0) return GemmPath::kTensorGroup;
+  if (m <= gemv::max_tokens()) return GemmPath::kGemv;
+  return GemmPath::kTensorChannel;
+}
+
+qk_status gemm_check(int m, int n, int k, int group_k) {
+  if (m < 0 || n < 0 || k <= 0) return QK_ERR_INVALID_ARG;
+  if ((k % 16) != 0 || (n % 8) != 0) return QK_ERR_INVALID_ARG;
+  if (group_k != 0 && group_k != 128) return QK_ERR_INVALID_ARG;
+  if (group_k == 128 && (k % 128) != 0) return QK_ERR_INVALID_ARG;
+  if (k > kMaxK) return QK_ERR_OVERFLOW_BOUND;
+  return QK_OK;
+}
+
+// Device-side bounded-wait check: one thread waits on a barrier that no one
+// arrives at.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    fence_mbar_init();
+    mbar_wait(smem_addr(&bar), 0u, nullptr, limit_ns);
+  }
+}
+
+}  // namespace
+}  // namespace qk
+
+using namespace qk;
+
+extern "C" {
+
+int qk_abi_version(void) { return QK_ABI_VERSION; }
+
+const char* qk_status_string(int status) {
+  switch (status) {
+    case QK_OK: return "ok";
+    case QK_ERR_INVALID_ARG: return "invalid argument";
+    case QK_ERR_MISALIGNED: return "misaligned pointer or row stride";
+    case QK_ERR_UNSUPPORTED: return "unsupported (needs a compute capability 10.0 device)";
+    case QK_ERR_OVERFLOW_BOUND: return "k too large: k * 127^2 must stay below 2^31";
+    case QK_ERR_CUDA: return "CUDA error";
+    case QK_ERR_TIMEOUT: return "a kernel's bounded wait expired";
+    case QK_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+qk_status qk_quantize_per_token(int m, int k, const void* x, qk_dtype x_dtype, int8_t* q,
+                                float* scale, qk_stream stream) {
+  return quant_common(m, k, x, nullptr, k, x_dtype, q, scale, stream, false);
+}
+
+qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, const void* up,
+                                      int64_t ld_in, qk_dtype in_dtype, int8_t* q, float* scale,
+                                      qk_stream stream) {
+  return quant_common(m, k, gate, up, ld_in, in_dtype, q, scale, stream, true);
+}
+
+size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
+  (void)m;
+  (void)n;
+  (void)k;
+  (void)group_k;
+  return 0;
+}
+
+qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
+                       const float* scale_a, const float* scale_b, int group_k,
+                       float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
+                       void* workspace, size_t workspace_bytes, qk_stream stream) {
+  qk_status st = gemm_check(m, n, k, group_k);
+  if (st != QK_OK) return st;
+  if (out != nullptr && out_dtype != QK_F32 && out_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return QK_OK;
+  if (a == nullptr || b == nullptr || (c == nullptr && out == nullptr)) return QK_ERR_INVALID_ARG;
+  if (out != nullptr && (scale_a == nullptr || scale_b == nullptr)) return QK_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(c, 16) || !aligned(out, 16) ||
+      !aligned(scale_a, 16) || !aligned(scale_b, 16))
+    return QK_ERR_MISALIGNED;
+  const size_t need = qk_w8a8_gemm_workspace_size(m, n, k, group_k);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
+    return QK_ERR_WORKSPACE;
+  const DeviceInfo* dev = nullptr;
+  st = check_device(&dev);
+  if (st != QK_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const GemmPath path = gemm_path(m, group_k);
+  if (path == GemmPath::kGemv) {
+    gemv::Args g;
+    g.m = m;
+    g.n = n;
+    g.k = k;
+    g.a = a;
+    g.w = b;
+    g.sa = scale_a;
+    g.sw = scale_b;
+    g.alpha = output_scale;
+    g.c = c;
+    g.out = out;
+    g.out_bf16 = out_dtype == QK_BF16;
+    return gemv::launch(g, dev->sms, s) == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  }
+  gemm::Args g;
+  g.m = m;
+  g.n = n;
+  g.k = k;
+  g.sa = scale_a;
+  g.sw = scale_b;
+  g.alpha = output_scale;
+  g.c = c;
+  g.out = out;
+  g.out_bf16 = out_dtype == QK_BF16;
+  cudaError_t e = cudaSuccess;
+  const int r = gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev->sms, s, &e);
+  if (r == 1) return QK_ERR_CUDA;
+  return r == 0 ? QK_OK : QK_ERR_CUDA;
+}
+
+qk_status qk_device_status(qk_stream stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QK_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, qk::g_status, sizeof v) != cudaSuccess) return QK_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(qk::g_status, &zero, sizeof zero) != cudaSuccess) return QK_ERR_CUDA;
+  return static_cast<qk_status>(v);
+}
+
+qk_status qk_selftest_bounded_wait(int timeout_us, qk_stream stream) {
+  if (timeout_us < 1 || timeout_us > 2000000) return QK_ERR_INVALID_ARG;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+}
+
+}  // extern "C"

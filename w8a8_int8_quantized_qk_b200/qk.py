@@ -1,0 +1,234 @@
+"""Python binding of libqk.so -- argument marshalling only.
+
+Two layers:
+
+* ctypes functions with the C names (``qk_quantize_per_token``,
+  ``qk_silu_mul_quant_per_token``, ``qk_w8a8_gemm``, ...) taking plain ints,
+  device pointers and a stream handle, exactly as ``include/qk.h`` declares
+  them (the ctypes binding shape follows "16. Deploying Custom Kernels",
+  Python Bindings: sizes as ints, tensors as pointers, a status return);
+* torch helpers (:func:`quantize_per_token`, :func:`silu_mul_quant_per_token`,
+  :func:`w8a8_gemm`, :func:`linear`) that allocate outputs with torch, pass
+  ``data_ptr()`` and the current stream, and raise :class:`QKError` on a
+  non-zero status.
+
+Every arithmetic step runs in the library's CUDA kernels; there is no CPU
+fallback: a missing library or a non-CUDA tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libqk.so")
+
+ABI_VERSION = 1
+
+QK_OK = 0
+QK_ERR_INVALID_ARG = 1
+QK_ERR_MISALIGNED = 2
+QK_ERR_UNSUPPORTED = 3
+QK_ERR_OVERFLOW_BOUND = 4
+QK_ERR_CUDA = 5
+QK_ERR_TIMEOUT = 6
+QK_ERR_WORKSPACE = 7
+
+QK_F32 = 0
+QK_BF16 = 1
+
+# name -> (restype, argtypes), in include/qk.h order
+_P = ctypes.c_void_p
+_SIGNATURES = {
+    "qk_abi_version": (ctypes.c_int, []),
+    "qk_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qk_quantize_per_token": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P]),
+    "qk_silu_mul_quant_per_token": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int64,
+                                                   ctypes.c_int, _P, _P, _P]),
+    "qk_w8a8_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
+                                    ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "qk_w8a8_gemm_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "qk_device_status": (ctypes.c_int, [_P]),
+    "qk_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_int, _P]),
+}
+
+_lib: ctypes.CDLL | None = None
+
+
+class QKError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        msg = status_string(status) if _lib is not None else str(status)
+        super().__init__(f"{where}: qk status {status} ({msg})" if where else f"qk status {status} ({msg})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqk.so and check its ABI number; raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m w8a8_int8_quantized_qk_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        got = L.qk_abi_version()
+        if got != ABI_VERSION:
+            raise RuntimeError(f"libqk.so ABI {got} != binding ABI {ABI_VERSION}: rebuild the library")
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().qk_status_string(status).decode()
+
+
+# ---------------------------------------------------------------- C names
+def qk_abi_version() -> int:
+    return lib().qk_abi_version()
+
+
+def qk_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def qk_quantize_per_token(m, k, x, x_dtype, q, scale, stream) -> int:
+    return lib().qk_quantize_per_token(m, k, x, x_dtype, q, scale, stream)
+
+
+def qk_silu_mul_quant_per_token(m, k, gate, up, ld_in, in_dtype, q, scale, stream) -> int:
+    return lib().qk_silu_mul_quant_per_token(m, k, gate, up, ld_in, in_dtype, q, scale, stream)
+
+
+def qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
+                 workspace, workspace_bytes, stream) -> int:
+    return lib().qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
+                              out_dtype, workspace, workspace_bytes, stream)
+
+
+def qk_w8a8_gemm_workspace_size(m, n, k, group_k) -> int:
+    return lib().qk_w8a8_gemm_workspace_size(m, n, k, group_k)
+
+
+def qk_device_status(stream) -> int:
+    return lib().qk_device_status(stream)
+
+
+def qk_selftest_bounded_wait(timeout_us, stream) -> int:
+    return lib().qk_selftest_bounded_wait(timeout_us, stream)
+
+
+# ---------------------------------------------------------------- torch helpers
+def _torch():
+    import torch
+
+    return torch
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p | None:
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return QK_BF16
+    if t.dtype == torch.float32:
+        return QK_F32
+    raise TypeError(f"expected bfloat16 or float32, got {t.dtype}")
+
+
+def _check(st: int, where: str) -> None:
+    if st != QK_OK:
+        raise QKError(st, where)
+
+
+def _need_cuda(*ts) -> None:
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libqk works on CUDA tensors only (no CPU fallback)")
+
+
+def quantize_per_token(x, q=None, scale=None, stream=None):
+    """x [m, k] bf16/fp32 (CUDA, contiguous) -> (q int8 [m, k], scale fp32 [m])."""
+    torch = _torch()
+    _need_cuda(x)
+    assert x.dim() == 2 and x.is_contiguous()
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=x.device) if q is None else q
+    scale = torch.empty((m,), dtype=torch.float32, device=x.device) if scale is None else scale
+    _check(qk_quantize_per_token(m, k, _ptr(x), _dtype_code(x), _ptr(q), _ptr(scale), _stream(stream)),
+           "qk_quantize_per_token")
+    return q, scale
+
+
+def silu_mul_quant_per_token(gate, up, q=None, scale=None, stream=None):
+    """gate, up [m, k] (same dtype and row stride) -> (q int8 [m, k], scale fp32 [m]).
+    gate/up may be the two halves of one [m, 2k] tensor (row stride 2k)."""
+    torch = _torch()
+    _need_cuda(gate, up)
+    assert gate.shape == up.shape and gate.dtype == up.dtype and gate.dim() == 2
+    assert gate.stride(1) == 1 and up.stride(1) == 1 and gate.stride(0) == up.stride(0)
+    m, k = gate.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=gate.device) if q is None else q
+    scale = torch.empty((m,), dtype=torch.float32, device=gate.device) if scale is None else scale
+    _check(qk_silu_mul_quant_per_token(m, k, _ptr(gate), _ptr(up), gate.stride(0), _dtype_code(gate),
+                                       _ptr(q), _ptr(scale), _stream(stream)),
+           "qk_silu_mul_quant_per_token")
+    return q, scale
+
+
+def silu_mul_quant_packed(gu, stream=None):
+    """gu [m, 2k]: gate = gu[:, :k], up = gu[:, k:]."""
+    k = gu.shape[1] // 2
+    return silu_mul_quant_per_token(gu[:, :k], gu[:, k:], stream=stream)
+
+
+def w8a8_gemm(a, b, scale_a, scale_b, group_k: int = 0, output_scale: float = 1.0,
+              out_dtype=None, want_out: bool = True, want_c: bool = False, out=None, c=None,
+              workspace=None, stream=None):
+    """a int8 [m, k], b int8 [n, k] -> (out [m, n] or None, c int32 [m, n] or None)."""
+    torch = _torch()
+    _need_cuda(a, b, scale_a, scale_b)
+    m, k = a.shape
+    n = b.shape[0]
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if want_out and out is None:
+        out = torch.empty((m, n), dtype=out_dtype, device=a.device)
+    if want_c and c is None:
+        c = torch.empty((m, n), dtype=torch.int32, device=a.device)
+    need = qk_w8a8_gemm_workspace_size(m, n, k, group_k)
+    if need and workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=a.device)
+    code = _dtype_code(out) if out is not None else QK_BF16
+    _check(qk_w8a8_gemm(m, n, k, _ptr(a), _ptr(b), _ptr(scale_a), _ptr(scale_b), group_k,
+                        float(output_scale), _ptr(c), _ptr(out), code, _ptr(workspace),
+                        0 if workspace is None else workspace.numel(), _stream(stream)),
+           "qk_w8a8_gemm")
+    return out, c
+
+
+def linear(x, w_q, sw, group_k: int = 0, output_scale: float = 1.0, out_dtype=None, stream=None):
+    """The whole W8A8 linear layer: quantise x per token, INT8 GEMM, dequant."""
+    q, sa = quantize_per_token(x, stream=stream)
+    out, _ = w8a8_gemm(q, w_q, sa, sw, group_k, output_scale, out_dtype, stream=stream)
+    return out
+
+
+def mlp_down(gate, up, w_q, sw, output_scale: float = 1.0, out_dtype=None, stream=None):
+    """silu(gate) * up, quantised per token, then the INT8 down projection."""
+    q, sa = silu_mul_quant_per_token(gate, up, stream=stream)
+    out, _ = w8a8_gemm(q, w_q, sa, sw, 0, output_scale, out_dtype, stream=stream)
+    return out
+
+
+def device_status(stream=None) -> int:
+    return qk_device_status(_stream(stream))
