@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""Benchmark of the W8A8 INT8 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One STEP is one pass of the whole hot path over one batch: per-token INT8
+quantisation of the activation, then the INT8 GEMM with its fused dequant
+epilogue.  The headline workload is the prefill linear layer (X bf16
+[4096, 4096], W int8 [4096, 4096], per-channel scales, bf16 out); ``value``
+is INT8 TOPS of the whole step (2*M*N*K per step / step time).  The same JSON
+line carries:
+
+* ``decode``   -- the decode linear layer's weight-stream GB/s (X bf16
+  [4, 4096], W int8 [14336, 4096]) with its HBM roofline;
+* ``stages``   -- per-stage device time and roofline fraction of all five
+  workloads (quantiser, fused SiLU quantiser, GEMV, tcgen05 GEMM per channel
+  and per 128-group);
+* ``roofline`` -- the dominant kernel (the GEMM) against the tensor peak;
+* ``e2e``      -- the same metric through the public API with host buffers
+  (pinned host -> device copy of X and device -> host copy of the output
+  inside the timed region);
+* ``cpu_baseline`` -- the CPU oracle on a bounded sample of rows.
+
+L2 (126 MB) is defeated by rotating several copies of every input and output
+(working set >= 3x L2), so steps run back to back.  Times are CUDA events on
+the launching stream; with N GPUs (torchrun) each rank runs an independent
+replica (no collective on the data path), the time is the max over ranks and
+``value`` sums all ranks' work ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill INT8 TOPS and decode weight-stream GB/s, % of B200 roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks() -> dict:
+    """Roofline denominators: the driver's measured peaks when present."""
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        p = {"hbm_gbs": float(m["hbm_gbs"]), "bf16_tflops": float(m["bf16_tflops"]),
+             "bf16_tflops_sustained": float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+             "source": "measured"}
+    # dense INT8 on B200 is nominally twice dense bf16 (4.5 vs 2.25 POPS)
+    p["int8_tops"] = 2.0 * p["bf16_tflops"]
+    return p
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML every ~2 ms, and runs
+    the nvidia-smi sampler (200 ms) alongside; use as a context manager around
+    the timed region."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, smi_csv: str | None = None):
+        self.index = index
+        self.samples: list[tuple[int, int]] = []
+        self.max_mhz = None
+        self.smi_csv = smi_csv
+        self._stop = threading.Event()
+        self._thr = None
+        self._smi = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: report no samples
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.smi_csv:
+            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            try:
+                self._smi = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv",
+                                              "-lms", "200", "-i", str(self.index)],
+                                             stdout=open(self.smi_csv, "w"), stderr=subprocess.DEVNULL)
+            except OSError:
+                self._smi = None
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+        if self._smi is not None:
+            self._smi.terminate()
+            self._smi.wait()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [name for b, name in self.REASONS.items() if bits & b]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(mhz), "reasons": reasons, "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------- helpers
+def _dev(torch, a, bf16=False):
+    import numpy as np
+
+    if bf16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _copies(bytes_per_copy: int, floor: int = 2) -> int:
+    return max(floor, -(-3 * L2_BYTES // max(bytes_per_copy, 1)))
+
+
+class Timer:
+    """Per-stage CUDA events on one stream."""
+
+    def __init__(self, torch, stream, stages: list[str], steps: int):
+        self.torch = torch
+        self.stream = stream
+        self.stages = stages
+        self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+                   for _ in range(steps)]
+
+    def mark(self, step: int, i: int):
+        self.ev[step][i].record(self.stream)
+
+    def per_stage_ms(self) -> dict:
+        out = {}
+        for i, name in enumerate(self.stages):
+            out[name] = statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in self.ev)
+        out["step"] = statistics.fmean(e[0].elapsed_time(e[-1]) for e in self.ev)
+        return out
+
+
+class Linear:
+    """A workload resident on the device in R rotating copies; step(i, timer)
+    runs quantise + GEMM through the C ABI on copy i % R."""
+
+    def __init__(self, torch, qk, w, stream, copies: int | None = None):
+        import ctypes
+
+        self.torch, self.qk, self.w = torch, qk, w
+        self.stream = ctypes.c_void_p(stream.cuda_stream)
+        m, n, k = w.m, w.n, w.k
+        silu = w.gate is not None
+        xb = (w.gate.nbytes + w.up.nbytes) if silu else w.x.nbytes
+        per_copy = xb + w.w_q.nbytes + m * k + m * n * (4 if w.out_dtype == "f32" else 2)
+        self.R = copies or _copies(per_copy)
+        bf = w.x_dtype == "bf16"
+        if silu:
+            g0, u0 = _dev(torch, w.gate, bf), _dev(torch, w.up, bf)
+            self.xs = [(g0.clone(), u0.clone()) for _ in range(self.R)]
+        else:
+            x0 = _dev(torch, w.x, bf)
+            self.xs = [x0.clone() for _ in range(self.R)]
+        w0 = _dev(torch, w.w_q)
+        self.ws = [w0.clone() for _ in range(self.R)]
+        self.sw = _dev(torch, w.sw)
+        self.qs = [torch.empty((m, k), dtype=torch.int8, device="cuda") for _ in range(self.R)]
+        self.sas = [torch.empty((m,), dtype=torch.float32, device="cuda") for _ in range(self.R)]
+        odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+        self.outs = [torch.empty((m, n), dtype=odt, device="cuda") for _ in range(self.R)]
+        self.xdt = qk.QK_BF16 if bf else qk.QK_F32
+        self.odt = qk.QK_F32 if w.out_dtype == "f32" else qk.QK_BF16
+        P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        self.p = []
+        for j in range(self.R):
+            xp = (P(self.xs[j][0]), P(self.xs[j][1])) if silu else (P(self.xs[j]), None)
+            self.p.append((xp, P(self.ws[j]), P(self.qs[j]), P(self.sas[j]), P(self.outs[j])))
+        self.swp = P(self.sw)
+        self.silu = silu
+        self.launches_per_step = 2
+        ws = qk.qk_w8a8_gemm_workspace_size(m, n, k, w.group_k)
+        self.wsb = torch.empty((max(ws, 1),), dtype=torch.uint8, device="cuda")
+        self.wsp, self.wsn = P(self.wsb), ws
+
+    def quant(self, j: int):
+        w, qk = self.w, self.qk
+        (xp, up), _, qp, sap, _ = self.p[j]
+        if self.silu:
+            st = qk.qk_silu_mul_quant_per_token(w.m, w.k, xp, up, w.k, self.xdt, qp, sap, self.stream)
+        else:
+            st = qk.qk_quantize_per_token(w.m, w.k, xp, self.xdt, qp, sap, self.stream)
+        if st != 0:
+            raise qk.QKError(st, "quantize")
+
+    def gemm(self, j: int):
+        w, qk = self.w, self.qk
+        _, wp, qp, sap, op = self.p[j]
+        st = qk.qk_w8a8_gemm(w.m, w.n, w.k, qp, wp, sap, self.swp, w.group_k, w.alpha, None, op,
+                             self.odt, self.wsp, self.wsn, self.stream)
+        if st != 0:
+            raise qk.QKError(st, "gemm")
+
+    def step(self, i: int, timer: Timer | None = None, ti: int = 0):
+        j = i % self.R
+        if timer:
+            timer.mark(ti, 0)
+        self.quant(j)
+        if timer:
+            timer.mark(ti, 1)
+        self.gemm(j)
+        if timer:
+            timer.mark(ti, 2)
+
+
+def _bytes(w) -> dict:
+    """Algorithmic bytes of each stage: every operand read once, every result
+    written once."""
+    m, n, k = w.m, w.n, w.k
+    if w.gate is not None:
+        qb = w.gate.nbytes + w.up.nbytes + m * k + 4 * m
+    else:
+        qb = w.x.nbytes + m * k + 4 * m
+    ob = m * n * (4 if w.out_dtype == "f32" else 2)
+    gb = m * k + w.w_q.nbytes + 4 * m + w.sw.nbytes + ob
+    return {"quant": qb, "gemm": gb}
+
+
+def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
+    from w8a8_int8_quantized_qk_b200 import synth
+
+    w = synth.make(name)
+    if w.w_q is None:  # tiny: quantise the fp32 weight per output channel first
+        wq, sw = qk.quantize_per_token(_dev(torch, w.w_f32))
+        torch.cuda.synchronize()
+        w.w_q, w.sw = wq.cpu().numpy(), sw.cpu().numpy()
+    stream = torch.cuda.current_stream()
+    L = Linear(torch, qk, w, stream)
+    for i in range(5):
+        L.step(i)
+    t = Timer(torch, stream, ["quant", "gemm"], iters)
+    for i in range(iters):
+        L.step(i, t, i)
+    torch.cuda.synchronize()
+    ms = t.per_stage_ms()
+    by = _bytes(w)
+    ops = 2.0 * w.m * w.n * w.k
+    gemm_kernel = "gemv (CUDA cores)" if (w.m <= 8 and not w.group_k) else (
+        "tcgen05 group-128" if w.group_k else "tcgen05 per-channel")
+    res = {"m": w.m, "n": w.n, "k": w.k, "copies": L.R,
+           "quant_kernel": "silu_mul_quant" if w.gate is not None else "quantize_per_token",
+           "quant_us": ms["quant"] * 1e3, "quant_GBs": by["quant"] / (ms["quant"] * 1e-3) / 1e9,
+           "quant_hbm_frac": by["quant"] / (ms["quant"] * 1e-3) / 1e9 / pk["hbm_gbs"],
+           "gemm_kernel": gemm_kernel, "gemm_us": ms["gemm"] * 1e3,
+           "gemm_TOPS": ops / (ms["gemm"] * 1e-3) / 1e12,
+           "gemm_GBs": by["gemm"] / (ms["gemm"] * 1e-3) / 1e9,
+           "gemm_tensor_frac": ops / (ms["gemm"] * 1e-3) / 1e12 / pk["int8_tops"],
+           "gemm_hbm_frac": by["gemm"] / (ms["gemm"] * 1e-3) / 1e9 / pk["hbm_gbs"],
+           "step_us": ms["step"] * 1e3, "bytes": by}
+    del L
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline(seconds: float = 10.0) -> dict:
+    """The oracle, as it stands, on a bounded sample of rows of the prefill
+    workload: quantise those rows, INT8 GEMM + per-channel epilogue."""
+    import numpy as np
+
+    from oracle.oracle import Oracle
+    from w8a8_int8_quantized_qk_b200 import synth
+
+    w = synth.make("prefill")
+    O = Oracle()
+
+    def run(rows):
+        x = np.ascontiguousarray(w.x[:rows])
+        t0 = time.perf_counter()
+        O.linear(x, w.w_q, w.sw)
+        return time.perf_counter() - t0
+
+    rows = max(1, min(O.nthreads, 64))
+    t = run(rows)
+    rows = int(min(w.m, max(rows, rows * seconds / max(t, 1e-3))))
+    t = run(rows)
+    ops = 2.0 * rows * w.n * w.k
+    return {"value": ops / t / 1e12, "unit": "TOPS", "cores": min(O.nthreads, rows),
+            "kind": "oracle", "seconds": t,
+            "sample": f"{rows} of {w.m} rows of the prefill workload (quantise + INT8 GEMM + "
+                      f"per-channel epilogue, {2 * rows * w.n * w.k / 1e9:.1f} Gop)"}
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args):
+    """The oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    from oracle.oracle import Oracle
+    from w8a8_int8_quantized_qk_b200 import synth
+
+    w = synth.make("prefill")
+    O = Oracle()
+    # rows per step sized so that warmup + steps stay around two minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = max(1, min(O.nthreads, 32))
+    t0 = time.perf_counter()
+    O.linear(np.ascontiguousarray(w.x[:rows]), w.w_q, w.sw)
+    t1 = time.perf_counter() - t0
+    rows = int(min(w.m, max(1, rows * budget / max(t1, 1e-3))))
+    x = np.ascontiguousarray(w.x[:rows])
+    for _ in range(args.warmup):
+        O.linear(x, w.w_q, w.sw)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.linear(x, w.w_q, w.sw)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    ops = 2.0 * rows * w.n * w.k
+    val = ops / dt / 1e12
+    sample = f"{rows} of {w.m} rows of the prefill workload per step"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "prefill linear X bf16 [4096,4096] x W int8 [4096,4096]^T, "
+                                   "per-token x per-channel scales, bf16 out (CPU oracle sample)",
+                       "m": rows, "n": w.n, "k": w.k},
+            "cpu_baseline": {"value": val, "unit": "TOPS", "cores": min(O.nthreads, rows),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    from w8a8_int8_quantized_qk_b200 import qk, synth
+
+    qk.lib()
+    pk = peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---- headline: prefill step (quantise + GEMM), device-resident inputs
+    w = synth.make("prefill")
+    L = Linear(torch, qk, w, stream)
+    for i in range(args.warmup):
+        L.step(i)
+    timer = Timer(torch, stream, ["quant", "gemm"], args.steps)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                          if args.smi else None)
+    barrier()
+    with clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            L.step(args.warmup + i, timer, i)
+        end.record(stream)
+        barrier()
+    total_ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st = timer.per_stage_ms()
+    ops_step = 2.0 * w.m * w.n * w.k
+    ms_per_step = total_ms / args.steps
+    value = world * ops_step * args.steps / (total_ms * 1e-3) / 1e12
+    by = _bytes(w)
+    gemm_tops = ops_step / (st["gemm"] * 1e-3) / 1e12
+    roof = {"kernel": "gemm_i8_channel_kernel (tcgen05)", "bound": "tensor",
+            "achieved": gemm_tops, "peak": pk["int8_tops"], "unit": "TFLOP/s",
+            "frac": gemm_tops / pk["int8_tops"], "traffic": args.gemm_traffic,
+            "peak_note": f"2 x {pk['source']} bf16 burst ({pk['bf16_tflops']} TFLOP/s): the nominal "
+                         "dense int8:bf16 ratio; int8 ops counted as 2*M*N*K",
+            "algorithmic_bytes": by["gemm"],
+            "launch_us": st["gemm"] * 1e3, "quant_us": st["quant"] * 1e3,
+            "quant_GBs": by["quant"] / (st["quant"] * 1e-3) / 1e9,
+            "quant_hbm_frac": by["quant"] / (st["quant"] * 1e-3) / 1e9 / pk["hbm_gbs"]}
+
+    # ---- e2e through the public API with host buffers
+    e2e = None
+    if not args.quick:
+        import numpy as np
+
+        xh = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+        oh = torch.empty((w.m, w.n), dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty((w.m, w.k), dtype=torch.bfloat16, device="cuda")
+        wd, swd = L.ws[0], L.sw
+        for _ in range(3):
+            xd.copy_(xh, non_blocking=True)
+            oh.copy_(qk.linear(xd, wd, swd), non_blocking=True)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        steps_e2e = max(3, min(args.steps, 20))
+        e0.record(stream)
+        for _ in range(steps_e2e):
+            xd.copy_(xh, non_blocking=True)
+            oh.copy_(qk.linear(xd, wd, swd), non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * ops_step * steps_e2e / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 2),
+               "ms_per_step": e2e_ms / steps_e2e, "steps": steps_e2e,
+               "api": "qk.linear (qk_quantize_per_token + qk_w8a8_gemm) on pinned host buffers"}
+    del L
+    torch.cuda.empty_cache()
+
+    # ---- decode + per-stage table of every workload
+    stages = {}
+    decode = None
+    if not args.quick:
+        for name in ("decode", "prefill", "mlp_down", "group", "tiny"):
+            stages[name] = measure_workload(torch, qk, name, args.stage_iters, pk)
+        d = stages["decode"]
+        gbs = d["bytes"]["gemm"] / (d["gemm_us"] * 1e-6) / 1e9
+        decode = {"value": gbs, "unit": "GB/s", "workload": "decode linear X bf16 [4,4096] x W int8 "
+                  "[14336,4096]^T, bf16 out", "kernel": "gemv_i8_kernel (dp4a, CUDA cores)",
+                  "gemv_us": d["gemm_us"], "algorithmic_bytes": d["bytes"]["gemm"],
+                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                               "traffic": args.gemv_traffic},
+                  "quant_us": d["quant_us"], "step_us": d["step_us"]}
+    if dist is not None:
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    cpu = None
+    if not args.quick and not args.no_cpu and world == 1:
+        cpu = cpu_baseline(args.cpu_seconds)
+    line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "prefill linear: X bf16 [4096,4096] quantised per token to int8, "
+                                   "W int8 [4096,4096], per-channel fp32 scales, INT32 accumulation, "
+                                   "bf16 out", "m": w.m, "n": w.n, "k": w.k,
+                       "parallelism": f"replicas x{world}",
+                       "l2": f"rotating {_copies(w.x.nbytes + w.w_q.nbytes + w.m * w.k + 2 * w.m * w.n)}"
+                             " copies of inputs/outputs (working set >= 3x L2)"},
+            "gpu_launches": args.steps * 2, "roofline": roof, "clocks": clocks.summary(),
+            "e2e": e2e, "decode": decode, "cpu_baseline": cpu, "stages": stages,
+            "peaks": pk, "gpu": torch.cuda.get_device_name(local)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline only (for profiling runs)")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-smi", dest="smi", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--stage-iters", type=int, default=50)
+    ap.add_argument("--gemm-traffic", type=float, default=None,
+                    help="ncu dram bytes per GEMM launch, when captured for the current build")
+    ap.add_argument("--gemv-traffic", type=float, default=None)
+    ap.add_argument("--only", choices=["tiny", "decode", "prefill", "mlp_down", "group"],
+                    help="profiling aid: time one workload's stages and print them")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.only:
+        import torch
+
+        from w8a8_int8_quantized_qk_b200 import qk
+
+        res = measure_workload(torch, qk, args.only, args.steps, peaks())
+        print(json.dumps({"only": args.only, **res}), flush=True)
+        return 0
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
