@@ -206,7 +206,7 @@ class Linear:
         self.silu = silu
         self.launches_per_step = 2
         ws = qk.qk_w8a8_gemm_workspace_size(m, n, k, w.group_k)
-        self.wsb = torch.empty((max(ws, 1),), dtype=torch.uint8, device="cuda")
+        self.wsb = torch.zeros((max(ws, 1),), dtype=torch.uint8, device="cuda")
         self.wsp, self.wsn = P(self.wsb), ws
 
     def quant(self, j: int):

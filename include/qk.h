@@ -163,8 +163,16 @@ QK_API qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, con
  * out            optional [m, n] output in out_dtype (QK_BF16 or QK_F32);
  *                NULL to skip; 16-B aligned.  At least one of c, out non-NULL.
  * workspace      device scratch of at least qk_w8a8_gemm_workspace_size()
- *                bytes, 256-B aligned; may be NULL when that size is 0.  The
- *                call owns it until the work on `stream` completes.
+ *                bytes, 256-B aligned; may be NULL when that size is 0.  It
+ *                is used when the output has too few tiles to occupy the GPU
+ *                and K is split across CTA pairs (partial INT32 sums plus a
+ *                4 KB header of arrival counters).  It must be zero-filled
+ *                before its first use; every completed call leaves the
+ *                header zero again, so one workspace (sized for the largest
+ *                problem) can be reused across calls and shapes.  The call
+ *                owns it until the work on `stream` completes: calls that
+ *                may overlap need separate workspaces.  After a call that
+ *                ended in QK_ERR_TIMEOUT, zero-fill it again.
  * Errors: QK_ERR_INVALID_ARG, QK_ERR_MISALIGNED, QK_ERR_OVERFLOW_BOUND,
  *         QK_ERR_WORKSPACE, QK_ERR_UNSUPPORTED, QK_ERR_CUDA.
  */
@@ -173,7 +181,8 @@ QK_API qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t
                        float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
                        void* workspace, size_t workspace_bytes, qk_stream stream);
 
-/* Bytes of workspace qk_w8a8_gemm needs for this problem (0 when none).
+/* Bytes of workspace qk_w8a8_gemm needs for this problem on the current
+ * device (0 when none; the split depends on the device's SM count).
  * Returns 0 for arguments qk_w8a8_gemm would reject. */
 QK_API size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k);
 

@@ -76,6 +76,32 @@ def test_gemm_fp32_out_and_c_only(O, m, n, k):
     assert_bits(out3, ref["out_bf16"], "bf16 (out only)")
 
 
+SPLIT_SHAPES = [(200, 512, 4096), (300, 520, 2048), (256, 1024, 14336), (129, 264, 1024)]
+
+
+@pytest.mark.parametrize("m,n,k", SPLIT_SHAPES)
+def test_gemm_split_k(O, m, n, k):
+    # few output tiles: K is split across CTA pairs and the partial sums meet
+    # in the workspace; run twice (the arrival counters must be back at zero)
+    a, w, sa, sw = _problem(m, n, k, 0, seed=m + 3 * n + k)
+    ref = O.linear_from_q(a, sa, w, sw, 0, 1.5)
+    for _ in range(2):
+        out, c = _run(a, w, sa, sw, 0, 1.5)
+        assert_bits(c, ref["acc"], "acc")
+        assert_bits(out, ref["out_bf16"], "bf16 out")
+
+
+def test_gemm_split_k_needs_workspace(O):
+    m, n, k = 200, 512, 4096
+    need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 0)
+    assert need > 0
+    a, w, sa, sw = (dev(t) for t in _problem(m, n, k, 0, seed=1))
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    st = qk.qk_w8a8_gemm(m, n, k, qk._ptr(a), qk._ptr(w), qk._ptr(sa), qk._ptr(sw), 0, 1.0, None,
+                         qk._ptr(out), qk.QK_BF16, None, 0, qk._stream())
+    assert st == qk.QK_ERR_WORKSPACE
+
+
 GROUP_SHAPES = [(1, 128, 128), (7, 136, 256), (129, 136, 256), (200, 264, 384), (256, 512, 1024),
                 (333, 1032, 2048)]
 

@@ -67,6 +67,25 @@ def test_silu_wide_range(O):
     assert_bits(host(s), sr, "scale")
 
 
+def test_quant_half_amax_ties(O):
+    # x = amax / 2 makes RN(x * inv) an exact tie at +-63.5 for most amax while
+    # the exact product is not a tie; q must come from the rounded product
+    # (two roundings, as written), not from a fused multiply-add.
+    r = np.random.default_rng(21)
+    amax = (r.uniform(1, 100, 512)).astype(np.float32)
+    x = np.zeros((512, 64), np.float32)
+    x[:, 0] = amax
+    x[:, 1:33] = (amax / 2)[:, None] * np.where(r.random((512, 32)) < 0.5, -1, 1)
+    x[:, 33:] = (r.standard_normal((512, 31)) * (amax / 8)[:, None])
+    import torch
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    for xin in (x, xb.view(torch.int16).numpy().view(np.uint16)):
+        q, s = qk.quantize_per_token(x_dev(xin))
+        qr, sr = O.quantize_per_token(xin)
+        assert_bits(host(q), qr, "q")
+        assert_bits(host(s), sr, "scale")
+
+
 def test_quant_special_rows(O):
     k = 256
     x = np.zeros((8, k), np.float32)

@@ -48,6 +48,12 @@ struct Args {
   void* out;        // [m, n] or null
   int out_bf16;
   int tiles_m, tiles_n, num_kb, groups;
+  // split-K (pair kernel): each tile's K range is cut into `splits` pieces of
+  // `kb_per_split` K blocks; partial sums meet in `ws` with per-region
+  // arrival counters `cnt` (zero before the call, zero again after it).
+  int splits, kb_per_split;
+  int32_t* ws;
+  int* cnt;
 };
 
 template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
@@ -64,10 +70,15 @@ struct alignas(1024) Storage {
   int abort;
 };
 
-// Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
-// all lanes saw the phase complete.
+// Warp-uniform bounded wait: lane 0 polls (so a waiting warp does not flood
+// the shared-memory pipe the tensor core reads its operands through), then
+// every lane confirms the completed phase once for itself; the warp
+// proceeds only if all lanes saw it complete.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort);
+  ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+  if (ok) ok = mbar_wait(bar, parity, abort);
   const bool all = __all_sync(0xFFFFFFFFu, ok);
   if (!all) *abort = 1;
   return all;
@@ -455,6 +466,312 @@ __global__ void __launch_bounds__(kGroupThreads, 1)
   teardown(s, tmem);
 }
 
+// ---------------------------------------------------------------- CTA-pair kernel
+// Pair tile 256 x 256: CTA rank r of the cluster owns rows [128 r, 128 r + 128)
+// of the tile and loads them (A) plus rows [128 r, 128 r + 128) of the
+// tile's 256 B rows (the N half the MMA reads from it).  The leader's single
+// MMA thread issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32); each
+// CTA's TMEM receives its 128 rows x 256 columns.  Per SM and stage this
+// moves 32 KB for 128 x 256 x 128 MACs, two thirds of the single-CTA
+// 128 x 256 tile's 48 KB.  Both CTAs' copies complete on the leader's full
+// barrier; the leader's commits arrive on both CTAs' empty / acc_full
+// barriers; both CTAs' epilogue warps arrive on the leader's acc_empty.
+constexpr int kPairBM = 256;
+constexpr int kPairBN = 256;
+constexpr int kPairStages = 6;
+constexpr int kPairEpiWarps = 8;  // two per TMEM lane quadrant, 128 columns each
+constexpr int kPairThreads = 64 + kPairEpiWarps * 32;
+constexpr uint32_t kPairStageBytes = 2u * 128u * BK;  // per CTA: A half + B half
+
+struct alignas(1024) PairStorage {
+  uint8_t a[kPairStages][128 * BK];
+  uint8_t b[kPairStages][128 * BK];
+  float sw_tile[kPairEpiWarps][kPairBN / 2];  // each epilogue warp's channel scales
+  uint64_t full[kPairStages];
+  uint64_t empty[kPairStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUtensorMap* tmB,
+                             const Args& p, uint32_t rank) {
+  const int nunits = p.tiles_m * p.tiles_n * p.splits;
+  const int npairs = gridDim.x >> 1;
+  uint32_t stage = 0, phase = 0, issued = 0;
+  bool ok = true;
+  for (int unit = blockIdx.x >> 1; ok && unit < nunits; unit += npairs) {
+    const int tile = unit / p.splits, split = unit % p.splits;
+    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    const int ya = tm * kPairBM + static_cast<int>(rank) * 128;
+    const int yb = tn * kPairBN + static_cast<int>(rank) * 128;
+    const int kb0 = split * p.kb_per_split;
+    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, &s.abort)) {
+        ok = false;
+        break;
+      }
+      const uint32_t fb_local = smem_addr(&s.full[stage]);
+      if (rank == 0) mbar_arrive_expect_tx(fb_local, 2u * kPairStageBytes);
+      const uint32_t fb = map_to_rank(fb_local, 0);
+      tma_load_2d_pair(smem_addr(s.a[stage]), tmA, fb, kb * BK, ya);
+      tma_load_2d_pair(smem_addr(s.b[stage]), tmB, fb, kb * BK, yb);
+      ++issued;
+      if (++stage == kPairStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  // Both CTAs' copies complete on the leader's barriers: the leader waits
+  // (bounded) for the last phases it armed before the pair may exit.
+  if (rank == 0) {
+    const uint32_t first = issued > kPairStages ? issued - kPairStages : 0u;
+    for (uint32_t i = first; i < issued; ++i)
+      mbar_wait(smem_addr(&s.full[i % kPairStages]), (i / kPairStages) & 1u, nullptr);
+  }
+}
+
+__device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p) {
+  const int nunits = p.tiles_m * p.tiles_n * p.splits;
+  const int npairs = gridDim.x >> 1;
+  constexpr uint32_t idesc = idesc_i8(kPairBM, kPairBN);
+  uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
+  bool ok = true;
+  for (int unit = blockIdx.x >> 1; ok && unit < nunits; unit += npairs) {
+    const int split = unit % p.splits;
+    const int kb0 = split * p.kb_per_split;
+    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+    if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) break;
+    tc_fence_after();
+    const uint32_t d = tmem + abuf * kPairBN;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(smem_addr(&s.full[stage]), phase, &s.abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a0 = smem_addr(s.a[stage]);
+      const uint32_t b0 = smem_addr(s.b[stage]);
+#pragma unroll
+      for (int kk = 0; kk < BK / UMMA_K; ++kk)
+        mma_i8_pair(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc,
+                    (kb > kb0 || kk > 0) ? 1u : 0u);
+      mma_commit_pair(smem_addr(&s.empty[stage]), 0x3);
+      if (++stage == kPairStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok) break;
+    mma_commit_pair(smem_addr(&s.acc_full[abuf]), 0x3);
+    if (++abuf == 2) {
+      abuf = 0;
+      aphase ^= 1u;
+    }
+  }
+  mma_commit_pair(smem_addr(&s.drain), 0x1);
+  mbar_wait(smem_addr(&s.drain), 0u, nullptr);
+}
+
+// 32 outputs of one row (columns col0 .. col0 + 31) from 32 accumulators;
+// channel scales come from shared memory.
+__device__ __forceinline__ void store32_channel(const Args& p, int row, int col0, float sa,
+                                                const float* sw, const uint32_t (&v)[32]) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int col = col0 + g * 8;
+    if (col >= p.n) break;
+    const int64_t o = static_cast<int64_t>(row) * p.n + col;
+    if (p.c) {
+      int4* dst = reinterpret_cast<int4*>(p.c + o);
+      dst[0] = make_int4(v[g * 8 + 0], v[g * 8 + 1], v[g * 8 + 2], v[g * 8 + 3]);
+      dst[1] = make_int4(v[g * 8 + 4], v[g * 8 + 5], v[g * 8 + 6], v[g * 8 + 7]);
+    }
+    if (p.out) {
+      const float4 s0 = *reinterpret_cast<const float4*>(sw + g * 8);
+      const float4 s1 = *reinterpret_cast<const float4*>(sw + g * 8 + 4);
+      const float s8[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      float f[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float t = __int2float_rn(static_cast<int>(v[g * 8 + j]));
+        t = __fmul_rn(t, sa);
+        t = __fmul_rn(t, s8[j]);
+        f[j] = __fmul_rn(t, p.alpha);
+      }
+      if (p.out_bf16) {
+        uint4 pk;
+        pk.x = pack_bf16x2(f[0], f[1]);
+        pk.y = pack_bf16x2(f[2], f[3]);
+        pk.z = pack_bf16x2(f[4], f[5]);
+        pk.w = pack_bf16x2(f[6], f[7]);
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o) = pk;
+      } else {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
+        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+      }
+    }
+  }
+}
+
+// Epilogue of the pair kernel: 8 warps per CTA; warp w (2..9) reads TMEM
+// lanes 32*(w%4) (rows) and columns [128 h, 128 h + 128), h = (w - 2) / 4.
+// The tile's channel scales are staged per warp in shared memory, the row's
+// token scale is fetched before the accumulator is ready, and the four
+// 32-column TMEM loads are double-buffered so the next load is in flight
+// while the current chunk is converted and stored.
+__device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t rank) {
+  const int nunits = p.tiles_m * p.tiles_n * p.splits;
+  const int npairs = gridDim.x >> 1;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int quad = warp & 3;
+  const int half = (warp - 2) >> 2;
+  const int region = static_cast<int>(rank) * kPairEpiWarps + (warp - 2);  // 0..15
+  float* sws = s.sw_tile[warp - 2];
+  uint32_t abuf = 0, aphase = 0;
+  for (int unit = blockIdx.x >> 1; unit < nunits; unit += npairs) {
+    const int tile = unit / p.splits, split = unit % p.splits;
+    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    const int row = tm * kPairBM + static_cast<int>(rank) * 128 + quad * 32 + lane;
+    const bool rv = row < p.m;
+    const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
+    const int colbase = tn * kPairBN + half * (kPairBN / 2);
+    if (p.out) {
+      const int c4 = colbase + lane * 4;  // n % 8 == 0: a group of 4 is all in or all out
+      const float4 v4 = c4 < p.n ? __ldg(reinterpret_cast<const float4*>(p.sw + c4))
+                                 : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      *reinterpret_cast<float4*>(sws + lane * 4) = v4;
+    }
+    __syncwarp();
+    if (!warp_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) break;
+    tc_fence_after();
+    const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * kPairBN +
+                        half * (kPairBN / 2);
+    uint32_t va[32], vb[32];
+    if (p.splits == 1) {
+      tmem_ld_32x32b_x32(tb, va);
+      tmem_ld_wait();
+#pragma unroll
+      for (int ch = 0; ch < 4; ch += 2) {
+        tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
+        if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
+        tmem_ld_wait();
+        if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
+        if (rv) store32_channel(p, row, colbase + (ch + 1) * 32, sa, sws + (ch + 1) * 32, vb);
+        tmem_ld_wait();
+      }
+    } else {
+      // This warp's 32 x 128 region of the tile: publish the partial sum in
+      // slice `split` of the workspace, laid out [column quad][lane][4] so a
+      // warp's 16-byte stores and loads are contiguous.
+      constexpr int kRegionInts = 32 * (kPairBN / 2);
+      int32_t* my_slice = p.ws + (static_cast<int64_t>(tile * p.splits + split) * 16 + region) *
+                                     kRegionInts;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        tmem_ld_32x32b_x32(tb + ch * 32, va);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<int4*>(my_slice + ((ch * 8 + q4) * 32 + lane) * 4) =
+              make_int4(va[q4 * 4], va[q4 * 4 + 1], va[q4 * 4 + 2], va[q4 * 4 + 3]);
+      }
+      __threadfence();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) last = atomicAdd(p.cnt + tile * 16 + region, 1) == p.splits - 1;
+      last = __shfl_sync(0xFFFFFFFFu, last, 0);
+      if (last) {
+        // Every other piece of this region is published: sum them with this
+        // unit's own partial (still in TMEM), dequantise and store.
+        __threadfence();
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          tmem_ld_32x32b_x32(tb + ch * 32, va);
+          tmem_ld_wait();
+          for (int o = 0; o < p.splits; ++o) {
+            if (o == split) continue;
+            const int32_t* other = p.ws + (static_cast<int64_t>(tile * p.splits + o) * 16 + region) *
+                                              kRegionInts;
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const int4 t4 = __ldcg(reinterpret_cast<const int4*>(other + ((ch * 8 + q4) * 32 + lane) * 4));
+              va[q4 * 4] += t4.x;
+              va[q4 * 4 + 1] += t4.y;
+              va[q4 * 4 + 2] += t4.z;
+              va[q4 * 4 + 3] += t4.w;
+            }
+          }
+          if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
+        }
+        if (lane == 0) p.cnt[tile * 16 + region] = 0;  // ready for the next call
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_addr(&s.acc_empty[abuf]), 0));
+    if (++abuf == 2) {
+      abuf = 0;
+      aphase ^= 1u;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+    gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const Args p) {
+  extern __shared__ uint8_t smem_raw[];
+  PairStorage& s = storage<PairStorage>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPairStages; ++i) {
+      mbar_init(smem_addr(&s.full[i]), 1);
+      mbar_init(smem_addr(&s.empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&s.acc_full[i]), 1);
+      mbar_init(smem_addr(&s.acc_empty[i]), 2 * kPairEpiWarps);  // epilogue warps of both CTAs
+    }
+    mbar_init(smem_addr(&s.drain), 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_addr(&s.tmem_base), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers exist before anyone signals them
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  if (warp == 0) {
+    if (lane == 0) produce_pair(s, &tmA, &tmB, p, rank);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) mma_issue_pair(s, tmem, p);
+    __syncwarp();
+  } else {
+    epilogue_pair(s, tmem, p, rank);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the leader's MMAs on this CTA's smem / TMEM are done
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -490,6 +807,113 @@ inline bool make_tmap(CUtensorMap* map, const void* base, int rows, int k, int b
 }
 
 inline size_t channel_smem() { return sizeof(ChannelStorage) + 1024; }
+inline size_t pair_smem() { return sizeof(PairStorage) + 1024; }
+
+// Largest number of co-resident CTA pairs (queried once per device).
+inline int max_pairs(int dev, int num_sms) {
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int pairs = num_sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = pair_smem();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(gemm_i8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pair_smem())) == cudaSuccess &&
+      cudaOccupancyMaxActiveClusters(&n, gemm_i8_pair_kernel, &cfg) == cudaSuccess && n > 0)
+    pairs = n < pairs ? n : pairs;
+  else
+    cudaGetLastError();
+  if (dev >= 0 && dev < 64) cache[dev] = pairs;
+  return pairs;
+}
+
+// CTA-pair kernel for m > 128.  0 ok, 1 tensor-map failure, 2 CUDA error.
+// Workspace of the pair kernel's split-K: a fixed header of arrival counters
+// (16 per tile; split-K only runs with fewer than 64 tiles), then the
+// partial-sum slices.  Because the header is at a fixed place and every call
+// leaves its counters at zero, one workspace can serve problems of any shape.
+constexpr size_t kCounterHeaderBytes = 4096;
+constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeaderBytes / (16 * 4));
+
+// Split-K plan of the pair kernel: when the output has fewer tiles than
+// three quarters of the SM pairs, cut K into pieces (>= 8 K blocks each) so
+// that about one unit lands on every pair.
+struct PairPlan {
+  int tiles, splits, kb_per_split;
+};
+
+inline PairPlan pair_plan(int m, int n, int k, int pairs) {
+  PairPlan pl;
+  pl.tiles = ((m + kPairBM - 1) / kPairBM) * ((n + kPairBN - 1) / kPairBN);
+  const int num_kb = (k + BK - 1) / BK;
+  int s = 1;
+  if (4 * pl.tiles < 3 * pairs && pl.tiles <= kMaxSplitTiles) {
+    s = pairs / pl.tiles;
+    const int by_k = num_kb / 8;
+    s = s < by_k ? s : by_k;
+    s = s > 1 ? s : 1;
+  }
+  pl.kb_per_split = (num_kb + s - 1) / s;
+  pl.splits = (num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
+  return pl;
+}
+
+inline size_t pair_workspace_bytes(const PairPlan& pl) {
+  if (pl.splits <= 1) return 0;
+  return kCounterHeaderBytes +
+         static_cast<size_t>(pl.tiles) * pl.splits * 16 * 32 * (kPairBN / 2) * 4;
+}
+
+inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int num_sms,
+                       void* workspace, cudaStream_t stream, cudaError_t* err) {
+  a.tiles_m = (a.m + kPairBM - 1) / kPairBM;
+  a.tiles_n = (a.n + kPairBN - 1) / kPairBN;
+  a.num_kb = (a.k + BK - 1) / BK;
+  a.groups = 0;
+  const int pairs = max_pairs(dev, num_sms);
+  const PairPlan pl = pair_plan(a.m, a.n, a.k, pairs);
+  a.splits = pl.splits;
+  a.kb_per_split = pl.kb_per_split;
+  a.ws = nullptr;
+  a.cnt = nullptr;
+  if (pl.splits > 1) {
+    a.cnt = static_cast<int*>(workspace);
+    a.ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kCounterHeaderBytes);
+  }
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, A, a.m, a.k, 128) || !make_tmap(&tb, B, a.n, a.k, 128)) return 1;
+  const int ntiles = a.tiles_m * a.tiles_n * a.splits;
+  const int grid_pairs = ntiles < pairs ? ntiles : pairs;
+  cudaError_t e = cudaFuncSetAttribute(gemm_i8_pair_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(pair_smem()));
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * grid_pairs, 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = pair_smem();
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel, ta, tb, a);
+  }
+  *err = e;
+  return e == cudaSuccess ? 0 : 2;
+}
 inline size_t group_smem() { return sizeof(GroupStorage) + 1024; }
 
 // 0 ok, 1 tensor-map failure, 2 CUDA error

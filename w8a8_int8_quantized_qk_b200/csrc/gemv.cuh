@@ -4,9 +4,10 @@
 // used for M multiply-adds only ("dynquant-kernels" page, What is in here:
 // the decode GEMV is the memory-bound case; "KV-cache kernels" section 01:
 // INT8 moves the memory-bound ceiling).  The design goal is HBM rate:
-//  - a CTA owns R consecutive rows of W and sweeps K with all its threads,
-//    so every thread has R independent 16-byte streaming loads in flight
-//    and the activation chunk it loads is reused R times;
+//  - a CTA owns groups of R consecutive rows of W and sweeps K with all its
+//    threads, so every thread has R independent 16-byte streaming loads in
+//    flight per group (two groups deep) and reuses each activation chunk R
+//    times;
 //  - the int8 dot products use dp4a (4 MACs per instruction, int32
 //    accumulation, exact);
 //  - per-(row, token) sums are reduced with warp redux and shared memory,
@@ -109,7 +110,152 @@ __global__ void __launch_bounds__(kThreads) gemv_i8_kernel(Args p) {
 
 inline int max_tokens() { return 8; }
 
+// ---------------------------------------------------------------------------
+// Persistent prefetching form (the default for K <= 16384): two CTAs per SM,
+// each walking row groups g = blockIdx, blockIdx + grid, ...  A group is R
+// rows; thread t owns the 16-byte K chunks t, t + 256, ... (J of them), so its
+// activation chunks for all tokens are loaded once and stay in registers, and
+// the W chunks of the next D - 1 groups are already in flight while the
+// current group is multiplied and reduced.  (Streaming W through shared
+// memory with one-dimensional bulk copies was measured and rejected: on this
+// part its throughput grows with the copy size and stays far below the
+// register path.)
+// ---------------------------------------------------------------------------
+constexpr int kPrefThreads = 256;
+constexpr int kPrefDepth = 2;
+
+// Rows per group for <MT tokens, J chunks per thread>: as many as the
+// 128-register budget of two resident CTAs per SM allows (two groups of W
+// chunks, R x MT accumulators and MT x J activation chunks per thread).
+__host__ __device__ constexpr int pref_rows(int mt, int j) {
+  return mt <= 2 ? 8 / j
+                 : (mt == 4 ? (j == 1 ? 8 : (j == 2 ? 4 : (j == 3 ? 2 : 1)))
+                            : (j == 1 ? 4 : (j == 2 ? 2 : 1)));
+}
+
+// The activation chunks of all tokens stay in registers: MT x J <= 16.
+inline bool pref_supported(int m, int k) {
+  const int j = (k / 16 + kPrefThreads - 1) / kPrefThreads;
+  const int mt = m <= 1 ? 1 : (m <= 2 ? 2 : (m <= 4 ? 4 : 8));
+  return k <= 16384 && mt * j <= 16;
+}
+
+template <int MT, int J>
+__global__ void __launch_bounds__(kPrefThreads, 2) gemv_i8_prefetch_kernel(Args p) {
+  constexpr int R = pref_rows(MT, J);
+  constexpr int D = kPrefDepth;
+  __shared__ int red[kPrefThreads / 32][R * MT];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cpr = p.k >> 4;
+  const int ngroups = (p.n + R - 1) / R;
+  uint4 av[MT][J];
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int kc = tid + j * kPrefThreads;
+      av[t][j] = (t < p.m && kc < cpr) ? ld_nc_v4(p.a + static_cast<int64_t>(t) * p.k + kc * 16)
+                                       : make_uint4(0, 0, 0, 0);
+    }
+  uint4 buf[D][R][J];
+  auto fetch = [&](uint4 (&b)[R][J], int g) {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < J; ++j) {
+        const int row = g * R + r;
+        const int kc = tid + j * kPrefThreads;
+        b[r][j] = (g < ngroups && row < p.n && kc < cpr)
+                      ? ld_stream_v4(p.w + static_cast<int64_t>(row) * p.k + kc * 16)
+                      : make_uint4(0, 0, 0, 0);
+      }
+  };
+#pragma unroll
+  for (int d = 0; d < D; ++d) fetch(buf[d], blockIdx.x + d * gridDim.x);
+  const int my_r = tid / MT, my_t = tid % MT;  // output owned by thread tid < R * MT
+  const float my_sa = (tid < R * MT && my_t < p.m && p.out) ? __ldg(p.sa + my_t) : 0.0f;
+  int slot = 0;
+  for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
+    const int my_row = g * R + my_r;
+    const float my_sw = (tid < R * MT && my_row < p.n && p.out) ? __ldg(p.sw + my_row) : 0.0f;
+    int acc[R][MT];
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      if (d == slot) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            int a = 0;
+#pragma unroll
+            for (int j = 0; j < J; ++j) a = dot16(buf[d][r][j], av[t][j], a);
+            acc[r][t] = a;
+          }
+        fetch(buf[d], g + D * gridDim.x);
+      }
+    }
+    slot = slot + 1 == D ? 0 : slot + 1;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const int v = __reduce_add_sync(0xFFFFFFFFu, acc[r][t]);
+        if (lane == 0) red[warp][r * MT + t] = v;
+      }
+    __syncthreads();
+    if (tid < R * MT && my_row < p.n && my_t < p.m) {
+      int sum = 0;
+#pragma unroll
+      for (int w = 0; w < kPrefThreads / 32; ++w) sum += red[w][tid];
+      const int64_t o = static_cast<int64_t>(my_t) * p.n + my_row;
+      if (p.c) p.c[o] = sum;
+      if (p.out) {
+        float v = __int2float_rn(sum);
+        v = __fmul_rn(v, my_sa);
+        v = __fmul_rn(v, my_sw);
+        v = __fmul_rn(v, p.alpha);
+        if (p.out_bf16)
+          static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(v);
+        else
+          static_cast<float*>(p.out)[o] = v;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <int MT>
+inline cudaError_t launch_pref_mt(const Args& a, int num_sms, cudaStream_t stream) {
+  const int J = (a.k / 16 + kPrefThreads - 1) / kPrefThreads;
+  int rows = 0;
+  switch (J) {
+    case 1: rows = pref_rows(MT, 1); break;
+    case 2: rows = pref_rows(MT, 2); break;
+    case 3: rows = pref_rows(MT, 3); break;
+    default: rows = pref_rows(MT, 4); break;
+  }
+  const int ngroups = (a.n + rows - 1) / rows;
+  const int grid = ngroups < 2 * num_sms ? ngroups : 2 * num_sms;
+  switch (J) {
+    case 1: gemv_i8_prefetch_kernel<MT, 1><<<grid, kPrefThreads, 0, stream>>>(a); break;
+    case 2: gemv_i8_prefetch_kernel<MT, 2><<<grid, kPrefThreads, 0, stream>>>(a); break;
+    case 3:
+      if constexpr (MT <= 4) gemv_i8_prefetch_kernel<MT, 3><<<grid, kPrefThreads, 0, stream>>>(a);
+      break;
+    default:
+      if constexpr (MT <= 4) gemv_i8_prefetch_kernel<MT, 4><<<grid, kPrefThreads, 0, stream>>>(a);
+      break;
+  }
+  return cudaGetLastError();
+}
+
 inline cudaError_t launch(const Args& a, int num_sms, cudaStream_t stream) {
+  if (pref_supported(a.m, a.k)) {
+    if (a.m <= 1) return launch_pref_mt<1>(a, num_sms, stream);
+    if (a.m <= 2) return launch_pref_mt<2>(a, num_sms, stream);
+    if (a.m <= 4) return launch_pref_mt<4>(a, num_sms, stream);
+    return launch_pref_mt<8>(a, num_sms, stream);
+  }
   const int ngroups = (a.n + kRows - 1) / kRows;
   const int grid = ngroups < 64 * num_sms ? ngroups : 64 * num_sms;
   if (a.m <= 1)

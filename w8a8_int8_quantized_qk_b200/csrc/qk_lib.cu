@@ -91,12 +91,13 @@ qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, 
 }
 
 // Which kernel runs a GEMM of this shape.
-enum class GemmPath { kGemv, kTensorChannel, kTensorGroup };
+enum class GemmPath { kGemv, kTensorChannel, kTensorPair, kTensorGroup };
 
 GemmPath gemm_path(int m, int group_k) {
   if (group_k != 0) return GemmPath::kTensorGroup;
   if (m <= gemv::max_tokens()) return GemmPath::kGemv;
-  return GemmPath::kTensorChannel;
+  if (m <= 128) return GemmPath::kTensorChannel;
+  return GemmPath::kTensorPair;
 }
 
 qk_status gemm_check(int m, int n, int k, int group_k) {
@@ -154,11 +155,14 @@ qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, const void
 }
 
 size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
-  (void)m;
-  (void)n;
-  (void)k;
-  (void)group_k;
-  return 0;
+  if (gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return 0;
+  if (gemm_path(m, group_k) != GemmPath::kTensorPair) return 0;
+  const DeviceInfo* dev = nullptr;
+  if (check_device(&dev) != QK_OK) return 0;
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const gemm::PairPlan pl = gemm::pair_plan(m, n, k, gemm::max_pairs(dev_id, dev->sms));
+  return gemm::pair_workspace_bytes(pl);
 }
 
 qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
@@ -207,8 +211,16 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   g.c = c;
   g.out = out;
   g.out_bf16 = out_dtype == QK_BF16;
+  g.splits = 1;
+  g.kb_per_split = 0;
+  g.ws = nullptr;
+  g.cnt = nullptr;
   cudaError_t e = cudaSuccess;
-  const int r = gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev->sms, s, &e);
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const int r = path == GemmPath::kTensorPair
+                    ? gemm::launch_pair(g, a, b, dev_id, dev->sms, workspace, s, &e)
+                    : gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev->sms, s, &e);
   if (r == 1) return QK_ERR_CUDA;
   return r == 0 ? QK_OK : QK_ERR_CUDA;
 }

@@ -22,7 +22,6 @@ namespace quant {
 
 namespace cg = cooperative_groups;
 
-constexpr int kVecPerThread = 8;  // 16-byte vectors held per thread
 constexpr int kMaxThreads = 512;  // threads per CTA (128 registers each)
 
 struct Args {
@@ -34,80 +33,100 @@ struct Args {
   float* scale;     // [m]
 };
 
+// 1.5 * 2^23: adding it to |y| < 2^22 rounds y to an integer, ties to even
+// (the sum lies in [2^23, 2^24), where the spacing is 1), and the low 22
+// mantissa bits of the sum hold that integer offset by 2^22.  The multiply
+// that produces y and the add are separate __fmul_rn / __fadd_rn intrinsics,
+// which are never contracted into a fused multiply-add.
+constexpr float kRoundMagic = 12582912.0f;
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
 // ---------------------------------------------------------------------------
 // The fixed binary32 exponential used by the fused SiLU: Cody & Waite
 // argument reduction (t = n ln2 + r, ln2 as a binary32 head plus tail, both
 // subtractions fused), e^r by the degree-7 Taylor polynomial in Horner form,
 // scaling by 2^n through the exponent field.  t is clamped to [-87, 88] so
-// 2^n stays a normal number.  Every step is an explicit round-to-nearest
-// operation so the result does not depend on compiler contraction choices.
+// 2^n stays a normal number; n = rint(RN(t log2 e)) is formed with the
+// round-to-integer constant above.  Every step is one IEEE round-to-nearest
+// operation in the order written.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float fixed_exp(float t) {
   constexpr float kLog2e = static_cast<float>(1.4426950408889634074);
   constexpr float kLn2Hi = static_cast<float>(0.69314718055994530942);
   constexpr float kLn2Lo =
       static_cast<float>(0.69314718055994530942 - static_cast<double>(kLn2Hi));
-  constexpr float kC7 = static_cast<float>(1.0 / 5040.0);
-  constexpr float kC6 = static_cast<float>(1.0 / 720.0);
-  constexpr float kC5 = static_cast<float>(1.0 / 120.0);
-  constexpr float kC4 = static_cast<float>(1.0 / 24.0);
-  constexpr float kC3 = static_cast<float>(1.0 / 6.0);
   t = fminf(fmaxf(t, -87.0f), 88.0f);
-  const float n = rintf(__fmul_rn(t, kLog2e));
+  const float nb = __fadd_rn(__fmul_rn(t, kLog2e), kRoundMagic);
+  const float n = __fsub_rn(nb, kRoundMagic);
   float r = __fmaf_rn(-n, kLn2Hi, t);
   r = __fmaf_rn(-n, kLn2Lo, r);
-  float p = kC7;
-  p = __fmaf_rn(p, r, kC6);
-  p = __fmaf_rn(p, r, kC5);
-  p = __fmaf_rn(p, r, kC4);
-  p = __fmaf_rn(p, r, kC3);
+  float p = static_cast<float>(1.0 / 5040.0);
+  p = __fmaf_rn(p, r, static_cast<float>(1.0 / 720.0));
+  p = __fmaf_rn(p, r, static_cast<float>(1.0 / 120.0));
+  p = __fmaf_rn(p, r, static_cast<float>(1.0 / 24.0));
+  p = __fmaf_rn(p, r, static_cast<float>(1.0 / 6.0));
   p = __fmaf_rn(p, r, 0.5f);
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
-  const int e = static_cast<int>(n) + 127;
-  return __fmul_rn(p, __int_as_float(e << 23));
+  // 2^n: exponent field n + 127, with n = (bits of nb) - bits of 1.5 * 2^23
+  const float two_n = __uint_as_float((__float_as_uint(nb) - kRoundMagicBits + 127u) << 23);
+  return __fmul_rn(p, two_n);
 }
 
 // h = silu(g) * u = (g / (1 + exp(-g))) * u
 __device__ __forceinline__ float silu_mul(float g, float u) {
   const float e = fixed_exp(-g);
-  const float d = __fadd_rn(1.0f, e);
-  return __fmul_rn(__fdiv_rn(g, d), u);
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, e)), u);
 }
 
-__device__ __forceinline__ int quant1(float x, float inv) {
-  const int r = __float2int_rn(__fmul_rn(x, inv));  // round half to even
-  return min(max(r, -127), 127);
+// Quantise one value: the low byte of (x * inv + 1.5 * 2^23) is
+// round_half_even(x * inv) as a two's-complement int8.  The clamp to
+// [-127, 127] is never active: |x| <= amax and inv = RN(1 / RN(a / 127)) with
+// a = max(amax, 1e-12) give |x * inv| <= 127 (1 + 2^-23), which rounds to at
+// most 127.
+__device__ __forceinline__ uint32_t quant_bits(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), kRoundMagic));
 }
 
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+// Four quantised values (low bytes of a..d) -> one packed int8x4 word.
+__device__ __forceinline__ uint32_t pack_q4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// Elements of one 16-byte vector, widened to fp32.
+// A 16-byte vector widened to binary32 (8 values for bf16, 4 for fp32).
 template <bool BF16>
 __device__ __forceinline__ void widen(const uint4& v, float (&f)[BF16 ? 8 : 4]) {
   if constexpr (BF16) {
-    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
-    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+    f[0] = __uint_as_float(v.x << 16); f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(v.y << 16); f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+    f[4] = __uint_as_float(v.z << 16); f[5] = __uint_as_float(v.z & 0xFFFF0000u);
+    f[6] = __uint_as_float(v.w << 16); f[7] = __uint_as_float(v.w & 0xFFFF0000u);
   } else {
     f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
     f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
   }
 }
 
-template <bool BF16>
-__device__ __forceinline__ void store_q(int8_t* dst, const float (&f)[BF16 ? 8 : 4], float inv) {
-  if constexpr (BF16) {
+// Quantise E values and store E int8 at dst.
+template <int E>
+__device__ __forceinline__ void store_q(int8_t* dst, const float (&f)[E], float inv) {
+  if constexpr (E == 8) {
     uint2 o;
-    o.x = pack4(quant1(f[0], inv), quant1(f[1], inv), quant1(f[2], inv), quant1(f[3], inv));
-    o.y = pack4(quant1(f[4], inv), quant1(f[5], inv), quant1(f[6], inv), quant1(f[7], inv));
+    o.x = pack_q4(quant_bits(f[0], inv), quant_bits(f[1], inv), quant_bits(f[2], inv),
+                  quant_bits(f[3], inv));
+    o.y = pack_q4(quant_bits(f[4], inv), quant_bits(f[5], inv), quant_bits(f[6], inv),
+                  quant_bits(f[7], inv));
     *reinterpret_cast<uint2*>(dst) = o;
   } else {
-    *reinterpret_cast<uint32_t*>(dst) =
-        pack4(quant1(f[0], inv), quant1(f[1], inv), quant1(f[2], inv), quant1(f[3], inv));
+    *reinterpret_cast<uint32_t*>(dst) = pack_q4(quant_bits(f[0], inv), quant_bits(f[1], inv),
+                                                quant_bits(f[2], inv), quant_bits(f[3], inv));
   }
+}
+
+// Cluster barrier without memory ordering: used only to keep a CTA's shared
+// memory alive until its peers have finished reading it.
+__device__ __forceinline__ void cluster_arrive_wait_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -138,16 +157,17 @@ __device__ __forceinline__ float row_max(float v, float* red /*[33]*/) {
   return v;
 }
 
+// scale = max(amax, 1e-12) / 127 and inv = 1 / scale, both IEEE RN.
 __device__ __forceinline__ void scale_and_inverse(float amax, float& scale, float& inv) {
   scale = __fdiv_rn(fmaxf(amax, 1e-12f), 127.0f);
   inv = __fdiv_rn(1.0f, scale);
 }
 
 // One row per CTA (CLUSTER = false) or per cluster.  The row's 16-byte vectors
-// are dealt round-robin to the row's threads; each thread holds up to
-// kVecPerThread of them.  SILU: x is gate, p.up is up, h = silu(g) * u is kept
-// in fp32 registers.
-template <bool BF16, bool SILU, bool CLUSTER>
+// are dealt round-robin to the row's threads; each thread holds up to V of
+// them, widened to fp32 in registers.  SILU: x is gate, p.up is up, and the
+// registers hold h = silu(g) * u.
+template <bool BF16, bool SILU, bool CLUSTER, int V>
 __global__ void __launch_bounds__(kMaxThreads) quant_rows_kernel(Args p) {
   constexpr int E = BF16 ? 8 : 4;  // elements per 16-byte vector
   constexpr int ES = BF16 ? 2 : 4;
@@ -167,15 +187,14 @@ __global__ void __launch_bounds__(kMaxThreads) quant_rows_kernel(Args p) {
   const int stride = nranks * blockDim.x;
   const int t0 = rank * blockDim.x + threadIdx.x;
   const char* xr = static_cast<const char*>(p.x) + static_cast<int64_t>(row) * p.ld * ES;
-  const char* ur = SILU ? static_cast<const char*>(p.up) + static_cast<int64_t>(row) * p.ld * ES
-                        : nullptr;
-
-  float vals[kVecPerThread][E];
-  float amax = 0.0f;
+  int8_t* qr = p.q + static_cast<int64_t>(row) * p.k;
+  float vals[V][E];
+  float m = 0.0f;
   if constexpr (SILU) {
-    uint4 gv[kVecPerThread], uv[kVecPerThread];
+    const char* ur = static_cast<const char*>(p.up) + static_cast<int64_t>(row) * p.ld * ES;
+    uint4 gv[V], uv[V];
 #pragma unroll
-    for (int j = 0; j < kVecPerThread; ++j) {
+    for (int j = 0; j < V; ++j) {
       const int v = t0 + j * stride;
       if (v < nvec) {
         gv[j] = ld_nc_v4(xr + static_cast<int64_t>(v) * 16);
@@ -186,41 +205,110 @@ __global__ void __launch_bounds__(kMaxThreads) quant_rows_kernel(Args p) {
       }
     }
 #pragma unroll
-    for (int j = 0; j < kVecPerThread; ++j) {
+    for (int j = 0; j < V; ++j) {
       float g[E], u[E];
       widen<BF16>(gv[j], g);
       widen<BF16>(uv[j], u);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         vals[j][e] = silu_mul(g[e], u[e]);
-        amax = fmaxf(amax, fabsf(vals[j][e]));
+        m = fmaxf(m, fabsf(vals[j][e]));
       }
     }
   } else {
-    uint4 xv[kVecPerThread];
+    uint4 xv[V];
 #pragma unroll
-    for (int j = 0; j < kVecPerThread; ++j) {
+    for (int j = 0; j < V; ++j) {
       const int v = t0 + j * stride;
       xv[j] = v < nvec ? ld_nc_v4(xr + static_cast<int64_t>(v) * 16) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int j = 0; j < kVecPerThread; ++j) {
+    for (int j = 0; j < V; ++j) {
       widen<BF16>(xv[j], vals[j]);
 #pragma unroll
-      for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(vals[j][e]));
+      for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(vals[j][e]));
     }
   }
-  amax = row_max<CLUSTER>(amax, red);
+  const float amax = row_max<CLUSTER>(m, red);
   float scale, inv;
   scale_and_inverse(amax, scale, inv);
-  int8_t* qr = p.q + static_cast<int64_t>(row) * p.k;
 #pragma unroll
-  for (int j = 0; j < kVecPerThread; ++j) {
+  for (int j = 0; j < V; ++j) {
     const int v = t0 + j * stride;
-    if (v < nvec) store_q<BF16>(qr + static_cast<int64_t>(v) * E, vals[j], inv);
+    if (v < nvec) store_q<E>(qr + static_cast<int64_t>(v) * E, vals[j], inv);
   }
   if (t0 == 0) p.scale[row] = scale;
-  if constexpr (CLUSTER) cg::this_cluster().sync();  // peers may still read red[32]
+  if constexpr (CLUSTER) cluster_arrive_wait_relaxed();  // peers may still read red[32]
+}
+
+// Many rows: persistent CTAs of 256 threads walk rows blockIdx, blockIdx +
+// grid, ...; each row's V 16-byte vectors per thread are loaded one row
+// ahead, so the next row's loads are in flight while the current row is
+// reduced and quantised.  The per-warp maxima are double-buffered by row
+// parity: one CTA barrier per row suffices.
+constexpr int kPersistThreads = 256;
+
+template <bool BF16, bool SILU, int V>
+__global__ void __launch_bounds__(kPersistThreads) quant_rows_persistent_kernel(Args p) {
+  constexpr int E = BF16 ? 8 : 4;
+  constexpr int ES = BF16 ? 2 : 4;
+  constexpr int NW = kPersistThreads / 32;
+  __shared__ float red[2][NW];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nvec = p.k / E;
+  uint4 xc[V], uc[SILU ? V : 1];
+  auto fetch = [&](uint4 (&xv)[V], uint4 (&uv)[SILU ? V : 1], int row) {
+    const char* xr = static_cast<const char*>(p.x) + static_cast<int64_t>(row) * p.ld * ES;
+    const char* ur = SILU ? static_cast<const char*>(p.up) + static_cast<int64_t>(row) * p.ld * ES
+                          : nullptr;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const int v = tid + j * kPersistThreads;
+      const bool in = row < p.m && v < nvec;
+      xv[j] = in ? ld_nc_v4(xr + static_cast<int64_t>(v) * 16) : make_uint4(0, 0, 0, 0);
+      if constexpr (SILU) uv[j] = in ? ld_nc_v4(ur + static_cast<int64_t>(v) * 16) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  fetch(xc, uc, blockIdx.x);
+  int par = 0;
+  for (int row = blockIdx.x; row < p.m; row += gridDim.x) {
+    uint4 xn[V], un[SILU ? V : 1];
+    fetch(xn, un, row + gridDim.x);
+    float vals[V][E];
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      widen<BF16>(xc[j], vals[j]);
+      if constexpr (SILU) {
+        float u[E];
+        widen<BF16>(uc[j], u);
+#pragma unroll
+        for (int e = 0; e < E; ++e) vals[j][e] = silu_mul(vals[j][e], u[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(vals[j][e]));
+    }
+    m = warp_max(m);
+    if (lane == 0) red[par][warp] = m;
+    __syncthreads();
+    float amax = lane < NW ? red[par][lane] : 0.0f;
+    amax = warp_max(amax);
+    float scale, inv;
+    scale_and_inverse(amax, scale, inv);
+    int8_t* qr = p.q + static_cast<int64_t>(row) * p.k;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const int v = tid + j * kPersistThreads;
+      if (v < nvec) store_q<E>(qr + static_cast<int64_t>(v) * E, vals[j], inv);
+    }
+    if (tid == 0) p.scale[row] = scale;
+    par ^= 1;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      xc[j] = xn[j];
+      if constexpr (SILU) uc[j] = un[j];
+    }
+  }
 }
 
 // Rows too long to hold on chip: the two-phase form (phase 1 absmax, phase 2
@@ -261,47 +349,65 @@ __global__ void __launch_bounds__(512) quant_rows_twopass_kernel(Args p) {
 #pragma unroll
       for (int e = 0; e < E; ++e) f[e] = silu_mul(f[e], u[e]);
     }
-    store_q<BF16>(qr + static_cast<int64_t>(v) * E, f, inv);
+    store_q<E>(qr + static_cast<int64_t>(v) * E, f, inv);
   }
   if (threadIdx.x == 0) p.scale[row] = scale;
 }
 
-// Launch geometry: threads per row T = ceil(nvec / 8).  A row is split over a
-// cluster of CL CTAs when T exceeds one CTA (512 threads), or when there are too few rows to
-// give every SM two CTAs (and each CTA keeps >= 64 threads).
+// Launch geometry: V vectors per thread (4 plain, 2 with SiLU, whose
+// per-element work is larger), T = ceil(nvec / V) threads per row.  A row is
+// split over a cluster of CL CTAs when T exceeds one CTA (512 threads), or
+// when there are too few rows to give every SM four CTAs (and each CTA keeps
+// >= 64 threads).
+template <bool SILU>
+constexpr int vec_per_thread() { return SILU ? 2 : 4; }
+
 struct Plan {
   int cluster;   // CTAs per row (1 = plain launch), 0 = two-pass kernel
   int threads;   // threads per CTA
 };
 
-inline Plan plan(int m, int k, bool bf16, int num_sms) {
+inline Plan plan(int m, int k, bool bf16, int V, int num_sms) {
   const int E = bf16 ? 8 : 4;
   const int nvec = k / E;
-  const int T = (nvec + kVecPerThread - 1) / kVecPerThread;
+  const int T = (nvec + V - 1) / V;
   int cl = 1;
   while (cl < 8 && (T + cl - 1) / cl > kMaxThreads) cl *= 2;
   if ((T + cl - 1) / cl > kMaxThreads) return {0, 512};
-  while (cl < 8 && static_cast<int64_t>(m) * cl < 2LL * num_sms && T / (2 * cl) >= 64) cl *= 2;
+  while (cl < 8 && static_cast<int64_t>(m) * cl < 4LL * num_sms && T / (2 * cl) >= 64) cl *= 2;
   int threads = (T + cl - 1) / cl;
   threads = ((threads + 31) / 32) * 32;
   return {cl, threads};
 }
 
-template <bool SILU>
-inline cudaError_t launch(const Args& a, bool bf16, int num_sms, cudaStream_t stream) {
-  const Plan pl = plan(a.m, a.k, bf16, num_sms);
+template <bool BF16, bool SILU, int V>
+inline cudaError_t launch_persistent(const Args& a, int num_sms, cudaStream_t stream) {
+  const int grid = a.m < 4 * num_sms ? a.m : 4 * num_sms;
+  quant_rows_persistent_kernel<BF16, SILU, V><<<grid, kPersistThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <bool BF16, bool SILU>
+inline cudaError_t launch_typed(const Args& a, int num_sms, cudaStream_t stream) {
+  // Many rows of a size the persistent kernel holds (<= 4 vectors per thread):
+  // persistent row loop with prefetch.
+  const int E = BF16 ? 8 : 4;
+  const int vp = (a.k / E + kPersistThreads - 1) / kPersistThreads;
+  if (a.m >= 2 * num_sms && vp <= 4) {
+    switch (vp) {
+      case 1: return launch_persistent<BF16, SILU, 1>(a, num_sms, stream);
+      case 2: return launch_persistent<BF16, SILU, 2>(a, num_sms, stream);
+      default: return launch_persistent<BF16, SILU, 4>(a, num_sms, stream);
+    }
+  }
+  constexpr int V = vec_per_thread<SILU>();
+  const Plan pl = plan(a.m, a.k, BF16, V, num_sms);
   if (pl.cluster == 0) {
-    if (bf16)
-      quant_rows_twopass_kernel<true, SILU><<<a.m, pl.threads, 0, stream>>>(a);
-    else
-      quant_rows_twopass_kernel<false, SILU><<<a.m, pl.threads, 0, stream>>>(a);
+    quant_rows_twopass_kernel<BF16, SILU><<<a.m, pl.threads, 0, stream>>>(a);
     return cudaGetLastError();
   }
   if (pl.cluster == 1) {
-    if (bf16)
-      quant_rows_kernel<true, SILU, false><<<a.m, pl.threads, 0, stream>>>(a);
-    else
-      quant_rows_kernel<false, SILU, false><<<a.m, pl.threads, 0, stream>>>(a);
+    quant_rows_kernel<BF16, SILU, false, V><<<a.m, pl.threads, 0, stream>>>(a);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -316,8 +422,13 @@ inline cudaError_t launch(const Args& a, bool bf16, int num_sms, cudaStream_t st
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (bf16) return cudaLaunchKernelEx(&cfg, quant_rows_kernel<true, SILU, true>, a);
-  return cudaLaunchKernelEx(&cfg, quant_rows_kernel<false, SILU, true>, a);
+  return cudaLaunchKernelEx(&cfg, quant_rows_kernel<BF16, SILU, true, V>, a);
+}
+
+template <bool SILU>
+inline cudaError_t launch(const Args& a, bool bf16, int num_sms, cudaStream_t stream) {
+  return bf16 ? launch_typed<true, SILU>(a, num_sms, stream)
+              : launch_typed<false, SILU>(a, num_sms, stream);
 }
 
 }  // namespace quant

@@ -207,13 +207,29 @@ def w8a8_gemm(a, b, scale_a, scale_b, group_k: int = 0, output_scale: float = 1.
         c = torch.empty((m, n), dtype=torch.int32, device=a.device)
     need = qk_w8a8_gemm_workspace_size(m, n, k, group_k)
     if need and workspace is None:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=a.device)
+        workspace = cached_workspace(need, a.device)
     code = _dtype_code(out) if out is not None else QK_BF16
     _check(qk_w8a8_gemm(m, n, k, _ptr(a), _ptr(b), _ptr(scale_a), _ptr(scale_b), group_k,
                         float(output_scale), _ptr(c), _ptr(out), code, _ptr(workspace),
                         0 if workspace is None else workspace.numel(), _stream(stream)),
            "qk_w8a8_gemm")
     return out, c
+
+
+_workspaces: dict = {}
+
+
+def cached_workspace(nbytes: int, device):
+    """A zero-filled workspace of at least `nbytes` on `device`, kept for reuse.
+    The library leaves its counter header zero after every completed call, so
+    the buffer can be shared by calls of any shape on one stream."""
+    torch = _torch()
+    key = torch.device(device).index
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros((max(nbytes, 1 << 20),), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
 
 
 def linear(x, w_q, sw, group_k: int = 0, output_scale: float = 1.0, out_dtype=None, stream=None):
