@@ -187,6 +187,40 @@ QK_API qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t
 QK_API size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k);
 
 /*
+ * qk_w8a8_gemm_noalloc -- qk_w8a8_gemm without a caller-provided workspace.
+ *
+ * (No counterpart on the pages: an addition for callers that cannot allocate
+ * device memory.)  Some callers cannot call cudaMalloc on the path that runs
+ * the layer: a plugin inside an inference runtime that owns all device
+ * memory, a latency-critical path where an allocation would synchronise the
+ * device, or an embedded caller with a fixed memory budget.  This entry point
+ * takes the same arguments as qk_w8a8_gemm minus the workspace, and when the
+ * problem needs split-K scratch it uses a scratch array built into the
+ * library instead: QK_NOALLOC_SCRATCH_BYTES bytes of device memory that every
+ * GPU which loads the library holds until the process exits.
+ *
+ * - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ *   library routine.  The inputs and outputs are still the caller's.
+ * - The first call on a device looks up the scratch array's device address
+ *   (once per device, with that device current); make that first call before
+ *   any stream capture on the device.
+ * - Each call clears the scratch array's counter header on `stream` before
+ *   its kernel, so it does not depend on what an earlier call left there.
+ * - Every call shares the one array: calls that can overlap on the GPU (on
+ *   different streams, or from different threads) race and give wrong
+ *   results.  Serialise them.
+ * - A problem whose split-K needs more than QK_NOALLOC_SCRATCH_BYTES (see
+ *   qk_w8a8_gemm_workspace_size) is rejected with QK_ERR_WORKSPACE and
+ *   nothing is launched.  Other errors are those of qk_w8a8_gemm.
+ */
+#define QK_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u + 4096u)
+
+QK_API qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_t* b,
+                                      const float* scale_a, const float* scale_b, int group_k,
+                                      float output_scale, int32_t* c, void* out,
+                                      qk_dtype out_dtype, qk_stream stream);
+
+/*
  * qk_device_status -- read and clear the library's device status word on the
  * current device.  Kernels that wait on a barrier give up after a bounded
  * time (about one second) instead of hanging; when that happens they record

@@ -1,0 +1,91 @@
+"""GPU test of qk_w8a8_gemm_noalloc, the GEMM entry point for callers that
+cannot allocate device memory (for example a plugin inside an inference
+runtime that owns all device memory, or a path where cudaMalloc's device
+synchronisation is not acceptable).  Instead of a caller workspace it uses a
+scratch array built into the library.
+
+The test calls it through the C ABI on a problem that needs split-K scratch,
+twice in a row, and checks each result against the regular entry point
+(qk_w8a8_gemm with its own zero-filled workspace): int32 sums identical,
+bf16 outputs within the suite's tolerance.  It also checks that a problem
+needing more scratch than the built-in array is refused.  It works both alone
+in a fresh process and after the rest of the suite.
+"""
+import numpy as np
+import pytest
+
+from gpu_util import check_out, dev, host, need_gpu
+from w8a8_int8_quantized_qk_b200 import qk, synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024 + 4096  # QK_NOALLOC_SCRATCH_BYTES in include/qk.h
+
+
+def _inputs(m, n, k, seed):
+    r = synth.streams(seed, ["a", "w", "sa", "sw"])
+    return (synth.int8_uniform(r["a"], (m, k)), synth.int8_uniform(r["w"], (n, k)),
+            synth.scales_uniform(r["sa"], (m,), 0.001, 0.05), synth.scales_uniform(r["sw"], (n,)))
+
+
+def _call_noalloc(m, n, k, a, w, sa, sw, alpha):
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    c = torch.empty((m, n), dtype=torch.int32, device="cuda")
+    st = qk.qk_w8a8_gemm_noalloc(m, n, k, qk._ptr(a), qk._ptr(w), qk._ptr(sa), qk._ptr(sw), 0,
+                                 alpha, qk._ptr(c), qk._ptr(out), qk.QK_BF16, qk._stream())
+    assert st == qk.QK_OK, qk.qk_status_string(st)
+    torch.cuda.synchronize()
+    assert qk.device_status() == qk.QK_OK
+    return host(out), host(c)
+
+
+def _call_regular(m, n, k, a, w, sa, sw, alpha):
+    need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 0)
+    ws = torch.zeros((max(need, 1),), dtype=torch.uint8, device="cuda")
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    c = torch.empty((m, n), dtype=torch.int32, device="cuda")
+    st = qk.qk_w8a8_gemm(m, n, k, qk._ptr(a), qk._ptr(w), qk._ptr(sa), qk._ptr(sw), 0, alpha,
+                         qk._ptr(c), qk._ptr(out), qk.QK_BF16, qk._ptr(ws), ws.numel(), qk._stream())
+    assert st == qk.QK_OK, qk.qk_status_string(st)
+    torch.cuda.synchronize()
+    return host(out), host(c)
+
+
+@pytest.mark.parametrize("m,n,k", [(256, 1024, 14336), (200, 512, 4096)])
+def test_noalloc_matches_regular_entry_point(m, n, k):
+    need_gpu()
+    need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 0)
+    assert 0 < need <= NOALLOC_SCRATCH_BYTES  # the split-K path, within the built-in scratch
+    a_h, w_h, sa_h, sw_h = _inputs(m, n, k, seed=m + n + k)
+    a, w, sa, sw = dev(a_h), dev(w_h), dev(sa_h), dev(sw_h)
+    ref_out, ref_c = _call_regular(m, n, k, a, w, sa, sw, 0.5)
+    ref_f32 = synth.bf16_bits_to_f32(ref_out)
+    for _ in range(2):  # two calls in a row share the built-in scratch
+        out, c = _call_noalloc(m, n, k, a, w, sa, sw, 0.5)
+        assert np.array_equal(c, ref_c)
+        check_out(out, ref_f32, ref_out)
+
+
+def test_noalloc_without_split_k_and_refusal():
+    need_gpu()
+    # a shape that needs no scratch behaves like the regular call
+    m, n, k = 512, 1024, 512
+    a_h, w_h, sa_h, sw_h = _inputs(m, n, k, seed=7)
+    a, w, sa, sw = dev(a_h), dev(w_h), dev(sa_h), dev(sw_h)
+    assert qk.qk_w8a8_gemm_workspace_size(m, n, k, 0) == 0
+    out, c = _call_noalloc(m, n, k, a, w, sa, sw, 1.0)
+    ref_out, ref_c = _call_regular(m, n, k, a, w, sa, sw, 1.0)
+    assert np.array_equal(c, ref_c) and np.array_equal(out, ref_out)
+    # a shape whose split-K would need more than the built-in scratch is refused
+    m, n, k = 200, 256, 131072
+    if qk.qk_w8a8_gemm_workspace_size(m, n, k, 0) > NOALLOC_SCRATCH_BYTES:
+        a = torch.zeros((m, k), dtype=torch.int8, device="cuda")
+        w = torch.zeros((n, k), dtype=torch.int8, device="cuda")
+        sa = torch.ones((m,), dtype=torch.float32, device="cuda")
+        sw = torch.ones((n,), dtype=torch.float32, device="cuda")
+        out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+        st = qk.qk_w8a8_gemm_noalloc(m, n, k, qk._ptr(a), qk._ptr(w), qk._ptr(sa), qk._ptr(sw), 0,
+                                     1.0, None, qk._ptr(out), qk.QK_BF16, qk._stream())
+        assert st == qk.QK_ERR_WORKSPACE

@@ -120,6 +120,28 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   }
 }
 
+// Scratch for qk_w8a8_gemm_noalloc: a split-K workspace that lives in the
+// library's own device memory (zero at module load).  Host code only ever sees
+// a stand-in for this symbol; its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QK_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, or nullptr.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
 }  // namespace
 }  // namespace qk
 
@@ -223,6 +245,27 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
                     : gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev->sms, s, &e);
   if (r == 1) return QK_ERR_CUDA;
   return r == 0 ? QK_OK : QK_ERR_CUDA;
+}
+
+qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_t* b,
+                               const float* scale_a, const float* scale_b, int group_k,
+                               float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
+                               qk_stream stream) {
+  const qk_status st = gemm_check(m, n, k, group_k);
+  if (st != QK_OK) return st;
+  const size_t need = qk_w8a8_gemm_workspace_size(m, n, k, group_k);
+  if (need == 0)
+    return qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
+                        out_dtype, nullptr, 0, stream);
+  if (need > QK_NOALLOC_SCRATCH_BYTES) return QK_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch();
+  if (scratch == nullptr) return QK_ERR_CUDA;
+  // The arrival counters sit in the first 4 KB and must start at zero.
+  if (cudaMemsetAsync(scratch, 0, gemm::kCounterHeaderBytes,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QK_ERR_CUDA;
+  return qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
+                      scratch, QK_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 qk_status qk_device_status(qk_stream stream) {

@@ -48,6 +48,8 @@ _SIGNATURES = {
     "qk_w8a8_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
                                     ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "qk_w8a8_gemm_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "qk_w8a8_gemm_noalloc": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
+                                            ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P]),
     "qk_device_status": (ctypes.c_int, [_P]),
     "qk_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_int, _P]),
 }
@@ -110,6 +112,14 @@ def qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
 
 def qk_w8a8_gemm_workspace_size(m, n, k, group_k) -> int:
     return lib().qk_w8a8_gemm_workspace_size(m, n, k, group_k)
+
+
+def qk_w8a8_gemm_noalloc(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
+                         stream) -> int:
+    """qk_w8a8_gemm for callers that cannot allocate device memory: split-K
+    scratch comes from an array built into the library (see include/qk.h)."""
+    return lib().qk_w8a8_gemm_noalloc(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
+                                      out_dtype, stream)
 
 
 def qk_device_status(stream) -> int:
