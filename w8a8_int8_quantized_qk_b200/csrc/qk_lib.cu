@@ -7,6 +7,8 @@
 // (GemmConfig's m, n, k, int8 a / b, int32 c, scale_a, scale_b,
 // output_scale, stream; a status-returning entry point) and Python Bindings
 // (the same fields passed as plain integers, pointers and a float).
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "gemm_sm100.cuh"
@@ -54,6 +56,15 @@ qk_status check_device(const DeviceInfo** out) {
   return QK_OK;
 }
 
+// With QK_DEBUG set in the environment, a failing CUDA call is reported on
+// stderr (the call still just returns QK_ERR_CUDA).
+qk_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return QK_OK;
+  static const bool debug = std::getenv("QK_DEBUG") != nullptr;
+  if (debug) std::fprintf(stderr, "libqk: %s: %s\n", where, cudaGetErrorString(e));
+  return QK_ERR_CUDA;
+}
+
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
@@ -87,14 +98,14 @@ qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, 
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = silu ? quant::launch<true>(a, dt == QK_BF16, dev->sms, s)
                              : quant::launch<false>(a, dt == QK_BF16, dev->sms, s);
-  return e == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  return cuda_status(e, "quantize launch");
 }
 
 // Which kernel runs a GEMM of this shape.
-enum class GemmPath { kGemv, kTensorChannel, kTensorPair, kTensorGroup };
+enum class GemmPath { kGemv, kTensorChannel, kTensorPair, kTensorGroup, kTensorPairGroup };
 
 GemmPath gemm_path(int m, int group_k) {
-  if (group_k != 0) return GemmPath::kTensorGroup;
+  if (group_k != 0) return m <= 128 ? GemmPath::kTensorGroup : GemmPath::kTensorPairGroup;
   if (m <= gemv::max_tokens()) return GemmPath::kGemv;
   if (m <= 128) return GemmPath::kTensorChannel;
   return GemmPath::kTensorPair;
@@ -221,7 +232,7 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
     g.c = c;
     g.out = out;
     g.out_bf16 = out_dtype == QK_BF16;
-    return gemv::launch(g, dev->sms, s) == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+    return cuda_status(gemv::launch(g, dev->sms, s), "gemv launch");
   }
   gemm::Args g;
   g.m = m;
@@ -240,11 +251,27 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   cudaError_t e = cudaSuccess;
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  const int r = path == GemmPath::kTensorPair
-                    ? gemm::launch_pair(g, a, b, dev_id, dev->sms, workspace, s, &e)
-                    : gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev->sms, s, &e);
-  if (r == 1) return QK_ERR_CUDA;
-  return r == 0 ? QK_OK : QK_ERR_CUDA;
+  int r = 0;
+  if (path == GemmPath::kTensorPair) {
+    r = gemm::launch_pair(g, a, b, dev_id, dev->sms, workspace, s, &e);
+  } else if (path == GemmPath::kTensorPairGroup) {
+    // The group kernel produces the scaled output; the full-K int32 sum, when
+    // asked for, comes from a per-channel pass (same MMA, no scales needed).
+    if (out != nullptr) {
+      gemm::Args go = g;
+      go.c = nullptr;
+      r = gemm::launch_pair_group(go, a, b, dev_id, dev->sms, s, &e);
+    }
+    if (r == 0 && c != nullptr) {
+      gemm::Args gc = g;
+      gc.out = nullptr;
+      r = gemm::launch_pair(gc, a, b, dev_id, dev->sms, nullptr, s, &e, false);
+    }
+  } else {
+    r = gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev->sms, s, &e);
+  }
+  if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
+  return r == 0 ? QK_OK : cuda_status(e, "gemm launch");
 }
 
 qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_t* b,
