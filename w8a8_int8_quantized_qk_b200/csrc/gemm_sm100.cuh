@@ -29,6 +29,9 @@
 // the TMEM is freed before the CTA exits.
 #pragma once
 
+#include <atomic>
+#include <mutex>
+
 #include "qk_common.cuh"
 
 namespace qk {
@@ -482,6 +485,7 @@ constexpr int kPairStages = 6;
 constexpr int kPairEpiWarps = 8;  // two per TMEM lane quadrant, 128 columns each
 constexpr int kPairThreads = 64 + kPairEpiWarps * 32;
 constexpr uint32_t kPairStageBytes = 2u * 128u * BK;  // per CTA: A half + B half
+constexpr int kRedBatch = 4;  // split-K slices summed per round of loads
 
 struct alignas(1024) PairStorage {
   uint8_t a[kPairStages][128 * BK];
@@ -689,24 +693,40 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
       last = __shfl_sync(0xFFFFFFFFu, last, 0);
       if (last) {
         // Every other piece of this region is published: sum them with this
-        // unit's own partial (still in TMEM), dequantise and store.
+        // unit's own partial (still in TMEM), dequantise and store.  The
+        // other slices' loads for a chunk are issued together, kRedBatch
+        // slices at a time, so a chunk costs one L2 round trip, not one per
+        // slice.
         __threadfence();
+        const int32_t* slices = p.ws + (static_cast<int64_t>(tile * p.splits) * 16 + region) *
+                                           kRegionInts;
+        constexpr int64_t kSliceStride = 16LL * kRegionInts;
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
           tmem_ld_32x32b_x32(tb + ch * 32, va);
-          tmem_ld_wait();
-          for (int o = 0; o < p.splits; ++o) {
-            if (o == split) continue;
-            const int32_t* other = p.ws + (static_cast<int64_t>(tile * p.splits + o) * 16 + region) *
-                                              kRegionInts;
+#pragma unroll 1
+          for (int o0 = 0; o0 < p.splits; o0 += kRedBatch) {
+            int4 t4[kRedBatch][8];
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const int4 t4 = __ldcg(reinterpret_cast<const int4*>(other + ((ch * 8 + q4) * 32 + lane) * 4));
-              va[q4 * 4] += t4.x;
-              va[q4 * 4 + 1] += t4.y;
-              va[q4 * 4 + 2] += t4.z;
-              va[q4 * 4 + 3] += t4.w;
+            for (int b = 0; b < kRedBatch; ++b) {
+              const int o = o0 + b;
+              const bool use = o < p.splits && o != split;
+              const int32_t* src = slices + o * kSliceStride + (ch * 8 * 32 + lane) * 4;
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                t4[b][q4] = use ? __ldcg(reinterpret_cast<const int4*>(src + q4 * 32 * 4))
+                                : make_int4(0, 0, 0, 0);
             }
+            if (o0 == 0) tmem_ld_wait();
+#pragma unroll
+            for (int b = 0; b < kRedBatch; ++b)
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4) {
+                va[q4 * 4] += t4[b][q4].x;
+                va[q4 * 4 + 1] += t4[b][q4].y;
+                va[q4 * 4 + 2] += t4[b][q4].z;
+                va[q4 * 4 + 3] += t4[b][q4].w;
+              }
           }
           if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
         }
@@ -772,359 +792,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
-// ---------------------------------------------------------------- CTA-pair group-128 kernel
-// Pair tile 256 x 128 (CTA rank r: rows [128 r, 128 r + 128) of A and rows
-// [64 r, 64 r + 64) of the tile's 128 B rows); every K block of 128 is one
-// scale group.  Four 128-column TMEM buffers take turns holding a group's
-// partial sum.  Each buffer is pre-loaded with the integer 0x4B400000 (the
-// bits of 1.5 * 2^23) and the MMA accumulates the group's products onto it,
-// so the epilogue reads 1.5 * 2^23 + P_g as a float: one packed subtract gives
-// (float)P_g exactly (|P_g| <= 128 * 127^2 < 2^22) and one packed fused
-// multiply-add folds it into the fp32 accumulator, f = fmaf(P_g, s[n, g], f),
-// in ascending g.  The epilogue writes the bias back into the buffer before
-// handing it back to the MMA.
-constexpr int kGroupPairBN = 128;
-constexpr int kGroupPairStages = 8;
-constexpr int kGroupPairBufs = 4;
-constexpr int kGroupPairScaleGroups = 8;  // scale groups staged per refill
-constexpr int kGroupPairEpiWarps = 8;     // two per TMEM lane quadrant
-constexpr int kGroupPairCols = kGroupPairBN / 2;  // columns per epilogue warp
-constexpr int kGroupPairThreads = 64 + kGroupPairEpiWarps * 32;
-constexpr uint32_t kGroupPairStageBytes = 128u * BK + 64u * BK;  // per CTA
-constexpr uint32_t kPartialBias = 0x4B400000u;
-
-struct alignas(1024) PairGroupStorage {
-  uint8_t a[kGroupPairStages][128 * BK];
-  uint8_t b[kGroupPairStages][64 * BK];
-  // per epilogue warp: two alternating [groups][columns] scale buffers
-  float sw_tile[kGroupPairEpiWarps][2][kGroupPairScaleGroups][kGroupPairCols];
-  uint64_t full[kGroupPairStages];
-  uint64_t empty[kGroupPairStages];
-  uint64_t acc_full[kGroupPairBufs];
-  uint64_t acc_empty[kGroupPairBufs];  // this CTA's 16 epilogue warps (CTA scope)
-  uint64_t peer_empty[kGroupPairBufs];  // leader only: one forwarded arrival from the peer
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort;
-};
-
-__device__ void produce_pair_group(PairGroupStorage& s, const CUtensorMap* tmA,
-                                   const CUtensorMap* tmB, const Args& p, uint32_t rank) {
-  const int ntiles = p.tiles_m * p.tiles_n;
-  const int npairs = gridDim.x >> 1;
-  uint32_t stage = 0, phase = 0, issued = 0;
-  bool ok = true;
-  for (int tile = blockIdx.x >> 1; ok && tile < ntiles; tile += npairs) {
-    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    const int ya = tm * kPairBM + static_cast<int>(rank) * 128;
-    const int yb = tn * kGroupPairBN + static_cast<int>(rank) * 64;
-    for (int kb = 0; kb < p.num_kb; ++kb) {
-      if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, &s.abort)) {
-        ok = false;
-        break;
-      }
-      const uint32_t fb_local = smem_addr(&s.full[stage]);
-      if (rank == 0) mbar_arrive_expect_tx(fb_local, 2u * kGroupPairStageBytes);
-      const uint32_t fb = map_to_rank(fb_local, 0);
-      tma_load_2d_pair(smem_addr(s.a[stage]), tmA, fb, kb * BK, ya);
-      tma_load_2d_pair(smem_addr(s.b[stage]), tmB, fb, kb * BK, yb);
-      ++issued;
-      if (++stage == kGroupPairStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-  }
-  if (rank == 0) {
-    const uint32_t first = issued > kGroupPairStages ? issued - kGroupPairStages : 0u;
-    for (uint32_t i = first; i < issued; ++i)
-      mbar_wait(smem_addr(&s.full[i % kGroupPairStages]), (i / kGroupPairStages) & 1u, nullptr);
-  }
-}
-
-// The n-th use of buffer b waits for the n-th "empty" round of b (round 0 is
-// the epilogue's initial bias fill).
-__device__ void mma_issue_pair_group(PairGroupStorage& s, uint32_t tmem, const Args& p) {
-  const int ntiles = p.tiles_m * p.tiles_n;
-  const int npairs = gridDim.x >> 1;
-  constexpr uint32_t idesc = idesc_i8(kPairBM, kGroupPairBN);
-  uint32_t stage = 0, phase = 0, gcount = 0;
-  bool ok = true;
-  for (int tile = blockIdx.x >> 1; ok && tile < ntiles; tile += npairs) {
-    for (int kb = 0; kb < p.num_kb; ++kb, ++gcount) {
-      const uint32_t buf = gcount % kGroupPairBufs;
-      const uint32_t use = (gcount / kGroupPairBufs) & 1u;
-      if (!mbar_wait(smem_addr(&s.acc_empty[buf]), use, &s.abort) ||
-          !mbar_wait(smem_addr(&s.peer_empty[buf]), use, &s.abort)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (!mbar_wait(smem_addr(&s.full[stage]), phase, &s.abort)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d = tmem + buf * kGroupPairBN;
-      const uint32_t a0 = smem_addr(s.a[stage]);
-      const uint32_t b0 = smem_addr(s.b[stage]);
-#pragma unroll
-      for (int kk = 0; kk < BK / UMMA_K; ++kk)  // always accumulate: onto the bias
-        mma_i8_pair(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc,
-                    1u);
-      mma_commit_pair(smem_addr(&s.empty[stage]), 0x3);
-      mma_commit_pair(smem_addr(&s.acc_full[buf]), 0x3);
-      if (++stage == kGroupPairStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-  }
-  mma_commit_pair(smem_addr(&s.drain), 0x1);
-  mbar_wait(smem_addr(&s.drain), 0u, nullptr);
-}
-
-// Peer CTA only: forward each completed round of this CTA's acc_empty[b] (its
-// 16 epilogue warps, CTA scope) to the leader's peer_empty[b] as one
-// cluster-scope arrival, so the epilogue warps never pay for a cluster-wide
-// release themselves.
-__device__ void forward_pair_group(PairGroupStorage& s, const Args& p) {
-  const int ntiles = p.tiles_m * p.tiles_n;
-  const int npairs = gridDim.x >> 1;
-  int ntile_local = 0;
-  for (int tile = blockIdx.x >> 1; tile < ntiles; tile += npairs) ++ntile_local;
-  const uint32_t total = static_cast<uint32_t>(ntile_local) * static_cast<uint32_t>(p.groups) +
-                         kGroupPairBufs;  // + the initial bias-fill round of each buffer
-  for (uint32_t r = 0; r < total; ++r) {
-    const uint32_t buf = r % kGroupPairBufs;
-    const uint32_t use = (r / kGroupPairBufs) & 1u;
-    if (!mbar_wait(smem_addr(&s.acc_empty[buf]), use, &s.abort)) break;
-    mbar_arrive_cluster(map_to_rank(smem_addr(&s.peer_empty[buf]), 0));
-  }
-}
-
-// All lanes of a warp wait on the barrier themselves (short waits: no
-// lane-0 relay); the warp proceeds only if every lane saw the phase complete.
-__device__ __forceinline__ bool warp_wait_lanes(uint32_t bar, uint32_t parity,
-                                                volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
-  const bool all = __all_sync(0xFFFFFFFFu, ok);
-  if (!all) *abort = 1;
-  return all;
-}
-
-// f[j] = fmaf(P, s, f[j]) for 16 columns: v holds 1.5 * 2^23 + P (bits),
-// sc the 16 channel scales.
-__device__ __forceinline__ void fold16(uint64_t* f, const uint32_t (&v)[16], const float* sc,
-                                       uint64_t neg_bias2) {
-  const float4* s4p = reinterpret_cast<const float4*>(sc);
-#pragma unroll
-  for (int j4 = 0; j4 < 4; ++j4) {
-    const float4 s4 = s4p[j4];
-    const uint64_t p0 = f32x2_add(pack2(v[4 * j4], v[4 * j4 + 1]), neg_bias2);  // P exactly
-    const uint64_t p1 = f32x2_add(pack2(v[4 * j4 + 2], v[4 * j4 + 3]), neg_bias2);
-    f[2 * j4] = f32x2_fma(p0, pack2(__float_as_uint(s4.x), __float_as_uint(s4.y)), f[2 * j4]);
-    f[2 * j4 + 1] =
-        f32x2_fma(p1, pack2(__float_as_uint(s4.z), __float_as_uint(s4.w)), f[2 * j4 + 1]);
-  }
-}
-
-// Epilogue warp w (2..9): TMEM lanes 32*(w%4) (rows) and columns
-// [64 h, 64 h + 64), h = (w - 2) / 4, of every partial buffer.  The fp32
-// accumulation over groups must run in ascending order, so each warp
-// pipelines inside its own sequence: a group is read in four 16-column
-// chunks, and the TMEM load of the next chunk (the rest of this group, then
-// the first chunk of the next group) is in flight while the chunk in hand is
-// folded in.  Buffer hand-backs are CTA-scope arrivals on this CTA's
-// acc_empty (the peer's are forwarded to the leader by forward_pair_group).
-__device__ void epilogue_pair_group(PairGroupStorage& s, uint32_t tmem, const Args& p,
-                                    uint32_t rank) {
-  const int ntiles = p.tiles_m * p.tiles_n;
-  const int npairs = gridDim.x >> 1;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int quad = warp & 3;
-  const int slice = (warp - 2) >> 2;  // which 64-column half of the tile
-  float (*sws)[kGroupPairScaleGroups][kGroupPairCols] = s.sw_tile[warp - 2];
-  const uint32_t tcol = (static_cast<uint32_t>(quad * 32) << 16) |
-                        static_cast<uint32_t>(slice * kGroupPairCols);
-  // Round 0 of every buffer's "empty" barrier: the initial bias fill.
-#pragma unroll
-  for (int buf = 0; buf < kGroupPairBufs; ++buf) {
-    tmem_st_32x32b_x32_fill(tmem + tcol + buf * kGroupPairBN, kPartialBias);
-    tmem_st_32x32b_x32_fill(tmem + tcol + buf * kGroupPairBN + 32, kPartialBias);
-  }
-  tmem_st_wait();
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0)
-    for (int buf = 0; buf < kGroupPairBufs; ++buf) mbar_arrive(smem_addr(&s.acc_empty[buf]));
-  const uint64_t neg_bias2 = pack2(__float_as_uint(-12582912.0f), __float_as_uint(-12582912.0f));
-  uint32_t gcount = 0;
-  bool ok = true;
-  for (int tile = blockIdx.x >> 1; ok && tile < ntiles; tile += npairs) {
-    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    const int colbase = tn * kGroupPairBN + slice * kGroupPairCols;
-    // Scales of groups [g0, g0 + 8) go to buffer (g0 / 8) & 1 by cp.async, one
-    // refill ahead of their use; lane stages column colbase + lane.
-    auto stage_scales = [&](int g0) {
-#pragma unroll
-      for (int c = 0; c < kGroupPairCols / 32; ++c) {
-        const int col = colbase + lane + 32 * c;
-        float* dst = &sws[(g0 / kGroupPairScaleGroups) & 1][0][lane + 32 * c];
-#pragma unroll
-        for (int gg = 0; gg < kGroupPairScaleGroups; ++gg) {
-          const bool in = col < p.n && g0 + gg < p.groups;
-          cp_async4(smem_addr(dst + gg * kGroupPairCols),
-                    in ? p.sw + static_cast<int64_t>(col) * p.groups + g0 + gg : p.sw, in);
-        }
-      }
-      cp_async_commit();
-    };
-    __syncwarp();
-    stage_scales(0);
-    uint64_t f[kGroupPairCols / 2];  // fp32 accumulators of this row's 64 columns, as pairs
-#pragma unroll
-    for (int j = 0; j < kGroupPairCols / 2; ++j) f[j] = 0ull;
-    uint32_t va[16], vb[16];
-    // prologue: first 16 columns of group 0
-    {
-      const uint32_t buf = gcount % kGroupPairBufs, use = (gcount / kGroupPairBufs) & 1u;
-      if (!warp_wait_lanes(smem_addr(&s.acc_full[buf]), use, &s.abort)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_ld_32x32b_x16(tmem + tcol + buf * kGroupPairBN, va);
-      tmem_ld_wait();
-    }
-    for (int g = 0; g < p.groups; ++g, ++gcount) {
-      const uint32_t buf = gcount % kGroupPairBufs;
-      const uint32_t tb = tmem + tcol + buf * kGroupPairBN;
-      const int gs = g % kGroupPairScaleGroups;
-      if (gs == 0) {
-        cp_async_wait_all();  // this refill's scales have landed
-        __syncwarp();
-        if (g + kGroupPairScaleGroups < p.groups) stage_scales(g + kGroupPairScaleGroups);
-      }
-      const float* sc = sws[(g / kGroupPairScaleGroups) & 1][gs];
-      // four 16-column chunks; the next chunk's load is in flight during each fold
-      tmem_ld_32x32b_x16(tb + 16, vb);
-      fold16(f, va, sc, neg_bias2);
-      tmem_ld_wait();
-      tmem_ld_32x32b_x16(tb + 32, va);
-      fold16(f + 8, vb, sc + 16, neg_bias2);
-      tmem_ld_wait();
-      tmem_ld_32x32b_x16(tb + 48, vb);
-      fold16(f + 16, va, sc + 32, neg_bias2);
-      tmem_ld_wait();
-      // group g is read: re-bias its buffer, then start on the next group
-      tmem_st_32x32b_x32_fill(tb, kPartialBias);
-      tmem_st_32x32b_x32_fill(tb + 32, kPartialBias);
-      if (g + 1 < p.groups) {
-        const uint32_t nb = (gcount + 1) % kGroupPairBufs;
-        const uint32_t nu = ((gcount + 1) / kGroupPairBufs) & 1u;
-        if (!warp_wait_lanes(smem_addr(&s.acc_full[nb]), nu, &s.abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_ld_32x32b_x16(tmem + tcol + nb * kGroupPairBN, va);
-      }
-      fold16(f + 24, vb, sc + 48, neg_bias2);
-      tmem_ld_wait();
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[buf]));
-    }
-    if (!ok) break;
-    const int row = tm * kPairBM + static_cast<int>(rank) * 128 + quad * 32 + lane;
-    if (row < p.m && p.out) {
-      const float sa = __ldg(p.sa + row);
-      if (p.out_bf16) {
-        // out = bf16((f * sa) * alpha); the pairs become packed bf16 words
-        uint32_t w[kGroupPairCols / 2];
-#pragma unroll
-        for (int j = 0; j < kGroupPairCols / 2; ++j)
-          w[j] = pack_bf16x2(__fmul_rn(__fmul_rn(lo_of(f[j]), sa), p.alpha),
-                             __fmul_rn(__fmul_rn(hi_of(f[j]), sa), p.alpha));
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.n;
-#pragma unroll
-        for (int g8 = 0; g8 < kGroupPairCols / 8; ++g8)
-          if (colbase + g8 * 8 < p.n)
-            *reinterpret_cast<uint4*>(orow + colbase + g8 * 8) =
-                make_uint4(w[4 * g8], w[4 * g8 + 1], w[4 * g8 + 2], w[4 * g8 + 3]);
-      } else {
-        float* orow = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.n;
-#pragma unroll
-        for (int g4 = 0; g4 < kGroupPairCols / 4; ++g4)
-          if (colbase + g4 * 4 < p.n)
-            *reinterpret_cast<float4*>(orow + colbase + g4 * 4) =
-                make_float4(__fmul_rn(__fmul_rn(lo_of(f[2 * g4]), sa), p.alpha),
-                            __fmul_rn(__fmul_rn(hi_of(f[2 * g4]), sa), p.alpha),
-                            __fmul_rn(__fmul_rn(lo_of(f[2 * g4 + 1]), sa), p.alpha),
-                            __fmul_rn(__fmul_rn(hi_of(f[2 * g4 + 1]), sa), p.alpha));
-      }
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kGroupPairThreads, 1)
-    gemm_i8_pair_group_kernel(const __grid_constant__ CUtensorMap tmA,
-                              const __grid_constant__ CUtensorMap tmB, const Args p) {
-  extern __shared__ uint8_t smem_raw[];
-  PairGroupStorage& s = storage<PairGroupStorage>(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-  }
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kGroupPairStages; ++i) {
-      mbar_init(smem_addr(&s.full[i]), 1);
-      mbar_init(smem_addr(&s.empty[i]), 1);
-    }
-    for (int i = 0; i < kGroupPairBufs; ++i) {
-      mbar_init(smem_addr(&s.acc_full[i]), 1);
-      mbar_init(smem_addr(&s.acc_empty[i]), kGroupPairEpiWarps);
-      mbar_init(smem_addr(&s.peer_empty[i]), 1);
-    }
-    mbar_init(smem_addr(&s.drain), 1);
-    s.abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_addr(&s.tmem_base), kTmemCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem = s.tmem_base;
-  if (warp == 0) {
-    if (lane == 0) produce_pair_group(s, &tmA, &tmB, p, rank);
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      if (rank == 0)
-        mma_issue_pair_group(s, tmem, p);
-      else
-        forward_pair_group(s, p);
-    }
-    __syncwarp();
-  } else {
-    epilogue_pair_group(s, tmem, p, rank);
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
-}
-
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -1159,6 +826,51 @@ inline bool make_tmap(CUtensorMap* map, const void* base, int rows, int k, int b
          CUDA_SUCCESS;
 }
 
+// Tensor maps depend only on (base, rows, k, box_rows): the recent ones are
+// kept so that repeated calls on the same buffers skip the driver's encoder
+// (a few microseconds of host time per map).
+inline bool cached_tmap(CUtensorMap* map, const void* base, int rows, int k, int box_rows) {
+  struct Entry {
+    const void* base;
+    int rows, k, box_rows;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 32;
+  static Entry entries[kEntries];
+  static int used = 0, next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i) {
+    const Entry& e = entries[i];
+    if (e.base == base && e.rows == rows && e.k == k && e.box_rows == box_rows) {
+      *map = e.map;
+      return true;
+    }
+  }
+  if (!make_tmap(map, base, rows, k, box_rows)) return false;
+  Entry& e = entries[next];
+  e.base = base;
+  e.rows = rows;
+  e.k = k;
+  e.box_rows = box_rows;
+  e.map = *map;
+  next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
+  return true;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel).
+template <class K>
+inline cudaError_t set_smem_once(K kernel, int dev, int slot, size_t bytes) {
+  static std::atomic<unsigned long long> done[4] = {};
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done[slot].load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess && bit) done[slot].fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 inline size_t channel_smem() { return sizeof(ChannelStorage) + 1024; }
 inline size_t pair_smem() { return sizeof(PairStorage) + 1024; }
 
@@ -1189,51 +901,12 @@ inline int max_pairs(int dev, int num_sms) {
   return pairs;
 }
 
-// CTA-pair kernel for m > 128.  0 ok, 1 tensor-map failure, 2 CUDA error.
 // Workspace of the pair kernel's split-K: a fixed header of arrival counters
 // (16 per tile; split-K only runs with fewer than 64 tiles), then the
 // partial-sum slices.  Because the header is at a fixed place and every call
 // leaves its counters at zero, one workspace can serve problems of any shape.
 constexpr size_t kCounterHeaderBytes = 4096;
 constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeaderBytes / (16 * 4));
-
-inline size_t pair_group_smem() { return sizeof(PairGroupStorage) + 1024; }
-
-// Group-128 pair kernel (m > 128).  0 ok, 1 tensor-map failure, 2 CUDA error.
-inline int launch_pair_group(Args a, const int8_t* A, const int8_t* B, int dev, int num_sms,
-                             cudaStream_t stream, cudaError_t* err) {
-  a.tiles_m = (a.m + kPairBM - 1) / kPairBM;
-  a.tiles_n = (a.n + kGroupPairBN - 1) / kGroupPairBN;
-  a.num_kb = a.k / BK;  // k % 128 == 0 in group mode
-  a.groups = a.k / 128;
-  a.splits = 1;
-  a.kb_per_split = a.num_kb;
-  CUtensorMap ta, tb;
-  if (!make_tmap(&ta, A, a.m, a.k, 128) || !make_tmap(&tb, B, a.n, a.k, 64)) return 1;
-  const int ntiles = a.tiles_m * a.tiles_n;
-  const int pairs = max_pairs(dev, num_sms);
-  const int grid_pairs = ntiles < pairs ? ntiles : pairs;
-  cudaError_t e = cudaFuncSetAttribute(gemm_i8_pair_group_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(pair_group_smem()));
-  if (e == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * grid_pairs, 1, 1);
-    cfg.blockDim = dim3(kGroupPairThreads, 1, 1);
-    cfg.dynamicSmemBytes = pair_group_smem();
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gemm_i8_pair_group_kernel, ta, tb, a);
-  }
-  *err = e;
-  return e == cudaSuccess ? 0 : 2;
-}
 
 // Split-K plan of the pair kernel: when the output has fewer tiles than
 // three quarters of the SM pairs, cut K into pieces (>= 8 K blocks each) so
@@ -1264,6 +937,7 @@ inline size_t pair_workspace_bytes(const PairPlan& pl) {
          static_cast<size_t>(pl.tiles) * pl.splits * 16 * 32 * (kPairBN / 2) * 4;
 }
 
+// CTA-pair kernel for m > 128.  0 ok, 1 tensor-map failure, 2 CUDA error.
 inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int num_sms,
                        void* workspace, cudaStream_t stream, cudaError_t* err,
                        bool allow_split = true) {
@@ -1286,12 +960,10 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
     a.ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kCounterHeaderBytes);
   }
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, A, a.m, a.k, 128) || !make_tmap(&tb, B, a.n, a.k, 128)) return 1;
+  if (!cached_tmap(&ta, A, a.m, a.k, 128) || !cached_tmap(&tb, B, a.n, a.k, 128)) return 1;
   const int ntiles = a.tiles_m * a.tiles_n * a.splits;
   const int grid_pairs = ntiles < pairs ? ntiles : pairs;
-  cudaError_t e = cudaFuncSetAttribute(gemm_i8_pair_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(pair_smem()));
+  cudaError_t e = set_smem_once(gemm_i8_pair_kernel, dev, 0, pair_smem());
   if (e == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * grid_pairs, 1, 1);
@@ -1313,7 +985,7 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
 inline size_t group_smem() { return sizeof(GroupStorage) + 1024; }
 
 // 0 ok, 1 tensor-map failure, 2 CUDA error
-inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int num_sms,
+inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev, int num_sms,
                   cudaStream_t stream, cudaError_t* err) {
   const int bn = group ? kGroupBN : kChannelBN;
   a.tiles_m = (a.m + BM - 1) / BM;
@@ -1321,14 +993,13 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int num_
   a.num_kb = (a.k + BK - 1) / BK;
   a.groups = group ? a.k / 128 : 0;
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, A, a.m, a.k, BM) || !make_tmap(&tb, B, a.n, a.k, bn)) return 1;
+  if (!cached_tmap(&ta, A, a.m, a.k, BM) || !cached_tmap(&tb, B, a.n, a.k, bn)) return 1;
   const int ntiles = a.tiles_m * a.tiles_n;
   const int grid = ntiles < num_sms ? ntiles : num_sms;
   cudaError_t e;
   if (!group) {
     const size_t smem = channel_smem();
-    e = cudaFuncSetAttribute(gemm_i8_channel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = set_smem_once(gemm_i8_channel_kernel, dev, 1, smem);
     if (e == cudaSuccess) {
       gemm_i8_channel_kernel<<<grid, kChannelThreads, smem, stream>>>(ta, tb, a);
       e = cudaGetLastError();
@@ -1336,15 +1007,13 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int num_
   } else {
     const size_t smem = group_smem();
     if (a.c) {
-      e = cudaFuncSetAttribute(gemm_i8_group_kernel<true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      e = set_smem_once(gemm_i8_group_kernel<true>, dev, 2, smem);
       if (e == cudaSuccess) {
         gemm_i8_group_kernel<true><<<grid, kGroupThreads, smem, stream>>>(ta, tb, a);
         e = cudaGetLastError();
       }
     } else {
-      e = cudaFuncSetAttribute(gemm_i8_group_kernel<false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      e = set_smem_once(gemm_i8_group_kernel<false>, dev, 3, smem);
       if (e == cudaSuccess) {
         gemm_i8_group_kernel<false><<<grid, kGroupThreads, smem, stream>>>(ta, tb, a);
         e = cudaGetLastError();

@@ -102,10 +102,10 @@ qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, 
 }
 
 // Which kernel runs a GEMM of this shape.
-enum class GemmPath { kGemv, kTensorChannel, kTensorPair, kTensorGroup, kTensorPairGroup };
+enum class GemmPath { kGemv, kTensorChannel, kTensorPair, kTensorGroup };
 
 GemmPath gemm_path(int m, int group_k) {
-  if (group_k != 0) return m <= 128 ? GemmPath::kTensorGroup : GemmPath::kTensorPairGroup;
+  if (group_k != 0) return GemmPath::kTensorGroup;
   if (m <= gemv::max_tokens()) return GemmPath::kGemv;
   if (m <= 128) return GemmPath::kTensorChannel;
   return GemmPath::kTensorPair;
@@ -254,21 +254,8 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   int r = 0;
   if (path == GemmPath::kTensorPair) {
     r = gemm::launch_pair(g, a, b, dev_id, dev->sms, workspace, s, &e);
-  } else if (path == GemmPath::kTensorPairGroup) {
-    // The group kernel produces the scaled output; the full-K int32 sum, when
-    // asked for, comes from a per-channel pass (same MMA, no scales needed).
-    if (out != nullptr) {
-      gemm::Args go = g;
-      go.c = nullptr;
-      r = gemm::launch_pair_group(go, a, b, dev_id, dev->sms, s, &e);
-    }
-    if (r == 0 && c != nullptr) {
-      gemm::Args gc = g;
-      gc.out = nullptr;
-      r = gemm::launch_pair(gc, a, b, dev_id, dev->sms, nullptr, s, &e, false);
-    }
   } else {
-    r = gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev->sms, s, &e);
+    r = gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev_id, dev->sms, s, &e);
   }
   if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
   return r == 0 ? QK_OK : cuda_status(e, "gemm launch");
