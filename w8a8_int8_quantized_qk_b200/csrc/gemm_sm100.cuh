@@ -68,6 +68,8 @@ struct alignas(1024) Storage {
   uint64_t empty[STAGES];
   uint64_t acc_full[NACC];
   uint64_t acc_empty[NACC];
+  uint64_t aux_full[2];   // group kernel: scale slice staged
+  uint64_t aux_empty[2];  // group kernel: scale slice consumed
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -254,13 +256,88 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p) {
   }
 }
 
-// Per-group epilogue, 8 warps: warp w (2..9) owns TMEM lanes 32*(w%4) and
-// columns [64*h, 64*h + 64) of the 128-column tile, h = (w - 2) / 4.  Each
-// warp stages the scales of its 64 columns for SG groups at a time in its own
-// slice of shared memory (only __syncwarp is needed, so an abort can never
-// strand a warp at a CTA-wide barrier).
+// Per-group epilogue.  Warp roles of the group kernel: 0 TMA producer, 1 MMA
+// issuer, 2..9 epilogue, 10 scale stager.  Epilogue warp w owns TMEM lanes
+// 32*(w%4) and columns [64*h, 64*h + 64) of the 128-column tile,
+// h = (w - 2) / 4.
+//
+// The stager copies the weight scales of the tile's 128 columns for SG
+// groups at a time from [n, groups] (global) into a shared slice laid out
+// [group][column], double buffered: slice i is published on aux_full[i]
+// (32 lane arrivals) and handed back on aux_empty[i] (8 warp arrivals).  So
+// the epilogue warps read their 64 scales of a group as 16 broadcast float4
+// loads and never wait on global memory.
+//
+// Accumulation per element, in ascending group order as the definition
+// states: pf = (float)P_g (exact: |P_g| < 2^22, via the bits of 1.5 * 2^23),
+// f = fma(pf, sw[n, g], f).
 constexpr int kGroupCols = 64;
 constexpr int kScaleGroups = 16;
+constexpr int kGroupEpiWarps = 8;
+
+template <int BN, class S>
+__device__ void stage_group_scales(S& s, const Args& p) {
+  const int ntiles = p.tiles_m * p.tiles_n;
+  const int lane = threadIdx.x & 31;
+  const int batches = (p.groups + kScaleGroups - 1) / kScaleGroups;
+  uint32_t buf = 0, phase = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int col0 = (tile / p.tiles_m) * BN;
+    for (int b = 0; b < batches; ++b) {
+      if (!warp_wait(smem_addr(&s.aux_empty[buf]), phase ^ 1u, &s.abort)) return;
+      float* dst = s.scales + buf * (kScaleGroups * BN);
+#pragma unroll 1
+      for (int i = 0; i < BN / 32; ++i) {
+        const int col = col0 + lane + 32 * i;
+        const float* src = p.sw + static_cast<int64_t>(col) * p.groups + b * kScaleGroups;
+        float v[kScaleGroups];
+#pragma unroll
+        for (int gg = 0; gg < kScaleGroups; ++gg)
+          v[gg] = (col < p.n && b * kScaleGroups + gg < p.groups) ? __ldg(src + gg) : 0.0f;
+#pragma unroll
+        for (int gg = 0; gg < kScaleGroups; ++gg) dst[gg * BN + lane + 32 * i] = v[gg];
+      }
+      mbar_arrive(smem_addr(&s.aux_full[buf]));  // release: this lane's stores
+      if (++buf == 2) {
+        buf = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+}
+
+// f[c] = fma((float)P[c], sw[c], f[c]) for the 32 columns C0 .. C0 + 31 of
+// this warp's 64, plus the int32 sums when NC == 64.
+template <int C0, int NC>
+__device__ __forceinline__ void group_fma32(float (&f)[kGroupCols], int (&cs)[NC],
+                                            const uint32_t (&v)[32], const float* sc) {
+  const float4* sc4 = reinterpret_cast<const float4*>(sc + C0);
+#pragma unroll
+  for (int j4 = 0; j4 < 8; ++j4) {
+    const float4 s4 = sc4[j4];
+    const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j4 * 4 + e;
+      // |P| < 2^22: the bits of 1.5 * 2^23 plus P, minus 1.5 * 2^23, is (float)P exactly
+      const float pf = __fsub_rn(__int_as_float(static_cast<int>(v[j]) + 0x4B400000), 12582912.0f);
+      f[C0 + j] = __fmaf_rn(pf, sv[e], f[C0 + j]);
+      if constexpr (NC == kGroupCols) cs[C0 + j] += static_cast<int>(v[j]);
+    }
+  }
+}
+
+// The warp is done reading accumulator buffer abuf: hand it back to the MMA.
+template <int NACC, class S>
+__device__ __forceinline__ void release_acc(S& s, uint32_t& abuf, uint32_t& aphase, int lane) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[abuf]));
+  if (++abuf == NACC) {
+    abuf = 0;
+    aphase ^= 1u;
+  }
+}
 
 template <int BN, int NACC, bool WITH_C, class S>
 __device__ void epilogue_group(S& s, uint32_t tmem, const Args& p) {
@@ -269,8 +346,7 @@ __device__ void epilogue_group(S& s, uint32_t tmem, const Args& p) {
   const int warp = threadIdx.x >> 5;
   const int quad = warp & 3;
   const int half = (warp - 2) >> 2;
-  float* ws = s.scales + (warp - 2) * (kScaleGroups * kGroupCols);  // [SG][64]
-  uint32_t abuf = 0, aphase = 0;
+  uint32_t abuf = 0, aphase = 0, sbuf = 0, sphase = 0;
   bool ok = true;
   for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
@@ -285,53 +361,44 @@ __device__ void epilogue_group(S& s, uint32_t tmem, const Args& p) {
     }
     for (int g = 0; g < p.groups; ++g) {
       const int gs = g % kScaleGroups;
-      if (gs == 0) {
-        __syncwarp();
-        // lane owns columns lane and lane + 32 of this warp's 64
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int col = colbase + lane + 32 * cc;
-          const float* src = p.sw + static_cast<int64_t>(col) * p.groups + g;
-#pragma unroll 4
-          for (int gg = 0; gg < kScaleGroups; ++gg) {
-            const bool in = col < p.n && g + gg < p.groups;
-            ws[gg * kGroupCols + lane + 32 * cc] = in ? __ldg(src + gg) : 0.0f;
-          }
-        }
-        __syncwarp();
+      if (gs == 0 && !warp_wait(smem_addr(&s.aux_full[sbuf]), sphase, &s.abort)) {
+        ok = false;
+        break;
       }
       if (!warp_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t v[kGroupCols];
       const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN +
                           half * kGroupCols;
-      tmem_ld_32x32b_x32(tb, *reinterpret_cast<uint32_t(*)[32]>(v));
-      tmem_ld_32x32b_x32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[abuf]));
-      if (++abuf == NACC) {
-        abuf = 0;
-        aphase ^= 1u;
+      const float* sc = s.scales + sbuf * (kScaleGroups * BN) + gs * BN + half * kGroupCols;
+      if constexpr (WITH_C) {
+        // the int32 sums take 64 more registers: read the 64 columns as two
+        // loads of 32 so that everything stays in registers
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tb, v);
+        tmem_ld_wait();
+        group_fma32<0>(f, cs, v, sc);
+        tmem_ld_32x32b_x32(tb + 32, v);
+        tmem_ld_wait();
+        release_acc<NACC>(s, abuf, aphase, lane);
+        group_fma32<32>(f, cs, v, sc);
+      } else {
+        uint32_t v[32], w[32];
+        tmem_ld_32x32b_x32(tb, v);
+        tmem_ld_32x32b_x32(tb + 32, w);
+        tmem_ld_wait();
+        release_acc<NACC>(s, abuf, aphase, lane);
+        group_fma32<0>(f, cs, v, sc);
+        group_fma32<32>(f, cs, w, sc);
       }
-      const float4* sc = reinterpret_cast<const float4*>(ws + gs * kGroupCols);
-#pragma unroll
-      for (int j4 = 0; j4 < kGroupCols / 4; ++j4) {
-        const float4 s4 = sc[j4];
-        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = j4 * 4 + e;
-          // |P| < 2^22: adding P to the bits of 1.5 * 2^23 and subtracting
-          // 1.5 * 2^23 gives (float)P exactly.
-          const float pf = __fsub_rn(__int_as_float(static_cast<int>(v[j]) + 0x4B400000),
-                                     12582912.0f);
-          f[j] = __fmaf_rn(pf, sv[e], f[j]);
-          if constexpr (WITH_C) cs[j] += static_cast<int>(v[j]);
+      if (gs == kScaleGroups - 1 || g + 1 == p.groups) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&s.aux_empty[sbuf]));
+        if (++sbuf == 2) {
+          sbuf = 0;
+          sphase ^= 1u;
         }
       }
     }
@@ -389,6 +456,10 @@ __device__ __forceinline__ void setup(S& s) {
       mbar_init(smem_addr(&s.acc_full[i]), 1);
       mbar_init(smem_addr(&s.acc_empty[i]), EPI_WARPS);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&s.aux_full[i]), 32);
+      mbar_init(smem_addr(&s.aux_empty[i]), EPI_WARPS);
+    }
     mbar_init(smem_addr(&s.drain), 1);
     s.abort = 0;
     fence_mbar_init();
@@ -441,8 +512,8 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
 
 constexpr int kGroupBN = 128;
 constexpr int kGroupStages = 5;
-constexpr int kGroupThreads = 64 + 8 * 32;
-using GroupStorage = Storage<kGroupBN, kGroupStages, 4, 8 * kScaleGroups * kGroupCols>;
+constexpr int kGroupThreads = 64 + kGroupEpiWarps * 32 + 32;
+using GroupStorage = Storage<kGroupBN, kGroupStages, 4, 2 * kScaleGroups * kGroupBN>;
 
 template <bool WITH_C>
 __global__ void __launch_bounds__(kGroupThreads, 1)
@@ -455,7 +526,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  setup<GroupStorage, kGroupStages, 4, 8>(s);
+  setup<GroupStorage, kGroupStages, 4, kGroupEpiWarps>(s);
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
     if (lane == 0) produce<kGroupBN, kGroupStages>(s, &tmA, &tmB, p);
@@ -463,8 +534,10 @@ __global__ void __launch_bounds__(kGroupThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) mma_issue<kGroupBN, kGroupStages, 4, true>(s, tmem, p);
     __syncwarp();
-  } else {
+  } else if (warp < 2 + kGroupEpiWarps) {
     epilogue_group<kGroupBN, 4, WITH_C>(s, tmem, p);
+  } else {
+    stage_group_scales<kGroupBN>(s, p);
   }
   teardown(s, tmem);
 }
