@@ -257,23 +257,32 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p) {
 }
 
 // Per-group epilogue.  Warp roles of the group kernel: 0 TMA producer, 1 MMA
-// issuer, 2..9 epilogue, 10 scale stager.  Epilogue warp w owns TMEM lanes
-// 32*(w%4) and columns [64*h, 64*h + 64) of the 128-column tile,
-// h = (w - 2) / 4.
+// issuer, then E epilogue warps, then one scale stager.  Epilogue warp w owns
+// TMEM lanes 32*(w%4) and columns [C*h, C*h + C) of the 128-column tile,
+// h = (w - 2) / 4, C = 4 * 128 / E.
 //
 // The stager copies the weight scales of the tile's 128 columns for SG
 // groups at a time from [n, groups] (global) into a shared slice laid out
 // [group][column], double buffered: slice i is published on aux_full[i]
-// (32 lane arrivals) and handed back on aux_empty[i] (8 warp arrivals).  So
-// the epilogue warps read their 64 scales of a group as 16 broadcast float4
-// loads and never wait on global memory.
+// (32 lane arrivals) and handed back on aux_empty[i] (one arrival per
+// epilogue warp).  So the epilogue warps read their scales of a group as
+// broadcast float4 loads and never wait on global memory.
 //
 // Accumulation per element, in ascending group order as the definition
 // states: pf = (float)P_g (exact: |P_g| < 2^22, via the bits of 1.5 * 2^23),
 // f = fma(pf, sw[n, g], f).
-constexpr int kGroupCols = 64;
 constexpr int kScaleGroups = 16;
-constexpr int kGroupEpiWarps = 8;
+
+// Epilogue width of the group kernel: 16 warps of 32 columns (four per TMEM
+// lane quadrant, so that more warps hide each one's waits), or 8 warps of 64
+// columns when the int32 sums are also kept (64 more registers per thread;
+// with 16 warps a thread has at most 96).
+template <bool WITH_C>
+struct GroupCfg {
+  static constexpr int epi_warps = WITH_C ? 8 : 16;
+  static constexpr int cols = 4 * 128 / epi_warps;  // columns per warp
+  static constexpr int threads = 64 + epi_warps * 32 + 32;
+};
 
 template <int BN, class S>
 __device__ void stage_group_scales(S& s, const Args& p) {
@@ -307,9 +316,9 @@ __device__ void stage_group_scales(S& s, const Args& p) {
 }
 
 // f[c] = fma((float)P[c], sw[c], f[c]) for the 32 columns C0 .. C0 + 31 of
-// this warp's 64, plus the int32 sums when NC == 64.
-template <int C0, int NC>
-__device__ __forceinline__ void group_fma32(float (&f)[kGroupCols], int (&cs)[NC],
+// this warp's COLS, plus the int32 sums when NC == COLS.
+template <int C0, int COLS, int NC>
+__device__ __forceinline__ void group_fma32(float (&f)[COLS], int (&cs)[NC],
                                             const uint32_t (&v)[32], const float* sc) {
   const float4* sc4 = reinterpret_cast<const float4*>(sc + C0);
 #pragma unroll
@@ -322,7 +331,7 @@ __device__ __forceinline__ void group_fma32(float (&f)[kGroupCols], int (&cs)[NC
       // |P| < 2^22: the bits of 1.5 * 2^23 plus P, minus 1.5 * 2^23, is (float)P exactly
       const float pf = __fsub_rn(__int_as_float(static_cast<int>(v[j]) + 0x4B400000), 12582912.0f);
       f[C0 + j] = __fmaf_rn(pf, sv[e], f[C0 + j]);
-      if constexpr (NC == kGroupCols) cs[C0 + j] += static_cast<int>(v[j]);
+      if constexpr (NC == COLS) cs[C0 + j] += static_cast<int>(v[j]);
     }
   }
 }
@@ -341,23 +350,24 @@ __device__ __forceinline__ void release_acc(S& s, uint32_t& abuf, uint32_t& apha
 
 template <int BN, int NACC, bool WITH_C, class S>
 __device__ void epilogue_group(S& s, uint32_t tmem, const Args& p) {
+  constexpr int COLS = GroupCfg<WITH_C>::cols;
   const int ntiles = p.tiles_m * p.tiles_n;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int quad = warp & 3;
-  const int half = (warp - 2) >> 2;
+  const int sub = (warp - 2) >> 2;  // column slice of the tile
   uint32_t abuf = 0, aphase = 0, sbuf = 0, sphase = 0;
   bool ok = true;
   for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    const int colbase = tn * BN + half * kGroupCols;
-    float f[kGroupCols];
-    int cs[WITH_C ? kGroupCols : 1];
+    const int colbase = tn * BN + sub * COLS;
+    float f[COLS];
+    int cs[WITH_C ? COLS : 1];
 #pragma unroll
-    for (int j = 0; j < kGroupCols; ++j) f[j] = 0.0f;
+    for (int j = 0; j < COLS; ++j) f[j] = 0.0f;
     if constexpr (WITH_C) {
 #pragma unroll
-      for (int j = 0; j < kGroupCols; ++j) cs[j] = 0;
+      for (int j = 0; j < COLS; ++j) cs[j] = 0;
     }
     for (int g = 0; g < p.groups; ++g) {
       const int gs = g % kScaleGroups;
@@ -371,27 +381,25 @@ __device__ void epilogue_group(S& s, uint32_t tmem, const Args& p) {
       }
       tc_fence_after();
       const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN +
-                          half * kGroupCols;
-      const float* sc = s.scales + sbuf * (kScaleGroups * BN) + gs * BN + half * kGroupCols;
-      if constexpr (WITH_C) {
-        // the int32 sums take 64 more registers: read the 64 columns as two
-        // loads of 32 so that everything stays in registers
+                          sub * COLS;
+      const float* sc = s.scales + sbuf * (kScaleGroups * BN) + gs * BN + sub * COLS;
+      if constexpr (COLS == 64) {
+        // 8 warps of 64 columns (the int32-sum form): two loads of 32 so
+        // that the sums and the accumulators stay in registers
         uint32_t v[32];
         tmem_ld_32x32b_x32(tb, v);
         tmem_ld_wait();
-        group_fma32<0>(f, cs, v, sc);
+        group_fma32<0, COLS>(f, cs, v, sc);
         tmem_ld_32x32b_x32(tb + 32, v);
         tmem_ld_wait();
         release_acc<NACC>(s, abuf, aphase, lane);
-        group_fma32<32>(f, cs, v, sc);
+        group_fma32<32, COLS>(f, cs, v, sc);
       } else {
-        uint32_t v[32], w[32];
+        uint32_t v[32];
         tmem_ld_32x32b_x32(tb, v);
-        tmem_ld_32x32b_x32(tb + 32, w);
         tmem_ld_wait();
         release_acc<NACC>(s, abuf, aphase, lane);
-        group_fma32<0>(f, cs, v, sc);
-        group_fma32<32>(f, cs, w, sc);
+        group_fma32<0, COLS>(f, cs, v, sc);
       }
       if (gs == kScaleGroups - 1 || g + 1 == p.groups) {
         __syncwarp();
@@ -407,7 +415,7 @@ __device__ void epilogue_group(S& s, uint32_t tmem, const Args& p) {
     if (row < p.m) {
       const float sa = __ldg(p.sa + row);
 #pragma unroll
-      for (int g8 = 0; g8 < kGroupCols / 8; ++g8) {
+      for (int g8 = 0; g8 < COLS / 8; ++g8) {
         const int col = colbase + g8 * 8;
         if (col >= p.n) break;
         const int64_t o = static_cast<int64_t>(row) * p.n + col;
@@ -512,11 +520,10 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
 
 constexpr int kGroupBN = 128;
 constexpr int kGroupStages = 5;
-constexpr int kGroupThreads = 64 + kGroupEpiWarps * 32 + 32;
 using GroupStorage = Storage<kGroupBN, kGroupStages, 4, 2 * kScaleGroups * kGroupBN>;
 
 template <bool WITH_C>
-__global__ void __launch_bounds__(kGroupThreads, 1)
+__global__ void __launch_bounds__(GroupCfg<WITH_C>::threads, 1)
     gemm_i8_group_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, const Args p) {
   extern __shared__ uint8_t smem_raw[];
@@ -526,7 +533,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  setup<GroupStorage, kGroupStages, 4, kGroupEpiWarps>(s);
+  constexpr int kEpiWarps = GroupCfg<WITH_C>::epi_warps;
+  setup<GroupStorage, kGroupStages, 4, kEpiWarps>(s);
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
     if (lane == 0) produce<kGroupBN, kGroupStages>(s, &tmA, &tmB, p);
@@ -534,7 +542,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) mma_issue<kGroupBN, kGroupStages, 4, true>(s, tmem, p);
     __syncwarp();
-  } else if (warp < 2 + kGroupEpiWarps) {
+  } else if (warp < 2 + kEpiWarps) {
     epilogue_group<kGroupBN, 4, WITH_C>(s, tmem, p);
   } else {
     stage_group_scales<kGroupBN>(s, p);
@@ -1082,13 +1090,13 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
     if (a.c) {
       e = set_smem_once(gemm_i8_group_kernel<true>, dev, 2, smem);
       if (e == cudaSuccess) {
-        gemm_i8_group_kernel<true><<<grid, kGroupThreads, smem, stream>>>(ta, tb, a);
+        gemm_i8_group_kernel<true><<<grid, GroupCfg<true>::threads, smem, stream>>>(ta, tb, a);
         e = cudaGetLastError();
       }
     } else {
       e = set_smem_once(gemm_i8_group_kernel<false>, dev, 3, smem);
       if (e == cudaSuccess) {
-        gemm_i8_group_kernel<false><<<grid, kGroupThreads, smem, stream>>>(ta, tb, a);
+        gemm_i8_group_kernel<false><<<grid, GroupCfg<false>::threads, smem, stream>>>(ta, tb, a);
         e = cudaGetLastError();
       }
     }
