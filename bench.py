@@ -42,6 +42,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill INT8 TOPS and decode weight-stream GB/s, % of B200 roofline"
+# ncu counters of the current kernels (see the --gemm-traffic help)
+GEMM_TRAFFIC_BYTES = 33.788160e6 + 1.123840e6
+GEMV_TRAFFIC_BYTES = 58.813440e6 + 0.028928e6
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -146,30 +149,9 @@ def _copies(bytes_per_copy: int, floor: int = 2) -> int:
     return max(floor, -(-3 * L2_BYTES // max(bytes_per_copy, 1)))
 
 
-class Timer:
-    """Per-stage CUDA events on one stream."""
-
-    def __init__(self, torch, stream, stages: list[str], steps: int):
-        self.torch = torch
-        self.stream = stream
-        self.stages = stages
-        self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
-                   for _ in range(steps)]
-
-    def mark(self, step: int, i: int):
-        self.ev[step][i].record(self.stream)
-
-    def per_stage_ms(self) -> dict:
-        out = {}
-        for i, name in enumerate(self.stages):
-            out[name] = statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in self.ev)
-        out["step"] = statistics.fmean(e[0].elapsed_time(e[-1]) for e in self.ev)
-        return out
-
-
 class Linear:
-    """A workload resident on the device in R rotating copies; step(i, timer)
-    runs quantise + GEMM through the C ABI on copy i % R."""
+    """A workload resident on the device in R rotating copies; step(i) runs
+    quantise + GEMM through the C ABI on copy i % R."""
 
     def __init__(self, torch, qk, w, stream, copies: int | None = None):
         import ctypes
@@ -227,16 +209,10 @@ class Linear:
         if st != 0:
             raise qk.QKError(st, "gemm")
 
-    def step(self, i: int, timer: Timer | None = None, ti: int = 0):
+    def step(self, i: int):
         j = i % self.R
-        if timer:
-            timer.mark(ti, 0)
         self.quant(j)
-        if timer:
-            timer.mark(ti, 1)
         self.gemm(j)
-        if timer:
-            timer.mark(ti, 2)
 
 
 def _bytes(w) -> dict:
@@ -252,7 +228,43 @@ def _bytes(w) -> dict:
     return {"quant": qb, "gemm": gb}
 
 
+def _graph_us(torch, L, body, iters: int, reps: int = 3) -> float:
+    """Average device time of one iteration of `body(i)`: `iters` iterations
+    are captured into one CUDA graph (so host-side launch cost cannot leave
+    the GPU idle between kernels) and the graph is replayed `reps` times
+    between CUDA events on the current stream."""
+    import ctypes
+
+    cur = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(cur)
+    g = torch.cuda.CUDAGraph()
+    saved = L.stream
+    L.stream = ctypes.c_void_p(cap.cuda_stream)
+    try:
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(iters):
+                body(i)
+    finally:
+        L.stream = saved
+    g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(reps):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * iters)
+    del g
+    return us
+
+
 def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
+    """Stage times of one workload: quantiser alone, GEMM alone and the whole
+    step, each as the average over `iters` back-to-back iterations (rotating
+    copies) replayed from a CUDA graph."""
     from w8a8_int8_quantized_qk_b200 import synth
 
     w = synth.make(name)
@@ -264,25 +276,25 @@ def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
     L = Linear(torch, qk, w, stream)
     for i in range(5):
         L.step(i)
-    t = Timer(torch, stream, ["quant", "gemm"], iters)
-    for i in range(iters):
-        L.step(i, t, i)
     torch.cuda.synchronize()
-    ms = t.per_stage_ms()
+    quant_us = _graph_us(torch, L, lambda i: L.quant(i % L.R), iters)
+    gemm_us = _graph_us(torch, L, lambda i: L.gemm(i % L.R), iters)
+    step_us = _graph_us(torch, L, lambda i: L.step(i), iters)
     by = _bytes(w)
     ops = 2.0 * w.m * w.n * w.k
     gemm_kernel = "gemv (CUDA cores)" if (w.m <= 8 and not w.group_k) else (
-        "tcgen05 group-128" if w.group_k else "tcgen05 per-channel")
-    res = {"m": w.m, "n": w.n, "k": w.k, "copies": L.R,
+        "tcgen05 group-128" if w.group_k else
+        ("tcgen05 per-channel, 1 SM" if w.m <= 128 else "tcgen05 per-channel, CTA pair"))
+    res = {"m": w.m, "n": w.n, "k": w.k, "copies": L.R, "timing": f"CUDA graph of {iters} iterations",
            "quant_kernel": "silu_mul_quant" if w.gate is not None else "quantize_per_token",
-           "quant_us": ms["quant"] * 1e3, "quant_GBs": by["quant"] / (ms["quant"] * 1e-3) / 1e9,
-           "quant_hbm_frac": by["quant"] / (ms["quant"] * 1e-3) / 1e9 / pk["hbm_gbs"],
-           "gemm_kernel": gemm_kernel, "gemm_us": ms["gemm"] * 1e3,
-           "gemm_TOPS": ops / (ms["gemm"] * 1e-3) / 1e12,
-           "gemm_GBs": by["gemm"] / (ms["gemm"] * 1e-3) / 1e9,
-           "gemm_tensor_frac": ops / (ms["gemm"] * 1e-3) / 1e12 / pk["int8_tops"],
-           "gemm_hbm_frac": by["gemm"] / (ms["gemm"] * 1e-3) / 1e9 / pk["hbm_gbs"],
-           "step_us": ms["step"] * 1e3, "bytes": by}
+           "quant_us": quant_us, "quant_GBs": by["quant"] / (quant_us * 1e-6) / 1e9,
+           "quant_hbm_frac": by["quant"] / (quant_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+           "gemm_kernel": gemm_kernel, "gemm_us": gemm_us,
+           "gemm_TOPS": ops / (gemm_us * 1e-6) / 1e12,
+           "gemm_GBs": by["gemm"] / (gemm_us * 1e-6) / 1e9,
+           "gemm_tensor_frac": ops / (gemm_us * 1e-6) / 1e12 / pk["int8_tops"],
+           "gemm_hbm_frac": by["gemm"] / (gemm_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+           "step_us": step_us, "bytes": by}
     del L
     torch.cuda.empty_cache()
     return res
@@ -387,12 +399,35 @@ def run_ours(args):
     pk = peaks()
     stream = torch.cuda.current_stream()
 
-    # ---- headline: prefill step (quantise + GEMM), device-resident inputs
+    # ---- headline: prefill step (quantise + GEMM), device-resident inputs.
+    # The W warm-up steps and the K timed steps are each captured into one
+    # CUDA graph (rotating copies, so every step reads fresh operands from
+    # HBM); the timed graph is replayed once between CUDA events.
+    import ctypes
+
     w = synth.make("prefill")
     L = Linear(torch, qk, w, stream)
-    for i in range(args.warmup):
+    for i in range(3):  # first calls set up tensor maps and kernel attributes
         L.step(i)
-    timer = Timer(torch, stream, ["quant", "gemm"], args.steps)
+    torch.cuda.synchronize()
+
+    def capture(first: int, count: int):
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        saved = L.stream
+        L.stream = ctypes.c_void_p(cap.cuda_stream)
+        try:
+            with torch.cuda.graph(g, stream=cap):
+                for i in range(first, first + count):
+                    L.step(i)
+        finally:
+            L.stream = saved
+        return g
+
+    g_warm = capture(0, args.warmup)
+    g_timed = capture(args.warmup, args.steps)
+    g_warm.replay()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
@@ -401,30 +436,36 @@ def run_ours(args):
     barrier()
     with clocks:
         start.record(stream)
-        for i in range(args.steps):
-            L.step(args.warmup + i, timer, i)
+        g_timed.replay()
         end.record(stream)
         barrier()
     total_ms = start.elapsed_time(end)
+    del g_warm, g_timed
     if dist is not None:
         t = torch.tensor([total_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    st = timer.per_stage_ms()
+    # the GEMM's and the quantiser's average launch durations: the same
+    # launches, each kernel alone in a graph of K back-to-back launches
+    iters = max(10, min(args.steps, 100))
+    quant_us = _graph_us(torch, L, lambda i: L.quant(i % L.R), iters)
+    gemm_us = _graph_us(torch, L, lambda i: L.gemm(i % L.R), iters)
     ops_step = 2.0 * w.m * w.n * w.k
     ms_per_step = total_ms / args.steps
     value = world * ops_step * args.steps / (total_ms * 1e-3) / 1e12
     by = _bytes(w)
-    gemm_tops = ops_step / (st["gemm"] * 1e-3) / 1e12
-    roof = {"kernel": "gemm_i8_channel_kernel (tcgen05)", "bound": "tensor",
+    gemm_tops = ops_step / (gemm_us * 1e-6) / 1e12
+    roof = {"kernel": "gemm_i8_pair_kernel (tcgen05.mma.cta_group::2, 256x256 tiles)", "bound": "tensor",
             "achieved": gemm_tops, "peak": pk["int8_tops"], "unit": "TFLOP/s",
-            "frac": gemm_tops / pk["int8_tops"], "traffic": args.gemm_traffic,
+            "frac": gemm_tops / pk["int8_tops"], "traffic": args.gemm_traffic or None,
             "peak_note": f"2 x {pk['source']} bf16 burst ({pk['bf16_tflops']} TFLOP/s): the nominal "
                          "dense int8:bf16 ratio; int8 ops counted as 2*M*N*K",
+            "timing": f"average of a CUDA graph of {iters} back-to-back GEMM launches on the "
+                      "headline's rotating buffers",
             "algorithmic_bytes": by["gemm"],
-            "launch_us": st["gemm"] * 1e3, "quant_us": st["quant"] * 1e3,
-            "quant_GBs": by["quant"] / (st["quant"] * 1e-3) / 1e9,
-            "quant_hbm_frac": by["quant"] / (st["quant"] * 1e-3) / 1e9 / pk["hbm_gbs"]}
+            "launch_us": gemm_us, "quant_us": quant_us,
+            "quant_GBs": by["quant"] / (quant_us * 1e-6) / 1e9,
+            "quant_hbm_frac": by["quant"] / (quant_us * 1e-6) / 1e9 / pk["hbm_gbs"]}
 
     # ---- e2e through the public API with host buffers
     e2e = None
@@ -469,11 +510,11 @@ def run_ours(args):
         d = stages["decode"]
         gbs = d["bytes"]["gemm"] / (d["gemm_us"] * 1e-6) / 1e9
         decode = {"value": gbs, "unit": "GB/s", "workload": "decode linear X bf16 [4,4096] x W int8 "
-                  "[14336,4096]^T, bf16 out", "kernel": "gemv_i8_kernel (dp4a, CUDA cores)",
+                  "[14336,4096]^T, bf16 out", "kernel": "gemv_i8_prefetch_kernel (dp4a, CUDA cores)",
                   "gemv_us": d["gemm_us"], "algorithmic_bytes": d["bytes"]["gemm"],
                   "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
-                               "traffic": args.gemv_traffic},
+                               "traffic": args.gemv_traffic or None},
                   "quant_us": d["quant_us"], "step_us": d["step_us"]}
     if dist is not None:
         torch.cuda.synchronize()
@@ -490,6 +531,8 @@ def run_ours(args):
                                    "W int8 [4096,4096], per-channel fp32 scales, INT32 accumulation, "
                                    "bf16 out", "m": w.m, "n": w.n, "k": w.k,
                        "parallelism": f"replicas x{world}",
+                       "timing": "warm-up and timed steps each captured as one CUDA graph; the timed "
+                                 "graph replayed once between CUDA events, max over ranks",
                        "l2": f"rotating {_copies(w.x.nbytes + w.w_q.nbytes + w.m * w.k + 2 * w.m * w.n)}"
                              " copies of inputs/outputs (working set >= 3x L2)"},
             "gpu_launches": args.steps * 2, "roofline": roof, "clocks": clocks.summary(),
@@ -510,9 +553,13 @@ def main():
     ap.add_argument("--no-smi", dest="smi", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--stage-iters", type=int, default=50)
-    ap.add_argument("--gemm-traffic", type=float, default=None,
-                    help="ncu dram bytes per GEMM launch, when captured for the current build")
-    ap.add_argument("--gemv-traffic", type=float, default=None)
+    # DRAM bytes (read + write) per launch from one ncu capture of the current
+    # build of each kernel; pass a new figure, or 0 for null, whenever the
+    # kernel changes.
+    ap.add_argument("--gemm-traffic", type=float, default=GEMM_TRAFFIC_BYTES,
+                    help="dram__bytes_read.sum + dram__bytes_write.sum of one prefill GEMM launch")
+    ap.add_argument("--gemv-traffic", type=float, default=GEMV_TRAFFIC_BYTES,
+                    help="the same for one decode GEMV launch")
     ap.add_argument("--only", choices=["tiny", "decode", "prefill", "mlp_down", "group"],
                     help="profiling aid: time one workload's stages and print them")
     args = ap.parse_args()
