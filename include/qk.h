@@ -165,11 +165,12 @@ QK_API qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, con
  * workspace      device scratch of at least qk_w8a8_gemm_workspace_size()
  *                bytes, 256-B aligned; may be NULL when that size is 0.  It
  *                is used when the output has too few tiles to occupy the GPU
- *                and K is split across CTA pairs (partial INT32 sums plus a
- *                4 KB header of arrival counters).  It must be zero-filled
- *                before its first use; every completed call leaves the
- *                header zero again, so one workspace (sized for the largest
- *                problem) can be reused across calls and shapes.  The call
+ *                and K is split across CTA pairs (a 4 KB header of arrival
+ *                counters, then one INT32 accumulator per output tile that
+ *                the K slices add into).  It must be zero-filled before its
+ *                first use; every completed call leaves it all zero again,
+ *                so one workspace (sized for the largest problem) can be
+ *                reused across calls and shapes.  The call
  *                owns it until the work on `stream` completes: calls that
  *                may overlap need separate workspaces.  After a call that
  *                ended in QK_ERR_TIMEOUT, zero-fill it again.
@@ -204,14 +205,17 @@ QK_API size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k);
  * - The first call on a device looks up the scratch array's device address
  *   (once per device, with that device current); make that first call before
  *   any stream capture on the device.
- * - Each call clears the scratch array's counter header on `stream` before
- *   its kernel, so it does not depend on what an earlier call left there.
+ * - Each call clears the part of the scratch array it uses (counters and
+ *   accumulators) on `stream` before its kernel, so it does not depend on
+ *   what an earlier call left there.
  * - Every call shares the one array: calls that can overlap on the GPU (on
  *   different streams, or from different threads) race and give wrong
  *   results.  Serialise them.
- * - A problem whose split-K needs more than QK_NOALLOC_SCRATCH_BYTES (see
- *   qk_w8a8_gemm_workspace_size) is rejected with QK_ERR_WORKSPACE and
- *   nothing is launched.  Other errors are those of qk_w8a8_gemm.
+ * - QK_NOALLOC_SCRATCH_BYTES covers every split-K problem (split-K runs
+ *   with fewer than 64 output tiles, 4 KB + 256 KB per tile); a problem
+ *   whose qk_w8a8_gemm_workspace_size exceeded it would be rejected with
+ *   QK_ERR_WORKSPACE and nothing launched.  Other errors are those of
+ *   qk_w8a8_gemm.
  */
 #define QK_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u + 4096u)
 

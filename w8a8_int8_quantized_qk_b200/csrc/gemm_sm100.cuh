@@ -566,7 +566,6 @@ constexpr int kPairStages = 6;
 constexpr int kPairEpiWarps = 8;  // two per TMEM lane quadrant, 128 columns each
 constexpr int kPairThreads = 64 + kPairEpiWarps * 32;
 constexpr uint32_t kPairStageBytes = 2u * 128u * BK;  // per CTA: A half + B half
-constexpr int kRedBatch = 4;  // split-K slices summed per round of loads
 
 struct alignas(1024) PairStorage {
   uint8_t a[kPairStages][128 * BK];
@@ -752,62 +751,56 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
         tmem_ld_wait();
       }
     } else {
-      // This warp's 32 x 128 region of the tile: publish the partial sum in
-      // slice `split` of the workspace, laid out [column quad][lane][4] so a
-      // warp's 16-byte stores and loads are contiguous.
+      // Split-K.  Every pair holds exactly one unit (the host plans at most
+      // one unit per pair), so once acc_full has fired the operand ring is
+      // idle and serves as staging space: this warp copies its 32 x 128
+      // partial region from TMEM into its own 16 KB of the ring, laid out
+      // [column quad][lane][4], and one bulk reduction adds it into the
+      // tile's int32 accumulator in the workspace (the additions happen at
+      // L2).  The warp that brings a region's arrival count to `splits`
+      // reads the finished sum, runs the epilogue, and leaves the region and
+      // its counter zero for the next call.
       constexpr int kRegionInts = 32 * (kPairBN / 2);
-      int32_t* my_slice = p.ws + (static_cast<int64_t>(tile * p.splits + split) * 16 + region) *
-                                     kRegionInts;
+      constexpr uint32_t kRegionBytes = kRegionInts * 4;
+      int32_t* acc_region = p.ws + (static_cast<int64_t>(tile) * 16 + region) * kRegionInts;
+      uint8_t* stg = &s.a[0][0] + (warp - 2) * kRegionBytes;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         tmem_ld_32x32b_x32(tb + ch * 32, va);
         tmem_ld_wait();
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<int4*>(my_slice + ((ch * 8 + q4) * 32 + lane) * 4) =
+          *reinterpret_cast<int4*>(stg + (((ch * 8 + q4) * 32 + lane) * 16)) =
               make_int4(va[q4 * 4], va[q4 * 4 + 1], va[q4 * 4 + 2], va[q4 * 4 + 3]);
       }
-      __threadfence();
+      fence_proxy_async_smem();
       __syncwarp();
       int last = 0;
-      if (lane == 0) last = atomicAdd(p.cnt + tile * 16 + region, 1) == p.splits - 1;
+      if (lane == 0) {
+        bulk_reduce_add_s32(acc_region, smem_addr(stg), kRegionBytes);
+        bulk_commit();
+        bulk_wait_all();
+        fence_proxy_async_global();
+        __threadfence();
+        last = atomicAdd(p.cnt + tile * 16 + region, 1) == p.splits - 1;
+      }
       last = __shfl_sync(0xFFFFFFFFu, last, 0);
       if (last) {
-        // Every other piece of this region is published: sum them with this
-        // unit's own partial (still in TMEM), dequantise and store.  The
-        // other slices' loads for a chunk are issued together, kRedBatch
-        // slices at a time, so a chunk costs one L2 round trip, not one per
-        // slice.
         __threadfence();
-        const int32_t* slices = p.ws + (static_cast<int64_t>(tile * p.splits) * 16 + region) *
-                                           kRegionInts;
-        constexpr int64_t kSliceStride = 16LL * kRegionInts;
+        const int4 zero = make_int4(0, 0, 0, 0);
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
-          tmem_ld_32x32b_x32(tb + ch * 32, va);
-#pragma unroll 1
-          for (int o0 = 0; o0 < p.splits; o0 += kRedBatch) {
-            int4 t4[kRedBatch][8];
+          int4 t4[8];
 #pragma unroll
-            for (int b = 0; b < kRedBatch; ++b) {
-              const int o = o0 + b;
-              const bool use = o < p.splits && o != split;
-              const int32_t* src = slices + o * kSliceStride + (ch * 8 * 32 + lane) * 4;
+          for (int q4 = 0; q4 < 8; ++q4)
+            t4[q4] = __ldcg(reinterpret_cast<const int4*>(acc_region + ((ch * 8 + q4) * 32 + lane) * 4));
 #pragma unroll
-              for (int q4 = 0; q4 < 8; ++q4)
-                t4[b][q4] = use ? __ldcg(reinterpret_cast<const int4*>(src + q4 * 32 * 4))
-                                : make_int4(0, 0, 0, 0);
-            }
-            if (o0 == 0) tmem_ld_wait();
-#pragma unroll
-            for (int b = 0; b < kRedBatch; ++b)
-#pragma unroll
-              for (int q4 = 0; q4 < 8; ++q4) {
-                va[q4 * 4] += t4[b][q4].x;
-                va[q4 * 4 + 1] += t4[b][q4].y;
-                va[q4 * 4 + 2] += t4[b][q4].z;
-                va[q4 * 4 + 3] += t4[b][q4].w;
-              }
+          for (int q4 = 0; q4 < 8; ++q4) {
+            va[q4 * 4] = t4[q4].x;
+            va[q4 * 4 + 1] = t4[q4].y;
+            va[q4 * 4 + 2] = t4[q4].z;
+            va[q4 * 4 + 3] = t4[q4].w;
+            __stcg(reinterpret_cast<int4*>(acc_region + ((ch * 8 + q4) * 32 + lane) * 4), zero);
           }
           if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
         }
@@ -983,9 +976,10 @@ inline int max_pairs(int dev, int num_sms) {
 }
 
 // Workspace of the pair kernel's split-K: a fixed header of arrival counters
-// (16 per tile; split-K only runs with fewer than 64 tiles), then the
-// partial-sum slices.  Because the header is at a fixed place and every call
-// leaves its counters at zero, one workspace can serve problems of any shape.
+// (16 per tile; split-K only runs with fewer than 64 tiles), then one int32
+// accumulator per output tile that the K slices add into.  The header is at
+// a fixed place and every completed call leaves counters and accumulators at
+// zero, so one zero-filled workspace can serve problems of any shape.
 constexpr size_t kCounterHeaderBytes = 4096;
 constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeaderBytes / (16 * 4));
 
@@ -1014,8 +1008,8 @@ inline PairPlan pair_plan(int m, int n, int k, int pairs) {
 
 inline size_t pair_workspace_bytes(const PairPlan& pl) {
   if (pl.splits <= 1) return 0;
-  return kCounterHeaderBytes +
-         static_cast<size_t>(pl.tiles) * pl.splits * 16 * 32 * (kPairBN / 2) * 4;
+  // counters, then one int32 accumulator tile (16 regions of 32 x 128) per tile
+  return kCounterHeaderBytes + static_cast<size_t>(pl.tiles) * 16 * 32 * (kPairBN / 2) * 4;
 }
 
 // CTA-pair kernel for m > 128.  0 ok, 1 tensor-map failure, 2 CUDA error.
@@ -1028,7 +1022,8 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
   a.groups = 0;
   const int pairs = max_pairs(dev, num_sms);
   PairPlan pl = pair_plan(a.m, a.n, a.k, pairs);
-  if (!allow_split) {
+  if (!allow_split || static_cast<int64_t>(pl.tiles) * pl.splits > pairs) {
+    // (split-K stages partials in the operand ring: one unit per pair)
     pl.splits = 1;
     pl.kb_per_split = a.num_kb;
   }

@@ -332,6 +332,36 @@ __device__ __forceinline__ void cp_async_wait_prior() {
 }
 
 // ---------------------------------------------------------------------------
+// Bulk element-wise reduction shared -> global, performed at L2 by the
+// asynchronous proxy: dst[i] += src[i] for `bytes` / 4 int32 values (both
+// addresses 16-B aligned, bytes a multiple of 16).  The issuing thread waits
+// for completion with bulk_wait_all(); threads whose generic stores filled
+// the source must first run fence_proxy_async_smem() (and synchronise with
+// the issuer).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void bulk_reduce_add_s32(void* dst, uint32_t src_smem, uint32_t bytes) {
+  asm volatile(
+      "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.s32 [%0], [%1], %2;" ::"l"(
+          reinterpret_cast<uint64_t>(dst)),
+      "r"(src_smem), "r"(bytes)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// generic-proxy writes to shared memory -> visible to the async proxy
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// async-proxy global writes <-> generic-proxy accesses of this thread
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Small helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {

@@ -274,9 +274,8 @@ qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_
   if (need > QK_NOALLOC_SCRATCH_BYTES) return QK_ERR_WORKSPACE;
   void* scratch = noalloc_scratch();
   if (scratch == nullptr) return QK_ERR_CUDA;
-  // The arrival counters sit in the first 4 KB and must start at zero.
-  if (cudaMemsetAsync(scratch, 0, gemm::kCounterHeaderBytes,
-                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // The arrival counters and the split-K accumulators must start at zero.
+  if (cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return QK_ERR_CUDA;
   return qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
                       scratch, QK_NOALLOC_SCRATCH_BYTES, stream);
