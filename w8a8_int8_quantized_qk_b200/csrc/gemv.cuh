@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(kThreads) gemv_i8_kernel(Args p) {
 inline int max_tokens() { return 8; }
 
 // ---------------------------------------------------------------------------
-// Persistent prefetching form (the default for K <= 16384): two CTAs per SM,
-// each walking row groups g = blockIdx, blockIdx + grid, ...  A group is R
+// Persistent prefetching form (the default for K <= 16384): a few CTAs per SM
+// (PrefCfg), each walking row groups g = blockIdx, blockIdx + grid, ...  A group is R
 // rows; thread t owns the 16-byte K chunks t, t + 256, ... (J of them), so its
 // activation chunks for all tokens are loaded once and stay in registers, and
 // the W chunks of the next D - 1 groups are already in flight while the
@@ -133,6 +133,20 @@ __host__ __device__ constexpr int pref_rows(int mt, int j) {
                             : (j == 1 ? 4 : (j == 2 ? 2 : 1)));
 }
 
+// Launch shape per <MT, J>: rows per group R, groups of W chunks in flight D,
+// resident CTAs per SM (the register budget is 65536 / (256 x minb)).  For
+// rows of up to 4096 bytes (J = 1) and up to 4 tokens, more resident CTAs of
+// smaller groups keep more warps issuing loads: 5 CTAs of 3-row groups (48
+// registers) read a 4 x 14336 x 4096 weight stream in 13.0 us where 2 CTAs of
+// 8-row groups, two groups deep, took 16.5 us (same launch method).
+template <int MT, int J>
+struct PrefCfg {
+  static constexpr bool narrow = J == 1 && MT <= 4;
+  static constexpr int rows = narrow ? 3 : pref_rows(MT, J);
+  static constexpr int depth = narrow ? 1 : kPrefDepth;
+  static constexpr int minb = narrow ? 5 : 2;
+};
+
 // The activation chunks of all tokens stay in registers: MT x J <= 16.
 inline bool pref_supported(int m, int k) {
   const int j = (k / 16 + kPrefThreads - 1) / kPrefThreads;
@@ -141,9 +155,10 @@ inline bool pref_supported(int m, int k) {
 }
 
 template <int MT, int J>
-__global__ void __launch_bounds__(kPrefThreads, 2) gemv_i8_prefetch_kernel(Args p) {
-  constexpr int R = pref_rows(MT, J);
-  constexpr int D = kPrefDepth;
+__global__ void __launch_bounds__(kPrefThreads, PrefCfg<MT, J>::minb)
+    gemv_i8_prefetch_kernel(Args p) {
+  constexpr int R = PrefCfg<MT, J>::rows;
+  constexpr int D = PrefCfg<MT, J>::depth;
   __shared__ int red[kPrefThreads / 32][R * MT];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cpr = p.k >> 4;
@@ -227,23 +242,21 @@ __global__ void __launch_bounds__(kPrefThreads, 2) gemv_i8_prefetch_kernel(Args 
 template <int MT>
 inline cudaError_t launch_pref_mt(const Args& a, int num_sms, cudaStream_t stream) {
   const int J = (a.k / 16 + kPrefThreads - 1) / kPrefThreads;
-  int rows = 0;
+  auto go = [&](auto kernel, int rows, int minb) {
+    const int ngroups = (a.n + rows - 1) / rows;
+    const int cap = minb * num_sms;
+    kernel<<<ngroups < cap ? ngroups : cap, kPrefThreads, 0, stream>>>(a);
+  };
   switch (J) {
-    case 1: rows = pref_rows(MT, 1); break;
-    case 2: rows = pref_rows(MT, 2); break;
-    case 3: rows = pref_rows(MT, 3); break;
-    default: rows = pref_rows(MT, 4); break;
-  }
-  const int ngroups = (a.n + rows - 1) / rows;
-  const int grid = ngroups < 2 * num_sms ? ngroups : 2 * num_sms;
-  switch (J) {
-    case 1: gemv_i8_prefetch_kernel<MT, 1><<<grid, kPrefThreads, 0, stream>>>(a); break;
-    case 2: gemv_i8_prefetch_kernel<MT, 2><<<grid, kPrefThreads, 0, stream>>>(a); break;
+    case 1: go(gemv_i8_prefetch_kernel<MT, 1>, PrefCfg<MT, 1>::rows, PrefCfg<MT, 1>::minb); break;
+    case 2: go(gemv_i8_prefetch_kernel<MT, 2>, PrefCfg<MT, 2>::rows, PrefCfg<MT, 2>::minb); break;
     case 3:
-      if constexpr (MT <= 4) gemv_i8_prefetch_kernel<MT, 3><<<grid, kPrefThreads, 0, stream>>>(a);
+      if constexpr (MT <= 4)
+        go(gemv_i8_prefetch_kernel<MT, 3>, PrefCfg<MT, 3>::rows, PrefCfg<MT, 3>::minb);
       break;
     default:
-      if constexpr (MT <= 4) gemv_i8_prefetch_kernel<MT, 4><<<grid, kPrefThreads, 0, stream>>>(a);
+      if constexpr (MT <= 4)
+        go(gemv_i8_prefetch_kernel<MT, 4>, PrefCfg<MT, 4>::rows, PrefCfg<MT, 4>::minb);
       break;
   }
   return cudaGetLastError();
