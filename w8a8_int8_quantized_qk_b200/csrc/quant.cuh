@@ -387,9 +387,31 @@ inline Plan plan(int m, int k, bool bf16, bool silu, int V, int num_sms) {
 template <bool BF16, bool SILU, int V>
 inline cudaError_t launch_rows(const Args& a, int num_sms, cudaStream_t stream);
 
+// Persistent grid: at most four CTAs per SM, and never more than can be
+// resident at once -- a CTA that waits for a second wave starts its rows
+// late and the whole launch waits for it (4 x 148 CTAs of the 4-vector
+// kernel, of which only 3 per SM fit, took 14.0 us at 2048 x 8192; all
+// resident, 12.4 us).
+template <bool BF16, bool SILU, int V>
+inline int persistent_ctas_per_sm() {
+  static int cached = 0;
+  if (cached == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, quant_rows_persistent_kernel<BF16, SILU, V>, kPersistThreads, 0) != cudaSuccess ||
+        n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    cached = n < 4 ? n : 4;
+  }
+  return cached;
+}
+
 template <bool BF16, bool SILU, int V>
 inline cudaError_t launch_persistent(const Args& a, int num_sms, cudaStream_t stream) {
-  const int grid = a.m < 4 * num_sms ? a.m : 4 * num_sms;
+  const int cap = persistent_ctas_per_sm<BF16, SILU, V>() * num_sms;
+  const int grid = a.m < cap ? a.m : cap;
   quant_rows_persistent_kernel<BF16, SILU, V><<<grid, kPersistThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
