@@ -505,6 +505,8 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
     prefetch_tmap(&tmB);
   }
   setup<ChannelStorage, kChannelStages, 2, 4>(s);
+  griddep_wait();  // set-up above overlapped the previous kernel
+  griddep_launch_dependents();
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
     if (lane == 0) produce<kChannelBN, kChannelStages>(s, &tmA, &tmB, p);
@@ -535,6 +537,8 @@ __global__ void __launch_bounds__(GroupCfg<WITH_C>::threads, 1)
   }
   constexpr int kEpiWarps = GroupCfg<WITH_C>::epi_warps;
   setup<GroupStorage, kGroupStages, 4, kEpiWarps>(s);
+  griddep_wait();  // set-up above overlapped the previous kernel
+  griddep_launch_dependents();
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
     if (lane == 0) produce<kGroupBN, kGroupStages>(s, &tmA, &tmB, p);
@@ -849,6 +853,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   __syncthreads();
   cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
+  griddep_wait();  // set-up above overlapped the previous kernel
+  griddep_launch_dependents();
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
     if (lane == 0) produce_pair(s, &tmA, &tmB, p, rank);
@@ -1041,19 +1047,8 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
   const int grid_pairs = ntiles < pairs ? ntiles : pairs;
   cudaError_t e = set_smem_once(gemm_i8_pair_kernel, dev, 0, pair_smem());
   if (e == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * grid_pairs, 1, 1);
-    cfg.blockDim = dim3(kPairThreads, 1, 1);
-    cfg.dynamicSmemBytes = pair_smem();
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel, ta, tb, a);
+    e = launch_pdl(gemm_i8_pair_kernel, dim3(2 * grid_pairs), dim3(kPairThreads), pair_smem(), stream,
+                   2, ta, tb, a);
   }
   *err = e;
   return e == cudaSuccess ? 0 : 2;
@@ -1077,22 +1072,22 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
     const size_t smem = channel_smem();
     e = set_smem_once(gemm_i8_channel_kernel, dev, 1, smem);
     if (e == cudaSuccess) {
-      gemm_i8_channel_kernel<<<grid, kChannelThreads, smem, stream>>>(ta, tb, a);
-      e = cudaGetLastError();
+      e = launch_pdl(gemm_i8_channel_kernel, dim3(grid), dim3(kChannelThreads), smem, stream, 1, ta,
+                     tb, a);
     }
   } else {
     const size_t smem = group_smem();
     if (a.c) {
       e = set_smem_once(gemm_i8_group_kernel<true>, dev, 2, smem);
       if (e == cudaSuccess) {
-        gemm_i8_group_kernel<true><<<grid, GroupCfg<true>::threads, smem, stream>>>(ta, tb, a);
-        e = cudaGetLastError();
+        e = launch_pdl(gemm_i8_group_kernel<true>, dim3(grid), dim3(GroupCfg<true>::threads), smem,
+                       stream, 1, ta, tb, a);
       }
     } else {
       e = set_smem_once(gemm_i8_group_kernel<false>, dev, 3, smem);
       if (e == cudaSuccess) {
-        gemm_i8_group_kernel<false><<<grid, GroupCfg<false>::threads, smem, stream>>>(ta, tb, a);
-        e = cudaGetLastError();
+        e = launch_pdl(gemm_i8_group_kernel<false>, dim3(grid), dim3(GroupCfg<false>::threads), smem,
+                       stream, 1, ta, tb, a);
       }
     }
   }

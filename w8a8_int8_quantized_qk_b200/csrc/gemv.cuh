@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(kThreads) gemv_i8_kernel(Args p) {
   __shared__ int red[kThreads / 32][kRows * MT];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nchunk = p.k >> 4;  // 16-byte chunks per row
+  griddep_wait();  // the previous kernel in the stream is done with our buffers
+  griddep_launch_dependents();
+
   const int ngroups = (p.n + kRows - 1) / kRows;
   for (int grp = blockIdx.x; grp < ngroups; grp += gridDim.x) {
     const int row0 = grp * kRows;
@@ -163,6 +166,9 @@ __global__ void __launch_bounds__(kPrefThreads, PrefCfg<MT, J>::minb)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cpr = p.k >> 4;
   const int ngroups = (p.n + R - 1) / R;
+  griddep_wait();  // the previous kernel in the stream is done with our buffers
+  griddep_launch_dependents();
+
   uint4 av[MT][J];
 #pragma unroll
   for (int t = 0; t < MT; ++t)
@@ -245,21 +251,22 @@ inline cudaError_t launch_pref_mt(const Args& a, int num_sms, cudaStream_t strea
   auto go = [&](auto kernel, int rows, int minb) {
     const int ngroups = (a.n + rows - 1) / rows;
     const int cap = minb * num_sms;
-    kernel<<<ngroups < cap ? ngroups : cap, kPrefThreads, 0, stream>>>(a);
+    return launch_pdl(kernel, dim3(ngroups < cap ? ngroups : cap), dim3(kPrefThreads), 0, stream, 1,
+                      a);
   };
   switch (J) {
-    case 1: go(gemv_i8_prefetch_kernel<MT, 1>, PrefCfg<MT, 1>::rows, PrefCfg<MT, 1>::minb); break;
-    case 2: go(gemv_i8_prefetch_kernel<MT, 2>, PrefCfg<MT, 2>::rows, PrefCfg<MT, 2>::minb); break;
+    case 1: return go(gemv_i8_prefetch_kernel<MT, 1>, PrefCfg<MT, 1>::rows, PrefCfg<MT, 1>::minb);
+    case 2: return go(gemv_i8_prefetch_kernel<MT, 2>, PrefCfg<MT, 2>::rows, PrefCfg<MT, 2>::minb);
     case 3:
       if constexpr (MT <= 4)
-        go(gemv_i8_prefetch_kernel<MT, 3>, PrefCfg<MT, 3>::rows, PrefCfg<MT, 3>::minb);
+        return go(gemv_i8_prefetch_kernel<MT, 3>, PrefCfg<MT, 3>::rows, PrefCfg<MT, 3>::minb);
       break;
     default:
       if constexpr (MT <= 4)
-        go(gemv_i8_prefetch_kernel<MT, 4>, PrefCfg<MT, 4>::rows, PrefCfg<MT, 4>::minb);
+        return go(gemv_i8_prefetch_kernel<MT, 4>, PrefCfg<MT, 4>::rows, PrefCfg<MT, 4>::minb);
       break;
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;  // (pref_supported rules these shapes out)
 }
 
 inline cudaError_t launch(const Args& a, int num_sms, cudaStream_t stream) {
@@ -271,15 +278,11 @@ inline cudaError_t launch(const Args& a, int num_sms, cudaStream_t stream) {
   }
   const int ngroups = (a.n + kRows - 1) / kRows;
   const int grid = ngroups < 64 * num_sms ? ngroups : 64 * num_sms;
-  if (a.m <= 1)
-    gemv_i8_kernel<1><<<grid, kThreads, 0, stream>>>(a);
-  else if (a.m <= 2)
-    gemv_i8_kernel<2><<<grid, kThreads, 0, stream>>>(a);
-  else if (a.m <= 4)
-    gemv_i8_kernel<4><<<grid, kThreads, 0, stream>>>(a);
-  else
-    gemv_i8_kernel<8><<<grid, kThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  const dim3 g(grid), b(kThreads);
+  if (a.m <= 1) return launch_pdl(gemv_i8_kernel<1>, g, b, 0, stream, 1, a);
+  if (a.m <= 2) return launch_pdl(gemv_i8_kernel<2>, g, b, 0, stream, 1, a);
+  if (a.m <= 4) return launch_pdl(gemv_i8_kernel<4>, g, b, 0, stream, 1, a);
+  return launch_pdl(gemv_i8_kernel<8>, g, b, 0, stream, 1, a);
 }
 
 }  // namespace gemv

@@ -184,6 +184,8 @@ __global__ void __launch_bounds__(kMaxThreads) quant_rows_kernel(Args p) {
     row = blockIdx.x;
   }
   const int nvec = p.k / E;
+  griddep_wait();  // the previous kernel in the stream is done with our buffers
+  griddep_launch_dependents();
   const int stride = nranks * blockDim.x;
   const int t0 = rank * blockDim.x + threadIdx.x;
   const char* xr = static_cast<const char*>(p.x) + static_cast<int64_t>(row) * p.ld * ES;
@@ -256,6 +258,8 @@ __global__ void __launch_bounds__(kPersistThreads) quant_rows_persistent_kernel(
   __shared__ float red[2][NW];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nvec = p.k / E;
+  griddep_wait();  // the previous kernel in the stream is done with our buffers
+  griddep_launch_dependents();
   uint4 xc[V], uc[SILU ? V : 1];
   auto fetch = [&](uint4 (&xv)[V], uint4 (&uv)[SILU ? V : 1], int row) {
     const char* xr = static_cast<const char*>(p.x) + static_cast<int64_t>(row) * p.ld * ES;
@@ -320,6 +324,8 @@ __global__ void __launch_bounds__(512) quant_rows_twopass_kernel(Args p) {
   __shared__ float red[33];
   const int row = blockIdx.x;
   const int nvec = p.k / E;
+  griddep_wait();  // the previous kernel in the stream is done with our buffers
+  griddep_launch_dependents();
   const char* xr = static_cast<const char*>(p.x) + static_cast<int64_t>(row) * p.ld * ES;
   const char* ur = SILU ? static_cast<const char*>(p.up) + static_cast<int64_t>(row) * p.ld * ES
                         : nullptr;
@@ -412,8 +418,8 @@ template <bool BF16, bool SILU, int V>
 inline cudaError_t launch_persistent(const Args& a, int num_sms, cudaStream_t stream) {
   const int cap = persistent_ctas_per_sm<BF16, SILU, V>() * num_sms;
   const int grid = a.m < cap ? a.m : cap;
-  quant_rows_persistent_kernel<BF16, SILU, V><<<grid, kPersistThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(quant_rows_persistent_kernel<BF16, SILU, V>, dim3(grid), dim3(kPersistThreads),
+                    0, stream, 1, a);
 }
 
 template <bool BF16, bool SILU>
@@ -436,26 +442,16 @@ template <bool BF16, bool SILU, int V>
 inline cudaError_t launch_rows(const Args& a, int num_sms, cudaStream_t stream) {
   const Plan pl = plan(a.m, a.k, BF16, SILU, V, num_sms);
   if (pl.cluster == 0) {
-    quant_rows_twopass_kernel<BF16, SILU><<<a.m, pl.threads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(quant_rows_twopass_kernel<BF16, SILU>, dim3(a.m), dim3(pl.threads), 0, stream,
+                      1, a);
   }
   if (pl.cluster == 1) {
-    quant_rows_kernel<BF16, SILU, false, V><<<a.m, pl.threads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(quant_rows_kernel<BF16, SILU, false, V>, dim3(a.m), dim3(pl.threads), 0,
+                      stream, 1, a);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.m) * pl.cluster, 1, 1);
-  cfg.blockDim = dim3(pl.threads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = pl.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quant_rows_kernel<BF16, SILU, true, V>, a);
+  return launch_pdl(quant_rows_kernel<BF16, SILU, true, V>,
+                    dim3(static_cast<unsigned>(a.m) * pl.cluster), dim3(pl.threads), 0, stream,
+                    static_cast<unsigned>(pl.cluster), a);
 }
 
 template <bool SILU>
