@@ -4,7 +4,7 @@ and repeated calls are deterministic."""
 import numpy as np
 import pytest
 
-from gpu_util import dev, host, need_gpu
+from gpu_util import dev, host, need_gpu, x_dev
 from w8a8_int8_quantized_qk_b200 import qk, synth
 
 pytestmark = pytest.mark.gpu
@@ -39,3 +39,55 @@ def test_side_stream_and_determinism():
     torch.cuda.synchronize()
     assert np.array_equal(host(out1), host(out2))
     assert qk.device_status() == qk.QK_OK
+
+
+def test_split_k_workspace_left_zero():
+    # split-K adds partial sums into the workspace; every completed call must
+    # leave the whole workspace (counters and accumulators) zero again
+    need_gpu()
+    for (m, n, k) in [(256, 1024, 14336), (200, 512, 4096)]:
+        need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 0)
+        assert need > 0
+        r = synth.streams(m + n, ["a", "w", "sa", "sw"])
+        a = dev(synth.int8_uniform(r["a"], (m, k)))
+        w = dev(synth.int8_uniform(r["w"], (n, k)))
+        sa = dev(synth.scales_uniform(r["sa"], (m,), 0.001, 0.05))
+        sw = dev(synth.scales_uniform(r["sw"], (n,)))
+        ws = torch.zeros((need,), dtype=torch.uint8, device="cuda")
+        outs = []
+        for _ in range(3):
+            out, _ = qk.w8a8_gemm(a, w, sa, sw, workspace=ws)
+            torch.cuda.synchronize()
+            assert qk.device_status() == qk.QK_OK
+            assert int(ws.count_nonzero()) == 0
+            outs.append(host(out))
+        assert all(np.array_equal(outs[0], o) for o in outs[1:])
+
+
+def test_graph_capture_of_the_layer():
+    # the same quantise + GEMM calls captured into a CUDA graph and replayed
+    # (as the benchmark runs them) give the eager results, including the
+    # split-K path and the SiLU prologue
+    need_gpu()
+    w = synth.make_linear(300, 520, 2048, seed=13)
+    x = x_dev(w.x)
+    wq, sw = dev(w.w_q), dev(w.sw)
+    g_, u_ = synth.make_silu(64, 2048, seed=14)
+    gd, ud = x_dev(g_), x_dev(u_)
+    ref = host(qk.linear(x, wq, sw))
+    q_ref, s_ref = (host(t) for t in qk.silu_mul_quant_per_token(gd, ud))
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        out = qk.linear(x, wq, sw)
+        q, s = qk.silu_mul_quant_per_token(gd, ud)
+    for _ in range(2):
+        out.zero_()
+        q.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert qk.device_status() == qk.QK_OK
+        assert np.array_equal(host(out), ref)
+        assert np.array_equal(host(q), q_ref) and np.array_equal(host(s), s_ref)
