@@ -76,13 +76,18 @@ def test_gemm_fp32_out_and_c_only(O, m, n, k):
     assert_bits(out3, ref["out_bf16"], "bf16 (out only)")
 
 
-SPLIT_SHAPES = [(200, 512, 4096), (300, 520, 2048), (256, 1024, 14336), (129, 264, 1024)]
+# few output tiles, so K is split across CTA pairs: the partial sums meet
+# through distributed shared memory in a cluster of the tile's pairs
+# (200x512x4096: 4 splits, 300x520x2048: 2, 256x4096x14336: 3) or in the
+# workspace (256x1024x14336 and 256x8960x4096); 129x264x1024 is not split
+SPLIT_SHAPES = [(200, 512, 4096), (300, 520, 2048), (256, 4096, 14336), (256, 1024, 14336),
+                (256, 8960, 4096), (129, 264, 1024)]
 
 
 @pytest.mark.parametrize("m,n,k", SPLIT_SHAPES)
 def test_gemm_split_k(O, m, n, k):
-    # few output tiles: K is split across CTA pairs and the partial sums meet
-    # in the workspace; run twice (the arrival counters must be back at zero)
+    # run twice: the workspace form's counters and accumulators must be back
+    # at zero
     a, w, sa, sw = _problem(m, n, k, 0, seed=m + 3 * n + k)
     ref = O.linear_from_q(a, sa, w, sw, 0, 1.5)
     for _ in range(2):
@@ -92,7 +97,7 @@ def test_gemm_split_k(O, m, n, k):
 
 
 def test_gemm_split_k_needs_workspace(O):
-    m, n, k = 200, 512, 4096
+    m, n, k = 256, 1024, 14336
     need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 0)
     assert need > 0
     a, w, sa, sw = (dev(t) for t in _problem(m, n, k, 0, seed=1))

@@ -57,6 +57,10 @@ struct Args {
   int splits, kb_per_split;
   int32_t* ws;
   int* cnt;
+  // pair kernel: 1 when the `splits` K slices of a tile are the CTA pairs of
+  // one cluster and are summed through distributed shared memory (no
+  // workspace); 0 for the workspace form above
+  int csplit;
 };
 
 template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
@@ -584,8 +588,10 @@ struct alignas(1024) PairStorage {
   int abort;
 };
 
+// pr: this CTA's rank within its pair; lead: the cluster rank of its pair's
+// leader (clusters hold one pair, or the `splits` pairs of one tile).
 __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUtensorMap* tmB,
-                             const Args& p, uint32_t rank) {
+                             const Args& p, uint32_t pr, uint32_t lead) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int npairs = gridDim.x >> 1;
   uint32_t stage = 0, phase = 0, issued = 0;
@@ -593,8 +599,8 @@ __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUten
   for (int unit = blockIdx.x >> 1; ok && unit < nunits; unit += npairs) {
     const int tile = unit / p.splits, split = unit % p.splits;
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    const int ya = tm * kPairBM + static_cast<int>(rank) * 128;
-    const int yb = tn * kPairBN + static_cast<int>(rank) * 128;
+    const int ya = tm * kPairBM + static_cast<int>(pr) * 128;
+    const int yb = tn * kPairBN + static_cast<int>(pr) * 128;
     const int kb0 = split * p.kb_per_split;
     const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
     for (int kb = kb0; kb < kb1; ++kb) {
@@ -603,8 +609,8 @@ __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUten
         break;
       }
       const uint32_t fb_local = smem_addr(&s.full[stage]);
-      if (rank == 0) mbar_arrive_expect_tx(fb_local, 2u * kPairStageBytes);
-      const uint32_t fb = map_to_rank(fb_local, 0);
+      if (pr == 0) mbar_arrive_expect_tx(fb_local, 2u * kPairStageBytes);
+      const uint32_t fb = map_to_rank(fb_local, lead);
       tma_load_2d_pair(smem_addr(s.a[stage]), tmA, fb, kb * BK, ya);
       tma_load_2d_pair(smem_addr(s.b[stage]), tmB, fb, kb * BK, yb);
       ++issued;
@@ -616,14 +622,15 @@ __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUten
   }
   // Both CTAs' copies complete on the leader's barriers: the leader waits
   // (bounded) for the last phases it armed before the pair may exit.
-  if (rank == 0) {
+  if (pr == 0) {
     const uint32_t first = issued > kPairStages ? issued - kPairStages : 0u;
     for (uint32_t i = first; i < issued; ++i)
       mbar_wait(smem_addr(&s.full[i % kPairStages]), (i / kPairStages) & 1u, nullptr);
   }
 }
 
-__device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p) {
+__device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t lead) {
+  const uint16_t pair_mask = static_cast<uint16_t>(0x3u << lead);
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int npairs = gridDim.x >> 1;
   constexpr uint32_t idesc = idesc_i8(kPairBM, kPairBN);
@@ -648,20 +655,20 @@ __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p) {
       for (int kk = 0; kk < BK / UMMA_K; ++kk)
         mma_i8_pair(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc,
                     (kb > kb0 || kk > 0) ? 1u : 0u);
-      mma_commit_pair(smem_addr(&s.empty[stage]), 0x3);
+      mma_commit_pair(smem_addr(&s.empty[stage]), pair_mask);
       if (++stage == kPairStages) {
         stage = 0;
         phase ^= 1u;
       }
     }
     if (!ok) break;
-    mma_commit_pair(smem_addr(&s.acc_full[abuf]), 0x3);
+    mma_commit_pair(smem_addr(&s.acc_full[abuf]), pair_mask);
     if (++abuf == 2) {
       abuf = 0;
       aphase ^= 1u;
     }
   }
-  mma_commit_pair(smem_addr(&s.drain), 0x1);
+  mma_commit_pair(smem_addr(&s.drain), static_cast<uint16_t>(1u << lead));
   mbar_wait(smem_addr(&s.drain), 0u, nullptr);
 }
 
@@ -713,20 +720,21 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
 // token scale is fetched before the accumulator is ready, and the four
 // 32-column TMEM loads are double-buffered so the next load is in flight
 // while the current chunk is converted and stored.
-__device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t rank) {
+__device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t pr,
+                              uint32_t lead) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int npairs = gridDim.x >> 1;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int quad = warp & 3;
   const int half = (warp - 2) >> 2;
-  const int region = static_cast<int>(rank) * kPairEpiWarps + (warp - 2);  // 0..15
+  const int region = static_cast<int>(pr) * kPairEpiWarps + (warp - 2);  // 0..15
   float* sws = s.sw_tile[warp - 2];
   uint32_t abuf = 0, aphase = 0;
   for (int unit = blockIdx.x >> 1; unit < nunits; unit += npairs) {
     const int tile = unit / p.splits, split = unit % p.splits;
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    const int row = tm * kPairBM + static_cast<int>(rank) * 128 + quad * 32 + lane;
+    const int row = tm * kPairBM + static_cast<int>(pr) * 128 + quad * 32 + lane;
     const bool rv = row < p.m;
     const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
     const int colbase = tn * kPairBN + half * (kPairBN / 2);
@@ -753,6 +761,21 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
         if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
         if (rv) store32_channel(p, row, colbase + (ch + 1) * 32, sa, sws + (ch + 1) * 32, vb);
         tmem_ld_wait();
+      }
+    } else if (p.csplit) {
+      // Split-K inside the cluster: stage this warp's 32 x 128 partial in its
+      // 16 KB slot of the (idle) operand ring, [column quad][lane][4]; the
+      // sum over the cluster's pairs is taken after the cluster barrier
+      // (cluster_reduce_pair).
+      uint8_t* stg = &s.a[0][0] + (warp - 2) * (32 * (kPairBN / 2) * 4);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        tmem_ld_32x32b_x32(tb + ch * 32, va);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<int4*>(stg + (((ch * 8 + q4) * 32 + lane) * 16)) =
+              make_int4(va[q4 * 4], va[q4 * 4 + 1], va[q4 * 4 + 2], va[q4 * 4 + 3]);
       }
     } else {
       // Split-K.  Every pair holds exactly one unit (the host plans at most
@@ -813,11 +836,87 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_addr(&s.acc_empty[abuf]), 0));
+    if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_addr(&s.acc_empty[abuf]), lead));
     if (++abuf == 2) {
       abuf = 0;
       aphase ^= 1u;
     }
+  }
+}
+
+// Split-K through distributed shared memory.  The cluster is the `splits`
+// CTA pairs of one tile (pair j computed K slice j); every CTA has staged
+// its 128 x 256 int32 partial in its operand ring as 8 slots of 32 rows x
+// 128 columns (slot = epilogue warp - 2, laid out [column quad][lane][4]).
+// After a cluster barrier, CTA (pair j, half h) takes the 32-column chunks
+// c = j, j + splits, ... of the tile's 256 columns: for its 128 rows it
+// sums chunk c over the `splits` CTAs of half h (plain integer adds, exact),
+// then dequantises and stores.  The two epilogue warps of a TMEM lane
+// quadrant take alternate chunks.
+// Before the cluster barrier: each epilogue warp copies the channel scales of
+// the (at most two) chunks it will reduce into its shared-memory slot.
+__device__ void cluster_reduce_scales(PairStorage& s, const Args& p, uint32_t crank) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int w2 = (warp - 2) >> 2;
+  const int j = static_cast<int>(crank >> 1);
+  const int tn = ((blockIdx.x >> 1) / p.splits) / p.tiles_m;
+  float* sws = s.sw_tile[warp - 2];
+  int t = 0;
+  for (int c = j + p.splits * w2; c < kPairBN / 32 && t < 2; c += 2 * p.splits, ++t) {
+    const int col = tn * kPairBN + c * 32 + lane;
+    sws[t * 32 + lane] = (p.out && col < p.n) ? __ldg(p.sw + col) : 0.0f;
+  }
+}
+
+__device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t crank) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int quad = warp & 3;
+  const int w2 = (warp - 2) >> 2;
+  const int j = static_cast<int>(crank >> 1), h = static_cast<int>(crank & 1u);
+  const int tile = (blockIdx.x >> 1) / p.splits;
+  const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+  const float* sws = s.sw_tile[warp - 2];
+  int t = 0;
+  const int row = tm * kPairBM + h * 128 + quad * 32 + lane;
+  const bool rv = row < p.m;
+  const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
+  const uint32_t base = smem_addr(&s.a[0][0]);
+  constexpr uint32_t kSlotBytes = 32 * (kPairBN / 2) * 4;
+  for (int c = j + p.splits * w2; c < kPairBN / 32; c += 2 * p.splits, ++t) {
+    const int hh = c >> 2, ch = c & 3;
+    const uint32_t slot = static_cast<uint32_t>(hh * 4 + ((quad + 2) & 3));  // staging warp of (quad, hh)
+    const uint32_t off = base + slot * kSlotBytes + static_cast<uint32_t>((ch * 8 * 32 + lane) * 16);
+    uint32_t va[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) va[i] = 0;
+    // all sources' loads of this chunk in flight together (splits <= 4):
+    // one round trip through the cluster per half chunk
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+      int4 t4[4][4];
+#pragma unroll
+      for (int o = 0; o < 4; ++o) {
+        const uint32_t peer = static_cast<uint32_t>(2 * o + h);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          t4[o][q] = o < p.splits ? ld_dsmem_v4(map_to_rank(off + (hq * 4 + q) * 32 * 16, peer))
+                                  : make_int4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int o = 0; o < 4; ++o)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int q4 = hq * 4 + q;
+          va[q4 * 4] += t4[o][q].x;
+          va[q4 * 4 + 1] += t4[o][q].y;
+          va[q4 * 4 + 2] += t4[o][q].z;
+          va[q4 * 4 + 3] += t4[o][q].w;
+        }
+    }
+    const int col0 = tn * kPairBN + c * 32;
+    if (rv && col0 < p.n) store32_channel(p, row, col0, sa, sws + t * 32, va);
   }
 }
 
@@ -827,7 +926,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   PairStorage& s = storage<PairStorage>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
+  const uint32_t crank = cluster_rank();
+  const uint32_t pr = crank & 1u, lead = crank & ~1u;
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
@@ -857,13 +957,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   griddep_launch_dependents();
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
-    if (lane == 0) produce_pair(s, &tmA, &tmB, p, rank);
+    if (lane == 0) produce_pair(s, &tmA, &tmB, p, pr, lead);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) mma_issue_pair(s, tmem, p);
+    if (lane == 0 && pr == 0) mma_issue_pair(s, tmem, p, lead);
     __syncwarp();
   } else {
-    epilogue_pair(s, tmem, p, rank);
+    epilogue_pair(s, tmem, p, pr, lead);
+  }
+  if (p.csplit) {
+    if (warp >= 2) cluster_reduce_scales(s, p, crank);
+    cluster_sync_all();  // every CTA of the cluster has staged its partial
+    if (warp >= 2) cluster_reduce_pair(s, p, crank);
   }
   tc_fence_before();
   __syncthreads();
@@ -954,6 +1059,35 @@ inline cudaError_t set_smem_once(K kernel, int dev, int slot, size_t bytes) {
 inline size_t channel_smem() { return sizeof(ChannelStorage) + 1024; }
 inline size_t pair_smem() { return sizeof(PairStorage) + 1024; }
 
+// Largest number of co-resident clusters of `cluster` CTAs of the pair
+// kernel (queried once per device and size; 0 when the size cannot run).
+inline int max_pair_clusters(int dev, int cluster) {
+  static int cache[64][5] = {};  // cluster 2, 4, 6, 8 (index cluster / 2)
+  const int ci = cluster / 2;
+  if (dev < 0 || dev >= 64 || ci < 1 || ci > 4 || cluster % 2) return 0;
+  if (cache[dev][ci] != 0) return cache[dev][ci] > 0 ? cache[dev][ci] : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cluster) * 16, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = pair_smem();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(gemm_i8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(pair_smem())) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, gemm_i8_pair_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache[dev][ci] = n > 0 ? n : -1;
+  return n > 0 ? n : 0;
+}
+
 // Largest number of co-resident CTA pairs (queried once per device).
 inline int max_pairs(int dev, int num_sms) {
   static int cache[64] = {0};
@@ -994,11 +1128,13 @@ constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeaderBytes / (16 * 4));
 // that about one unit lands on every pair.
 struct PairPlan {
   int tiles, splits, kb_per_split;
+  int csplit;  // 1: the splits of a tile are the pairs of one cluster (no workspace)
 };
 
-inline PairPlan pair_plan(int m, int n, int k, int pairs) {
+inline PairPlan pair_plan(int m, int n, int k, int pairs, int dev) {
   PairPlan pl;
   pl.tiles = ((m + kPairBM - 1) / kPairBM) * ((n + kPairBN - 1) / kPairBN);
+  pl.csplit = 0;
   const int num_kb = (k + BK - 1) / BK;
   int s = 1;
   if (4 * pl.tiles < 3 * pairs && pl.tiles <= kMaxSplitTiles) {
@@ -1009,11 +1145,31 @@ inline PairPlan pair_plan(int m, int n, int k, int pairs) {
   }
   pl.kb_per_split = (num_kb + s - 1) / s;
   pl.splits = (num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
+  if (pl.splits > 1) {
+    // The split-K tail through the workspace costs about 23 K-block times
+    // (measured at 256 x 4096 x 14336); summing the partials through
+    // distributed shared memory in a cluster of the tile's pairs costs about
+    // 3, but needs the clusters co-resident and allows at most 4 pairs per
+    // cluster.  Take whichever is estimated faster (ties: the workspace).
+    const double cost_ws = pl.kb_per_split + 23.0;
+    for (int cs = 4; cs >= 2; --cs) {
+      if (num_kb / cs < 8 || pl.tiles * cs > pairs) continue;
+      if (max_pair_clusters(dev, 2 * cs) < pl.tiles) continue;
+      const int kbps = (num_kb + cs - 1) / cs;
+      if ((num_kb + kbps - 1) / kbps != cs) continue;
+      if (kbps + 3.0 < cost_ws) {
+        pl.splits = cs;
+        pl.kb_per_split = kbps;
+        pl.csplit = 1;
+      }
+      break;
+    }
+  }
   return pl;
 }
 
 inline size_t pair_workspace_bytes(const PairPlan& pl) {
-  if (pl.splits <= 1) return 0;
+  if (pl.splits <= 1 || pl.csplit) return 0;
   // counters, then one int32 accumulator tile (16 regions of 32 x 128) per tile
   return kCounterHeaderBytes + static_cast<size_t>(pl.tiles) * 16 * 32 * (kPairBN / 2) * 4;
 }
@@ -1027,17 +1183,19 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
   a.num_kb = (a.k + BK - 1) / BK;
   a.groups = 0;
   const int pairs = max_pairs(dev, num_sms);
-  PairPlan pl = pair_plan(a.m, a.n, a.k, pairs);
+  PairPlan pl = pair_plan(a.m, a.n, a.k, pairs, dev);
   if (!allow_split || static_cast<int64_t>(pl.tiles) * pl.splits > pairs) {
     // (split-K stages partials in the operand ring: one unit per pair)
     pl.splits = 1;
     pl.kb_per_split = a.num_kb;
   }
+  if (pl.splits == 1) pl.csplit = 0;
   a.splits = pl.splits;
   a.kb_per_split = pl.kb_per_split;
+  a.csplit = pl.csplit;
   a.ws = nullptr;
   a.cnt = nullptr;
-  if (pl.splits > 1) {
+  if (pl.splits > 1 && !pl.csplit) {
     a.cnt = static_cast<int*>(workspace);
     a.ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kCounterHeaderBytes);
   }
@@ -1047,8 +1205,11 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
   const int grid_pairs = ntiles < pairs ? ntiles : pairs;
   cudaError_t e = set_smem_once(gemm_i8_pair_kernel, dev, 0, pair_smem());
   if (e == cudaSuccess) {
+    // cluster: one pair, or (cluster split-K) the splits pairs of one tile;
+    // the grid is then exactly tiles x splits pairs, one unit each
+    const unsigned cluster = pl.csplit ? 2u * static_cast<unsigned>(pl.splits) : 2u;
     e = launch_pdl(gemm_i8_pair_kernel, dim3(2 * grid_pairs), dim3(kPairThreads), pair_smem(), stream,
-                   2, ta, tb, a);
+                   cluster, ta, tb, a);
   }
   *err = e;
   return e == cudaSuccess ? 0 : 2;

@@ -194,7 +194,7 @@ size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
   if (check_device(&dev) != QK_OK) return 0;
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  const gemm::PairPlan pl = gemm::pair_plan(m, n, k, gemm::max_pairs(dev_id, dev->sms));
+  const gemm::PairPlan pl = gemm::pair_plan(m, n, k, gemm::max_pairs(dev_id, dev->sms), dev_id);
   return gemm::pair_workspace_bytes(pl);
 }
 
@@ -248,6 +248,7 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   g.kb_per_split = 0;
   g.ws = nullptr;
   g.cnt = nullptr;
+  g.csplit = 0;
   cudaError_t e = cudaSuccess;
   int dev_id = 0;
   cudaGetDevice(&dev_id);
