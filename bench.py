@@ -329,6 +329,18 @@ def cpu_baseline(seconds: float = 10.0) -> dict:
 
 
 # ---------------------------------------------------------------- arms
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of `value` over all ranks (every rank gets it); `dist` is
+    torch.distributed or None for a single process."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args):
     """The oracle as the reference arm (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -341,8 +353,8 @@ def run_reference(args):
 
     w = synth.make("prefill")
     O = Oracle()
-    # rows per step sized so that warmup + steps stay around two minutes
-    budget = 120.0 / max(1, args.steps + args.warmup)
+    # rows per step sized so that warmup + steps stay around --ref-seconds
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)
     rows = max(1, min(O.nthreads, 32))
     t0 = time.perf_counter()
     O.linear(np.ascontiguousarray(w.x[:rows]), w.w_q, w.sw)
@@ -441,10 +453,7 @@ def run_ours(args):
         barrier()
     total_ms = start.elapsed_time(end)
     del g_warm, g_timed
-    if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, "cuda")
     # the GEMM's and the quantiser's average launch durations: the same
     # launches, each kernel alone in a graph of K back-to-back launches
     iters = max(10, min(args.steps, 100))
@@ -506,10 +515,7 @@ def run_ours(args):
         e1.record(stream)
         barrier()
         e2e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
         e2e = {"value": world * ops_step * steps_e2e / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
                "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(ohs[0].numel() * 2),
                "ms_per_step": e2e_ms / steps_e2e, "steps": steps_e2e,
@@ -569,6 +575,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-smi", dest="smi", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="CPU time budget of the whole --impl reference run")
     ap.add_argument("--stage-iters", type=int, default=50)
     # DRAM bytes (read + write) per launch from one ncu capture of the current
     # build of each kernel; pass a new figure, or 0 for null, whenever the
