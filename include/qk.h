@@ -163,14 +163,17 @@ QK_API qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, con
  * out            optional [m, n] output in out_dtype (QK_BF16 or QK_F32);
  *                NULL to skip; 16-B aligned.  At least one of c, out non-NULL.
  * workspace      device scratch of at least qk_w8a8_gemm_workspace_size()
- *                bytes, 256-B aligned; may be NULL when that size is 0.  It
- *                is used when the output has too few tiles to occupy the GPU
- *                and K is split across CTA pairs (a 4 KB header of arrival
- *                counters, then one INT32 accumulator per output tile that
- *                the K slices add into).  It must be zero-filled before its
- *                first use; every completed call leaves it all zero again,
- *                so one workspace (sized for the largest problem) can be
- *                reused across calls and shapes.  The call
+ *                bytes, 256-B aligned; may be NULL when that size is 0.  When
+ *                the output has too few tiles to occupy the GPU, K is split
+ *                across CTA pairs; if the pairs of a tile can share a
+ *                cluster, the partial sums meet in distributed shared memory
+ *                and no workspace is needed (size 0), otherwise they meet in
+ *                the workspace (a 4 KB header of arrival counters, then one
+ *                INT32 accumulator per output tile that the K slices add
+ *                into).  It must be zero-filled before its first use; every
+ *                completed call leaves it all zero again, so one workspace
+ *                (sized for the largest problem) can be reused across calls
+ *                and shapes.  The call
  *                owns it until the work on `stream` completes: calls that
  *                may overlap need separate workspaces.  After a call that
  *                ended in QK_ERR_TIMEOUT, zero-fill it again.

@@ -114,15 +114,17 @@ __global__ void __launch_bounds__(kThreads) gemv_i8_kernel(Args p) {
 inline int max_tokens() { return 8; }
 
 // ---------------------------------------------------------------------------
-// Persistent prefetching form (the default for K <= 16384): a few CTAs per SM
-// (PrefCfg), each walking row groups g = blockIdx, blockIdx + grid, ...  A group is R
-// rows; thread t owns the 16-byte K chunks t, t + 256, ... (J of them), so its
-// activation chunks for all tokens are loaded once and stay in registers, and
-// the W chunks of the next D - 1 groups are already in flight while the
-// current group is multiplied and reduced.  (Streaming W through shared
-// memory with one-dimensional bulk copies was measured and rejected: on this
-// part its throughput grows with the copy size and stays far below the
-// register path.)
+// Persistent prefetching form (the default for K <= 16384): a few CTAs per
+// SM (PrefCfg), each walking row groups g = blockIdx, blockIdx + grid, ...
+// A group is R rows; thread t owns the 16-byte K chunks t, t + 256, ... (J of
+// them), so its activation chunks for all tokens are loaded once and stay in
+// registers.  D groups of W chunks are held in registers: as soon as a
+// group's dot products are done its registers are refilled with the group D
+// ahead, so those loads are in flight while the current group is reduced
+// (and, for D = 2, while the next one is multiplied).  (Streaming W through
+// shared memory with one-dimensional bulk copies was measured and rejected:
+// on this part its throughput grows with the copy size and stays far below
+// the register path.)
 // ---------------------------------------------------------------------------
 constexpr int kPrefThreads = 256;
 constexpr int kPrefDepth = 2;
