@@ -559,15 +559,18 @@ __global__ void __launch_bounds__(GroupCfg<WITH_C>::threads, 1)
 }
 
 // ---------------------------------------------------------------- CTA-pair kernel
-// Pair tile 256 x 256: CTA rank r of the cluster owns rows [128 r, 128 r + 128)
-// of the tile and loads them (A) plus rows [128 r, 128 r + 128) of the
-// tile's 256 B rows (the N half the MMA reads from it).  The leader's single
-// MMA thread issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32); each
-// CTA's TMEM receives its 128 rows x 256 columns.  Per SM and stage this
-// moves 32 KB for 128 x 256 x 128 MACs, two thirds of the single-CTA
-// 128 x 256 tile's 48 KB.  Both CTAs' copies complete on the leader's full
-// barrier; the leader's commits arrive on both CTAs' empty / acc_full
-// barriers; both CTAs' epilogue warps arrive on the leader's acc_empty.
+// Pair tile 256 x 256: the CTA of pair rank r (cluster rank & 1) owns rows
+// [128 r, 128 r + 128) of the tile and loads them (A) plus rows
+// [128 r, 128 r + 128) of the tile's 256 B rows (the N half the MMA reads
+// from it).  A cluster is one pair, or, for split-K through distributed
+// shared memory, the `splits` pairs of one tile; the pair's leader is the
+// even cluster rank.  The leader's single MMA thread issues
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32); each CTA's TMEM
+// receives its 128 rows x 256 columns.  Per SM and stage this moves 32 KB for
+// 128 x 256 x 128 MACs, two thirds of the single-CTA 128 x 256 tile's 48 KB.
+// Both CTAs' copies complete on the leader's full barrier; the leader's
+// commits arrive on both CTAs' empty / acc_full barriers; both CTAs'
+// epilogue warps arrive on the leader's acc_empty.
 constexpr int kPairBM = 256;
 constexpr int kPairBN = 256;
 constexpr int kPairStages = 6;
