@@ -50,7 +50,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 1
+#define QK_ABI_VERSION 2
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -189,6 +189,36 @@ QK_API qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t
  * device (0 when none; the split depends on the device's SM count).
  * Returns 0 for arguments qk_w8a8_gemm would reject. */
 QK_API size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k);
+
+/*
+ * qk_w8a8_linear -- the whole W8A8 linear layer in one call: dynamic
+ * per-token quantisation of x (as qk_quantize_per_token) into the
+ * workspace, then the INT8 GEMM and dequant epilogue (as qk_w8a8_gemm) on
+ * the same stream.  The two kernels are launched with programmatic
+ * dependent launch, so the GEMM's set-up overlaps the quantiser's tail.  The
+ * int8 values, scales and outputs are bit-identical to the two-call form.
+ * (A form with the quantiser inside every decode-GEMV CTA was built and
+ * measured slower on this part -- 15.6 us against 13.2 us at 4 x 14336 x
+ * 4096 -- because every CTA must read all of x to reduce the row maxima.)
+ *
+ * x              [m, k] activations, x_dtype QK_BF16 or QK_F32, 16-B aligned
+ * b, scale_b, group_k, output_scale   as qk_w8a8_gemm
+ * scale_a_out    optional [m] fp32: receives the per-token scales; NULL to skip
+ * out            [m, n] output in out_dtype, 16-B aligned (required)
+ * workspace      qk_w8a8_linear_workspace_size() bytes, 256-B aligned: the
+ *                GEMM's workspace (which must be zero-filled before its
+ *                first use and is left zero by every call), then q and the
+ *                scales.  Calls that may overlap need separate workspaces.
+ * Errors: those of qk_quantize_per_token and qk_w8a8_gemm.
+ */
+QK_API qk_status qk_w8a8_linear(int m, int n, int k, const void* x, qk_dtype x_dtype,
+                                const int8_t* b, const float* scale_b, int group_k,
+                                float output_scale, float* scale_a_out, void* out,
+                                qk_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                qk_stream stream);
+
+/* Bytes of workspace qk_w8a8_linear needs (0 for arguments it would reject). */
+QK_API size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k);
 
 /*
  * qk_w8a8_gemm_noalloc -- qk_w8a8_gemm without a caller-provided workspace.

@@ -735,7 +735,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
   float* sws = s.sw_tile[warp - 2];
   uint32_t abuf = 0, aphase = 0;
   for (int unit = blockIdx.x >> 1; unit < nunits; unit += npairs) {
-    const int tile = unit / p.splits, split = unit % p.splits;
+    const int tile = unit / p.splits;
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
     const int row = tm * kPairBM + static_cast<int>(pr) * 128 + quad * 32 + lane;
     const bool rv = row < p.m;

@@ -171,15 +171,8 @@ __global__ void __launch_bounds__(kPrefThreads, PrefCfg<MT, J>::minb)
   griddep_wait();  // the previous kernel in the stream is done with our buffers
   griddep_launch_dependents();
 
-  uint4 av[MT][J];
-#pragma unroll
-  for (int t = 0; t < MT; ++t)
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int kc = tid + j * kPrefThreads;
-      av[t][j] = (t < p.m && kc < cpr) ? ld_nc_v4(p.a + static_cast<int64_t>(t) * p.k + kc * 16)
-                                       : make_uint4(0, 0, 0, 0);
-    }
+  // the first groups of the weight stream are requested before the
+  // activations are read, so DRAM starts at once
   uint4 buf[D][R][J];
   auto fetch = [&](uint4 (&b)[R][J], int g) {
 #pragma unroll
@@ -195,6 +188,16 @@ __global__ void __launch_bounds__(kPrefThreads, PrefCfg<MT, J>::minb)
   };
 #pragma unroll
   for (int d = 0; d < D; ++d) fetch(buf[d], blockIdx.x + d * gridDim.x);
+  uint4 av[MT][J];
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int kc = tid + j * kPrefThreads;
+      av[t][j] = (t < p.m && kc < cpr) ? ld_nc_v4(p.a + static_cast<int64_t>(t) * p.k + kc * 16)
+                                       : make_uint4(0, 0, 0, 0);
+    }
+
   const int my_r = tid / MT, my_t = tid % MT;  // output owned by thread tid < R * MT
   const float my_sa = (tid < R * MT && my_t < p.m && p.out) ? __ldg(p.sa + my_t) : 0.0f;
   int slot = 0;
@@ -257,15 +260,19 @@ inline cudaError_t launch_pref_mt(const Args& a, int num_sms, cudaStream_t strea
                       a);
   };
   switch (J) {
-    case 1: return go(gemv_i8_prefetch_kernel<MT, 1>, PrefCfg<MT, 1>::rows, PrefCfg<MT, 1>::minb);
-    case 2: return go(gemv_i8_prefetch_kernel<MT, 2>, PrefCfg<MT, 2>::rows, PrefCfg<MT, 2>::minb);
+    case 1:
+      return go(gemv_i8_prefetch_kernel<MT, 1>, PrefCfg<MT, 1>::rows, PrefCfg<MT, 1>::minb);
+    case 2:
+      return go(gemv_i8_prefetch_kernel<MT, 2>, PrefCfg<MT, 2>::rows, PrefCfg<MT, 2>::minb);
     case 3:
       if constexpr (MT <= 4)
-        return go(gemv_i8_prefetch_kernel<MT, 3>, PrefCfg<MT, 3>::rows, PrefCfg<MT, 3>::minb);
+        return go(gemv_i8_prefetch_kernel<MT, 3>, PrefCfg<MT, 3>::rows,
+                  PrefCfg<MT, 3>::minb);
       break;
     default:
       if constexpr (MT <= 4)
-        return go(gemv_i8_prefetch_kernel<MT, 4>, PrefCfg<MT, 4>::rows, PrefCfg<MT, 4>::minb);
+        return go(gemv_i8_prefetch_kernel<MT, 4>, PrefCfg<MT, 4>::rows,
+                  PrefCfg<MT, 4>::minb);
       break;
   }
   return cudaErrorInvalidValue;  // (pref_supported rules these shapes out)

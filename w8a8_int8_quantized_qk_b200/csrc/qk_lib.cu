@@ -220,7 +220,7 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const GemmPath path = gemm_path(m, group_k);
   if (path == GemmPath::kGemv) {
-    gemv::Args g;
+    gemv::Args g = {};
     g.m = m;
     g.n = n;
     g.k = k;
@@ -260,6 +260,54 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   }
   if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
   return r == 0 ? QK_OK : cuda_status(e, "gemm launch");
+}
+
+// The linear layer's workspace: the GEMM's own (offset 0, so its
+// zero-on-return contract covers it), then q [m, k] int8, then the scales.
+namespace {
+inline size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+}  // namespace
+
+size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k) {
+  if (gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return 0;
+  const size_t g = round256(qk_w8a8_gemm_workspace_size(m, n, k, group_k));
+  return g + round256(static_cast<size_t>(m) * static_cast<size_t>(k)) +
+         round256(static_cast<size_t>(m) * 4);
+}
+
+qk_status qk_w8a8_linear(int m, int n, int k, const void* x, qk_dtype x_dtype, const int8_t* b,
+                         const float* scale_b, int group_k, float output_scale,
+                         float* scale_a_out, void* out, qk_dtype out_dtype, void* workspace,
+                         size_t workspace_bytes, qk_stream stream) {
+  qk_status st = gemm_check(m, n, k, group_k);
+  if (st != QK_OK) return st;
+  if (x_dtype != QK_F32 && x_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (out_dtype != QK_F32 && out_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return QK_OK;
+  if (x == nullptr || b == nullptr || scale_b == nullptr || out == nullptr)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(b, 16) || !aligned(scale_b, 16) || !aligned(out, 16) ||
+      !aligned(scale_a_out, 4))
+    return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  st = check_device(&dev);
+  if (st != QK_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t need = qk_w8a8_linear_workspace_size(m, n, k, group_k);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
+    return QK_ERR_WORKSPACE;
+  const size_t g_bytes = round256(qk_w8a8_gemm_workspace_size(m, n, k, group_k));
+  int8_t* q = reinterpret_cast<int8_t*>(static_cast<char*>(workspace) + g_bytes);
+  float* sa = reinterpret_cast<float*>(static_cast<char*>(workspace) + g_bytes +
+                                       round256(static_cast<size_t>(m) * static_cast<size_t>(k)));
+  st = quant_common(m, k, x, nullptr, k, x_dtype, q, sa, stream, false);
+  if (st != QK_OK) return st;
+  st = qk_w8a8_gemm(m, n, k, q, b, sa, scale_b, group_k, output_scale, nullptr, out, out_dtype,
+                    g_bytes > 0 ? workspace : nullptr, g_bytes, stream);
+  if (st != QK_OK || scale_a_out == nullptr) return st;
+  return cuda_status(cudaMemcpyAsync(scale_a_out, sa, static_cast<size_t>(m) * 4,
+                                     cudaMemcpyDeviceToDevice, s),
+                     "scale copy");
 }
 
 qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_t* b,

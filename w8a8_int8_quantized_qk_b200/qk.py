@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -48,6 +48,10 @@ _SIGNATURES = {
     "qk_w8a8_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
                                     ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "qk_w8a8_gemm_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "qk_w8a8_linear": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P,
+                                      ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t,
+                                      _P]),
+    "qk_w8a8_linear_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "qk_w8a8_gemm_noalloc": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
                                             ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P]),
     "qk_device_status": (ctypes.c_int, [_P]),
@@ -112,6 +116,18 @@ def qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
 
 def qk_w8a8_gemm_workspace_size(m, n, k, group_k) -> int:
     return lib().qk_w8a8_gemm_workspace_size(m, n, k, group_k)
+
+
+def qk_w8a8_linear(m, n, k, x, x_dtype, b, scale_b, group_k, output_scale, scale_a_out, out, out_dtype,
+                   workspace, workspace_bytes, stream) -> int:
+    """The whole layer (quantise + GEMM + epilogue) with q and the scales in
+    the workspace (see include/qk.h)."""
+    return lib().qk_w8a8_linear(m, n, k, x, x_dtype, b, scale_b, group_k, output_scale, scale_a_out, out,
+                                out_dtype, workspace, workspace_bytes, stream)
+
+
+def qk_w8a8_linear_workspace_size(m, n, k, group_k) -> int:
+    return lib().qk_w8a8_linear_workspace_size(m, n, k, group_k)
 
 
 def qk_w8a8_gemm_noalloc(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
@@ -242,8 +258,33 @@ def cached_workspace(nbytes: int, device):
     return ws
 
 
+def w8a8_linear(x, w_q, sw, group_k: int = 0, output_scale: float = 1.0, out_dtype=None,
+                want_scale: bool = False, workspace=None, stream=None):
+    """qk_w8a8_linear: x [m, k] bf16/fp32 -> (out [m, n], per-token scales [m] or None).
+    `workspace` (or a fresh zero-filled one) holds q and the scales between
+    the two kernels."""
+    torch = _torch()
+    _need_cuda(x, w_q, sw)
+    assert x.dim() == 2 and x.is_contiguous()
+    m, k = x.shape
+    n = w_q.shape[0]
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = torch.empty((m, n), dtype=out_dtype, device=x.device)
+    sa = torch.empty((m,), dtype=torch.float32, device=x.device) if want_scale else None
+    need = qk_w8a8_linear_workspace_size(m, n, k, group_k)
+    if need and workspace is None:
+        workspace = torch.zeros((need,), dtype=torch.uint8, device=x.device)
+    _check(qk_w8a8_linear(m, n, k, _ptr(x), _dtype_code(x), _ptr(w_q), _ptr(sw), group_k,
+                          float(output_scale), _ptr(sa), _ptr(out), _dtype_code(out), _ptr(workspace),
+                          0 if workspace is None else workspace.numel(), _stream(stream)),
+           "qk_w8a8_linear")
+    return out, sa
+
+
 def linear(x, w_q, sw, group_k: int = 0, output_scale: float = 1.0, out_dtype=None, stream=None):
-    """The whole W8A8 linear layer: quantise x per token, INT8 GEMM, dequant."""
+    """The whole W8A8 linear layer: quantise x per token, INT8 GEMM, dequant
+    (q and the scales in torch allocations, so concurrent calls on different
+    streams do not share buffers)."""
     q, sa = quantize_per_token(x, stream=stream)
     out, _ = w8a8_gemm(q, w_q, sa, sw, group_k, output_scale, out_dtype, stream=stream)
     return out
