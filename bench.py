@@ -228,6 +228,19 @@ def _bytes(w) -> dict:
     return {"quant": qb, "gemm": gb}
 
 
+def _upload_graph(g, stream) -> None:
+    """Upload an instantiated CUDA graph to the device (cuGraphUpload), so
+    the first replay inside a timed region does not also pay for it."""
+    import ctypes
+
+    cu = ctypes.CDLL("libcuda.so.1")
+    cu.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    rc = cu.cuGraphUpload(ctypes.c_void_p(int(g.raw_cuda_graph_exec())),
+                          ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"cuGraphUpload failed: {rc}")
+
+
 def _graph_us(torch, L, body, iters: int, reps: int = 3) -> float:
     """Average device time of one iteration of `body(i)`: `iters` iterations
     are captured into one CUDA graph (so host-side launch cost cannot leave
@@ -414,7 +427,8 @@ def run_ours(args):
     # ---- headline: prefill step (quantise + GEMM), device-resident inputs.
     # The W warm-up steps and the K timed steps are each captured into one
     # CUDA graph (rotating copies, so every step reads fresh operands from
-    # HBM); the timed graph is replayed once between CUDA events.
+    # HBM); both graphs are uploaded to the device first, and the timed graph
+    # is replayed once between CUDA events.
     import ctypes
 
     w = synth.make("prefill")
@@ -439,6 +453,8 @@ def run_ours(args):
 
     g_warm = capture(0, args.warmup)
     g_timed = capture(args.warmup, args.steps)
+    _upload_graph(g_warm, stream)
+    _upload_graph(g_timed, stream)
     g_warm.replay()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)

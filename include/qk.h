@@ -170,10 +170,17 @@ QK_API qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, con
  *                and no workspace is needed (size 0), otherwise they meet in
  *                the workspace (a 4 KB header of arrival counters, then one
  *                INT32 accumulator per output tile that the K slices add
- *                into).  It must be zero-filled before its first use; every
- *                completed call leaves it all zero again, so one workspace
- *                (sized for the largest problem) can be reused across calls
- *                and shapes.  The call
+ *                into).  When there are more tiles than CTA pairs but not a
+ *                whole number of waves, the tiles of the last partial wave
+ *                are cut into 2 to 4 K slices that run first; every slice
+ *                stores its INT32 partial in the workspace and the last to
+ *                finish adds them up (the same 4 KB header, 16 MB left for
+ *                the split-K accumulators, then 256 KB per partial).  It
+ *                must be zero-filled before its first use; every completed
+ *                call leaves the header and the split-K accumulators zero
+ *                again (the partials past them need no initialisation), so
+ *                one workspace (sized for the largest problem) can be
+ *                reused across calls and shapes.  The call
  *                owns it until the work on `stream` completes: calls that
  *                may overlap need separate workspaces.  After a call that
  *                ended in QK_ERR_TIMEOUT, zero-fill it again.
@@ -238,19 +245,20 @@ QK_API size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k);
  * - The first call on a device looks up the scratch array's device address
  *   (once per device, with that device current); make that first call before
  *   any stream capture on the device.
- * - Each call clears the part of the scratch array it uses (counters and
- *   accumulators) on `stream` before its kernel, so it does not depend on
- *   what an earlier call left there.
+ * - Each call clears the part of the scratch array that must start at zero
+ *   (counters and split-K accumulators) on `stream` before its kernel, so it
+ *   does not depend on what an earlier call left there.
  * - Every call shares the one array: calls that can overlap on the GPU (on
  *   different streams, or from different threads) race and give wrong
  *   results.  Serialise them.
- * - QK_NOALLOC_SCRATCH_BYTES covers every split-K problem (split-K runs
- *   with fewer than 64 output tiles, 4 KB + 256 KB per tile); a problem
+ * - QK_NOALLOC_SCRATCH_BYTES covers every split-K problem (a 4 KB header,
+ *   at most 64 split-K accumulator tiles and 128 tail-split partial tiles,
+ *   each 256 KB); a problem
  *   whose qk_w8a8_gemm_workspace_size exceeded it would be rejected with
  *   QK_ERR_WORKSPACE and nothing launched.  Other errors are those of
  *   qk_w8a8_gemm.
  */
-#define QK_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u + 4096u)
+#define QK_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u + 4096u)
 
 QK_API qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_t* b,
                                       const float* scale_a, const float* scale_b, int group_k,

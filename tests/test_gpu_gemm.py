@@ -96,6 +96,23 @@ def test_gemm_split_k(O, m, n, k):
         assert_bits(out, ref["out_bf16"], "bf16 out")
 
 
+# more output tiles than CTA pairs, not a whole number of waves: the tiles of
+# the last partial wave are cut into K slices that run first, and their
+# partials meet in the workspace (2, 3 and 4 slices; ragged M, N and K)
+TAIL_SHAPES = [(2304, 2304, 2048), (2500, 2056, 3008), (2560, 2048, 4096), (1280, 4096, 8192)]
+
+
+@pytest.mark.parametrize("m,n,k", TAIL_SHAPES)
+def test_gemm_tail_split(O, m, n, k):
+    assert qk.qk_w8a8_gemm_workspace_size(m, n, k, 0) > 0  # the tail split is planned
+    a, w, sa, sw = _problem(m, n, k, 0, seed=m + 5 * n + k)
+    ref = O.linear_from_q(a, sa, w, sw, 0, 0.5)
+    for _ in range(2):  # the workspace must be back at zero after each call
+        out, c = _run(a, w, sa, sw, 0, 0.5)
+        assert_bits(c, ref["acc"], "acc")
+        assert_bits(out, ref["out_bf16"], "bf16 out")
+
+
 def test_gemm_split_k_needs_workspace(O):
     m, n, k = 256, 1024, 14336
     need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 0)

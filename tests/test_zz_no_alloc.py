@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024 + 4096  # QK_NOALLOC_SCRATCH_BYTES in include/qk.h
+NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024 + 4096  # QK_NOALLOC_SCRATCH_BYTES in include/qk.h
 
 
 def _inputs(m, n, k, seed):
@@ -53,11 +53,12 @@ def _call_regular(m, n, k, a, w, sa, sw, alpha):
     return host(out), host(c)
 
 
-@pytest.mark.parametrize("m,n,k", [(256, 1024, 14336), (256, 8960, 4096)])
+@pytest.mark.parametrize("m,n,k", [(256, 1024, 14336), (256, 8960, 4096), (2304, 2304, 2048),
+                                   (4096, 4096, 4096)])
 def test_noalloc_matches_regular_entry_point(m, n, k):
     need_gpu()
     need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 0)
-    assert 0 < need <= NOALLOC_SCRATCH_BYTES  # the split-K path, within the built-in scratch
+    assert 0 < need <= NOALLOC_SCRATCH_BYTES  # split-K or tail split, within the built-in scratch
     a_h, w_h, sa_h, sw_h = _inputs(m, n, k, seed=m + n + k)
     a, w, sa, sw = dev(a_h), dev(w_h), dev(sa_h), dev(sw_h)
     ref_out, ref_c = _call_regular(m, n, k, a, w, sa, sw, 0.5)
@@ -79,6 +80,8 @@ def test_noalloc_without_split_k_and_scratch_bound():
     ref_out, ref_c = _call_regular(m, n, k, a, w, sa, sw, 1.0)
     assert np.array_equal(c, ref_c) and np.array_equal(out, ref_out)
     # every split-K problem fits the built-in scratch: split-K runs only with
-    # fewer than 64 output tiles and needs 4 KB + 256 KB per tile
-    for m, n, k in [(200, 256, 131072), (256, 4096, 14336), (1024, 3072, 8192), (2000, 1800, 4096)]:
+    # fewer than 64 output tiles (4 KB + 256 KB per tile), and the tail split
+    # keeps at most 128 partial tiles of 256 KB past 4 KB + 16 MB
+    for m, n, k in [(200, 256, 131072), (256, 4096, 14336), (1024, 3072, 8192), (2000, 1800, 4096),
+                    (4096, 4096, 4096), (4096, 14336, 4096), (2560, 2048, 4096), (9000, 2304, 8192)]:
         assert qk.qk_w8a8_gemm_workspace_size(m, n, k, 0) <= NOALLOC_SCRATCH_BYTES

@@ -61,6 +61,15 @@ struct Args {
   // one cluster and are summed through distributed shared memory (no
   // workspace); 0 for the workspace form above
   int csplit;
+  // pair kernel, tail split (tail_splits > 1, splits == 1): tiles
+  // [0, dp_tiles) are computed whole; each remaining tile is cut into
+  // `tail_splits` K slices of `tail_kbps` K blocks, and those slices are the
+  // first unit of pairs 0 .. (tiles - dp_tiles) * tail_splits - 1.  Every
+  // slice stores its partial in `tail_ws` and then counts itself in `cnt`;
+  // the slice that arrives last adds the others' partials to its own, runs
+  // the epilogue and leaves the counter zero (the partials are scratch).
+  int dp_tiles, tail_splits, tail_kbps;
+  int32_t* tail_ws;
 };
 
 template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
@@ -591,22 +600,59 @@ struct alignas(1024) PairStorage {
   int abort;
 };
 
+// One unit of a pair's work: K blocks [kb0, kb1) of output tile `tile`;
+// slice is the K slice index (0 for a whole tile).
+struct PairUnit {
+  int tile, kb0, kb1, slice;
+};
+
+// The i-th unit of pair `pi` (false past its last).  Without the tail split,
+// units pi, pi + npairs, ... of the tiles x splits list; with it, the pair's
+// tail slice first (if it has one), then data-parallel tiles pi,
+// pi + npairs, ... below dp_tiles.
+__device__ __forceinline__ bool pair_unit(const Args& p, int pi, int npairs, int i, PairUnit& u) {
+  if (p.tail_splits > 1) {
+    const int tail_units = (p.tiles_m * p.tiles_n - p.dp_tiles) * p.tail_splits;
+    if (pi < tail_units) {
+      if (i == 0) {
+        u.tile = p.dp_tiles + pi / p.tail_splits;
+        u.slice = pi % p.tail_splits;
+        u.kb0 = u.slice * p.tail_kbps;
+        u.kb1 = min(p.num_kb, u.kb0 + p.tail_kbps);
+        return true;
+      }
+      --i;
+    }
+    const int t = pi + i * npairs;
+    if (t >= p.dp_tiles) return false;
+    u.tile = t;
+    u.slice = 0;
+    u.kb0 = 0;
+    u.kb1 = p.num_kb;
+    return true;
+  }
+  const int unit = pi + i * npairs;
+  if (unit >= p.tiles_m * p.tiles_n * p.splits) return false;
+  u.tile = unit / p.splits;
+  u.slice = unit % p.splits;
+  u.kb0 = u.slice * p.kb_per_split;
+  u.kb1 = min(p.num_kb, u.kb0 + p.kb_per_split);
+  return true;
+}
+
 // pr: this CTA's rank within its pair; lead: the cluster rank of its pair's
 // leader (clusters hold one pair, or the `splits` pairs of one tile).
 __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUtensorMap* tmB,
                              const Args& p, uint32_t pr, uint32_t lead) {
-  const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int npairs = gridDim.x >> 1;
   uint32_t stage = 0, phase = 0, issued = 0;
   bool ok = true;
-  for (int unit = blockIdx.x >> 1; ok && unit < nunits; unit += npairs) {
-    const int tile = unit / p.splits, split = unit % p.splits;
-    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+  PairUnit u;
+  for (int i = 0; ok && pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
+    const int tm = u.tile % p.tiles_m, tn = u.tile / p.tiles_m;
     const int ya = tm * kPairBM + static_cast<int>(pr) * 128;
     const int yb = tn * kPairBN + static_cast<int>(pr) * 128;
-    const int kb0 = split * p.kb_per_split;
-    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
-    for (int kb = kb0; kb < kb1; ++kb) {
+    for (int kb = u.kb0; kb < u.kb1; ++kb) {
       if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, &s.abort)) {
         ok = false;
         break;
@@ -634,15 +680,13 @@ __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUten
 
 __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t lead) {
   const uint16_t pair_mask = static_cast<uint16_t>(0x3u << lead);
-  const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int npairs = gridDim.x >> 1;
   constexpr uint32_t idesc = idesc_i8(kPairBM, kPairBN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
-  for (int unit = blockIdx.x >> 1; ok && unit < nunits; unit += npairs) {
-    const int split = unit % p.splits;
-    const int kb0 = split * p.kb_per_split;
-    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+  PairUnit u;
+  for (int i = 0; ok && pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
+    const int kb0 = u.kb0, kb1 = u.kb1;
     if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) break;
     tc_fence_after();
     const uint32_t d = tmem + abuf * kPairBN;
@@ -717,6 +761,69 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
   }
 }
 
+// Tail split, one epilogue warp's 32 x 128 region (TMEM columns from tb) of
+// K slice `u.slice` of tile `u.tile`.  Partial slots in `tail_ws` are
+// [tail tile][slice][region][column quad][lane][4] int32, so each group of
+// 32 lanes moves 512 contiguous bytes.  Every slice stores its partial and
+// then takes a ticket on the region's counter (release); the slice whose
+// ticket is the last one knows the others' partials are complete (acquire),
+// adds them to its own accumulator, still in TMEM (integer adds, exact in
+// any order), runs the per-channel epilogue and resets the counter.  No
+// slice waits for another.
+__device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region, uint32_t tb,
+                                    int row, bool rv, float sa, int colbase, const float* sws) {
+  constexpr int kRegionInts = 32 * (kPairBN / 2);
+  const int lane = threadIdx.x & 31;
+  const int S = p.tail_splits;
+  const int tt = u.tile - p.dp_tiles;
+  int* cnt = p.cnt + tt * 16 + region;
+  int32_t* slots = p.tail_ws + static_cast<int64_t>(tt) * S * 16 * kRegionInts;
+  uint32_t va[32];
+  {
+    int4* dst = reinterpret_cast<int4*>(slots + (static_cast<int64_t>(u.slice) * 16 + region) * kRegionInts);
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+      tmem_ld_32x32b_x32(tb + ch * 32, va);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4)
+        __stcg(dst + (ch * 8 + q4) * 32 + lane,
+               make_int4(va[q4 * 4], va[q4 * 4 + 1], va[q4 * 4 + 2], va[q4 * 4 + 3]));
+    }
+  }
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = atomicAdd(cnt, 1) == S - 1;
+  last = __shfl_sync(0xFFFFFFFFu, last, 0);
+  if (!last) return;
+  __threadfence();
+#pragma unroll 1
+  for (int ch = 0; ch < 4; ++ch) {
+    tmem_ld_32x32b_x32(tb + ch * 32, va);
+#pragma unroll 1
+    for (int o = 0; o < S; ++o) {
+      if (o == u.slice) continue;
+      const int4* src =
+          reinterpret_cast<const int4*>(slots + (static_cast<int64_t>(o) * 16 + region) * kRegionInts);
+      int4 t4[8];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) t4[q4] = __ldcg(src + (ch * 8 + q4) * 32 + lane);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        va[q4 * 4] += t4[q4].x;
+        va[q4 * 4 + 1] += t4[q4].y;
+        va[q4 * 4 + 2] += t4[q4].z;
+        va[q4 * 4 + 3] += t4[q4].w;
+      }
+    }
+    if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
+  }
+  __syncwarp();
+  if (lane == 0) *cnt = 0;  // ready for the next call
+}
+
 // Epilogue of the pair kernel: 8 warps per CTA; warp w (2..9) reads TMEM
 // lanes 32*(w%4) (rows) and columns [128 h, 128 h + 128), h = (w - 2) / 4.
 // The tile's channel scales are staged per warp in shared memory, the row's
@@ -725,7 +832,6 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
 // while the current chunk is converted and stored.
 __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t pr,
                               uint32_t lead) {
-  const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int npairs = gridDim.x >> 1;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -734,8 +840,10 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
   const int region = static_cast<int>(pr) * kPairEpiWarps + (warp - 2);  // 0..15
   float* sws = s.sw_tile[warp - 2];
   uint32_t abuf = 0, aphase = 0;
-  for (int unit = blockIdx.x >> 1; unit < nunits; unit += npairs) {
-    const int tile = unit / p.splits;
+  PairUnit u;
+  for (int i = 0; pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
+    const int tile = u.tile;
+    const bool tail = p.tail_splits > 1 && tile >= p.dp_tiles;
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
     const int row = tm * kPairBM + static_cast<int>(pr) * 128 + quad * 32 + lane;
     const bool rv = row < p.m;
@@ -753,7 +861,9 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
     const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * kPairBN +
                         half * (kPairBN / 2);
     uint32_t va[32], vb[32];
-    if (p.splits == 1) {
+    if (tail) {
+      tail_slice_epilogue(p, u, region, tb, row, rv, sa, colbase, sws);
+    } else if (p.splits == 1) {
       tmem_ld_32x32b_x32(tb, va);
       tmem_ld_wait();
 #pragma unroll
@@ -1125,20 +1235,52 @@ inline int max_pairs(int dev, int num_sms) {
 // zero, so one zero-filled workspace can serve problems of any shape.
 constexpr size_t kCounterHeaderBytes = 4096;
 constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeaderBytes / (16 * 4));
+constexpr size_t kTileAccBytes = static_cast<size_t>(256) * 1024;  // one 256 x 256 int32 tile
+// Tail-split partials live past the split-K accumulators (so those stay
+// zero): at most kMaxTailSlots partial tiles.
+constexpr size_t kTailOffset = kCounterHeaderBytes + kMaxSplitTiles * kTileAccBytes;
+constexpr int kMaxTailSlots = 128;
 
 // Split-K plan of the pair kernel: when the output has fewer tiles than
 // three quarters of the SM pairs, cut K into pieces (>= 8 K blocks each) so
 // that about one unit lands on every pair.
+//
+// Tail split: with more tiles than pairs, the last wave of whole tiles
+// would leave pairs idle (4096 x 4096 is 256 tiles on 74 pairs: 3 full
+// waves, then 34 tiles).  Those r = tiles mod pairs tiles are instead cut
+// into S = min(pairs / r, 4) K slices (>= 8 K blocks each) that run first,
+// on r * S pairs, while the data-parallel tiles follow: the work takes
+// about (waves + 1 / S) tile times instead of (waves + 1).
 struct PairPlan {
   int tiles, splits, kb_per_split;
   int csplit;  // 1: the splits of a tile are the pairs of one cluster (no workspace)
+  int dp_tiles, tail_splits, tail_kbps;
 };
 
 inline PairPlan pair_plan(int m, int n, int k, int pairs, int dev) {
   PairPlan pl;
   pl.tiles = ((m + kPairBM - 1) / kPairBM) * ((n + kPairBN - 1) / kPairBN);
   pl.csplit = 0;
+  pl.dp_tiles = pl.tiles;
+  pl.tail_splits = 1;
+  pl.tail_kbps = 0;
   const int num_kb = (k + BK - 1) / BK;
+  if (pl.tiles > pairs && pairs > 0) {
+    const int r = pl.tiles % pairs;
+    int ts = r > 0 ? pairs / r : 1;
+    ts = ts < 4 ? ts : 4;
+    ts = ts < num_kb / 8 ? ts : num_kb / 8;
+    while (ts > 1 && (r > kMaxSplitTiles || ts * r > kMaxTailSlots)) --ts;
+    if (ts > 1) {
+      const int kbps = (num_kb + ts - 1) / ts;
+      pl.tail_splits = (num_kb + kbps - 1) / kbps;
+      pl.tail_kbps = kbps;
+      pl.dp_tiles = pl.tiles - r;
+    }
+    pl.splits = 1;
+    pl.kb_per_split = num_kb;
+    return pl;
+  }
   int s = 1;
   if (4 * pl.tiles < 3 * pairs && pl.tiles <= kMaxSplitTiles) {
     s = pairs / pl.tiles;
@@ -1171,7 +1313,22 @@ inline PairPlan pair_plan(int m, int n, int k, int pairs, int dev) {
   return pl;
 }
 
+// Leading bytes of the workspace that must be zero before a call (and that
+// every completed call leaves zero): the counters, and the split-K
+// accumulators when the plan adds into them.
+inline size_t pair_workspace_zero_bytes(const PairPlan& pl) {
+  if (pl.tail_splits > 1) return kCounterHeaderBytes;
+  if (pl.splits <= 1 || pl.csplit) return 0;
+  return kCounterHeaderBytes + static_cast<size_t>(pl.tiles) * kTileAccBytes;
+}
+
 inline size_t pair_workspace_bytes(const PairPlan& pl) {
+  if (pl.tail_splits > 1) {
+    // counters, the (unused) split-K accumulators, then every slice's
+    // partial of every tail tile
+    return kTailOffset +
+           static_cast<size_t>(pl.tiles - pl.dp_tiles) * pl.tail_splits * kTileAccBytes;
+  }
   if (pl.splits <= 1 || pl.csplit) return 0;
   // counters, then one int32 accumulator tile (16 regions of 32 x 128) per tile
   return kCounterHeaderBytes + static_cast<size_t>(pl.tiles) * 16 * 32 * (kPairBN / 2) * 4;
@@ -1192,19 +1349,28 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
     pl.splits = 1;
     pl.kb_per_split = a.num_kb;
   }
+  if (!allow_split) {
+    pl.tail_splits = 1;
+    pl.dp_tiles = pl.tiles;
+  }
   if (pl.splits == 1) pl.csplit = 0;
   a.splits = pl.splits;
   a.kb_per_split = pl.kb_per_split;
   a.csplit = pl.csplit;
+  a.dp_tiles = pl.dp_tiles;
+  a.tail_splits = pl.tail_splits;
+  a.tail_kbps = pl.tail_kbps;
   a.ws = nullptr;
   a.cnt = nullptr;
-  if (pl.splits > 1 && !pl.csplit) {
+  a.tail_ws = nullptr;
+  if ((pl.splits > 1 && !pl.csplit) || pl.tail_splits > 1) {
     a.cnt = static_cast<int*>(workspace);
     a.ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kCounterHeaderBytes);
+    a.tail_ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kTailOffset);
   }
   CUtensorMap ta, tb;
   if (!cached_tmap(&ta, A, a.m, a.k, 128) || !cached_tmap(&tb, B, a.n, a.k, 128)) return 1;
-  const int ntiles = a.tiles_m * a.tiles_n * a.splits;
+  const int ntiles = a.tiles_m * a.tiles_n * a.splits;  // > pairs whenever the tail split is on
   const int grid_pairs = ntiles < pairs ? ntiles : pairs;
   cudaError_t e = set_smem_once(gemm_i8_pair_kernel, dev, 0, pair_smem());
   if (e == cudaSuccess) {

@@ -187,15 +187,24 @@ qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, const void
   return quant_common(m, k, gate, up, ld_in, in_dtype, q, scale, stream, true);
 }
 
-size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
-  if (gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return 0;
-  if (gemm_path(m, group_k) != GemmPath::kTensorPair) return 0;
+namespace {
+// The pair kernel's plan for this problem on the current device; false when
+// the problem takes no workspace (another kernel, or bad arguments).
+bool pair_plan_for(int m, int n, int k, int group_k, gemm::PairPlan* pl) {
+  if (gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return false;
+  if (gemm_path(m, group_k) != GemmPath::kTensorPair) return false;
   const DeviceInfo* dev = nullptr;
-  if (check_device(&dev) != QK_OK) return 0;
+  if (check_device(&dev) != QK_OK) return false;
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  const gemm::PairPlan pl = gemm::pair_plan(m, n, k, gemm::max_pairs(dev_id, dev->sms), dev_id);
-  return gemm::pair_workspace_bytes(pl);
+  *pl = gemm::pair_plan(m, n, k, gemm::max_pairs(dev_id, dev->sms), dev_id);
+  return true;
+}
+}  // namespace
+
+size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
+  gemm::PairPlan pl;
+  return pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_bytes(pl) : 0;
 }
 
 qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
@@ -234,7 +243,7 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
     g.out_bf16 = out_dtype == QK_BF16;
     return cuda_status(gemv::launch(g, dev->sms, s), "gemv launch");
   }
-  gemm::Args g;
+  gemm::Args g = {};
   g.m = m;
   g.n = n;
   g.k = k;
@@ -323,8 +332,11 @@ qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_
   if (need > QK_NOALLOC_SCRATCH_BYTES) return QK_ERR_WORKSPACE;
   void* scratch = noalloc_scratch();
   if (scratch == nullptr) return QK_ERR_CUDA;
-  // The arrival counters and the split-K accumulators must start at zero.
-  if (cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // The arrival counters and the split-K accumulators must start at zero
+  // (the tail split's partials need no initialisation).
+  gemm::PairPlan pl;
+  const size_t zero = pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_zero_bytes(pl) : need;
+  if (cudaMemsetAsync(scratch, 0, zero, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return QK_ERR_CUDA;
   return qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
                       scratch, QK_NOALLOC_SCRATCH_BYTES, stream);
