@@ -70,6 +70,10 @@ struct Args {
   // the epilogue and leaves the counter zero (the partials are scratch).
   int dp_tiles, tail_splits, tail_kbps;
   int32_t* tail_ws;
+  // pair kernel: 1 when bf16 `out` (and no `c`) is written by TMA bulk
+  // tensor stores from shared memory (tensor map tmO) on the whole-tile and
+  // tail paths
+  int tma_out;
 };
 
 template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
@@ -587,9 +591,14 @@ constexpr int kPairEpiWarps = 8;  // two per TMEM lane quadrant, 128 columns eac
 constexpr int kPairThreads = 64 + kPairEpiWarps * 32;
 constexpr uint32_t kPairStageBytes = 2u * 128u * BK;  // per CTA: A half + B half
 
+// bf16 output staging of one epilogue warp: a 32-row x 32-column box
+// (64 bytes a row) for one TMA store
+constexpr int kOutBoxBytes = 32 * 32 * 2;
+
 struct alignas(1024) PairStorage {
   uint8_t a[kPairStages][128 * BK];
   uint8_t b[kPairStages][128 * BK];
+  uint8_t out_stage[kPairEpiWarps][kOutBoxBytes];
   float sw_tile[kPairEpiWarps][kPairBN / 2];  // each epilogue warp's channel scales
   uint64_t full[kPairStages];
   uint64_t empty[kPairStages];
@@ -761,6 +770,43 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
   }
 }
 
+// 32 bf16 outputs of one row (columns col0 .. col0 + 31), converted exactly
+// as store32_channel does, written by the warp into its staging box (row r =
+// lane at byte 64 r; 64-byte swizzle: 16-byte chunk j of row r sits at
+// 64 r + 16 (j ^ ((r >> 1) & 3))) and stored with one TMA bulk tensor copy
+// at (col0, row0), which clips rows >= m and columns >= n.  Lane 0 issues
+// the copies; before rewriting the box it waits until the previous copy has
+// read it.  Every lane of the warp must call this.
+__device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tmO, uint8_t* box,
+                                            int row0, int col0, float sa, const float* sw,
+                                            const uint32_t (&v)[32]) {
+  if (col0 >= p.n || row0 >= p.m) return;  // the box lies wholly outside (warp-uniform)
+  const int lane = threadIdx.x & 31;
+  uint32_t w[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float2 s2 = *reinterpret_cast<const float2*>(sw + 2 * j);
+    float t0 = __int2float_rn(static_cast<int>(v[2 * j]));
+    float t1 = __int2float_rn(static_cast<int>(v[2 * j + 1]));
+    t0 = __fmul_rn(__fmul_rn(__fmul_rn(t0, sa), s2.x), p.alpha);
+    t1 = __fmul_rn(__fmul_rn(__fmul_rn(t1, sa), s2.y), p.alpha);
+    w[j] = pack_bf16x2(t0, t1);
+  }
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+  const uint32_t rowaddr = smem_addr(box) + static_cast<uint32_t>(lane) * 64u;
+  const uint32_t sx = (static_cast<uint32_t>(lane) >> 1) & 3u;
+#pragma unroll
+  for (uint32_t j = 0; j < 4; ++j)
+    st_shared_v4(rowaddr + ((j ^ sx) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmO, smem_addr(box), col0, row0);
+    bulk_commit();
+  }
+}
+
 // Tail split, one epilogue warp's 32 x 128 region (TMEM columns from tb) of
 // K slice `u.slice` of tile `u.tile`.  Partial slots in `tail_ws` are
 // [tail tile][slice][region][column quad][lane][4] int32, so each group of
@@ -771,7 +817,8 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
 // any order), runs the per-channel epilogue and resets the counter.  No
 // slice waits for another.
 __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region, uint32_t tb,
-                                    int row, bool rv, float sa, int colbase, const float* sws) {
+                                    int row, bool rv, float sa, int colbase, const float* sws,
+                                    const CUtensorMap* tmO, uint8_t* box) {
   constexpr int kRegionInts = 32 * (kPairBN / 2);
   const int lane = threadIdx.x & 31;
   const int S = p.tail_splits;
@@ -818,7 +865,10 @@ __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region
         va[q4 * 4 + 3] += t4[q4].w;
       }
     }
-    if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
+    if (p.tma_out)
+      store32_tma(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
+    else if (rv)
+      store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
   }
   __syncwarp();
   if (lane == 0) *cnt = 0;  // ready for the next call
@@ -831,7 +881,7 @@ __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region
 // 32-column TMEM loads are double-buffered so the next load is in flight
 // while the current chunk is converted and stored.
 __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t pr,
-                              uint32_t lead) {
+                              uint32_t lead, const CUtensorMap* tmO) {
   const int npairs = gridDim.x >> 1;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -839,6 +889,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
   const int half = (warp - 2) >> 2;
   const int region = static_cast<int>(pr) * kPairEpiWarps + (warp - 2);  // 0..15
   float* sws = s.sw_tile[warp - 2];
+  uint8_t* box = s.out_stage[warp - 2];
   uint32_t abuf = 0, aphase = 0;
   PairUnit u;
   for (int i = 0; pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
@@ -862,7 +913,19 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
                         half * (kPairBN / 2);
     uint32_t va[32], vb[32];
     if (tail) {
-      tail_slice_epilogue(p, u, region, tb, row, rv, sa, colbase, sws);
+      tail_slice_epilogue(p, u, region, tb, row, rv, sa, colbase, sws, tmO, box);
+    } else if (p.tma_out) {
+      tmem_ld_32x32b_x32(tb, va);
+      tmem_ld_wait();
+#pragma unroll
+      for (int ch = 0; ch < 4; ch += 2) {
+        tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
+        store32_tma(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
+        tmem_ld_wait();
+        if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
+        store32_tma(p, tmO, box, row - lane, colbase + (ch + 1) * 32, sa, sws + (ch + 1) * 32, vb);
+        tmem_ld_wait();
+      }
     } else if (p.splits == 1) {
       tmem_ld_32x32b_x32(tb, va);
       tmem_ld_wait();
@@ -955,6 +1018,8 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
       aphase ^= 1u;
     }
   }
+  if (p.tma_out && lane == 0) bulk_wait_all();  // the output stores are complete
+  __syncwarp();
 }
 
 // Split-K through distributed shared memory.  The cluster is the `splits`
@@ -1035,7 +1100,8 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
 
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const Args p) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmO, const Args p) {
   extern __shared__ uint8_t smem_raw[];
   PairStorage& s = storage<PairStorage>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1044,6 +1110,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (p.tma_out) prefetch_tmap(&tmO);
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPairStages; ++i) {
@@ -1076,7 +1143,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     if (lane == 0 && pr == 0) mma_issue_pair(s, tmem, p, lead);
     __syncwarp();
   } else {
-    epilogue_pair(s, tmem, p, pr, lead);
+    epilogue_pair(s, tmem, p, pr, lead, &tmO);
   }
   if (p.csplit) {
     if (warp >= 2) cluster_reduce_scales(s, p, crank);
@@ -1124,13 +1191,31 @@ inline bool make_tmap(CUtensorMap* map, const void* base, int rows, int k, int b
          CUDA_SUCCESS;
 }
 
-// Tensor maps depend only on (base, rows, k, box_rows): the recent ones are
-// kept so that repeated calls on the same buffers skip the driver's encoder
-// (a few microseconds of host time per map).
-inline bool cached_tmap(CUtensorMap* map, const void* base, int rows, int k, int box_rows) {
+// bf16 [rows, cols] row-major output, box = 32 columns (64 bytes) x 32 rows,
+// 64-byte swizzle (the layout store32_tma writes); stores are clipped to
+// the tensor.
+inline bool make_out_tmap(CUtensorMap* map, const void* base, int rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps depend only on (base, rows, k, box_rows, kind): the recent
+// ones are kept so that repeated calls on the same buffers skip the
+// driver's encoder (a few microseconds of host time per map).  kind 0: an
+// int8 operand (make_tmap); kind 1: a bf16 output (make_out_tmap, k =
+// columns).
+inline bool cached_tmap(CUtensorMap* map, const void* base, int rows, int k, int box_rows,
+                        int kind = 0) {
   struct Entry {
     const void* base;
-    int rows, k, box_rows;
+    int rows, k, box_rows, kind;
     CUtensorMap map;
   };
   constexpr int kEntries = 32;
@@ -1140,17 +1225,19 @@ inline bool cached_tmap(CUtensorMap* map, const void* base, int rows, int k, int
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < used; ++i) {
     const Entry& e = entries[i];
-    if (e.base == base && e.rows == rows && e.k == k && e.box_rows == box_rows) {
+    if (e.base == base && e.rows == rows && e.k == k && e.box_rows == box_rows && e.kind == kind) {
       *map = e.map;
       return true;
     }
   }
-  if (!make_tmap(map, base, rows, k, box_rows)) return false;
+  if (!(kind == 1 ? make_out_tmap(map, base, rows, k) : make_tmap(map, base, rows, k, box_rows)))
+    return false;
   Entry& e = entries[next];
   e.base = base;
   e.rows = rows;
   e.k = k;
   e.box_rows = box_rows;
+  e.kind = kind;
   e.map = *map;
   next = (next + 1) % kEntries;
   if (used < kEntries) ++used;
@@ -1368,8 +1455,15 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
     a.ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kCounterHeaderBytes);
     a.tail_ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kTailOffset);
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to;
   if (!cached_tmap(&ta, A, a.m, a.k, 128) || !cached_tmap(&tb, B, a.n, a.k, 128)) return 1;
+  // bf16 out without c, outside split-K: TMA stores from shared memory
+  a.tma_out = (a.out != nullptr && a.out_bf16 && a.c == nullptr && a.splits == 1) ? 1 : 0;
+  if (a.tma_out) {
+    if (!cached_tmap(&to, a.out, a.m, a.n, 32, 1)) return 1;
+  } else {
+    to = ta;  // unused
+  }
   const int ntiles = a.tiles_m * a.tiles_n * a.splits;  // > pairs whenever the tail split is on
   const int grid_pairs = ntiles < pairs ? ntiles : pairs;
   cudaError_t e = set_smem_once(gemm_i8_pair_kernel, dev, 0, pair_smem());
@@ -1378,7 +1472,7 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
     // the grid is then exactly tiles x splits pairs, one unit each
     const unsigned cluster = pl.csplit ? 2u * static_cast<unsigned>(pl.splits) : 2u;
     e = launch_pdl(gemm_i8_pair_kernel, dim3(2 * grid_pairs), dim3(kPairThreads), pair_smem(), stream,
-                   cluster, ta, tb, a);
+                   cluster, ta, tb, to, a);
   }
   *err = e;
   return e == cudaSuccess ? 0 : 2;
