@@ -236,32 +236,140 @@ __device__ __forceinline__ void store8_channel(const Args& p, int row, int col, 
   }
 }
 
-// Per-channel epilogue, 4 warps; warp (w % 4) owns TMEM lanes 32*(w%4) ..
+// bf16 output staging of one epilogue warp: a 32-row x 32-column box
+// (64 bytes a row) for one TMA store
+constexpr int kOutBoxBytes = 32 * 32 * 2;
+
+// 32 outputs of one row (columns col0 .. col0 + 31) from 32 accumulators;
+// channel scales come from shared memory.
+__device__ __forceinline__ void store32_channel(const Args& p, int row, int col0, float sa,
+                                                const float* sw, const uint32_t (&v)[32]) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int col = col0 + g * 8;
+    if (col >= p.n) break;
+    const int64_t o = static_cast<int64_t>(row) * p.n + col;
+    if (p.c) {
+      int4* dst = reinterpret_cast<int4*>(p.c + o);
+      dst[0] = make_int4(v[g * 8 + 0], v[g * 8 + 1], v[g * 8 + 2], v[g * 8 + 3]);
+      dst[1] = make_int4(v[g * 8 + 4], v[g * 8 + 5], v[g * 8 + 6], v[g * 8 + 7]);
+    }
+    if (p.out) {
+      const float4 s0 = *reinterpret_cast<const float4*>(sw + g * 8);
+      const float4 s1 = *reinterpret_cast<const float4*>(sw + g * 8 + 4);
+      const float s8[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      float f[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float t = __int2float_rn(static_cast<int>(v[g * 8 + j]));
+        t = __fmul_rn(t, sa);
+        t = __fmul_rn(t, s8[j]);
+        f[j] = __fmul_rn(t, p.alpha);
+      }
+      if (p.out_bf16) {
+        uint4 pk;
+        pk.x = pack_bf16x2(f[0], f[1]);
+        pk.y = pack_bf16x2(f[2], f[3]);
+        pk.z = pack_bf16x2(f[4], f[5]);
+        pk.w = pack_bf16x2(f[6], f[7]);
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o) = pk;
+      } else {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
+        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+      }
+    }
+  }
+}
+
+// 32 bf16 outputs of one row (columns col0 .. col0 + 31), converted exactly
+// as store32_channel does, written by the warp into its staging box (row r =
+// lane at byte 64 r; 64-byte swizzle: 16-byte chunk j of row r sits at
+// 64 r + 16 (j ^ ((r >> 1) & 3))) and stored with one TMA bulk tensor copy
+// at (col0, row0), which clips rows >= m and columns >= n.  Lane 0 issues
+// the copies; before rewriting the box it waits until the previous copy has
+// read it.  Every lane of the warp must call this.
+__device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tmO, uint8_t* box,
+                                            int row0, int col0, float sa, const float* sw,
+                                            const uint32_t (&v)[32]) {
+  if (col0 >= p.n || row0 >= p.m) return;  // the box lies wholly outside (warp-uniform)
+  const int lane = threadIdx.x & 31;
+  uint32_t w[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float2 s2 = *reinterpret_cast<const float2*>(sw + 2 * j);
+    float t0 = __int2float_rn(static_cast<int>(v[2 * j]));
+    float t1 = __int2float_rn(static_cast<int>(v[2 * j + 1]));
+    t0 = __fmul_rn(__fmul_rn(__fmul_rn(t0, sa), s2.x), p.alpha);
+    t1 = __fmul_rn(__fmul_rn(__fmul_rn(t1, sa), s2.y), p.alpha);
+    w[j] = pack_bf16x2(t0, t1);
+  }
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+  const uint32_t rowaddr = smem_addr(box) + static_cast<uint32_t>(lane) * 64u;
+  const uint32_t sx = (static_cast<uint32_t>(lane) >> 1) & 3u;
+#pragma unroll
+  for (uint32_t j = 0; j < 4; ++j)
+    st_shared_v4(rowaddr + ((j ^ sx) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmO, smem_addr(box), col0, row0);
+    bulk_commit();
+  }
+}
+
+// Per-channel epilogue, 4 warps; warp w owns TMEM lanes 32*(w%4) (rows)
+// and all BN columns of the tile.  Before the accumulator is ready the warp
+// stages the tile's channel scales in its shared-memory slot and fetches its
+// row's token scale; the 32-column TMEM loads are double-buffered so the
+// next load is in flight while the current chunk is converted and stored.
+// bf16 output without c leaves through TMA stores (store32_tma).
 template <int BN, int NACC, class S>
-__device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p) {
+__device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUtensorMap* tmO) {
   const int ntiles = p.tiles_m * p.tiles_n;
   const int lane = threadIdx.x & 31;
+  const int ew = (threadIdx.x >> 5) - 2;  // epilogue warp 0..3
   const int quad = (threadIdx.x >> 5) & 3;
+  float* sws = s.sw_tile[ew];
+  uint8_t* box = s.out_stage[ew];
   uint32_t abuf = 0, aphase = 0;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    const int row0 = tm * BM + quad * 32, row = row0 + lane;
+    const bool rv = row < p.m;
+    const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
+    const int colbase = tn * BN;
+    if (p.out) {
+#pragma unroll
+      for (int c4 = lane * 4; c4 < BN; c4 += 128) {  // n % 8 == 0: a group of 4 is all in or out
+        const int col = colbase + c4;
+        *reinterpret_cast<float4*>(sws + c4) =
+            col < p.n ? __ldg(reinterpret_cast<const float4*>(p.sw + col))
+                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+    }
+    __syncwarp();
     if (!warp_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) break;
     tc_fence_after();
-    const int row = tm * BM + quad * 32 + lane;
-    const bool rv = row < p.m;
-    const float sa = rv ? __ldg(p.sa + row) : 0.0f;
     const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN;
+    uint32_t va[32], vb[32];
+    auto emit = [&](int ch, const uint32_t(&v)[32]) {
+      if (p.tma_out)
+        store32_tma(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
+      else if (rv)
+        store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
+    };
+    tmem_ld_32x32b_x32(tb, va);
+    tmem_ld_wait();
 #pragma unroll 1
-    for (int ch = 0; ch < BN / 32; ++ch) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tb + ch * 32, v);
+    for (int ch = 0; ch < BN / 32; ch += 2) {
+      tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
+      emit(ch, va);
       tmem_ld_wait();
-      const int col0 = tn * BN + ch * 32;
-      if (rv) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-          if (col0 + g * 8 < p.n) store8_channel(p, row, col0 + g * 8, sa, v + g * 8);
-      }
+      if (ch + 2 < BN / 32) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
+      emit(ch + 1, vb);
+      tmem_ld_wait();
     }
     tc_fence_before();
     __syncwarp();
@@ -271,6 +379,8 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p) {
       aphase ^= 1u;
     }
   }
+  if (p.tma_out && lane == 0) bulk_wait_all();  // the output stores are complete
+  __syncwarp();
 }
 
 // Per-group epilogue.  Warp roles of the group kernel: 0 TMA producer, 1 MMA
@@ -509,17 +619,33 @@ __device__ __forceinline__ void teardown(S& s, uint32_t tmem) {
 constexpr int kChannelBN = 256;
 constexpr int kChannelStages = 4;
 constexpr int kChannelThreads = 64 + 4 * 32;
-using ChannelStorage = Storage<kChannelBN, kChannelStages, 2, 0>;
+struct alignas(1024) ChannelStorage {
+  uint8_t a[kChannelStages][BM * BK];
+  uint8_t b[kChannelStages][kChannelBN * BK];
+  uint8_t out_stage[4][kOutBoxBytes];  // each epilogue warp's TMA store box
+  float sw_tile[4][kChannelBN];        // each epilogue warp's channel scales
+  uint64_t full[kChannelStages];
+  uint64_t empty[kChannelStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t aux_full[2];  // (unused by this kernel; set up with the others)
+  uint64_t aux_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
 
 __global__ void __launch_bounds__(kChannelThreads, 1)
     gemm_i8_channel_kernel(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB, const Args p) {
+                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmO, const Args p) {
   extern __shared__ uint8_t smem_raw[];
   ChannelStorage& s = storage<ChannelStorage>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (p.tma_out) prefetch_tmap(&tmO);
   }
   setup<ChannelStorage, kChannelStages, 2, 4>(s);
   griddep_wait();  // set-up above overlapped the previous kernel
@@ -532,7 +658,7 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
     if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false>(s, tmem, p);
     __syncwarp();
   } else {
-    epilogue_channel<kChannelBN, 2>(s, tmem, p);
+    epilogue_channel<kChannelBN, 2>(s, tmem, p, &tmO);
   }
   teardown(s, tmem);
 }
@@ -590,10 +716,6 @@ constexpr int kPairStages = 6;
 constexpr int kPairEpiWarps = 8;  // two per TMEM lane quadrant, 128 columns each
 constexpr int kPairThreads = 64 + kPairEpiWarps * 32;
 constexpr uint32_t kPairStageBytes = 2u * 128u * BK;  // per CTA: A half + B half
-
-// bf16 output staging of one epilogue warp: a 32-row x 32-column box
-// (64 bytes a row) for one TMA store
-constexpr int kOutBoxBytes = 32 * 32 * 2;
 
 struct alignas(1024) PairStorage {
   uint8_t a[kPairStages][128 * BK];
@@ -726,85 +848,6 @@ __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uin
   }
   mma_commit_pair(smem_addr(&s.drain), static_cast<uint16_t>(1u << lead));
   mbar_wait(smem_addr(&s.drain), 0u, nullptr);
-}
-
-// 32 outputs of one row (columns col0 .. col0 + 31) from 32 accumulators;
-// channel scales come from shared memory.
-__device__ __forceinline__ void store32_channel(const Args& p, int row, int col0, float sa,
-                                                const float* sw, const uint32_t (&v)[32]) {
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const int col = col0 + g * 8;
-    if (col >= p.n) break;
-    const int64_t o = static_cast<int64_t>(row) * p.n + col;
-    if (p.c) {
-      int4* dst = reinterpret_cast<int4*>(p.c + o);
-      dst[0] = make_int4(v[g * 8 + 0], v[g * 8 + 1], v[g * 8 + 2], v[g * 8 + 3]);
-      dst[1] = make_int4(v[g * 8 + 4], v[g * 8 + 5], v[g * 8 + 6], v[g * 8 + 7]);
-    }
-    if (p.out) {
-      const float4 s0 = *reinterpret_cast<const float4*>(sw + g * 8);
-      const float4 s1 = *reinterpret_cast<const float4*>(sw + g * 8 + 4);
-      const float s8[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      float f[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float t = __int2float_rn(static_cast<int>(v[g * 8 + j]));
-        t = __fmul_rn(t, sa);
-        t = __fmul_rn(t, s8[j]);
-        f[j] = __fmul_rn(t, p.alpha);
-      }
-      if (p.out_bf16) {
-        uint4 pk;
-        pk.x = pack_bf16x2(f[0], f[1]);
-        pk.y = pack_bf16x2(f[2], f[3]);
-        pk.z = pack_bf16x2(f[4], f[5]);
-        pk.w = pack_bf16x2(f[6], f[7]);
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o) = pk;
-      } else {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
-        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
-        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
-      }
-    }
-  }
-}
-
-// 32 bf16 outputs of one row (columns col0 .. col0 + 31), converted exactly
-// as store32_channel does, written by the warp into its staging box (row r =
-// lane at byte 64 r; 64-byte swizzle: 16-byte chunk j of row r sits at
-// 64 r + 16 (j ^ ((r >> 1) & 3))) and stored with one TMA bulk tensor copy
-// at (col0, row0), which clips rows >= m and columns >= n.  Lane 0 issues
-// the copies; before rewriting the box it waits until the previous copy has
-// read it.  Every lane of the warp must call this.
-__device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tmO, uint8_t* box,
-                                            int row0, int col0, float sa, const float* sw,
-                                            const uint32_t (&v)[32]) {
-  if (col0 >= p.n || row0 >= p.m) return;  // the box lies wholly outside (warp-uniform)
-  const int lane = threadIdx.x & 31;
-  uint32_t w[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float2 s2 = *reinterpret_cast<const float2*>(sw + 2 * j);
-    float t0 = __int2float_rn(static_cast<int>(v[2 * j]));
-    float t1 = __int2float_rn(static_cast<int>(v[2 * j + 1]));
-    t0 = __fmul_rn(__fmul_rn(__fmul_rn(t0, sa), s2.x), p.alpha);
-    t1 = __fmul_rn(__fmul_rn(__fmul_rn(t1, sa), s2.y), p.alpha);
-    w[j] = pack_bf16x2(t0, t1);
-  }
-  if (lane == 0) bulk_wait_read_all();
-  __syncwarp();
-  const uint32_t rowaddr = smem_addr(box) + static_cast<uint32_t>(lane) * 64u;
-  const uint32_t sx = (static_cast<uint32_t>(lane) >> 1) & 3u;
-#pragma unroll
-  for (uint32_t j = 0; j < 4; ++j)
-    st_shared_v4(rowaddr + ((j ^ sx) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_2d(tmO, smem_addr(box), col0, row0);
-    bulk_commit();
-  }
 }
 
 // Tail split, one epilogue warp's 32 x 128 region (TMEM columns from tb) of
@@ -1487,8 +1530,15 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   a.tiles_n = (a.n + bn - 1) / bn;
   a.num_kb = (a.k + BK - 1) / BK;
   a.groups = group ? a.k / 128 : 0;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to;
   if (!cached_tmap(&ta, A, a.m, a.k, BM) || !cached_tmap(&tb, B, a.n, a.k, bn)) return 1;
+  // channel kernel, bf16 out without c: TMA stores from shared memory
+  a.tma_out = (!group && a.out != nullptr && a.out_bf16 && a.c == nullptr) ? 1 : 0;
+  if (a.tma_out) {
+    if (!cached_tmap(&to, a.out, a.m, a.n, 32, 1)) return 1;
+  } else {
+    to = ta;  // unused
+  }
   const int ntiles = a.tiles_m * a.tiles_n;
   const int grid = ntiles < num_sms ? ntiles : num_sms;
   cudaError_t e;
@@ -1497,7 +1547,7 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
     e = set_smem_once(gemm_i8_channel_kernel, dev, 1, smem);
     if (e == cudaSuccess) {
       e = launch_pdl(gemm_i8_channel_kernel, dim3(grid), dim3(kChannelThreads), smem, stream, 1, ta,
-                     tb, a);
+                     tb, to, a);
     }
   } else {
     const size_t smem = group_smem();
