@@ -422,17 +422,21 @@ __device__ void stage_group_scales(S& s, const Args& p) {
     for (int b = 0; b < batches; ++b) {
       if (!warp_wait(smem_addr(&s.aux_empty[buf]), phase ^ 1u, &s.abort)) return;
       float* dst = s.scales + buf * (kScaleGroups * BN);
-#pragma unroll 1
+      // all BN / 32 x kScaleGroups loads of the slice in flight together:
+      // one memory round trip per slice
+      float v[BN / 32][kScaleGroups];
+#pragma unroll
       for (int i = 0; i < BN / 32; ++i) {
         const int col = col0 + lane + 32 * i;
         const float* src = p.sw + static_cast<int64_t>(col) * p.groups + b * kScaleGroups;
-        float v[kScaleGroups];
 #pragma unroll
         for (int gg = 0; gg < kScaleGroups; ++gg)
-          v[gg] = (col < p.n && b * kScaleGroups + gg < p.groups) ? __ldg(src + gg) : 0.0f;
-#pragma unroll
-        for (int gg = 0; gg < kScaleGroups; ++gg) dst[gg * BN + lane + 32 * i] = v[gg];
+          v[i][gg] = (col < p.n && b * kScaleGroups + gg < p.groups) ? __ldg(src + gg) : 0.0f;
       }
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i)
+#pragma unroll
+        for (int gg = 0; gg < kScaleGroups; ++gg) dst[gg * BN + lane + 32 * i] = v[i][gg];
       mbar_arrive(smem_addr(&s.aux_full[buf]));  // release: this lane's stores
       if (++buf == 2) {
         buf = 0;
