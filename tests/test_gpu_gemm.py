@@ -96,6 +96,27 @@ def test_gemm_split_k(O, m, n, k):
         assert_bits(out, ref["out_bf16"], "bf16 out")
 
 
+# few 128 x 256 tiles on the 1-SM kernel (m <= 128, or m <= 256 when that
+# gives each CTA fewer K blocks than the CTA-pair plan): K is split across
+# the CTAs of a cluster and the partials meet in distributed shared memory
+CHANNEL_SPLIT_SHAPES = [(64, 4096, 4096), (100, 1032, 3008), (17, 520, 2048), (256, 4096, 14336)]
+
+
+@pytest.mark.parametrize("m,n,k", CHANNEL_SPLIT_SHAPES)
+def test_gemm_channel_cluster_split(O, m, n, k):
+    assert qk.qk_w8a8_gemm_workspace_size(m, n, k, 0) == 0  # no workspace: DSMEM
+    a, w, sa, sw = _problem(m, n, k, 0, seed=m * 3 + n + 7 * k)
+    ref = O.linear_from_q(a, sa, w, sw, 0, 0.75)
+    for _ in range(2):
+        out, c = _run(a, w, sa, sw, 0, 0.75)
+        assert_bits(c, ref["acc"], "acc")
+        assert_bits(out, ref["out_bf16"], "bf16 out")
+    out32, _ = _run(a, w, sa, sw, 0, 0.75, out_dtype=torch.float32, want_c=False)
+    assert_bits(out32, ref["out_f32"], "fp32 out")
+    out16, _ = _run(a, w, sa, sw, 0, 0.75, want_c=False)  # bf16 through TMA stores
+    assert_bits(out16, ref["out_bf16"], "bf16 out, no c")
+
+
 # more output tiles than CTA pairs, not a whole number of waves: the tiles of
 # the last partial wave are cut into K slices that run first, and their
 # partials meet in the workspace (2, 3 and 4 slices; ragged M, N and K)

@@ -109,13 +109,16 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // ---------------------------------------------------------------- producer
 template <int BN, int STAGES, class S>
 __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, const Args& p) {
-  const int ntiles = p.tiles_m * p.tiles_n;
+  const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const uint32_t bytes = static_cast<uint32_t>((BM + BN) * BK);
   uint32_t stage = 0, phase = 0, issued = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+  for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
+    const int tile = unit / p.splits;
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    for (int kb = 0; kb < p.num_kb; ++kb) {
+    const int kb0 = (unit % p.splits) * p.kb_per_split;
+    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+    for (int kb = kb0; kb < kb1; ++kb) {
       if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, &s.abort)) {
         ok = false;
         break;
@@ -143,16 +146,18 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
 // otherwise one buffer per tile.
 template <int BN, int STAGES, int NACC, bool GROUP, class S>
 __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
-  const int ntiles = p.tiles_m * p.tiles_n;
+  const int nunits = p.tiles_m * p.tiles_n * p.splits;
   constexpr uint32_t idesc = idesc_i8(BM, BN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+  for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
+    const int kb0 = (unit % p.splits) * p.kb_per_split;
+    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
     if (!GROUP) {
       if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) break;
       tc_fence_after();
     }
-    for (int kb = 0; kb < p.num_kb; ++kb) {
+    for (int kb = kb0; kb < kb1; ++kb) {
       if (GROUP) {
         if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) {
           ok = false;
@@ -170,7 +175,7 @@ __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
       const uint32_t b0 = smem_addr(s.b[stage]);
 #pragma unroll
       for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-        const uint32_t acc = GROUP ? (kk > 0) : (kb > 0 || kk > 0);
+        const uint32_t acc = GROUP ? (kk > 0) : (kb > kb0 || kk > 0);
         mma_i8(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc, acc);
       }
       mma_commit(smem_addr(&s.empty[stage]));
@@ -327,14 +332,15 @@ __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tm
 // bf16 output without c leaves through TMA stores (store32_tma).
 template <int BN, int NACC, class S>
 __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUtensorMap* tmO) {
-  const int ntiles = p.tiles_m * p.tiles_n;
+  const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int lane = threadIdx.x & 31;
   const int ew = (threadIdx.x >> 5) - 2;  // epilogue warp 0..3
   const int quad = (threadIdx.x >> 5) & 3;
   float* sws = s.sw_tile[ew];
   uint8_t* box = s.out_stage[ew];
   uint32_t abuf = 0, aphase = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+  for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
+    const int tile = unit / p.splits;
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
     const int row0 = tm * BM + quad * 32, row = row0 + lane;
     const bool rv = row < p.m;
@@ -354,6 +360,27 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
     tc_fence_after();
     const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN;
     uint32_t va[32], vb[32];
+    if (p.csplit) {
+      // Split-K inside the cluster (one unit per CTA, so the operand ring is
+      // idle once acc_full has fired): stage this warp's 32 x BN partial in
+      // its 32 KB slot of the ring, laid out [chunk][column quad][lane][4];
+      // channel_cluster_reduce sums the slots over the cluster after a
+      // cluster barrier.
+      uint8_t* stg = &s.a[0][0] + quad * (32 * BN * 4);
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        tmem_ld_32x32b_x32(tb + ch * 32, va);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<int4*>(stg + (((ch * 8 + q4) * 32 + lane) * 16)) =
+              make_int4(va[q4 * 4], va[q4 * 4 + 1], va[q4 * 4 + 2], va[q4 * 4 + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[abuf]));
+      break;  // one unit per CTA
+    }
     auto emit = [&](int ch, const uint32_t(&v)[32]) {
       if (p.tma_out)
         store32_tma(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
@@ -620,6 +647,67 @@ __device__ __forceinline__ void teardown(S& s, uint32_t tmem) {
   if ((threadIdx.x >> 5) == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Split-K of the 1-SM kernel through distributed shared memory.  The
+// cluster is the `splits` CTAs of one tile (CTA j computed K slice j, and j
+// is its cluster rank); each has staged its 128 x BN int32 partial in its
+// operand ring as four 32 KB slots, one per TMEM lane quadrant (see
+// epilogue_channel).  After a cluster barrier, CTA j takes the 32-column
+// chunks c = j, j + splits, ... of the tile; for each, epilogue warp q sums
+// the chunk's 32 rows of quadrant q over the cluster's CTAs (all sources'
+// loads in flight together; integer adds, exact), then dequantises and
+// stores.  The scales of the whole tile were staged in the warp's slot
+// before the accumulator was ready.
+template <int BN, class S>
+__device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* tmO) {
+  const int lane = threadIdx.x & 31;
+  const int ew = (threadIdx.x >> 5) - 2;
+  const int quad = (threadIdx.x >> 5) & 3;
+  const int j = static_cast<int>(cluster_rank());
+  const int tile = static_cast<int>(blockIdx.x) / p.splits;
+  const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+  const float* sws = s.sw_tile[ew];
+  uint8_t* box = s.out_stage[ew];
+  const int row0 = tm * BM + quad * 32, row = row0 + lane;
+  const bool rv = row < p.m;
+  const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
+  const uint32_t slot = smem_addr(&s.a[0][0]) + static_cast<uint32_t>(quad * (32 * BN * 4));
+  for (int c = j; c < BN / 32; c += p.splits) {
+    const int col0 = tn * BN + c * 32;
+    uint32_t va[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) va[i] = 0;
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+      int4 t4[4][4];
+#pragma unroll
+      for (int o = 0; o < 4; ++o)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          t4[o][q] = o < p.splits
+                         ? ld_dsmem_v4(map_to_rank(
+                               slot + static_cast<uint32_t>(((c * 8 + hq * 4 + q) * 32 + lane) * 16),
+                               static_cast<uint32_t>(o)))
+                         : make_int4(0, 0, 0, 0);
+#pragma unroll
+      for (int o = 0; o < 4; ++o)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int q4 = hq * 4 + q;
+          va[q4 * 4] += t4[o][q].x;
+          va[q4 * 4 + 1] += t4[o][q].y;
+          va[q4 * 4 + 2] += t4[o][q].z;
+          va[q4 * 4 + 3] += t4[o][q].w;
+        }
+    }
+    if (p.tma_out)
+      store32_tma(p, tmO, box, row0, col0, sa, sws + c * 32, va);
+    else if (rv && col0 < p.n)
+      store32_channel(p, row, col0, sa, sws + c * 32, va);
+  }
+  if (p.tma_out && lane == 0) bulk_wait_all();
+  __syncwarp();
+}
+
 constexpr int kChannelBN = 256;
 constexpr int kChannelStages = 4;
 constexpr int kChannelThreads = 64 + 4 * 32;
@@ -663,6 +751,11 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
     __syncwarp();
   } else {
     epilogue_channel<kChannelBN, 2>(s, tmem, p, &tmO);
+  }
+  if (p.csplit) {
+    cluster_sync_all();  // every CTA of the cluster has staged its partial
+    if (warp >= 2) channel_cluster_reduce<kChannelBN>(s, p, &tmO);
+    cluster_sync_all();  // the peers are done reading this CTA's slots
   }
   teardown(s, tmem);
 }
@@ -1527,6 +1620,81 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
 inline size_t group_smem() { return sizeof(GroupStorage) + 1024; }
 
 // 0 ok, 1 tensor-map failure, 2 CUDA error
+// Largest number of co-resident clusters of `cluster` CTAs of the 1-SM
+// channel kernel (queried once per device and size; 0 when it cannot run).
+inline int max_channel_clusters(int dev, int cluster) {
+  static int cache[64][5] = {};
+  if (dev < 0 || dev >= 64 || cluster < 2 || cluster > 4) return 0;
+  if (cache[dev][cluster] != 0) return cache[dev][cluster] > 0 ? cache[dev][cluster] : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cluster) * 16, 1, 1);
+  cfg.blockDim = dim3(kChannelThreads, 1, 1);
+  cfg.dynamicSmemBytes = channel_smem();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(gemm_i8_channel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(channel_smem())) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, gemm_i8_channel_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache[dev][cluster] = n > 0 ? n : -1;
+  return n > 0 ? n : 0;
+}
+
+// Split-K plan of the 1-SM channel kernel: with fewer 128 x 256 tiles than
+// half the SMs, cut K into S <= 4 slices (>= 8 K blocks each), one CTA per
+// slice, the S CTAs of a tile forming one cluster whose partials meet in
+// distributed shared memory.  S = 1 when the clusters would not all be
+// co-resident.
+struct ChannelPlan {
+  int tiles, splits, kb_per_split;
+};
+
+inline ChannelPlan channel_plan(int m, int n, int k, int num_sms, int dev) {
+  ChannelPlan pl;
+  pl.tiles = ((m + BM - 1) / BM) * ((n + kChannelBN - 1) / kChannelBN);
+  const int num_kb = (k + BK - 1) / BK;
+  int s = 1;
+  if (2 * pl.tiles <= num_sms) {
+    s = num_sms / pl.tiles;
+    s = s < 4 ? s : 4;
+    s = s < num_kb / 8 ? s : num_kb / 8;
+  }
+  while (s > 1) {
+    const int kbps = (num_kb + s - 1) / s;
+    const int ns = (num_kb + kbps - 1) / kbps;
+    if (ns > 1 && max_channel_clusters(dev, ns) >= pl.tiles) {
+      s = ns;
+      break;
+    }
+    --s;
+  }
+  if (s < 1) s = 1;
+  pl.kb_per_split = (num_kb + s - 1) / s;
+  pl.splits = (num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
+  return pl;
+}
+
+// For 128 < m <= 256 (two 128-row tiles): the 1-SM kernel with cluster
+// split-K is preferred over the CTA-pair kernel when it gives each CTA fewer
+// K blocks (mlp_down, 256 x 4096 x 14336: 32 tiles x 4 slices of 28 K
+// blocks on 128 SMs, against 16 pair tiles x 3 slices of 38 on 96 SMs).
+inline bool prefer_channel_split(int m, int n, int k, int num_sms, int dev) {
+  if (m <= BM || m > 2 * BM) return false;
+  const ChannelPlan cp = channel_plan(m, n, k, num_sms, dev);
+  if (cp.splits < 2) return false;
+  const PairPlan pp = pair_plan(m, n, k, max_pairs(dev, num_sms), dev);
+  const int pair_kb = pp.splits > 1 ? pp.kb_per_split : (k + BK - 1) / BK;
+  return cp.kb_per_split < pair_kb;
+}
+
 inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev, int num_sms,
                   cudaStream_t stream, cudaError_t* err) {
   const int bn = group ? kGroupBN : kChannelBN;
@@ -1534,6 +1702,18 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   a.tiles_n = (a.n + bn - 1) / bn;
   a.num_kb = (a.k + BK - 1) / BK;
   a.groups = group ? a.k / 128 : 0;
+  a.splits = 1;
+  a.kb_per_split = a.num_kb;
+  a.csplit = 0;
+  a.tail_splits = 1;
+  if (!group) {
+    const ChannelPlan pl = channel_plan(a.m, a.n, a.k, num_sms, dev);
+    if (pl.splits > 1) {
+      a.splits = pl.splits;
+      a.kb_per_split = pl.kb_per_split;
+      a.csplit = 1;
+    }
+  }
   CUtensorMap ta, tb, to;
   if (!cached_tmap(&ta, A, a.m, a.k, BM) || !cached_tmap(&tb, B, a.n, a.k, bn)) return 1;
   // channel kernel, bf16 out without c: TMA stores from shared memory
@@ -1544,14 +1724,15 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
     to = ta;  // unused
   }
   const int ntiles = a.tiles_m * a.tiles_n;
-  const int grid = ntiles < num_sms ? ntiles : num_sms;
+  // split-K: exactly one CTA per (tile, K slice), in clusters of `splits`
+  const int grid = a.csplit ? ntiles * a.splits : (ntiles < num_sms ? ntiles : num_sms);
   cudaError_t e;
   if (!group) {
     const size_t smem = channel_smem();
     e = set_smem_once(gemm_i8_channel_kernel, dev, 1, smem);
     if (e == cudaSuccess) {
-      e = launch_pdl(gemm_i8_channel_kernel, dim3(grid), dim3(kChannelThreads), smem, stream, 1, ta,
-                     tb, to, a);
+      e = launch_pdl(gemm_i8_channel_kernel, dim3(grid), dim3(kChannelThreads), smem, stream,
+                     a.csplit ? static_cast<unsigned>(a.splits) : 1u, ta, tb, to, a);
     }
   } else {
     const size_t smem = group_smem();

@@ -104,10 +104,17 @@ qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, 
 // Which kernel runs a GEMM of this shape.
 enum class GemmPath { kGemv, kTensorChannel, kTensorPair, kTensorGroup };
 
-GemmPath gemm_path(int m, int group_k) {
+GemmPath gemm_path(int m, int n, int k, int group_k) {
   if (group_k != 0) return GemmPath::kTensorGroup;
   if (m <= gemv::max_tokens()) return GemmPath::kGemv;
   if (m <= 128) return GemmPath::kTensorChannel;
+  if (m <= 256) {
+    const DeviceInfo* dev = nullptr;
+    int dev_id = 0;
+    if (check_device(&dev) == QK_OK && cudaGetDevice(&dev_id) == cudaSuccess &&
+        gemm::prefer_channel_split(m, n, k, dev->sms, dev_id))
+      return GemmPath::kTensorChannel;
+  }
   return GemmPath::kTensorPair;
 }
 
@@ -192,7 +199,7 @@ namespace {
 // the problem takes no workspace (another kernel, or bad arguments).
 bool pair_plan_for(int m, int n, int k, int group_k, gemm::PairPlan* pl) {
   if (gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return false;
-  if (gemm_path(m, group_k) != GemmPath::kTensorPair) return false;
+  if (gemm_path(m, n, k, group_k) != GemmPath::kTensorPair) return false;
   const DeviceInfo* dev = nullptr;
   if (check_device(&dev) != QK_OK) return false;
   int dev_id = 0;
@@ -227,7 +234,7 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   st = check_device(&dev);
   if (st != QK_OK) return st;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const GemmPath path = gemm_path(m, group_k);
+  const GemmPath path = gemm_path(m, n, k, group_k);
   if (path == GemmPath::kGemv) {
     gemv::Args g = {};
     g.m = m;
