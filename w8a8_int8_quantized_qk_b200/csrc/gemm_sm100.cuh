@@ -676,35 +676,37 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
     uint32_t va[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) va[i] = 0;
+    // every source's part of the chunk requested at once (32 loads in
+    // flight per lane: one cluster round trip per chunk)
+    int4 t4[4][8];
 #pragma unroll
-    for (int hq = 0; hq < 2; ++hq) {
-      int4 t4[4][4];
+    for (int o = 0; o < 4; ++o)
 #pragma unroll
-      for (int o = 0; o < 4; ++o)
+      for (int q4 = 0; q4 < 8; ++q4)
+        t4[o][q4] = o < p.splits
+                        ? ld_dsmem_v4(map_to_rank(
+                              slot + static_cast<uint32_t>(((c * 8 + q4) * 32 + lane) * 16),
+                              static_cast<uint32_t>(o)))
+                        : make_int4(0, 0, 0, 0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          t4[o][q] = o < p.splits
-                         ? ld_dsmem_v4(map_to_rank(
-                               slot + static_cast<uint32_t>(((c * 8 + hq * 4 + q) * 32 + lane) * 16),
-                               static_cast<uint32_t>(o)))
-                         : make_int4(0, 0, 0, 0);
+    for (int o = 0; o < 4; ++o)
 #pragma unroll
-      for (int o = 0; o < 4; ++o)
+      for (int q4 = 0; q4 < 8; ++q4) order_after_loads(t4[o][q4]);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int q4 = hq * 4 + q;
-          va[q4 * 4] += t4[o][q].x;
-          va[q4 * 4 + 1] += t4[o][q].y;
-          va[q4 * 4 + 2] += t4[o][q].z;
-          va[q4 * 4 + 3] += t4[o][q].w;
-        }
-    }
+    for (int o = 0; o < 4; ++o)
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        va[q4 * 4] += t4[o][q4].x;
+        va[q4 * 4 + 1] += t4[o][q4].y;
+        va[q4 * 4 + 2] += t4[o][q4].z;
+        va[q4 * 4 + 3] += t4[o][q4].w;
+      }
     if (p.tma_out)
       store32_tma(p, tmO, box, row0, col0, sa, sws + c * 32, va);
     else if (rv && col0 < p.n)
       store32_channel(p, row, col0, sa, sws + c * 32, va);
   }
-  if (p.tma_out && lane == 0) bulk_wait_all();
+  if (p.tma_out && lane == 0) bulk_wait_all();  // the output stores are complete
   __syncwarp();
 }
 
@@ -1210,29 +1212,29 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
 #pragma unroll
     for (int i = 0; i < 32; ++i) va[i] = 0;
     // all sources' loads of this chunk in flight together (splits <= 4):
-    // one round trip through the cluster per half chunk
+    // one round trip through the cluster per chunk
+    int4 t4[4][8];
 #pragma unroll
-    for (int hq = 0; hq < 2; ++hq) {
-      int4 t4[4][4];
+    for (int o = 0; o < 4; ++o) {
+      const uint32_t peer = static_cast<uint32_t>(2 * o + h);
 #pragma unroll
-      for (int o = 0; o < 4; ++o) {
-        const uint32_t peer = static_cast<uint32_t>(2 * o + h);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          t4[o][q] = o < p.splits ? ld_dsmem_v4(map_to_rank(off + (hq * 4 + q) * 32 * 16, peer))
-                                  : make_int4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int o = 0; o < 4; ++o)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int q4 = hq * 4 + q;
-          va[q4 * 4] += t4[o][q].x;
-          va[q4 * 4 + 1] += t4[o][q].y;
-          va[q4 * 4 + 2] += t4[o][q].z;
-          va[q4 * 4 + 3] += t4[o][q].w;
-        }
+      for (int q4 = 0; q4 < 8; ++q4)
+        t4[o][q4] = o < p.splits ? ld_dsmem_v4(map_to_rank(off + q4 * 32 * 16, peer))
+                                 : make_int4(0, 0, 0, 0);
     }
+#pragma unroll
+    for (int o = 0; o < 4; ++o)
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) order_after_loads(t4[o][q4]);
+#pragma unroll
+    for (int o = 0; o < 4; ++o)
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        va[q4 * 4] += t4[o][q4].x;
+        va[q4 * 4 + 1] += t4[o][q4].y;
+        va[q4 * 4 + 2] += t4[o][q4].z;
+        va[q4 * 4 + 3] += t4[o][q4].w;
+      }
     const int col0 = tn * kPairBN + c * 32;
     if (rv && col0 < p.n) store32_channel(p, row, col0, sa, sws + t * 32, va);
   }

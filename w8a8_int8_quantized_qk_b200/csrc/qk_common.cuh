@@ -238,6 +238,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
 }
 
 // 16-byte load from another CTA's shared memory (address from mapa).
+// Keep the uses of v after every load issued before this point: volatile
+// asm statements keep their order, so loads issued earlier all stay ahead of
+// arithmetic on values passed through here (their latencies then overlap).
+__device__ __forceinline__ void order_after_loads(int4& v) {
+  asm volatile("" : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w));
+}
+
 __device__ __forceinline__ int4 ld_dsmem_v4(uint32_t cluster_addr) {
   int4 v;
   asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
