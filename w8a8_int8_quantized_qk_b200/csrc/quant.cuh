@@ -79,6 +79,49 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, e)), u);
 }
 
+__device__ __forceinline__ uint64_t splat2(float x) {
+  return pack2(__float_as_uint(x), __float_as_uint(x));
+}
+
+// Two silu_mul at once: the same operations in the same order, with the
+// reduction, polynomial and final multiply as packed pairs (per-lane IEEE
+// round-to-nearest), so each result is bit-identical to silu_mul's.  No
+// packed multiply feeds a packed add (the pair could be fused), and the
+// clamp, the 2^n scaling, the 1 + e and the divide stay scalar.
+__device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1, float& h0,
+                                          float& h1) {
+  constexpr float kLog2e = static_cast<float>(1.4426950408889634074);
+  constexpr float kLn2Hi = static_cast<float>(0.69314718055994530942);
+  constexpr float kLn2Lo =
+      static_cast<float>(0.69314718055994530942 - static_cast<double>(kLn2Hi));
+  const float t0 = fminf(fmaxf(-g0, -87.0f), 88.0f);
+  const float t1 = fminf(fmaxf(-g1, -87.0f), 88.0f);
+  const float nb0 = __fadd_rn(__fmul_rn(t0, kLog2e), kRoundMagic);
+  const float nb1 = __fadd_rn(__fmul_rn(t1, kLog2e), kRoundMagic);
+  const uint64_t t = pack2(__float_as_uint(t0), __float_as_uint(t1));
+  const uint64_t n =
+      f32x2_add(pack2(__float_as_uint(nb0), __float_as_uint(nb1)), splat2(-kRoundMagic));
+  const uint64_t mn = n ^ 0x8000000080000000ull;  // -n in both lanes
+  uint64_t r = f32x2_fma(mn, splat2(kLn2Hi), t);
+  r = f32x2_fma(mn, splat2(kLn2Lo), r);
+  uint64_t p = f32x2_fma(splat2(static_cast<float>(1.0 / 5040.0)), r,
+                         splat2(static_cast<float>(1.0 / 720.0)));
+  p = f32x2_fma(p, r, splat2(static_cast<float>(1.0 / 120.0)));
+  p = f32x2_fma(p, r, splat2(static_cast<float>(1.0 / 24.0)));
+  p = f32x2_fma(p, r, splat2(static_cast<float>(1.0 / 6.0)));
+  p = f32x2_fma(p, r, splat2(0.5f));
+  p = f32x2_fma(p, r, splat2(1.0f));
+  p = f32x2_fma(p, r, splat2(1.0f));
+  const float two0 = __uint_as_float((__float_as_uint(nb0) - kRoundMagicBits + 127u) << 23);
+  const float two1 = __uint_as_float((__float_as_uint(nb1) - kRoundMagicBits + 127u) << 23);
+  const float s0 = __fdiv_rn(g0, __fadd_rn(1.0f, __fmul_rn(lo_of(p), two0)));
+  const float s1 = __fdiv_rn(g1, __fadd_rn(1.0f, __fmul_rn(hi_of(p), two1)));
+  const uint64_t h = f32x2_mul(pack2(__float_as_uint(s0), __float_as_uint(s1)),
+                               pack2(__float_as_uint(u0), __float_as_uint(u1)));
+  h0 = lo_of(h);
+  h1 = hi_of(h);
+}
+
 // Quantise one value: the low byte of (x * inv + 1.5 * 2^23) is
 // round_half_even(x * inv) as a two's-complement int8.  The clamp to
 // [-127, 127] is never active: |x| <= amax and inv = RN(1 / RN(a / 127)) with
@@ -212,9 +255,10 @@ __global__ void __launch_bounds__(kMaxThreads) quant_rows_kernel(Args p) {
       widen<BF16>(gv[j], g);
       widen<BF16>(uv[j], u);
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        vals[j][e] = silu_mul(g[e], u[e]);
+      for (int e = 0; e < E; e += 2) {
+        silu_mul2(g[e], g[e + 1], u[e], u[e + 1], vals[j][e], vals[j][e + 1]);
         m = fmaxf(m, fabsf(vals[j][e]));
+        m = fmaxf(m, fabsf(vals[j][e + 1]));
       }
     }
   } else {
@@ -287,7 +331,8 @@ __global__ void __launch_bounds__(kPersistThreads) quant_rows_persistent_kernel(
         float u[E];
         widen<BF16>(uc[j], u);
 #pragma unroll
-        for (int e = 0; e < E; ++e) vals[j][e] = silu_mul(vals[j][e], u[e]);
+        for (int e = 0; e < E; e += 2)
+          silu_mul2(vals[j][e], vals[j][e + 1], u[e], u[e + 1], vals[j][e], vals[j][e + 1]);
       }
 #pragma unroll
       for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(vals[j][e]));
@@ -337,7 +382,7 @@ __global__ void __launch_bounds__(512) quant_rows_twopass_kernel(Args p) {
       float u[E];
       widen<BF16>(ld_nc_v4(ur + static_cast<int64_t>(v) * 16), u);
 #pragma unroll
-      for (int e = 0; e < E; ++e) f[e] = silu_mul(f[e], u[e]);
+      for (int e = 0; e < E; e += 2) silu_mul2(f[e], f[e + 1], u[e], u[e + 1], f[e], f[e + 1]);
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(f[e]));
@@ -353,7 +398,7 @@ __global__ void __launch_bounds__(512) quant_rows_twopass_kernel(Args p) {
       float u[E];
       widen<BF16>(ld_nc_v4(ur + static_cast<int64_t>(v) * 16), u);
 #pragma unroll
-      for (int e = 0; e < E; ++e) f[e] = silu_mul(f[e], u[e]);
+      for (int e = 0; e < E; e += 2) silu_mul2(f[e], f[e + 1], u[e], u[e + 1], f[e], f[e + 1]);
     }
     store_q<E>(qr + static_cast<int64_t>(v) * E, f, inv);
   }
