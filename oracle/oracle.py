@@ -22,6 +22,12 @@ Which page each function follows:
   (GemmConfig's scale_a, scale_b, output_scale).
 * :func:`gemm_group` -- "KV-cache kernels" section 03 (per-group scales every
   64-128 channels); group partials in int32, fp32 accumulation across groups.
+* :func:`quantize_per_token_fp8`, :func:`silu_mul_quant_per_token_fp8` -- the
+  vLLM PR's own FP8 form (Purpose/Algorithm: float8_e4m3fn,
+  scale = max(absmax, 1e-12) / fp8_max, optionally clamped by scale_ub).
+* :func:`gemm_fp8` -- the FP8 x FP8 product with the exact accumulator
+  (every e4m3 value is an integer multiple of 2^-9) and the per-channel
+  epilogue.
 """
 from __future__ import annotations
 
@@ -84,6 +90,20 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.qko_epilogue_per_channel.restype = i32
     lib.qko_gemm_group.argtypes = [i32, i32, i32, i32, P, P, P, P, f32, P, P, i32]
     lib.qko_gemm_group.restype = i32
+    lib.qko_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+    lib.qko_e4m3_to_f32.restype = f32
+    lib.qko_f32_to_e4m3.argtypes = [f32]
+    lib.qko_f32_to_e4m3.restype = ctypes.c_uint8
+    lib.qko_f32_to_e4m3_array.argtypes = [P, P, i64]
+    lib.qko_f32_to_e4m3_array.restype = None
+    lib.qko_quantize_row_fp8.argtypes = [P, i32, P, P, P]
+    lib.qko_quantize_row_fp8.restype = None
+    lib.qko_quantize_per_token_fp8.argtypes = [i32, i32, P, i32, P, P, P]
+    lib.qko_quantize_per_token_fp8.restype = i32
+    lib.qko_silu_mul_quant_per_token_fp8.argtypes = [i32, i32, P, P, i64, i32, P, P, P]
+    lib.qko_silu_mul_quant_per_token_fp8.restype = i32
+    lib.qko_gemm_fp8.argtypes = [i32, i32, i32, P, P, P, P, f32, P, P, i32]
+    lib.qko_gemm_fp8.restype = i32
     return lib
 
 
@@ -238,4 +258,73 @@ class Oracle:
         else:
             acc = self.gemm_s32(q, w_q)
             out = self.epilogue_per_channel(acc, sa, sw, alpha)
+        return {"q": q, "sa": sa, "acc": acc, "out_f32": out, "out_bf16": self.f32_to_bf16(out)}
+
+    # -- FP8 (e4m3) variant ---------------------------------------------------
+    def e4m3_to_f32(self, codes: np.ndarray) -> np.ndarray:
+        f = self.lib.qko_e4m3_to_f32
+        c = np.asarray(codes, np.uint8)
+        return np.array([f(int(b)) for b in c.ravel()], np.float32).reshape(c.shape)
+
+    def f32_to_e4m3(self, x: np.ndarray) -> np.ndarray:
+        x = np.ascontiguousarray(x, np.float32)
+        out = np.empty(x.shape, np.uint8)
+        self.lib.qko_f32_to_e4m3_array(_ptr(x), _ptr(out), x.size)
+        return out
+
+    def _ub(self, scale_ub):
+        if scale_ub is None:
+            return None, ctypes.c_void_p(0)
+        ub = np.array([scale_ub], np.float32)
+        return ub, _ptr(ub)
+
+    def quantize_per_token_fp8(self, x: np.ndarray, scale_ub: float | None = None):
+        """x [m, k] (float32 or bf16 bits) -> (q e4m3 codes uint8 [m, k], scale float32 [m])."""
+        x = np.ascontiguousarray(x)
+        m, k = x.shape
+        q = np.empty((m, k), np.uint8)
+        s = np.empty((m,), np.float32)
+        keep, ub = self._ub(scale_ub)
+        _check(self.lib.qko_quantize_per_token_fp8(m, k, _ptr(x), _dtype_code(x), ub, _ptr(q),
+                                                   _ptr(s)), "quantize_per_token_fp8")
+        return q, s
+
+    def silu_mul_quant_per_token_fp8(self, gate: np.ndarray, up: np.ndarray,
+                                     scale_ub: float | None = None):
+        """gate, up [m, k] (same dtype) -> (q e4m3 codes uint8 [m, k], scale float32 [m])."""
+        gate = np.ascontiguousarray(gate)
+        up = np.ascontiguousarray(up)
+        assert gate.shape == up.shape and gate.dtype == up.dtype
+        m, k = gate.shape
+        q = np.empty((m, k), np.uint8)
+        s = np.empty((m,), np.float32)
+        keep, ub = self._ub(scale_ub)
+        _check(self.lib.qko_silu_mul_quant_per_token_fp8(m, k, _ptr(gate), _ptr(up), k,
+                                                         _dtype_code(gate), ub, _ptr(q), _ptr(s)),
+               "silu_mul_quant_per_token_fp8")
+        return q, s
+
+    def gemm_fp8(self, a: np.ndarray, w: np.ndarray, sa: np.ndarray | None = None,
+                 sw: np.ndarray | None = None, alpha: float = 1.0):
+        """a [m, k], w [n, k] e4m3 codes -> (exact acc float64 [m, n], fp32 out [m, n] or None)."""
+        a = np.ascontiguousarray(a, np.uint8)
+        w = np.ascontiguousarray(w, np.uint8)
+        m, k = a.shape
+        n = w.shape[0]
+        acc = np.empty((m, n), np.float64)
+        out = None
+        if sa is not None:
+            sa = np.ascontiguousarray(sa, np.float32)
+            sw = np.ascontiguousarray(sw, np.float32)
+            out = np.empty((m, n), np.float32)
+        _check(self.lib.qko_gemm_fp8(m, n, k, _ptr(a), _ptr(w),
+                                     _ptr(sa) if sa is not None else ctypes.c_void_p(0),
+                                     _ptr(sw) if sw is not None else ctypes.c_void_p(0),
+                                     ctypes.c_float(alpha), _ptr(acc),
+                                     _ptr(out) if out is not None else ctypes.c_void_p(0),
+                                     self.nthreads), "gemm_fp8")
+        return acc, out
+
+    def linear_fp8_from_q(self, q, sa, w_q, sw, alpha: float = 1.0):
+        acc, out = self.gemm_fp8(q, w_q, sa, sw, alpha)
         return {"q": q, "sa": sa, "acc": acc, "out_f32": out, "out_bf16": self.f32_to_bf16(out)}

@@ -36,6 +36,22 @@
  *    f = fmaf((float)P_g, sw[n][g], f); o = (f * sa[m]) * alpha.
  *  - bf16 output = round-to-nearest-even of o.
  *
+ * FP8 variant (same vLLM PR, Purpose / Algorithm: the pages' own kernel
+ * quantises to float8_e4m3fn, scale = max(absmax, 1e-12) / fp8_max,
+ * "optionally clamped by scale_ub"; "The Quantization Ladder" page (day 11)
+ * on e4m3 spending its bits on mantissa):
+ *  - e4m3 is the OCP E4M3FN format: 1 sign, 4 exponent bits (bias 7), 3
+ *    mantissa bits, no infinities, S.1111.111 NaN; largest finite 448,
+ *    smallest normal 2^-6, smallest subnormal 2^-9.
+ *  - scale = max(amax, 1e-12f) / 448 (fp32 RN); with an upper bound ub the
+ *    written scale is min(that, ub) (the scale itself is clamped, as the
+ *    page's sentence reads); inv = 1 / scale (fp32 RN).
+ *  - q = e4m3(clamp(x * inv, -448, 448)), converted round-to-nearest-even.
+ *  - the FP8 GEMM's accumulator is the exact dot product of the decoded
+ *    values (every e4m3 value is an integer multiple of 2^-9, so products
+ *    are integer multiples of 2^-18 and the sum is exact in int64), rounded
+ *    once to fp32; the epilogue is the per-channel one above.
+ *
  * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread (no fast-math),
  * so every float operation below is a single IEEE binary32 RN operation.
  *
@@ -329,4 +345,181 @@ int qko_gemm_group(int m, int n, int k, int group, const int8_t* a, const int8_t
   j.acc = acc;
   j.out = out;
   return qko_run_rows(&j, m, nthreads);
+}
+
+/* ----------------------------------------------------------------------- */
+/* FP8 e4m3 (E4M3FN) encode / decode                                       */
+/* ----------------------------------------------------------------------- */
+
+/* value of an e4m3 code: subnormal (exponent field 0) m * 2^-9, normal
+ * (8 + m) * 2^(e - 10) = (1 + m / 8) * 2^(e - 7); S.1111.111 is NaN. */
+float qko_e4m3_to_f32(uint8_t b) {
+  const int e = (b >> 3) & 15, m = b & 7;
+  if (e == 15 && m == 7) return NAN;
+  const float v = e == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
+  return (b & 0x80) ? -v : v;
+}
+
+/* The code's value in units of 2^-9 (an integer for every finite code). */
+static int64_t qko_e4m3_units(uint8_t b) {
+  const int e = (b >> 3) & 15, m = b & 7;
+  const int64_t u = e == 0 ? (int64_t)m : (int64_t)(8 + m) << (e - 1);
+  return (b & 0x80) ? -u : u;
+}
+
+/* Nearest e4m3 value to a finite x, ties to the even code; |x| >= 448 gives
+ * +-448 (the quantiser clamps to [-448, 448] before converting).  The
+ * spacing in [2^E, 2^(E+1)) is 2^(E-3) for E >= -6, and 2^-9 below 2^-6;
+ * dividing by a power of two is exact, so nearbyintf does the rounding. */
+uint8_t qko_f32_to_e4m3(float x) {
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  const float a = fabsf(x);
+  if (a >= 448.0f) return sign | 0x7E;
+  if (a == 0.0f) return sign;
+  int ex;
+  frexpf(a, &ex);  /* a = f * 2^ex, f in [0.5, 1) */
+  int E = ex - 1;  /* a in [2^E, 2^(E+1)) */
+  if (E < -6) E = -6;
+  const float spacing = ldexpf(1.0f, E - 3);
+  const float steps = nearbyintf(a / spacing); /* ties to even */
+  const float v = steps * spacing;             /* exact */
+  if (v == 0.0f) return sign;
+  frexpf(v, &ex);
+  const int E2 = ex - 1;
+  if (E2 < -6) return sign | (uint8_t)(int)(v / ldexpf(1.0f, -9));
+  const int m = (int)(v / ldexpf(1.0f, E2 - 3)) - 8; /* 0..7 */
+  return sign | (uint8_t)(((E2 + 7) << 3) | m);
+}
+
+void qko_f32_to_e4m3_array(const float* in, uint8_t* out, int64_t count) {
+  for (int64_t i = 0; i < count; ++i) out[i] = qko_f32_to_e4m3(in[i]);
+}
+
+/* ----------------------------------------------------------------------- */
+/* Dynamic per-token FP8 quantisation                                      */
+/* ----------------------------------------------------------------------- */
+
+/* One row: amax = max|x|, scale = max(amax, 1e-12f) / 448, clamped above by
+ * *ub when ub is given; inv = 1 / scale; q = e4m3(clamp(x * inv, +-448)). */
+void qko_quantize_row_fp8(const float* x, int k, const float* ub, uint8_t* q, float* scale) {
+  float amax = 0.0f;
+  for (int i = 0; i < k; ++i) {
+    float ax = fabsf(x[i]);
+    if (ax > amax) amax = ax;
+  }
+  float s = fmaxf(amax, 1e-12f) / 448.0f;
+  if (ub && s > *ub) s = *ub;
+  float inv = 1.0f / s;
+  for (int i = 0; i < k; ++i) {
+    float y = x[i] * inv;
+    if (y > 448.0f) y = 448.0f;
+    if (y < -448.0f) y = -448.0f;
+    q[i] = qko_f32_to_e4m3(y);
+  }
+  *scale = s;
+}
+
+int qko_quantize_per_token_fp8(int m, int k, const void* x, int dtype, const float* ub,
+                               uint8_t* q, float* scale) {
+  if (m < 0 || k <= 0 || (dtype != QKO_F32 && dtype != QKO_BF16)) return QKO_ERR_ARG;
+  float* row = (float*)malloc(sizeof(float) * (size_t)k);
+  if (!row) return QKO_ERR_ARG;
+  for (int r = 0; r < m; ++r) {
+    for (int i = 0; i < k; ++i) row[i] = qko_load(x, dtype, (int64_t)r * k + i);
+    qko_quantize_row_fp8(row, k, ub, q + (int64_t)r * k, scale + r);
+  }
+  free(row);
+  return QKO_OK;
+}
+
+/* silu(gate) * up (fp32, as qko_silu_mul_quant_per_token), then the FP8
+ * per-token quantisation of the row. */
+int qko_silu_mul_quant_per_token_fp8(int m, int k, const void* gate, const void* up, int64_t ld,
+                                     int dtype, const float* ub, uint8_t* q, float* scale) {
+  if (m < 0 || k <= 0 || ld < k || (dtype != QKO_F32 && dtype != QKO_BF16)) return QKO_ERR_ARG;
+  float* h = (float*)malloc(sizeof(float) * (size_t)k);
+  if (!h) return QKO_ERR_ARG;
+  for (int r = 0; r < m; ++r) {
+    for (int i = 0; i < k; ++i) {
+      float gv = qko_load(gate, dtype, (int64_t)r * ld + i);
+      float uv = qko_load(up, dtype, (int64_t)r * ld + i);
+      h[i] = qko_silu(gv) * uv;
+    }
+    qko_quantize_row_fp8(h, k, ub, q + (int64_t)r * k, scale + r);
+  }
+  free(h);
+  return QKO_OK;
+}
+
+/* ----------------------------------------------------------------------- */
+/* FP8 x FP8 GEMM (exact accumulator) and its per-channel epilogue          */
+/* ----------------------------------------------------------------------- */
+
+typedef struct {
+  int m0, m1, n, k;
+  const uint8_t* a;
+  const uint8_t* w;
+  const float* sa;
+  const float* sw;
+  float alpha;
+  double* acc;
+  float* out;
+} qko_fp8_job;
+
+static void* qko_fp8_worker(void* p) {
+  qko_fp8_job* j = (qko_fp8_job*)p;
+  for (int r = j->m0; r < j->m1; ++r) {
+    const uint8_t* ar = j->a + (int64_t)r * j->k;
+    for (int c = 0; c < j->n; ++c) {
+      const uint8_t* wr = j->w + (int64_t)c * j->k;
+      int64_t s = 0; /* units of 2^-18 */
+      for (int i = 0; i < j->k; ++i) s += qko_e4m3_units(ar[i]) * qko_e4m3_units(wr[i]);
+      const double exact = ldexp((double)s, -18);
+      if (j->acc) j->acc[(int64_t)r * j->n + c] = exact;
+      if (j->out) {
+        float o = (float)exact; /* the exact sum rounded once to fp32 */
+        o = o * j->sa[r];
+        o = o * j->sw[c];
+        o = o * j->alpha;
+        j->out[(int64_t)r * j->n + c] = o;
+      }
+    }
+  }
+  return NULL;
+}
+
+/* a: [m, k] e4m3 codes, w: [n, k] e4m3 codes.  acc (nullable): the exact dot
+ * products as double (exact while |sum| < 2^35, i.e. k * 448^2 < 2^35 --
+ * always so below k = 171,000); out (nullable): the fp32 epilogue. */
+int qko_gemm_fp8(int m, int n, int k, const uint8_t* a, const uint8_t* w, const float* sa,
+                 const float* sw, float alpha, double* acc, float* out, int nthreads) {
+  if (m < 0 || n < 0 || k <= 0 || k > 171000) return QKO_ERR_ARG;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > m) nthreads = m > 0 ? m : 1;
+  qko_fp8_job* jobs = (qko_fp8_job*)calloc((size_t)nthreads, sizeof(qko_fp8_job));
+  pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+  if (!jobs || !th) {
+    free(jobs);
+    free(th);
+    return QKO_ERR_ARG;
+  }
+  for (int t = 0; t < nthreads; ++t) {
+    jobs[t].m0 = (int)((int64_t)m * t / nthreads);
+    jobs[t].m1 = (int)((int64_t)m * (t + 1) / nthreads);
+    jobs[t].n = n;
+    jobs[t].k = k;
+    jobs[t].a = a;
+    jobs[t].w = w;
+    jobs[t].sa = sa;
+    jobs[t].sw = sw;
+    jobs[t].alpha = alpha;
+    jobs[t].acc = acc;
+    jobs[t].out = out;
+  }
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, qko_fp8_worker, &jobs[t]);
+  qko_fp8_worker(&jobs[0]);
+  for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+  free(jobs);
+  free(th);
+  return QKO_OK;
 }

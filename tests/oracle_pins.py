@@ -22,6 +22,16 @@ What pins what:
                        left-to-right fp32 chain; exact power-of-two cases;
                        group mode against a float64 sum of per-group terms.
 * whole chain       -- hand-worked example (golden ``linear_hand.json``).
+* FP8 e4m3 codec    -- torch's float8_e4m3fn (decode of all 256 codes; the
+                       float32 -> e4m3 cast on random values, every
+                       representable value and every tie midpoint);
+                       closed forms from the format (448, 2^-6, 2^-9, ties
+                       to the even code).
+* FP8 quantiser     -- absmax element -> +-448; scale * 448 ~ absmax;
+                       round-trip bound of half an e4m3 spacing; the
+                       scale_ub clamp; a hand-worked row.
+* FP8 GEMM          -- numpy float64 matmul of the decoded operands (exact
+                       at these sizes); closed forms (all-448 operands).
 """
 from __future__ import annotations
 
@@ -266,6 +276,129 @@ def pin_linear_golden(O) -> None:
     assert res["out_f32"].tolist() == g["out"]
 
 
+# --------------------------------------------------------------------------- FP8 e4m3
+def _torch_e4m3(x: np.ndarray) -> np.ndarray:
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.float8_e4m3fn) \
+        .view(torch.uint8).numpy()
+
+
+def _e4m3_values() -> np.ndarray:
+    """The finite non-negative e4m3 values, from torch's float8_e4m3fn decode."""
+    import torch
+
+    codes = torch.arange(0, 0x7F, dtype=torch.uint8)  # 0x00 .. 0x7E, NaN is 0x7F
+    return codes.view(torch.float8_e4m3fn).float().numpy()
+
+
+def pin_e4m3_codec(O) -> None:
+    import torch
+
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy()
+    got = O.e4m3_to_f32(codes)
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin]) and np.all(np.isnan(got[~fin]))
+    assert sorted(np.where(~fin)[0].tolist()) == [0x7F, 0xFF]
+    vals = _e4m3_values()
+    mids = ((vals[:-1].astype(np.float64) + vals[1:]) / 2).astype(np.float32)
+    rng = np.random.default_rng(11)
+    x = np.concatenate([vals, -vals, mids, -mids, rng.uniform(-448, 448, 20000).astype(np.float32),
+                        (rng.standard_normal(20000) * 0.02).astype(np.float32)])
+    assert np.array_equal(O.f32_to_e4m3(x), _torch_e4m3(x))
+    # closed forms of the format: largest finite, smallest normal and
+    # subnormal, 1.0, and ties to the even code
+    fixed = {448.0: 0x7E, -448.0: 0xFE, 2.0 ** -6: 0x08, 2.0 ** -9: 0x01, 1.0: 0x38,
+             2.0 ** -10: 0x00, 3 * 2.0 ** -10: 0x02, 1.0625: 0x38, 1.1875: 0x3A, 0.0: 0x00,
+             240.0: 0x77, 232.0: 0x76, 0.01953125: 0x0A}
+    got = O.f32_to_e4m3(np.float32(list(fixed)))
+    assert got.tolist() == list(fixed.values()), (got.tolist(), list(fixed.values()))
+
+
+def _check_fp8_quant(O, x32, q, s, ub=None) -> None:
+    x64 = x32.astype(np.float64)
+    dec = O.e4m3_to_f32(q).astype(np.float64)
+    for r in range(x32.shape[0]):
+        amax = float(np.abs(x64[r]).max())
+        sc = float(s[r])
+        want = max(amax, float(np.float32(1e-12))) / 448.0
+        if ub is not None and want > ub:
+            assert sc == np.float32(ub), (r, sc, ub)
+        else:
+            assert abs(sc - want) <= ulp32(sc), (r, sc, want)
+        y = x64[r] / sc
+        inside = np.abs(y) <= 448.0
+        # half an e4m3 spacing at |y| (2^-10 in the subnormal range), plus the
+        # fp32 rounding of x * inv
+        e = np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** -6)))
+        half = np.where(np.abs(y) < 2.0 ** -6, 2.0 ** -10, 2.0 ** (e - 4))
+        err = np.abs(dec[r] - y)
+        assert np.all(err[inside] <= half[inside] * (1 + 1e-6) + np.abs(y[inside]) * 2.0 ** -22)
+        # clamped elements saturate at +-448
+        assert np.all(np.abs(dec[r][~inside]) == 448.0)
+        assert np.all(np.sign(dec[r][~inside]) == np.sign(y[~inside]))
+        if ub is None and amax >= 1e-12:
+            i = int(np.argmax(np.abs(x64[r])))
+            assert dec[r, i] == 448.0 * np.sign(x64[r, i]), (r, dec[r, i])
+
+
+def pin_fp8_quant(O) -> None:
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((6, 257)).astype(np.float32)
+    x[1] *= 1e-4
+    x[2, 40] = -300.0
+    x[3] = 0.0
+    q, s = O.quantize_per_token_fp8(x)
+    _check_fp8_quant(O, x, q, s)
+    assert np.all(q[3] == 0) and s[3] == np.float32(np.float32(1e-12) / np.float32(448.0))
+    # an upper bound on the scale: rows whose absmax / 448 exceeds it clamp
+    ub = 0.002
+    q2, s2 = O.quantize_per_token_fp8(x, scale_ub=ub)
+    _check_fp8_quant(O, x, q2, s2, ub)
+    assert np.any(np.abs(O.e4m3_to_f32(q2[0])) == 448.0)
+    # hand-worked row: absmax 448 -> scale 1, inv 1; each value is its own
+    # nearest e4m3 or a tie
+    row = np.float32([[448.0, -1.0, 1.0625, 1.1875, 3.0 * 2.0 ** -10, 17.0, -0.0]])
+    q3, s3 = O.quantize_per_token_fp8(row)
+    assert s3.tolist() == [1.0]
+    assert q3.tolist() == [[0x7E, 0xB8, 0x38, 0x3A, 0x02, 0x58, 0x80]], q3.tolist()  # 17 ties to 16
+
+
+def pin_fp8_silu_quant(O) -> None:
+    rng = np.random.default_rng(13)
+    g = rng.standard_normal((3, 100)).astype(np.float32) * 3
+    u = rng.standard_normal((3, 100)).astype(np.float32)
+    q, s = O.silu_mul_quant_per_token_fp8(g, u)
+    h = np.array([[O.silu(float(a)) for a in row] for row in g], np.float32) * u
+    q2, s2 = O.quantize_per_token_fp8(h.astype(np.float32))
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+def pin_fp8_gemm(O) -> None:
+    rng = np.random.default_rng(14)
+    vals = _e4m3_values()
+    a = rng.integers(0, 256, (7, 300)).astype(np.uint8)
+    w = rng.integers(0, 256, (5, 300)).astype(np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0x10  # no NaN codes
+    w[(w & 0x7F) == 0x7F] = 0x22
+    da = O.e4m3_to_f32(a).astype(np.float64)
+    dw = O.e4m3_to_f32(w).astype(np.float64)
+    del vals
+    acc, _ = O.gemm_fp8(a, w)
+    # every e4m3 value is a multiple of 2^-9: the float64 products and their
+    # sums at this size are exact, in any order
+    assert np.array_equal(acc, da @ dw.T)
+    # closed form: all operands 448 -> k * 448^2
+    k = 1000
+    acc2, out2 = O.gemm_fp8(np.full((2, k), 0x7E, np.uint8), np.full((3, k), 0xFE, np.uint8),
+                            np.float32([1.0, 0.5]), np.float32([1.0, 2.0, 0.25]), 1.0)
+    assert np.all(acc2 == -k * 448.0 ** 2)
+    assert out2.tolist() == [[-k * 448.0 ** 2, -2 * k * 448.0 ** 2, -k * 448.0 ** 2 / 4],
+                             [-k * 448.0 ** 2 / 2, -k * 448.0 ** 2, -k * 448.0 ** 2 / 8]]
+
+
 ALL_PINS = [pin_exp, pin_silu, pin_bf16_rounding, pin_quant_golden, pin_quant_invariants,
             pin_quant_bf16_path, pin_silu_quant, pin_gemm_bruteforce, pin_gemm_closed_forms,
-            pin_epilogue_per_channel, pin_group, pin_linear_golden]
+            pin_epilogue_per_channel, pin_group, pin_linear_golden, pin_e4m3_codec, pin_fp8_quant,
+            pin_fp8_silu_quant, pin_fp8_gemm]

@@ -44,6 +44,21 @@ MUTANTS = [
     ("bf16_widen_wrong", "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)b) << 15;"),
     ("silu_ld_ignored", "float u = qko_load(up, dtype, (int64_t)r * ld + i);",
      "float u = qko_load(up, dtype, (int64_t)r * k + i);"),
+    ("fp8_ties_away", "const float steps = nearbyintf(a / spacing); /* ties to even */",
+     "const float steps = roundf(a / spacing);"),
+    ("fp8_no_subnormal_floor", "if (E < -6) E = -6;", ""),
+    ("fp8_bias_8", "return sign | (uint8_t)(((E2 + 7) << 3) | m);",
+     "return sign | (uint8_t)(((E2 + 8) << 3) | m);"),
+    ("fp8_decode_bias", ": ldexpf((float)(8 + m), e - 10);", ": ldexpf((float)(8 + m), e - 11);"),
+    ("fp8_qmax_240", "float s = fmaxf(amax, 1e-12f) / 448.0f;", "float s = fmaxf(amax, 1e-12f) / 240.0f;"),
+    ("fp8_ub_ignored", "if (ub && s > *ub) s = *ub;", ""),
+    ("fp8_absmax_signed", "float ax = fabsf(x[i]);", "float ax = x[i];"),
+    ("fp8_clamp_240", "if (y > 448.0f) y = 448.0f;", "if (y > 240.0f) y = 240.0f;"),
+    ("fp8_silu_up_from_gate", "float uv = qko_load(up, dtype, (int64_t)r * ld + i);",
+     "float uv = qko_load(gate, dtype, (int64_t)r * ld + i);"),
+    ("fp8_gemm_units", ": (int64_t)(8 + m) << (e - 1);", ": (int64_t)(8 + m) << e;"),
+    ("fp8_gemm_dropped_term", "for (int i = 0; i < j->k; ++i) s += qko_e4m3_units(ar[i]) * qko_e4m3_units(wr[i]);",
+     "for (int i = 1; i < j->k; ++i) s += qko_e4m3_units(ar[i]) * qko_e4m3_units(wr[i]);"),
 ]
 
 
