@@ -50,7 +50,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 2
+#define QK_ABI_VERSION 3
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -126,6 +126,32 @@ QK_API qk_status qk_quantize_per_token(int m, int k, const void* x, qk_dtype x_d
 QK_API qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, const void* up,
                                       int64_t ld_in, qk_dtype in_dtype, int8_t* q, float* scale,
                                       qk_stream stream);
+
+/*
+ * qk_quantize_per_token_fp8 / qk_silu_mul_quant_per_token_fp8 -- the same
+ * two quantisers with float8 e4m3 output: the form of the vLLM PR "fused
+ * silu_and_mul + dynamic per-token FP8 quantization" itself (Purpose /
+ * Algorithm: float8_e4m3fn, scale = max(absmax, 1e-12) / fp8_max, optionally
+ * clamped by scale_ub, quantisation with the per-token inverse scale).
+ *
+ * Per row: amax = max |x| (or |h|, h = silu(gate) * up in fp32);
+ * scale = max(amax, 1e-12f) / 448 (fp32 RN), then scale = min(scale,
+ * *scale_ub) when scale_ub is given; inv = 1 / scale (fp32 RN);
+ * q = e4m3(clamp(x * inv, -448, 448)) rounded to nearest, ties to even.
+ * e4m3 is the OCP E4M3FN format (no infinities, largest finite 448).
+ *
+ * scale_ub       optional device pointer to one fp32 upper bound of the
+ *                written scale (NULL: none), 4-byte aligned
+ * q              [m, k] e4m3 codes (one byte each), 16-B aligned
+ * other arguments, layouts and errors as the int8 forms above.
+ */
+QK_API qk_status qk_quantize_per_token_fp8(int m, int k, const void* x, qk_dtype x_dtype,
+                                           const float* scale_ub, uint8_t* q, float* scale,
+                                           qk_stream stream);
+QK_API qk_status qk_silu_mul_quant_per_token_fp8(int m, int k, const void* gate, const void* up,
+                                                 int64_t ld_in, qk_dtype in_dtype,
+                                                 const float* scale_ub, uint8_t* q, float* scale,
+                                                 qk_stream stream);
 
 /*
  * qk_w8a8_gemm -- INT8 x INT8 GEMM with INT32 accumulation and a fused

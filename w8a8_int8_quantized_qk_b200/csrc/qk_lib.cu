@@ -73,7 +73,8 @@ inline bool aligned(const void* p, uintptr_t a) {
 constexpr int kMaxK = 133144;
 
 qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, qk_dtype dt,
-                       int8_t* q, float* scale, qk_stream stream, bool silu) {
+                       int8_t* q, float* scale, qk_stream stream, bool silu, bool fp8 = false,
+                       const float* ub = nullptr) {
   if (m < 0 || k <= 0 || (k % 16) != 0) return QK_ERR_INVALID_ARG;
   if (dt != QK_F32 && dt != QK_BF16) return QK_ERR_INVALID_ARG;
   if (ld < k) return QK_ERR_INVALID_ARG;
@@ -82,7 +83,7 @@ qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, 
     return QK_ERR_INVALID_ARG;
   const int64_t esize = dt == QK_BF16 ? 2 : 4;
   if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale, 4) || (silu && !aligned(up, 16)) ||
-      (ld * esize) % 16 != 0)
+      !aligned(ub, 4) || (ld * esize) % 16 != 0)
     return QK_ERR_MISALIGNED;
   const DeviceInfo* dev = nullptr;
   const qk_status st = check_device(&dev);
@@ -95,6 +96,8 @@ qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, 
   a.ld = ld;
   a.q = q;
   a.scale = scale;
+  a.fp8 = fp8 ? 1 : 0;
+  a.ub = fp8 ? ub : nullptr;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = silu ? quant::launch<true>(a, dt == QK_BF16, dev->sms, s)
                              : quant::launch<false>(a, dt == QK_BF16, dev->sms, s);
@@ -192,6 +195,20 @@ qk_status qk_silu_mul_quant_per_token(int m, int k, const void* gate, const void
                                       int64_t ld_in, qk_dtype in_dtype, int8_t* q, float* scale,
                                       qk_stream stream) {
   return quant_common(m, k, gate, up, ld_in, in_dtype, q, scale, stream, true);
+}
+
+qk_status qk_quantize_per_token_fp8(int m, int k, const void* x, qk_dtype x_dtype,
+                                    const float* scale_ub, uint8_t* q, float* scale,
+                                    qk_stream stream) {
+  return quant_common(m, k, x, nullptr, k, x_dtype, reinterpret_cast<int8_t*>(q), scale, stream,
+                      false, true, scale_ub);
+}
+
+qk_status qk_silu_mul_quant_per_token_fp8(int m, int k, const void* gate, const void* up,
+                                          int64_t ld_in, qk_dtype in_dtype, const float* scale_ub,
+                                          uint8_t* q, float* scale, qk_stream stream) {
+  return quant_common(m, k, gate, up, ld_in, in_dtype, reinterpret_cast<int8_t*>(q), scale,
+                      stream, true, true, scale_ub);
 }
 
 namespace {

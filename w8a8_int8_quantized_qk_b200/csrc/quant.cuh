@@ -29,8 +29,10 @@ struct Args {
   const void* x;    // plain: [m, k]
   const void* up;   // silu: gate = x, up = up, row stride ld
   int64_t ld;       // row stride of x / up in elements
-  int8_t* q;        // [m, k]
+  int8_t* q;        // [m, k]: int8 codes, or e4m3 codes when fp8
   float* scale;     // [m]
+  int fp8;          // 0: int8, qmax 127; 1: float8 e4m3, qmax 448
+  const float* ub;  // fp8 only, optional: upper bound of the written scale
 };
 
 // 1.5 * 2^23: adding it to |y| < 2^22 rounds y to an integer, ties to even
@@ -127,6 +129,16 @@ __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1
 // [-127, 127] is never active: |x| <= amax and inv = RN(1 / RN(a / 127)) with
 // a = max(amax, 1e-12) give |x * inv| <= 127 (1 + 2^-23), which rounds to at
 // most 127.
+// Four binary32 values -> four float8 e4m3 codes (bytes in order a..d),
+// each rounded to nearest, ties to even, saturating to +-448.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  // cvt's first source goes to the upper byte of the pair
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
 __device__ __forceinline__ uint32_t quant_bits(float x, float inv) {
   return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), kRoundMagic));
 }
@@ -152,7 +164,24 @@ __device__ __forceinline__ void widen(const uint4& v, float (&f)[BF16 ? 8 : 4]) 
 
 // Quantise E values and store E int8 at dst.
 template <int E>
-__device__ __forceinline__ void store_q(int8_t* dst, const float (&f)[E], float inv) {
+__device__ __forceinline__ void store_q(const Args& p, int8_t* dst, const float (&f)[E], float inv) {
+  if (p.fp8) {
+    // e4m3: y = x * inv (fp32 RN), converted round-to-nearest-even; the
+    // satfinite conversion gives +-448 for |y| beyond it, as the clamp to
+    // [-448, 448] before an exact conversion does
+    if constexpr (E == 8) {
+      uint2 o;
+      o.x = e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
+                   __fmul_rn(f[3], inv));
+      o.y = e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
+                   __fmul_rn(f[7], inv));
+      *reinterpret_cast<uint2*>(dst) = o;
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv),
+                                                 __fmul_rn(f[2], inv), __fmul_rn(f[3], inv));
+    }
+    return;
+  }
   if constexpr (E == 8) {
     uint2 o;
     o.x = pack_q4(quant_bits(f[0], inv), quant_bits(f[1], inv), quant_bits(f[2], inv),
@@ -201,8 +230,14 @@ __device__ __forceinline__ float row_max(float v, float* red /*[33]*/) {
 }
 
 // scale = max(amax, 1e-12) / 127 and inv = 1 / scale, both IEEE RN.
-__device__ __forceinline__ void scale_and_inverse(float amax, float& scale, float& inv) {
-  scale = __fdiv_rn(fmaxf(amax, 1e-12f), 127.0f);
+__device__ __forceinline__ void scale_and_inverse(const Args& p, float amax, float& scale,
+                                                  float& inv) {
+  if (p.fp8) {
+    scale = __fdiv_rn(fmaxf(amax, 1e-12f), 448.0f);
+    if (p.ub != nullptr) scale = fminf(scale, __ldg(p.ub));
+  } else {
+    scale = __fdiv_rn(fmaxf(amax, 1e-12f), 127.0f);
+  }
   inv = __fdiv_rn(1.0f, scale);
 }
 
@@ -277,11 +312,11 @@ __global__ void __launch_bounds__(kMaxThreads) quant_rows_kernel(Args p) {
   }
   const float amax = row_max<CLUSTER>(m, red);
   float scale, inv;
-  scale_and_inverse(amax, scale, inv);
+  scale_and_inverse(p, amax, scale, inv);
 #pragma unroll
   for (int j = 0; j < V; ++j) {
     const int v = t0 + j * stride;
-    if (v < nvec) store_q<E>(qr + static_cast<int64_t>(v) * E, vals[j], inv);
+    if (v < nvec) store_q<E>(p, qr + static_cast<int64_t>(v) * E, vals[j], inv);
   }
   if (t0 == 0) p.scale[row] = scale;
   if constexpr (CLUSTER) cluster_arrive_wait_relaxed();  // peers may still read red[32]
@@ -343,12 +378,12 @@ __global__ void __launch_bounds__(kPersistThreads) quant_rows_persistent_kernel(
     float amax = lane < NW ? red[par][lane] : 0.0f;
     amax = warp_max(amax);
     float scale, inv;
-    scale_and_inverse(amax, scale, inv);
+    scale_and_inverse(p, amax, scale, inv);
     int8_t* qr = p.q + static_cast<int64_t>(row) * p.k;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const int v = tid + j * kPersistThreads;
-      if (v < nvec) store_q<E>(qr + static_cast<int64_t>(v) * E, vals[j], inv);
+      if (v < nvec) store_q<E>(p, qr + static_cast<int64_t>(v) * E, vals[j], inv);
     }
     if (tid == 0) p.scale[row] = scale;
     par ^= 1;
@@ -389,7 +424,7 @@ __global__ void __launch_bounds__(512) quant_rows_twopass_kernel(Args p) {
   }
   amax = row_max<false>(amax, red);
   float scale, inv;
-  scale_and_inverse(amax, scale, inv);
+  scale_and_inverse(p, amax, scale, inv);
   int8_t* qr = p.q + static_cast<int64_t>(row) * p.k;
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float f[E];
@@ -400,7 +435,7 @@ __global__ void __launch_bounds__(512) quant_rows_twopass_kernel(Args p) {
 #pragma unroll
       for (int e = 0; e < E; e += 2) silu_mul2(f[e], f[e + 1], u[e], u[e + 1], f[e], f[e + 1]);
     }
-    store_q<E>(qr + static_cast<int64_t>(v) * E, f, inv);
+    store_q<E>(p, qr + static_cast<int64_t>(v) * E, f, inv);
   }
   if (threadIdx.x == 0) p.scale[row] = scale;
 }

@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -45,6 +45,10 @@ _SIGNATURES = {
     "qk_quantize_per_token": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P]),
     "qk_silu_mul_quant_per_token": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int64,
                                                    ctypes.c_int, _P, _P, _P]),
+    "qk_quantize_per_token_fp8": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P,
+                                                 _P]),
+    "qk_silu_mul_quant_per_token_fp8": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int64,
+                                                       ctypes.c_int, _P, _P, _P, _P]),
     "qk_w8a8_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
                                     ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "qk_w8a8_gemm_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
@@ -106,6 +110,15 @@ def qk_quantize_per_token(m, k, x, x_dtype, q, scale, stream) -> int:
 
 def qk_silu_mul_quant_per_token(m, k, gate, up, ld_in, in_dtype, q, scale, stream) -> int:
     return lib().qk_silu_mul_quant_per_token(m, k, gate, up, ld_in, in_dtype, q, scale, stream)
+
+
+def qk_quantize_per_token_fp8(m, k, x, x_dtype, scale_ub, q, scale, stream) -> int:
+    return lib().qk_quantize_per_token_fp8(m, k, x, x_dtype, scale_ub, q, scale, stream)
+
+
+def qk_silu_mul_quant_per_token_fp8(m, k, gate, up, ld_in, in_dtype, scale_ub, q, scale, stream) -> int:
+    return lib().qk_silu_mul_quant_per_token_fp8(m, k, gate, up, ld_in, in_dtype, scale_ub, q, scale,
+                                                 stream)
 
 
 def qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
@@ -209,6 +222,35 @@ def silu_mul_quant_per_token(gate, up, q=None, scale=None, stream=None):
     _check(qk_silu_mul_quant_per_token(m, k, _ptr(gate), _ptr(up), gate.stride(0), _dtype_code(gate),
                                        _ptr(q), _ptr(scale), _stream(stream)),
            "qk_silu_mul_quant_per_token")
+    return q, scale
+
+
+def quantize_per_token_fp8(x, scale_ub=None, q=None, scale=None, stream=None):
+    """x [m, k] bf16/fp32 -> (q e4m3 codes uint8 [m, k], scale fp32 [m]); scale_ub:
+    optional one-element fp32 CUDA tensor bounding the scale."""
+    torch = _torch()
+    _need_cuda(x)
+    assert x.dim() == 2 and x.is_contiguous()
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.uint8, device=x.device) if q is None else q
+    scale = torch.empty((m,), dtype=torch.float32, device=x.device) if scale is None else scale
+    _check(qk_quantize_per_token_fp8(m, k, _ptr(x), _dtype_code(x), _ptr(scale_ub), _ptr(q), _ptr(scale),
+                                     _stream(stream)), "qk_quantize_per_token_fp8")
+    return q, scale
+
+
+def silu_mul_quant_per_token_fp8(gate, up, scale_ub=None, q=None, scale=None, stream=None):
+    """gate, up [m, k] -> (q e4m3 codes uint8 [m, k], scale fp32 [m])."""
+    torch = _torch()
+    _need_cuda(gate, up)
+    assert gate.shape == up.shape and gate.dtype == up.dtype and gate.dim() == 2
+    assert gate.stride(1) == 1 and up.stride(1) == 1 and gate.stride(0) == up.stride(0)
+    m, k = gate.shape
+    q = torch.empty((m, k), dtype=torch.uint8, device=gate.device) if q is None else q
+    scale = torch.empty((m,), dtype=torch.float32, device=gate.device) if scale is None else scale
+    _check(qk_silu_mul_quant_per_token_fp8(m, k, _ptr(gate), _ptr(up), gate.stride(0), _dtype_code(gate),
+                                           _ptr(scale_ub), _ptr(q), _ptr(scale), _stream(stream)),
+           "qk_silu_mul_quant_per_token_fp8")
     return q, scale
 
 
