@@ -218,6 +218,29 @@ QK_API qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t
                        float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
                        void* workspace, size_t workspace_bytes, qk_stream stream);
 
+/*
+ * qk_fp8_gemm -- float8 e4m3 x e4m3 GEMM (tcgen05.mma kind::f8f6f4, fp32
+ * accumulation in the tensor core) with the per-token x per-channel
+ * dequantisation epilogue: out = ((acc * scale_a[m]) * scale_b[n]) *
+ * output_scale, rounded to out_dtype.  The FP8 counterpart of qk_w8a8_gemm
+ * for the e4m3 codes of qk_quantize_per_token_fp8 (the vLLM PR's W8A8-FP8
+ * use; "KV-cache kernels" section 02 for the epilogue order).
+ *
+ * a              [m, k] e4m3 codes, K contiguous, 16-B aligned
+ * b              [n, k] e4m3 codes (one output channel per row), 16-B aligned
+ * scale_a, scale_b   [m] and [n] fp32 dequant scales, 16-B aligned
+ * out            [m, n] in out_dtype (QK_BF16 or QK_F32), 16-B aligned
+ * m, n, k        k % 16 == 0, n % 8 == 0 (either of m, n 0: no-op)
+ * The accumulation order inside the tensor core is the hardware's, so the
+ * results match the exact dot product to within fp32 summation error, not
+ * bit for bit.  No workspace (whole tiles, no split-K).
+ * Errors: QK_ERR_INVALID_ARG, QK_ERR_MISALIGNED, QK_ERR_UNSUPPORTED,
+ *         QK_ERR_CUDA.
+ */
+QK_API qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
+                             const float* scale_a, const float* scale_b, float output_scale,
+                             void* out, qk_dtype out_dtype, qk_stream stream);
+
 /* Bytes of workspace qk_w8a8_gemm needs for this problem on the current
  * device (0 when none; the split depends on the device's SM count).
  * Returns 0 for arguments qk_w8a8_gemm would reject. */

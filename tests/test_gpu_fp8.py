@@ -112,3 +112,88 @@ def test_fp8_workload_mlp_down_prologue(O):
     qr, sr = O.silu_mul_quant_per_token_fp8(w.gate, w.up)
     assert_bits(host(q), qr, "q")
     assert_bits(host(s), sr, "scale")
+
+
+# ---------------------------------------------------------------- FP8 GEMM
+def _fp8_problem(m, n, k, seed):
+    r = synth.streams(seed, ["a", "w", "sa", "sw"])
+    return (synth.e4m3_codes(r["a"], (m, k)), synth.e4m3_codes(r["w"], (n, k)),
+            synth.scales_uniform(r["sa"], (m,), 0.001, 0.05), synth.scales_uniform(r["sw"], (n,)))
+
+
+def _fp8_bound(O, a, w, sa, sw, alpha, rows=None):
+    """Per-element bound on |gpu - exact| for the fp32 output: fp32 summation
+    of k products inside the tensor core (at most k * 2^-24 of the sum of the
+    products' magnitudes, the worst case of any summation order) plus the
+    three fp32 multiplies of the epilogue (2^-22 of the value)."""
+    da = np.abs(O.e4m3_to_f32(a).astype(np.float64))
+    dw = np.abs(O.e4m3_to_f32(w).astype(np.float64))
+    s_abs = da @ dw.T
+    k = a.shape[1]
+    scale = np.abs(sa.astype(np.float64))[:, None] * np.abs(sw.astype(np.float64))[None, :] * abs(alpha)
+    return (k * 2.0 ** -24 * s_abs) * scale
+
+
+def _check_fp8(O, got, acc_exact, bound, sa, sw, alpha, bf16):
+    ref = acc_exact * sa.astype(np.float64)[:, None] * sw.astype(np.float64)[None, :] * alpha
+    g = synth.bf16_bits_to_f32(got).astype(np.float64) if bf16 else got.astype(np.float64)
+    extra = np.abs(ref) * (2.0 ** -8 if bf16 else 2.0 ** -22)
+    err = np.abs(g - ref)
+    assert np.all(err <= bound + extra), float((err - bound - extra).max())
+    # the norm criterion of the INT8 path holds as well
+    l2 = np.sqrt(np.sum(ref * ref, axis=1, keepdims=True))
+    assert float((err / np.where(l2 > 0, l2, 1.0)).max(initial=0.0)) <= 2e-2
+
+
+FP8_GEMM_SHAPES = [(1, 64, 32), (4, 136, 272), (9, 256, 128), (100, 1032, 3008), (128, 256, 4096),
+                   (130, 264, 272), (257, 520, 1040), (300, 1000, 1552), (1024, 2048, 512)]
+
+
+@pytest.mark.parametrize("m,n,k", FP8_GEMM_SHAPES)
+def test_fp8_gemm(O, m, n, k):
+    a, w, sa, sw = _fp8_problem(m, n, k, seed=m * 13 + n + 3 * k)
+    alpha = 0.75
+    acc, _ = O.gemm_fp8(a, w)
+    bound = _fp8_bound(O, a, w, sa, sw, alpha)
+    for dt in (torch.float32, torch.bfloat16):
+        out = qk.fp8_gemm(torch.from_numpy(a).cuda(), torch.from_numpy(w).cuda(),
+                          torch.from_numpy(sa).cuda(), torch.from_numpy(sw).cuda(), alpha, dt)
+        torch.cuda.synchronize()
+        assert qk.device_status() == qk.QK_OK
+        _check_fp8(O, host(out), acc, bound, sa, sw, alpha, dt == torch.bfloat16)
+
+
+def test_fp8_linear_chain(O):
+    # quantise per token to e4m3 on the GPU (bit-exact), then the FP8 GEMM of
+    # those codes against e4m3 weights, the prefill shape on sampled rows
+    w = synth.make("prefill")
+    x = x_dev(w.x)
+    q, sa = qk.quantize_per_token_fp8(x)
+    r = synth.streams(99, ["w", "sw"])
+    wq = synth.e4m3_codes(r["w"], (w.n, w.k))
+    sw = synth.scales_uniform(r["sw"], (w.n,))
+    out = qk.fp8_gemm(q, torch.from_numpy(wq).cuda(), sa, torch.from_numpy(sw).cuda(), 1.0)
+    torch.cuda.synchronize()
+    assert qk.device_status() == qk.QK_OK
+    rows = np.random.default_rng(5).choice(w.m, 48, replace=False)
+    qh, sah = host(q), host(sa)
+    qr, sr = O.quantize_per_token_fp8(w.x[rows])
+    assert_bits(qh[rows], qr, "q rows")
+    assert_bits(sah[rows], sr, "scale rows")
+    acc, _ = O.gemm_fp8(qh[rows], wq)
+    bound = _fp8_bound(O, qh[rows], wq, sah[rows], sw, 1.0)
+    _check_fp8(O, host(out)[rows], acc, bound, sah[rows], sw, 1.0, True)
+
+
+def test_fp8_gemm_errors():
+    need_gpu()
+    a = torch.zeros((4, 40), dtype=torch.uint8, device="cuda")
+    w = torch.zeros((16, 40), dtype=torch.uint8, device="cuda")
+    s = torch.ones((16,), dtype=torch.float32, device="cuda")
+    out = torch.empty((4, 16), dtype=torch.bfloat16, device="cuda")
+    st = qk.qk_fp8_gemm(4, 16, 40, qk._ptr(a), qk._ptr(w), qk._ptr(s), qk._ptr(s), 1.0, qk._ptr(out),
+                        qk.QK_BF16, qk._stream())
+    assert st == qk.QK_ERR_INVALID_ARG  # k % 16 != 0
+    st = qk.qk_fp8_gemm(4, 16, 32, qk._ptr(a), qk._ptr(w), qk._ptr(s), qk._ptr(s), 1.0, None,
+                        qk.QK_BF16, qk._stream())
+    assert st == qk.QK_ERR_INVALID_ARG  # out is required

@@ -74,6 +74,9 @@ struct Args {
   // tensor stores from shared memory (tensor map tmO) on the whole-tile and
   // tail paths
   int tma_out;
+  // 1: a and b are float8 e4m3 codes, the MMA is kind::f8f6f4 and the
+  // accumulator fp32 (channel and pair kernels, whole tiles only, no c)
+  int f8;
 };
 
 template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
@@ -147,7 +150,7 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
 template <int BN, int STAGES, int NACC, bool GROUP, class S>
 __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
-  constexpr uint32_t idesc = idesc_i8(BM, BN);
+  const uint32_t idesc = p.f8 ? idesc_e4m3(BM, BN) : idesc_i8(BM, BN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
   for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
@@ -176,7 +179,10 @@ __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
 #pragma unroll
       for (int kk = 0; kk < BK / UMMA_K; ++kk) {
         const uint32_t acc = GROUP ? (kk > 0) : (kb > kb0 || kk > 0);
-        mma_i8(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc, acc);
+        if (!GROUP && p.f8)
+          mma_e4m3(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc, acc);
+        else
+          mma_i8(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc, acc);
       }
       mma_commit(smem_addr(&s.empty[stage]));
       if (++stage == STAGES) {
@@ -245,8 +251,17 @@ __device__ __forceinline__ void store8_channel(const Args& p, int row, int col, 
 // (64 bytes a row) for one TMA store
 constexpr int kOutBoxBytes = 32 * 32 * 2;
 
+// The accumulator's value as binary32: an int32 sum converted (exact below
+// 2^24, round-to-nearest above), or, for the FP8 kind, the fp32 sum itself.
+template <bool F8>
+__device__ __forceinline__ float acc_value(uint32_t v) {
+  if constexpr (F8) return __uint_as_float(v);
+  return __int2float_rn(static_cast<int>(v));
+}
+
 // 32 outputs of one row (columns col0 .. col0 + 31) from 32 accumulators;
 // channel scales come from shared memory.
+template <bool F8 = false>
 __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0, float sa,
                                                 const float* sw, const uint32_t (&v)[32]) {
 #pragma unroll
@@ -254,7 +269,7 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
     const int col = col0 + g * 8;
     if (col >= p.n) break;
     const int64_t o = static_cast<int64_t>(row) * p.n + col;
-    if (p.c) {
+    if (!F8 && p.c) {
       int4* dst = reinterpret_cast<int4*>(p.c + o);
       dst[0] = make_int4(v[g * 8 + 0], v[g * 8 + 1], v[g * 8 + 2], v[g * 8 + 3]);
       dst[1] = make_int4(v[g * 8 + 4], v[g * 8 + 5], v[g * 8 + 6], v[g * 8 + 7]);
@@ -266,7 +281,7 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
       float f[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        float t = __int2float_rn(static_cast<int>(v[g * 8 + j]));
+        float t = acc_value<F8>(v[g * 8 + j]);
         t = __fmul_rn(t, sa);
         t = __fmul_rn(t, s8[j]);
         f[j] = __fmul_rn(t, p.alpha);
@@ -294,6 +309,7 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
 // at (col0, row0), which clips rows >= m and columns >= n.  Lane 0 issues
 // the copies; before rewriting the box it waits until the previous copy has
 // read it.  Every lane of the warp must call this.
+template <bool F8 = false>
 __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tmO, uint8_t* box,
                                             int row0, int col0, float sa, const float* sw,
                                             const uint32_t (&v)[32]) {
@@ -303,8 +319,8 @@ __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tm
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float2 s2 = *reinterpret_cast<const float2*>(sw + 2 * j);
-    float t0 = __int2float_rn(static_cast<int>(v[2 * j]));
-    float t1 = __int2float_rn(static_cast<int>(v[2 * j + 1]));
+    float t0 = acc_value<F8>(v[2 * j]);
+    float t1 = acc_value<F8>(v[2 * j + 1]);
     t0 = __fmul_rn(__fmul_rn(__fmul_rn(t0, sa), s2.x), p.alpha);
     t1 = __fmul_rn(__fmul_rn(__fmul_rn(t1, sa), s2.y), p.alpha);
     w[j] = pack_bf16x2(t0, t1);
@@ -382,10 +398,16 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
       break;  // one unit per CTA
     }
     auto emit = [&](int ch, const uint32_t(&v)[32]) {
-      if (p.tma_out)
+      if (p.f8) {
+        if (p.tma_out)
+          store32_tma<true>(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
+        else if (rv)
+          store32_channel<true>(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
+      } else if (p.tma_out) {
         store32_tma(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
-      else if (rv)
+      } else if (rv) {
         store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
+      }
     };
     tmem_ld_32x32b_x32(tb, va);
     tmem_ld_wait();
@@ -911,7 +933,7 @@ __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUten
 __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t lead) {
   const uint16_t pair_mask = static_cast<uint16_t>(0x3u << lead);
   const int npairs = gridDim.x >> 1;
-  constexpr uint32_t idesc = idesc_i8(kPairBM, kPairBN);
+  const uint32_t idesc = p.f8 ? idesc_e4m3(kPairBM, kPairBN) : idesc_i8(kPairBM, kPairBN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
   PairUnit u;
@@ -929,9 +951,14 @@ __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uin
       const uint32_t a0 = smem_addr(s.a[stage]);
       const uint32_t b0 = smem_addr(s.b[stage]);
 #pragma unroll
-      for (int kk = 0; kk < BK / UMMA_K; ++kk)
-        mma_i8_pair(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc,
-                    (kb > kb0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+        if (p.f8)
+          mma_e4m3_pair(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc,
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
+        else
+          mma_i8_pair(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc,
+                      (kb > kb0 || kk > 0) ? 1u : 0u);
+      }
       mma_commit_pair(smem_addr(&s.empty[stage]), pair_mask);
       if (++stage == kPairStages) {
         stage = 0;
@@ -1056,6 +1083,25 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
     uint32_t va[32], vb[32];
     if (tail) {
       tail_slice_epilogue(p, u, region, tb, row, rv, sa, colbase, sws, tmO, box);
+    } else if (p.f8) {
+      // FP8 kind (fp32 accumulator; whole tiles only)
+      auto emit = [&](int ch, const uint32_t(&v)[32]) {
+        if (p.tma_out)
+          store32_tma<true>(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, v);
+        else if (rv)
+          store32_channel<true>(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
+      };
+      tmem_ld_32x32b_x32(tb, va);
+      tmem_ld_wait();
+#pragma unroll
+      for (int ch = 0; ch < 4; ch += 2) {
+        tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
+        emit(ch, va);
+        tmem_ld_wait();
+        if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
+        emit(ch + 1, vb);
+        tmem_ld_wait();
+      }
     } else if (p.tma_out) {
       tmem_ld_32x32b_x32(tb, va);
       tmem_ld_wait();
@@ -1578,7 +1624,9 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
     pl.splits = 1;
     pl.kb_per_split = a.num_kb;
   }
-  if (!allow_split) {
+  if (!allow_split || a.f8) {  // (the FP8 kind runs whole tiles only)
+    pl.splits = 1;
+    pl.kb_per_split = a.num_kb;
     pl.tail_splits = 1;
     pl.dp_tiles = pl.tiles;
   }
@@ -1708,7 +1756,7 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   a.kb_per_split = a.num_kb;
   a.csplit = 0;
   a.tail_splits = 1;
-  if (!group) {
+  if (!group && !a.f8) {  // (the FP8 kind runs whole tiles only)
     const ChannelPlan pl = channel_plan(a.m, a.n, a.k, num_sms, dev);
     if (pl.splits > 1) {
       a.splits = pl.splits;

@@ -295,6 +295,46 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   return r == 0 ? QK_OK : cuda_status(e, "gemm launch");
 }
 
+qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
+                      const float* scale_a, const float* scale_b, float output_scale, void* out,
+                      qk_dtype out_dtype, qk_stream stream) {
+  if (m < 0 || n < 0 || k <= 0 || (k % 16) != 0 || (n % 8) != 0) return QK_ERR_INVALID_ARG;
+  if (out_dtype != QK_F32 && out_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return QK_OK;
+  if (a == nullptr || b == nullptr || scale_a == nullptr || scale_b == nullptr || out == nullptr)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(scale_a, 16) ||
+      !aligned(scale_b, 16))
+    return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  gemm::Args g = {};
+  g.m = m;
+  g.n = n;
+  g.k = k;
+  g.sa = scale_a;
+  g.sw = scale_b;
+  g.alpha = output_scale;
+  g.c = nullptr;
+  g.out = out;
+  g.out_bf16 = out_dtype == QK_BF16;
+  g.splits = 1;
+  g.f8 = 1;
+  cudaError_t e = cudaSuccess;
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int8_t* ai = reinterpret_cast<const int8_t*>(a);
+  const int8_t* bi = reinterpret_cast<const int8_t*>(b);
+  // m <= 128: the 1-SM kernel (rows beyond m read as zero); otherwise the
+  // CTA-pair kernel; whole tiles only
+  const int r = m <= 128 ? gemm::launch(g, ai, bi, false, dev_id, dev->sms, s, &e)
+                         : gemm::launch_pair(g, ai, bi, dev_id, dev->sms, nullptr, s, &e);
+  if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
+  return r == 0 ? QK_OK : cuda_status(e, "fp8 gemm launch");
+}
+
 // The linear layer's workspace: the GEMM's own (offset 0, so its
 // zero-on-return contract covers it), then q [m, k] int8, then the scales.
 namespace {

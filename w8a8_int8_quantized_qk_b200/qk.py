@@ -51,6 +51,8 @@ _SIGNATURES = {
                                                        ctypes.c_int, _P, _P, _P, _P]),
     "qk_w8a8_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
                                     ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "qk_fp8_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_float,
+                                   _P, ctypes.c_int, _P]),
     "qk_w8a8_gemm_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "qk_w8a8_linear": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P,
                                       ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t,
@@ -125,6 +127,10 @@ def qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
                  workspace, workspace_bytes, stream) -> int:
     return lib().qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
                               out_dtype, workspace, workspace_bytes, stream)
+
+
+def qk_fp8_gemm(m, n, k, a, b, scale_a, scale_b, output_scale, out, out_dtype, stream) -> int:
+    return lib().qk_fp8_gemm(m, n, k, a, b, scale_a, scale_b, output_scale, out, out_dtype, stream)
 
 
 def qk_w8a8_gemm_workspace_size(m, n, k, group_k) -> int:
@@ -282,6 +288,19 @@ def w8a8_gemm(a, b, scale_a, scale_b, group_k: int = 0, output_scale: float = 1.
                         0 if workspace is None else workspace.numel(), _stream(stream)),
            "qk_w8a8_gemm")
     return out, c
+
+
+def fp8_gemm(a, b, scale_a, scale_b, output_scale: float = 1.0, out_dtype=None, out=None, stream=None):
+    """a [m, k], b [n, k] e4m3 codes (uint8, CUDA) -> out [m, n] (bf16 by default)."""
+    torch = _torch()
+    _need_cuda(a, b, scale_a, scale_b)
+    m, k = a.shape
+    n = b.shape[0]
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = torch.empty((m, n), dtype=out_dtype, device=a.device) if out is None else out
+    _check(qk_fp8_gemm(m, n, k, _ptr(a), _ptr(b), _ptr(scale_a), _ptr(scale_b), float(output_scale),
+                       _ptr(out), _dtype_code(out), _stream(stream)), "qk_fp8_gemm")
+    return out
 
 
 _workspaces: dict = {}

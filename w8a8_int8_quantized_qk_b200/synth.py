@@ -101,6 +101,14 @@ def int8_uniform(rng: np.random.Generator, shape) -> np.ndarray:
     return rng.integers(-127, 128, size=shape, dtype=np.int8)
 
 
+def e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
+    """Float8 e4m3 codes drawn uniformly from the 254 finite ones (the two NaN
+    codes 0x7F and 0xFF excluded); one byte each."""
+    c = rng.integers(0, 254, size=shape, dtype=np.int64)
+    c = np.where(c >= 0x7F, c + 1, c)  # skip 0x7F
+    return c.astype(np.uint8)
+
+
 def scales_uniform(rng: np.random.Generator, shape, lo: float = 0.001, hi: float = 0.01):
     return rng.uniform(lo, hi, size=shape).astype(np.float32)
 
