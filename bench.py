@@ -313,6 +313,85 @@ def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
     return res
 
 
+class LinearFP8:
+    """The prefill workload's FP8 (e4m3) form, resident in R rotating copies:
+    the activation quantised per token to e4m3 (qk_quantize_per_token_fp8),
+    then the e4m3 x e4m3 GEMM with the per-channel epilogue (qk_fp8_gemm).
+    The weights are synthetic e4m3 codes with per-channel scales."""
+
+    def __init__(self, torch, qk, w, stream):
+        import ctypes
+
+        from w8a8_int8_quantized_qk_b200 import synth
+
+        self.torch, self.qk, self.w = torch, qk, w
+        self.stream = ctypes.c_void_p(stream.cuda_stream)
+        m, n, k = w.m, w.n, w.k
+        r = synth.streams(7, ["w", "sw"])
+        wq = torch.from_numpy(synth.e4m3_codes(r["w"], (n, k))).cuda()
+        self.sw = torch.from_numpy(synth.scales_uniform(r["sw"], (n,))).cuda()
+        per_copy = w.x.nbytes + wq.numel() + m * k + m * n * 2
+        self.R = _copies(per_copy)
+        x0 = _dev(torch, w.x, True)
+        self.xs = [x0.clone() for _ in range(self.R)]
+        self.ws = [wq.clone() for _ in range(self.R)]
+        self.qs = [torch.empty((m, k), dtype=torch.uint8, device="cuda") for _ in range(self.R)]
+        self.sas = [torch.empty((m,), dtype=torch.float32, device="cuda") for _ in range(self.R)]
+        self.outs = [torch.empty((m, n), dtype=torch.bfloat16, device="cuda") for _ in range(self.R)]
+        P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        self.p = [(P(self.xs[j]), P(self.ws[j]), P(self.qs[j]), P(self.sas[j]), P(self.outs[j]))
+                  for j in range(self.R)]
+        self.swp = P(self.sw)
+
+    def quant(self, j: int):
+        w, qk = self.w, self.qk
+        xp, _, qp, sap, _ = self.p[j]
+        st = qk.qk_quantize_per_token_fp8(w.m, w.k, xp, qk.QK_BF16, None, qp, sap, self.stream)
+        if st != 0:
+            raise qk.QKError(st, "quantize fp8")
+
+    def gemm(self, j: int):
+        w, qk = self.w, self.qk
+        _, wp, qp, sap, op = self.p[j]
+        st = qk.qk_fp8_gemm(w.m, w.n, w.k, qp, wp, sap, self.swp, 1.0, op, qk.QK_BF16, self.stream)
+        if st != 0:
+            raise qk.QKError(st, "fp8 gemm")
+
+    def step(self, i: int):
+        j = i % self.R
+        self.quant(j)
+        self.gemm(j)
+
+
+def measure_fp8(torch, qk, iters: int, pk: dict) -> dict:
+    """Stage times of the prefill workload in its FP8 (e4m3) form."""
+    from w8a8_int8_quantized_qk_b200 import synth
+
+    w = synth.make("prefill")
+    L = LinearFP8(torch, qk, w, torch.cuda.current_stream())
+    for i in range(5):
+        L.step(i)
+    torch.cuda.synchronize()
+    quant_us = _graph_us(torch, L, lambda i: L.quant(i % L.R), iters)
+    gemm_us = _graph_us(torch, L, lambda i: L.gemm(i % L.R), iters)
+    step_us = _graph_us(torch, L, lambda i: L.step(i), iters)
+    m, n, k = w.m, w.n, w.k
+    qb = w.x.nbytes + m * k + 4 * m
+    ops = 2.0 * m * n * k
+    res = {"m": m, "n": n, "k": k, "copies": L.R, "timing": f"CUDA graph of {iters} iterations",
+           "quant_kernel": "quantize_per_token_fp8 (e4m3)", "quant_us": quant_us,
+           "quant_GBs": qb / (quant_us * 1e-6) / 1e9,
+           "quant_hbm_frac": qb / (quant_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+           "gemm_kernel": "tcgen05 kind::f8f6f4 (e4m3, fp32 accumulate), CTA pair, whole tiles",
+           "gemm_us": gemm_us, "gemm_TOPS": ops / (gemm_us * 1e-6) / 1e12,
+           "gemm_tensor_frac": ops / (gemm_us * 1e-6) / 1e12 / pk["int8_tops"],
+           "tensor_peak_note": "dense e4m3 peak taken equal to the int8 one (nominal 4.5 PFLOP/s both)",
+           "step_us": step_us}
+    del L
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(seconds: float = 10.0) -> dict:
     """The oracle, as it stands, on a bounded sample of rows of the prefill
     workload: quantise those rows, INT8 GEMM + per-channel epilogue."""
@@ -546,6 +625,7 @@ def run_ours(args):
     if not args.quick:
         for name in ("decode", "prefill", "mlp_down", "group", "tiny"):
             stages[name] = measure_workload(torch, qk, name, args.stage_iters, pk)
+        stages["prefill_fp8"] = measure_fp8(torch, qk, args.stage_iters, pk)
         d = stages["decode"]
         gbs = d["bytes"]["gemm"] / (d["gemm_us"] * 1e-6) / 1e9
         decode = {"value": gbs, "unit": "GB/s", "workload": "decode linear X bf16 [4,4096] x W int8 "
@@ -601,7 +681,7 @@ def main():
                     help="dram__bytes_read.sum + dram__bytes_write.sum of one prefill GEMM launch")
     ap.add_argument("--gemv-traffic", type=float, default=GEMV_TRAFFIC_BYTES,
                     help="the same for one decode GEMV launch")
-    ap.add_argument("--only", choices=["tiny", "decode", "prefill", "mlp_down", "group"],
+    ap.add_argument("--only", choices=["tiny", "decode", "prefill", "mlp_down", "group", "prefill_fp8"],
                     help="profiling aid: time one workload's stages and print them")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
@@ -612,7 +692,8 @@ def main():
 
         from w8a8_int8_quantized_qk_b200 import qk
 
-        res = measure_workload(torch, qk, args.only, args.steps, peaks())
+        res = (measure_fp8(torch, qk, args.steps, peaks()) if args.only == "prefill_fp8"
+               else measure_workload(torch, qk, args.only, args.steps, peaks()))
         print(json.dumps({"only": args.only, **res}), flush=True)
         return 0
     return run_ours(args)
