@@ -25,6 +25,10 @@ Which page each function follows:
 * :func:`quantize_per_token_fp8`, :func:`silu_mul_quant_per_token_fp8` -- the
   vLLM PR's own FP8 form (Purpose/Algorithm: float8_e4m3fn,
   scale = max(absmax, 1e-12) / fp8_max, optionally clamped by scale_ub).
+* :func:`quantize_per_token_asym`, :func:`gemm_s32_asym` -- asymmetric
+  per-token INT8 ("write-int8-quantized-kernel", Inputs: asymmetric maps
+  [-128, 127] to an arbitrary range with a non-zero zero-point) and the
+  GEMM with the zero-point correction.
 * :func:`gemm_fp8` -- the FP8 x FP8 product with the exact accumulator
   (every e4m3 value is an integer multiple of 2^-9) and the per-channel
   epilogue.
@@ -104,6 +108,14 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.qko_silu_mul_quant_per_token_fp8.restype = i32
     lib.qko_gemm_fp8.argtypes = [i32, i32, i32, P, P, P, P, f32, P, P, i32]
     lib.qko_gemm_fp8.restype = i32
+    lib.qko_quantize_row_asym.argtypes = [P, i32, P, P, P]
+    lib.qko_quantize_row_asym.restype = None
+    lib.qko_quantize_per_token_asym.argtypes = [i32, i32, P, i32, P, P, P]
+    lib.qko_quantize_per_token_asym.restype = i32
+    lib.qko_weight_row_sums.argtypes = [i32, i32, P, P]
+    lib.qko_weight_row_sums.restype = i32
+    lib.qko_gemm_s32_asym.argtypes = [i32, i32, i32, P, P, P, P]
+    lib.qko_gemm_s32_asym.restype = i32
     return lib
 
 
@@ -328,3 +340,39 @@ class Oracle:
     def linear_fp8_from_q(self, q, sa, w_q, sw, alpha: float = 1.0):
         acc, out = self.gemm_fp8(q, w_q, sa, sw, alpha)
         return {"q": q, "sa": sa, "acc": acc, "out_f32": out, "out_bf16": self.f32_to_bf16(out)}
+
+    # -- asymmetric per-token INT8 --------------------------------------------
+    def quantize_per_token_asym(self, x: np.ndarray):
+        """x [m, k] -> (q int8 [m, k], scale float32 [m], zero-point int32 [m])."""
+        x = np.ascontiguousarray(x)
+        m, k = x.shape
+        q = np.empty((m, k), np.int8)
+        s = np.empty((m,), np.float32)
+        z = np.empty((m,), np.int32)
+        _check(self.lib.qko_quantize_per_token_asym(m, k, _ptr(x), _dtype_code(x), _ptr(q), _ptr(s),
+                                                    _ptr(z)), "quantize_per_token_asym")
+        return q, s, z
+
+    def weight_row_sums(self, w: np.ndarray) -> np.ndarray:
+        w = np.ascontiguousarray(w, np.int8)
+        n, k = w.shape
+        out = np.empty((n,), np.int32)
+        _check(self.lib.qko_weight_row_sums(n, k, _ptr(w), _ptr(out)), "weight_row_sums")
+        return out
+
+    def gemm_s32_asym(self, a: np.ndarray, zp: np.ndarray, w: np.ndarray) -> np.ndarray:
+        """sum_k (a[m, k] - zp[m]) * w[n, k] -> int32 [m, n]."""
+        a = np.ascontiguousarray(a, np.int8)
+        zp = np.ascontiguousarray(zp, np.int32)
+        w = np.ascontiguousarray(w, np.int8)
+        m, k = a.shape
+        n = w.shape[0]
+        acc = np.empty((m, n), np.int32)
+        _check(self.lib.qko_gemm_s32_asym(m, n, k, _ptr(a), _ptr(zp), _ptr(w), _ptr(acc)),
+               "gemm_s32_asym")
+        return acc
+
+    def linear_asym_from_q(self, q, sa, zp, w_q, sw, alpha: float = 1.0):
+        acc = self.gemm_s32_asym(q, zp, w_q)
+        out = self.epilogue_per_channel(acc, sa, sw, alpha)
+        return {"acc": acc, "out_f32": out, "out_bf16": self.f32_to_bf16(out)}

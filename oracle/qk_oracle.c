@@ -52,6 +52,16 @@
  *    are integer multiples of 2^-18 and the sum is exact in int64), rounded
  *    once to fp32; the epilogue is the per-channel one above.
  *
+ * Asymmetric per-token INT8 ("write-int8-quantized-kernel", Inputs the agent
+ * should gather first: asymmetric quantisation maps [-128, 127] to an
+ * arbitrary range with a non-zero zero-point):
+ *  - the row's range [lo, hi] is widened to hold 0 (so the zero-point is
+ *    representable); scale = max(hi - lo, 1e-12f) / 255, inv = 1 / scale;
+ *  - zp = clamp(rne(-128 - lo * inv), -128, 127);
+ *    q = clamp(rne(x * inv) + zp, -128, 127), x ~ (q - zp) * scale;
+ *  - the GEMM's accumulator is sum_k (q - zp) * w = acc - zp * wsum[n],
+ *    wsum[n] = sum_k w[n][k]; the epilogue is the per-channel one.
+ *
  * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread (no fast-math),
  * so every float operation below is a single IEEE binary32 RN operation.
  *
@@ -522,4 +532,78 @@ int qko_gemm_fp8(int m, int n, int k, const uint8_t* a, const uint8_t* w, const 
   free(jobs);
   free(th);
   return QKO_OK;
+}
+
+/* ----------------------------------------------------------------------- */
+/* Asymmetric per-token INT8 ("write-int8-quantized-kernel", Inputs:        */
+/* asymmetric maps [-128, 127] to an arbitrary range with a non-zero        */
+/* zero-point, which adds arithmetic to the hot loop).                      */
+/* ----------------------------------------------------------------------- */
+
+/* One row: lo = min(min x, 0), hi = max(max x, 0) (the range holds zero, so
+ * the zero-point lies in [-128, 127]); scale = max(hi - lo, 1e-12f) / 255;
+ * inv = 1 / scale; zp = clamp(round_half_even(-128 - lo * inv), -128, 127);
+ * q = clamp(round_half_even(x * inv) + zp, -128, 127); x ~ (q - zp) * scale. */
+void qko_quantize_row_asym(const float* x, int k, int8_t* q, float* scale, int32_t* zp) {
+  float lo = 0.0f, hi = 0.0f;
+  for (int i = 0; i < k; ++i) {
+    if (x[i] < lo) lo = x[i];
+    if (x[i] > hi) hi = x[i];
+  }
+  const float s = fmaxf(hi - lo, 1e-12f) / 255.0f;
+  const float inv = 1.0f / s;
+  float z = nearbyintf(-128.0f - lo * inv);
+  if (z < -128.0f) z = -128.0f;
+  if (z > 127.0f) z = 127.0f;
+  for (int i = 0; i < k; ++i) {
+    float r = nearbyintf(x[i] * inv) + z;
+    if (r > 127.0f) r = 127.0f;
+    if (r < -128.0f) r = -128.0f;
+    q[i] = (int8_t)(int)r;
+  }
+  *scale = s;
+  *zp = (int32_t)z;
+}
+
+int qko_quantize_per_token_asym(int m, int k, const void* x, int dtype, int8_t* q, float* scale,
+                                int32_t* zp) {
+  if (m < 0 || k <= 0 || (dtype != QKO_F32 && dtype != QKO_BF16)) return QKO_ERR_ARG;
+  float* row = (float*)malloc(sizeof(float) * (size_t)k);
+  if (!row) return QKO_ERR_ARG;
+  for (int r = 0; r < m; ++r) {
+    for (int i = 0; i < k; ++i) row[i] = qko_load(x, dtype, (int64_t)r * k + i);
+    qko_quantize_row_asym(row, k, q + (int64_t)r * k, scale + r, zp + r);
+  }
+  free(row);
+  return QKO_OK;
+}
+
+/* wsum[n] = sum_k w[n][k] (int64, checked against the int32 range). */
+int qko_weight_row_sums(int n, int k, const int8_t* w, int32_t* wsum) {
+  if (n < 0 || k <= 0) return QKO_ERR_ARG;
+  for (int c = 0; c < n; ++c) {
+    int64_t t = 0;
+    for (int i = 0; i < k; ++i) t += w[(int64_t)c * k + i];
+    if (t > INT32_MAX || t < INT32_MIN) return QKO_ERR_OVERFLOW;
+    wsum[c] = (int32_t)t;
+  }
+  return QKO_OK;
+}
+
+/* acc[m][n] = sum_k (a[m][k] - zp[m]) * w[n][k], in int64, checked against
+ * the int32 range; it equals the plain sum minus zp[m] * wsum[n]. */
+int qko_gemm_s32_asym(int m, int n, int k, const int8_t* a, const int32_t* zp, const int8_t* w,
+                      int32_t* acc) {
+  if (m < 0 || n < 0 || k <= 0) return QKO_ERR_ARG;
+  int overflow = 0;
+  for (int r = 0; r < m; ++r) {
+    for (int c = 0; c < n; ++c) {
+      int64_t s = 0;
+      for (int i = 0; i < k; ++i)
+        s += ((int64_t)a[(int64_t)r * k + i] - zp[r]) * (int64_t)w[(int64_t)c * k + i];
+      if (s > INT32_MAX || s < INT32_MIN) overflow = 1;
+      acc[(int64_t)r * n + c] = (int32_t)s;
+    }
+  }
+  return overflow ? QKO_ERR_OVERFLOW : QKO_OK;
 }

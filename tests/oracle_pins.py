@@ -32,6 +32,10 @@ What pins what:
                        scale_ub clamp; a hand-worked row.
 * FP8 GEMM          -- numpy float64 matmul of the decoded operands (exact
                        at these sizes); closed forms (all-448 operands).
+* asymmetric INT8   -- hand-worked rows with scale 1 (q = x - 128, ties to
+                       even); zero-point and extreme-element invariants;
+                       round-trip bound; numpy int64 brute force of the
+                       zero-point GEMM and of the weight row sums.
 """
 from __future__ import annotations
 
@@ -398,7 +402,51 @@ def pin_fp8_gemm(O) -> None:
                              [-k * 448.0 ** 2 / 2, -k * 448.0 ** 2, -k * 448.0 ** 2 / 8]]
 
 
+# --------------------------------------------------------------------------- asymmetric INT8
+def pin_asym_quant(O) -> None:
+    # range [0, 255]: scale 1, inv 1, zp -128, q = rne(x) - 128
+    row = np.float32([[0.0, 1.0, 127.0, 128.0, 255.0, 2.5, 3.5, 200.4]])
+    q, s, z = O.quantize_per_token_asym(row)
+    assert s.tolist() == [1.0] and z.tolist() == [-128]
+    assert q.tolist() == [[-128, -127, -1, 0, 127, -126, -124, 72]], q.tolist()
+    # range [-255, 0]: scale 1, zp = 127, q = rne(x) + 127
+    q2, s2, z2 = O.quantize_per_token_asym(np.float32([[-255.0, -100.0, 0.0, -0.5]]))
+    assert s2.tolist() == [1.0] and z2.tolist() == [127]
+    assert q2.tolist() == [[-128, 27, 127, 127]], q2.tolist()
+    # random rows: invariants
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((6, 301)).astype(np.float32)
+    x[1] = np.abs(x[1]) + 0.5  # all positive: lo widened to 0
+    x[2] = -np.abs(x[2]) * 9   # all negative
+    x[3] = 0.0
+    x[4, 10] = 40.0
+    q, s, z = O.quantize_per_token_asym(x)
+    x64 = x.astype(np.float64)
+    for r in range(x.shape[0]):
+        lo = min(float(x64[r].min()), 0.0)
+        hi = max(float(x64[r].max()), 0.0)
+        sc = float(s[r])
+        assert abs(sc * 255.0 - max(hi - lo, float(np.float32(1e-12)))) <= 255.0 * ulp32(sc)
+        assert -128 <= int(z[r]) <= 127
+        deq = (q[r].astype(np.float64) - float(z[r])) * sc
+        assert float(np.abs(deq - x64[r]).max()) <= sc * (0.5 + 2.0 ** -12) + 1e-30
+        if hi > lo:
+            assert abs(int(q[r, int(np.argmin(x64[r]))]) + 128) <= 1 or lo == 0.0
+            assert abs(int(q[r, int(np.argmax(x64[r]))]) - 127) <= 1 or hi == 0.0
+    assert np.all(q[3] == -128) and z[3] == -128
+
+
+def pin_asym_gemm(O) -> None:
+    rng = np.random.default_rng(22)
+    a = rng.integers(-128, 128, (6, 333)).astype(np.int8)
+    zp = rng.integers(-128, 128, (6,)).astype(np.int32)
+    w = rng.integers(-127, 128, (9, 333)).astype(np.int8)
+    ref = (a.astype(np.int64) - zp[:, None].astype(np.int64)) @ w.astype(np.int64).T
+    assert np.array_equal(O.gemm_s32_asym(a, zp, w), ref)
+    assert np.array_equal(O.weight_row_sums(w), w.astype(np.int64).sum(axis=1))
+
+
 ALL_PINS = [pin_exp, pin_silu, pin_bf16_rounding, pin_quant_golden, pin_quant_invariants,
             pin_quant_bf16_path, pin_silu_quant, pin_gemm_bruteforce, pin_gemm_closed_forms,
             pin_epilogue_per_channel, pin_group, pin_linear_golden, pin_e4m3_codec, pin_fp8_quant,
-            pin_fp8_silu_quant, pin_fp8_gemm]
+            pin_fp8_silu_quant, pin_fp8_gemm, pin_asym_quant, pin_asym_gemm]

@@ -56,6 +56,16 @@ MUTANTS = [
     ("fp8_clamp_240", "if (y > 448.0f) y = 448.0f;", "if (y > 240.0f) y = 240.0f;"),
     ("fp8_silu_up_from_gate", "float uv = qko_load(up, dtype, (int64_t)r * ld + i);",
      "float uv = qko_load(gate, dtype, (int64_t)r * ld + i);"),
+    ("asym_ties_away", "float r = nearbyintf(x[i] * inv) + z;", "float r = roundf(x[i] * inv) + z;"),
+    ("asym_range_without_zero", "float lo = 0.0f, hi = 0.0f;", "float lo = x[0], hi = x[0];"),
+    ("asym_qrange_256", "const float s = fmaxf(hi - lo, 1e-12f) / 255.0f;",
+     "const float s = fmaxf(hi - lo, 1e-12f) / 256.0f;"),
+    ("asym_zp_sign", "float z = nearbyintf(-128.0f - lo * inv);", "float z = nearbyintf(-128.0f + lo * inv);"),
+    ("asym_clamp_127", "if (r < -128.0f) r = -128.0f;", "if (r < -127.0f) r = -127.0f;"),
+    ("asym_gemm_zp_ignored", "s += ((int64_t)a[(int64_t)r * k + i] - zp[r]) * (int64_t)w[(int64_t)c * k + i];",
+     "s += ((int64_t)a[(int64_t)r * k + i]) * (int64_t)w[(int64_t)c * k + i];"),
+    ("asym_wsum_dropped", "for (int i = 0; i < k; ++i) t += w[(int64_t)c * k + i];",
+     "for (int i = 1; i < k; ++i) t += w[(int64_t)c * k + i];"),
     ("fp8_gemm_units", ": (int64_t)(8 + m) << (e - 1);", ": (int64_t)(8 + m) << e;"),
     ("fp8_gemm_dropped_term", "for (int i = 0; i < j->k; ++i) s += qko_e4m3_units(ar[i]) * qko_e4m3_units(wr[i]);",
      "for (int i = 1; i < j->k; ++i) s += qko_e4m3_units(ar[i]) * qko_e4m3_units(wr[i]);"),
