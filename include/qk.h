@@ -50,7 +50,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 3
+#define QK_ABI_VERSION 4
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -240,6 +240,42 @@ QK_API qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t
 QK_API qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
                              const float* scale_a, const float* scale_b, float output_scale,
                              void* out, qk_dtype out_dtype, qk_stream stream);
+
+/*
+ * Asymmetric per-token INT8 ("write-int8-quantized-kernel", Inputs the agent
+ * should gather first: asymmetric quantisation maps [-128, 127] to an
+ * arbitrary range with a non-zero zero-point; the zero-point adds
+ * arithmetic to the hot loop).
+ *
+ * qk_quantize_per_token_asym: per row, the range [lo, hi] = [min(min x, 0),
+ * max(max x, 0)]; scale = max(hi - lo, 1e-12f) / 255; inv = 1 / scale;
+ * zero_point = clamp(rne(-128 - lo * inv), -128, 127);
+ * q = clamp(rne(x * inv) + zero_point, -128, 127), so x ~ (q - zp) * scale.
+ *   x [m, k] (QK_BF16 / QK_F32, 16-B aligned, k % 16 == 0); q [m, k] int8
+ *   (16-B aligned); scale [m] fp32; zero_point [m] int32.
+ *
+ * qk_weight_row_sums: wsum[r] = sum_k w[r][k] (int32), the term the
+ *   zero-point correction needs; computed once per weight.  w [n, k] int8,
+ *   16-B aligned, k % 16 == 0.
+ *
+ * qk_w8a8_gemm_asym: qk_w8a8_gemm (per channel, group_k 0) for asymmetric
+ *   activations: acc = sum_k (a[m][k] - zero_point_a[m]) * b[n][k], formed
+ *   as the tensor-core sum minus zero_point_a[m] * wsum_b[n]; the epilogue
+ *   and c as qk_w8a8_gemm.  wsum_b [n] int32 (16-B aligned) from
+ *   qk_weight_row_sums.  k <= 66311, so that k * 255 * 127 < 2^31 (else
+ *   QK_ERR_OVERFLOW_BOUND).  Workspace as qk_w8a8_gemm.
+ */
+QK_API qk_status qk_quantize_per_token_asym(int m, int k, const void* x, qk_dtype x_dtype,
+                                            int8_t* q, float* scale, int32_t* zero_point,
+                                            qk_stream stream);
+QK_API qk_status qk_weight_row_sums(int n, int k, const int8_t* w, int32_t* wsum,
+                                    qk_stream stream);
+QK_API qk_status qk_w8a8_gemm_asym(int m, int n, int k, const int8_t* a,
+                                   const int32_t* zero_point_a, const int8_t* b,
+                                   const int32_t* wsum_b, const float* scale_a,
+                                   const float* scale_b, float output_scale, int32_t* c,
+                                   void* out, qk_dtype out_dtype, void* workspace,
+                                   size_t workspace_bytes, qk_stream stream);
 
 /* Bytes of workspace qk_w8a8_gemm needs for this problem on the current
  * device (0 when none; the split depends on the device's SM count).

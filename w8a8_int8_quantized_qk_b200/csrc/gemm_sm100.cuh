@@ -77,6 +77,10 @@ struct Args {
   // 1: a and b are float8 e4m3 codes, the MMA is kind::f8f6f4 and the
   // accumulator fp32 (channel and pair kernels, whole tiles only, no c)
   int f8;
+  // asymmetric activations (per channel only): zp [m] zero-points and wsum
+  // [n] = sum_k b[n][k]; the epilogues use acc - zp[m] * wsum[n]
+  const int32_t* zp;
+  const int32_t* wsum;
 };
 
 template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
@@ -147,10 +151,10 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
 // ---------------------------------------------------------------- MMA issuer
 // GROUP: one accumulator buffer per K block (each K block is one group);
 // otherwise one buffer per tile.
-template <int BN, int STAGES, int NACC, bool GROUP, class S>
+template <int BN, int STAGES, int NACC, bool GROUP, bool F8 = false, class S>
 __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
-  const uint32_t idesc = p.f8 ? idesc_e4m3(BM, BN) : idesc_i8(BM, BN);
+  constexpr uint32_t idesc = F8 ? idesc_e4m3(BM, BN) : idesc_i8(BM, BN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
   for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
@@ -179,7 +183,7 @@ __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
 #pragma unroll
       for (int kk = 0; kk < BK / UMMA_K; ++kk) {
         const uint32_t acc = GROUP ? (kk > 0) : (kb > kb0 || kk > 0);
-        if (!GROUP && p.f8)
+        if constexpr (F8)
           mma_e4m3(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc, acc);
         else
           mma_i8(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc, acc);
@@ -257,6 +261,24 @@ template <bool F8>
 __device__ __forceinline__ float acc_value(uint32_t v) {
   if constexpr (F8) return __uint_as_float(v);
   return __int2float_rn(static_cast<int>(v));
+}
+
+// Zero-point correction of 32 int32 accumulators of one row (columns col0 ..
+// col0 + 31): v -= zp[row] * wsum[col], in two's-complement arithmetic
+// (exact whenever the corrected sum fits in int32, which the host's bound
+// on k guarantees).  Rows >= m and columns >= n (n % 8 == 0) take 0.
+__device__ __forceinline__ void apply_zp(const Args& p, int row, int col0, uint32_t (&v)[32]) {
+  const uint32_t z = row < p.m ? static_cast<uint32_t>(__ldg(p.zp + row)) : 0u;
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const int col = col0 + g * 4;
+    const int4 w4 = col < p.n ? __ldg(reinterpret_cast<const int4*>(p.wsum + col))
+                              : make_int4(0, 0, 0, 0);
+    v[g * 4 + 0] -= z * static_cast<uint32_t>(w4.x);
+    v[g * 4 + 1] -= z * static_cast<uint32_t>(w4.y);
+    v[g * 4 + 2] -= z * static_cast<uint32_t>(w4.z);
+    v[g * 4 + 3] -= z * static_cast<uint32_t>(w4.w);
+  }
 }
 
 // 32 outputs of one row (columns col0 .. col0 + 31) from 32 accumulators;
@@ -346,7 +368,7 @@ __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tm
 // row's token scale; the 32-column TMEM loads are double-buffered so the
 // next load is in flight while the current chunk is converted and stored.
 // bf16 output without c leaves through TMA stores (store32_tma).
-template <int BN, int NACC, class S>
+template <int BN, int NACC, bool F8 = false, class S>
 __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUtensorMap* tmO) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int lane = threadIdx.x & 31;
@@ -397,16 +419,18 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
       if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[abuf]));
       break;  // one unit per CTA
     }
-    auto emit = [&](int ch, const uint32_t(&v)[32]) {
-      if (p.f8) {
+    auto emit = [&](int ch, uint32_t(&v)[32]) {
+      if constexpr (F8) {
         if (p.tma_out)
           store32_tma<true>(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
         else if (rv)
           store32_channel<true>(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
-      } else if (p.tma_out) {
-        store32_tma(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
-      } else if (rv) {
-        store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
+      } else {
+        if (p.zp) apply_zp(p, row, colbase + ch * 32, v);
+        if (p.tma_out)
+          store32_tma(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
+        else if (rv)
+          store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
       }
     };
     tmem_ld_32x32b_x32(tb, va);
@@ -723,6 +747,7 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
         va[q4 * 4 + 2] += t4[o][q4].z;
         va[q4 * 4 + 3] += t4[o][q4].w;
       }
+    if (p.zp) apply_zp(p, row, col0, va);
     if (p.tma_out)
       store32_tma(p, tmO, box, row0, col0, sa, sws + c * 32, va);
     else if (rv && col0 < p.n)
@@ -751,6 +776,7 @@ struct alignas(1024) ChannelStorage {
   int abort;
 };
 
+template <bool F8>
 __global__ void __launch_bounds__(kChannelThreads, 1)
     gemm_i8_channel_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
@@ -771,10 +797,10 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
     if (lane == 0) produce<kChannelBN, kChannelStages>(s, &tmA, &tmB, p);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false>(s, tmem, p);
+    if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false, F8>(s, tmem, p);
     __syncwarp();
   } else {
-    epilogue_channel<kChannelBN, 2>(s, tmem, p, &tmO);
+    epilogue_channel<kChannelBN, 2, F8>(s, tmem, p, &tmO);
   }
   if (p.csplit) {
     cluster_sync_all();  // every CTA of the cluster has staged its partial
@@ -930,10 +956,11 @@ __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUten
   }
 }
 
+template <bool F8>
 __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t lead) {
   const uint16_t pair_mask = static_cast<uint16_t>(0x3u << lead);
   const int npairs = gridDim.x >> 1;
-  const uint32_t idesc = p.f8 ? idesc_e4m3(kPairBM, kPairBN) : idesc_i8(kPairBM, kPairBN);
+  constexpr uint32_t idesc = F8 ? idesc_e4m3(kPairBM, kPairBN) : idesc_i8(kPairBM, kPairBN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
   PairUnit u;
@@ -952,7 +979,7 @@ __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uin
       const uint32_t b0 = smem_addr(s.b[stage]);
 #pragma unroll
       for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-        if (p.f8)
+        if constexpr (F8)
           mma_e4m3_pair(d, sdesc_k_sw128(a0 + kk * UMMA_K), sdesc_k_sw128(b0 + kk * UMMA_K), idesc,
                         (kb > kb0 || kk > 0) ? 1u : 0u);
         else
@@ -1034,6 +1061,7 @@ __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region
         va[q4 * 4 + 3] += t4[q4].w;
       }
     }
+    if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
     if (p.tma_out)
       store32_tma(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
     else if (rv)
@@ -1049,6 +1077,7 @@ __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region
 // token scale is fetched before the accumulator is ready, and the four
 // 32-column TMEM loads are double-buffered so the next load is in flight
 // while the current chunk is converted and stored.
+template <bool F8>
 __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t pr,
                               uint32_t lead, const CUtensorMap* tmO) {
   const int npairs = gridDim.x >> 1;
@@ -1083,7 +1112,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
     uint32_t va[32], vb[32];
     if (tail) {
       tail_slice_epilogue(p, u, region, tb, row, rv, sa, colbase, sws, tmO, box);
-    } else if (p.f8) {
+    } else if constexpr (F8) {
       // FP8 kind (fp32 accumulator; whole tiles only)
       auto emit = [&](int ch, const uint32_t(&v)[32]) {
         if (p.tma_out)
@@ -1108,9 +1137,11 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
 #pragma unroll
       for (int ch = 0; ch < 4; ch += 2) {
         tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
+        if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
         store32_tma(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
         tmem_ld_wait();
         if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
+        if (p.zp) apply_zp(p, row, colbase + (ch + 1) * 32, vb);
         store32_tma(p, tmO, box, row - lane, colbase + (ch + 1) * 32, sa, sws + (ch + 1) * 32, vb);
         tmem_ld_wait();
       }
@@ -1120,9 +1151,11 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
 #pragma unroll
       for (int ch = 0; ch < 4; ch += 2) {
         tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
+        if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
         if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
         tmem_ld_wait();
         if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
+        if (p.zp) apply_zp(p, row, colbase + (ch + 1) * 32, vb);
         if (rv) store32_channel(p, row, colbase + (ch + 1) * 32, sa, sws + (ch + 1) * 32, vb);
         tmem_ld_wait();
       }
@@ -1193,6 +1226,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
             va[q4 * 4 + 3] = t4[q4].w;
             __stcg(reinterpret_cast<int4*>(acc_region + ((ch * 8 + q4) * 32 + lane) * 4), zero);
           }
+          if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
           if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
         }
         if (lane == 0) p.cnt[tile * 16 + region] = 0;  // ready for the next call
@@ -1282,10 +1316,12 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
         va[q4 * 4 + 3] += t4[o][q4].w;
       }
     const int col0 = tn * kPairBN + c * 32;
+    if (p.zp) apply_zp(p, row, col0, va);
     if (rv && col0 < p.n) store32_channel(p, row, col0, sa, sws + t * 32, va);
   }
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -1328,10 +1364,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     if (lane == 0) produce_pair(s, &tmA, &tmB, p, pr, lead);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && pr == 0) mma_issue_pair(s, tmem, p, lead);
+    if (lane == 0 && pr == 0) mma_issue_pair<F8>(s, tmem, p, lead);
     __syncwarp();
   } else {
-    epilogue_pair(s, tmem, p, pr, lead, &tmO);
+    epilogue_pair<F8>(s, tmem, p, pr, lead, &tmO);
   }
   if (p.csplit) {
     if (warp >= 2) cluster_reduce_scales(s, p, crank);
@@ -1435,7 +1471,7 @@ inline bool cached_tmap(CUtensorMap* map, const void* base, int rows, int k, int
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel).
 template <class K>
 inline cudaError_t set_smem_once(K kernel, int dev, int slot, size_t bytes) {
-  static std::atomic<unsigned long long> done[4] = {};
+  static std::atomic<unsigned long long> done[6] = {};
   const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
   if (bit && (done[slot].load(std::memory_order_acquire) & bit)) return cudaSuccess;
   const cudaError_t e =
@@ -1466,9 +1502,9 @@ inline int max_pair_clusters(int dev, int cluster) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(gemm_i8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(gemm_i8_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(pair_smem())) != cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, gemm_i8_pair_kernel, &cfg) != cudaSuccess) {
+      cudaOccupancyMaxActiveClusters(&n, gemm_i8_pair_kernel<false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -1493,9 +1529,9 @@ inline int max_pairs(int dev, int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(gemm_i8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(gemm_i8_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(pair_smem())) == cudaSuccess &&
-      cudaOccupancyMaxActiveClusters(&n, gemm_i8_pair_kernel, &cfg) == cudaSuccess && n > 0)
+      cudaOccupancyMaxActiveClusters(&n, gemm_i8_pair_kernel<false>, &cfg) == cudaSuccess && n > 0)
     pairs = n < pairs ? n : pairs;
   else
     cudaGetLastError();
@@ -1656,12 +1692,14 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
   }
   const int ntiles = a.tiles_m * a.tiles_n * a.splits;  // > pairs whenever the tail split is on
   const int grid_pairs = ntiles < pairs ? ntiles : pairs;
-  cudaError_t e = set_smem_once(gemm_i8_pair_kernel, dev, 0, pair_smem());
+  cudaError_t e = a.f8 ? set_smem_once(gemm_i8_pair_kernel<true>, dev, 4, pair_smem())
+                       : set_smem_once(gemm_i8_pair_kernel<false>, dev, 0, pair_smem());
   if (e == cudaSuccess) {
     // cluster: one pair, or (cluster split-K) the splits pairs of one tile;
     // the grid is then exactly tiles x splits pairs, one unit each
     const unsigned cluster = pl.csplit ? 2u * static_cast<unsigned>(pl.splits) : 2u;
-    e = launch_pdl(gemm_i8_pair_kernel, dim3(2 * grid_pairs), dim3(kPairThreads), pair_smem(), stream,
+    e = launch_pdl(a.f8 ? gemm_i8_pair_kernel<true> : gemm_i8_pair_kernel<false>, dim3(2 * grid_pairs),
+                   dim3(kPairThreads), pair_smem(), stream,
                    cluster, ta, tb, to, a);
   }
   *err = e;
@@ -1688,9 +1726,9 @@ inline int max_channel_clusters(int dev, int cluster) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(gemm_i8_channel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(gemm_i8_channel_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(channel_smem())) != cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, gemm_i8_channel_kernel, &cfg) != cudaSuccess) {
+      cudaOccupancyMaxActiveClusters(&n, gemm_i8_channel_kernel<false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -1779,9 +1817,11 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   cudaError_t e;
   if (!group) {
     const size_t smem = channel_smem();
-    e = set_smem_once(gemm_i8_channel_kernel, dev, 1, smem);
+    e = a.f8 ? set_smem_once(gemm_i8_channel_kernel<true>, dev, 5, smem)
+             : set_smem_once(gemm_i8_channel_kernel<false>, dev, 1, smem);
     if (e == cudaSuccess) {
-      e = launch_pdl(gemm_i8_channel_kernel, dim3(grid), dim3(kChannelThreads), smem, stream,
+      e = launch_pdl(a.f8 ? gemm_i8_channel_kernel<true> : gemm_i8_channel_kernel<false>, dim3(grid),
+                     dim3(kChannelThreads), smem, stream,
                      a.csplit ? static_cast<unsigned>(a.splits) : 1u, ta, tb, to, a);
     }
   } else {

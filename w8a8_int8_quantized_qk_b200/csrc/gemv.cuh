@@ -32,7 +32,19 @@ struct Args {
   int32_t* c;       // [m, n] or null
   void* out;        // [m, n] or null
   int out_bf16;
+  // asymmetric activations: zp [m] zero-points and wsum [n] = sum_k w[n][k];
+  // the epilogue uses acc - zp[t] * wsum[row] (null: symmetric)
+  const int32_t* zp;
+  const int32_t* wsum;
 };
+
+// acc - zp * wsum in two's-complement arithmetic (exact when the corrected
+// sum fits in int32, which the host's bound on k guarantees)
+__device__ __forceinline__ int zp_correct(const Args& p, int acc, int t, int row) {
+  if (p.zp == nullptr) return acc;
+  return static_cast<int>(static_cast<uint32_t>(acc) -
+                          static_cast<uint32_t>(p.zp[t]) * static_cast<uint32_t>(p.wsum[row]));
+}
 
 __device__ __forceinline__ int dot16(const uint4& w, const uint4& a, int acc) {
   acc = __dp4a(static_cast<int>(w.x), static_cast<int>(a.x), acc);
@@ -93,6 +105,7 @@ __global__ void __launch_bounds__(kThreads) gemv_i8_kernel(Args p) {
         int s = 0;
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) s += red[w][threadIdx.x];
+        s = zp_correct(p, s, t, row);
         const int64_t o = static_cast<int64_t>(t) * p.n + row;
         if (p.c) p.c[o] = s;
         if (p.out) {
@@ -233,6 +246,7 @@ __global__ void __launch_bounds__(kPrefThreads, PrefCfg<MT, J>::minb)
       int sum = 0;
 #pragma unroll
       for (int w = 0; w < kPrefThreads / 32; ++w) sum += red[w][tid];
+      sum = zp_correct(p, sum, my_t, my_row);
       const int64_t o = static_cast<int64_t>(my_t) * p.n + my_row;
       if (p.c) p.c[o] = sum;
       if (p.out) {

@@ -71,6 +71,8 @@ inline bool aligned(const void* p, uintptr_t a) {
 
 // K * 127^2 < 2^31  <=>  K <= 133144
 constexpr int kMaxK = 133144;
+// asymmetric activations: |q - zp| <= 255, so k * 255 * 127 < 2^31
+constexpr int kMaxKAsym = 66311;
 
 qk_status quant_common(int m, int k, const void* x, const void* up, int64_t ld, qk_dtype dt,
                        int8_t* q, float* scale, qk_stream stream, bool silu, bool fp8 = false,
@@ -231,10 +233,78 @@ size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
   return pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_bytes(pl) : 0;
 }
 
+namespace {
+// The GEMM of qk_w8a8_gemm, and of qk_w8a8_gemm_asym when zp / wsum are
+// given (per channel only; the caller has checked them).
+qk_status gemm_common(int m, int n, int k, const int8_t* a, const int8_t* b,
+                      const float* scale_a, const float* scale_b, int group_k,
+                      float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
+                      void* workspace, size_t workspace_bytes, qk_stream stream,
+                      const int32_t* zp, const int32_t* wsum);
+}  // namespace
+
 qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
                        const float* scale_a, const float* scale_b, int group_k,
                        float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
                        void* workspace, size_t workspace_bytes, qk_stream stream) {
+  return gemm_common(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
+                     workspace, workspace_bytes, stream, nullptr, nullptr);
+}
+
+qk_status qk_w8a8_gemm_asym(int m, int n, int k, const int8_t* a, const int32_t* zero_point_a,
+                            const int8_t* b, const int32_t* wsum_b, const float* scale_a,
+                            const float* scale_b, float output_scale, int32_t* c, void* out,
+                            qk_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                            qk_stream stream) {
+  if (k > kMaxKAsym) return QK_ERR_OVERFLOW_BOUND;
+  if (m > 0 && n > 0 && (zero_point_a == nullptr || wsum_b == nullptr)) return QK_ERR_INVALID_ARG;
+  if (!aligned(zero_point_a, 4) || !aligned(wsum_b, 16)) return QK_ERR_MISALIGNED;
+  return gemm_common(m, n, k, a, b, scale_a, scale_b, 0, output_scale, c, out, out_dtype,
+                     workspace, workspace_bytes, stream, zero_point_a, wsum_b);
+}
+
+qk_status qk_quantize_per_token_asym(int m, int k, const void* x, qk_dtype x_dtype, int8_t* q,
+                                     float* scale, int32_t* zero_point, qk_stream stream) {
+  if (m < 0 || k <= 0 || (k % 16) != 0) return QK_ERR_INVALID_ARG;
+  if (x_dtype != QK_F32 && x_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (m == 0) return QK_OK;
+  if (x == nullptr || q == nullptr || scale == nullptr || zero_point == nullptr)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale, 4) || !aligned(zero_point, 4))
+    return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  quant::AsymArgs a;
+  a.m = m;
+  a.k = k;
+  a.x = x;
+  a.q = q;
+  a.scale = scale;
+  a.zp = zero_point;
+  return cuda_status(quant::launch_asym(a, x_dtype == QK_BF16, reinterpret_cast<cudaStream_t>(stream)),
+                     "asymmetric quantize launch");
+}
+
+qk_status qk_weight_row_sums(int n, int k, const int8_t* w, int32_t* wsum, qk_stream stream) {
+  if (n < 0 || k <= 0 || (k % 16) != 0) return QK_ERR_INVALID_ARG;
+  if (k > kMaxK) return QK_ERR_OVERFLOW_BOUND;
+  if (n == 0) return QK_OK;
+  if (w == nullptr || wsum == nullptr) return QK_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(wsum, 4)) return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  return cuda_status(quant::launch_weight_row_sums(n, k, w, wsum, reinterpret_cast<cudaStream_t>(stream)),
+                     "weight row sums launch");
+}
+
+namespace {
+qk_status gemm_common(int m, int n, int k, const int8_t* a, const int8_t* b,
+                      const float* scale_a, const float* scale_b, int group_k,
+                      float output_scale, int32_t* c, void* out, qk_dtype out_dtype,
+                      void* workspace, size_t workspace_bytes, qk_stream stream,
+                      const int32_t* zp, const int32_t* wsum) {
   qk_status st = gemm_check(m, n, k, group_k);
   if (st != QK_OK) return st;
   if (out != nullptr && out_dtype != QK_F32 && out_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
@@ -265,6 +335,8 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
     g.c = c;
     g.out = out;
     g.out_bf16 = out_dtype == QK_BF16;
+    g.zp = zp;
+    g.wsum = wsum;
     return cuda_status(gemv::launch(g, dev->sms, s), "gemv launch");
   }
   gemm::Args g = {};
@@ -282,6 +354,8 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   g.ws = nullptr;
   g.cnt = nullptr;
   g.csplit = 0;
+  g.zp = zp;
+  g.wsum = wsum;
   cudaError_t e = cudaSuccess;
   int dev_id = 0;
   cudaGetDevice(&dev_id);
@@ -294,6 +368,7 @@ qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t* b,
   if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
   return r == 0 ? QK_OK : cuda_status(e, "gemm launch");
 }
+}  // namespace
 
 qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
                       const float* scale_a, const float* scale_b, float output_scale, void* out,

@@ -542,5 +542,126 @@ inline cudaError_t launch(const Args& a, bool bf16, int num_sms, cudaStream_t st
               : launch_typed<false, SILU>(a, num_sms, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Asymmetric per-token INT8 ("write-int8-quantized-kernel", Inputs:
+// asymmetric quantisation maps [-128, 127] to an arbitrary range with a
+// non-zero zero-point).  Per row: the range [lo, hi] is widened to hold 0;
+// scale = max(hi - lo, 1e-12) / 255; inv = 1 / scale;
+// zp = clamp(rint(-128 - lo * inv), -128, 127);
+// q = clamp(rint(x * inv) + zp, -128, 127).  One CTA of 256 threads per row,
+// two passes over the row (the second from L2); every step one IEEE
+// round-to-nearest binary32 operation.
+// ---------------------------------------------------------------------------
+struct AsymArgs {
+  int m, k;
+  const void* x;  // [m, k]
+  int8_t* q;      // [m, k]
+  float* scale;   // [m]
+  int32_t* zp;    // [m]
+};
+
+constexpr int kAsymThreads = 256;
+
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// low byte of the int8 value r (an integer-valued float in [-128, 127])
+__device__ __forceinline__ uint32_t asym_byte(float x, float inv, float z) {
+  float r = __fadd_rn(rintf(__fmul_rn(x, inv)), z);
+  r = fminf(fmaxf(r, -128.0f), 127.0f);
+  return static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kAsymThreads) quant_asym_kernel(AsymArgs p) {
+  constexpr int E = BF16 ? 8 : 4;
+  constexpr int ES = BF16 ? 2 : 4;
+  __shared__ float rlo[kAsymThreads / 32], rhi[kAsymThreads / 32];
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  griddep_wait();
+  griddep_launch_dependents();
+  const char* xr = static_cast<const char*>(p.x) + static_cast<int64_t>(row) * p.k * ES;
+  const int nvec = p.k / E;
+  float lo = 0.0f, hi = 0.0f;
+  for (int v = tid; v < nvec; v += kAsymThreads) {
+    float f[E];
+    widen<BF16>(ld_nc_v4(xr + static_cast<int64_t>(v) * 16), f);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      lo = fminf(lo, f[e]);
+      hi = fmaxf(hi, f[e]);
+    }
+  }
+  lo = warp_min(lo);
+  hi = warp_max(hi);
+  if (lane == 0) {
+    rlo[warp] = lo;
+    rhi[warp] = hi;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kAsymThreads / 32; ++w) {
+    lo = fminf(lo, rlo[w]);
+    hi = fmaxf(hi, rhi[w]);
+  }
+  const float sc = __fdiv_rn(fmaxf(__fsub_rn(hi, lo), 1e-12f), 255.0f);
+  const float inv = __fdiv_rn(1.0f, sc);
+  const float z = fminf(fmaxf(rintf(__fsub_rn(-128.0f, __fmul_rn(lo, inv))), -128.0f), 127.0f);
+  int8_t* qr = p.q + static_cast<int64_t>(row) * p.k;
+  for (int v = tid; v < nvec; v += kAsymThreads) {
+    float f[E];
+    widen<BF16>(ld_nc_v4(xr + static_cast<int64_t>(v) * 16), f);
+    uint32_t w[E / 4];
+#pragma unroll
+    for (int j = 0; j < E / 4; ++j)
+      w[j] = asym_byte(f[4 * j], inv, z) | (asym_byte(f[4 * j + 1], inv, z) << 8) |
+             (asym_byte(f[4 * j + 2], inv, z) << 16) | (asym_byte(f[4 * j + 3], inv, z) << 24);
+    if constexpr (E == 8)
+      *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(v) * E) = make_uint2(w[0], w[1]);
+    else
+      *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(v) * E) = w[0];
+  }
+  if (tid == 0) {
+    p.scale[row] = sc;
+    p.zp[row] = static_cast<int32_t>(z);
+  }
+}
+
+inline cudaError_t launch_asym(const AsymArgs& a, bool bf16, cudaStream_t stream) {
+  return bf16 ? launch_pdl(quant_asym_kernel<true>, dim3(a.m), dim3(kAsymThreads), 0, stream, 1, a)
+              : launch_pdl(quant_asym_kernel<false>, dim3(a.m), dim3(kAsymThreads), 0, stream, 1, a);
+}
+
+// wsum[r] = sum_k w[r][k] for the zero-point correction: one warp per row,
+// 16-byte loads, dp4a against bytes of 1 (exact int32 sums).
+__global__ void __launch_bounds__(256) weight_row_sums_kernel(int n, int k, const int8_t* w,
+                                                              int32_t* wsum) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= n) return;
+  const char* wr = reinterpret_cast<const char*>(w) + static_cast<int64_t>(row) * k;
+  int acc = 0;
+  for (int v = lane; v < k / 16; v += 32) {
+    const uint4 x = ld_nc_v4(wr + static_cast<int64_t>(v) * 16);
+    acc = __dp4a(static_cast<int>(x.x), 0x01010101, acc);
+    acc = __dp4a(static_cast<int>(x.y), 0x01010101, acc);
+    acc = __dp4a(static_cast<int>(x.z), 0x01010101, acc);
+    acc = __dp4a(static_cast<int>(x.w), 0x01010101, acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if (lane == 0) wsum[row] = acc;
+}
+
+inline cudaError_t launch_weight_row_sums(int n, int k, const int8_t* w, int32_t* wsum,
+                                          cudaStream_t stream) {
+  return launch_pdl(weight_row_sums_kernel, dim3((n + 7) / 8), dim3(256), 0, stream, 1, n, k, w,
+                    wsum);
+}
+
 }  // namespace quant
 }  // namespace qk

@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 3
+ABI_VERSION = 4
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -53,6 +53,11 @@ _SIGNATURES = {
                                     ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "qk_fp8_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, ctypes.c_float,
                                    _P, ctypes.c_int, _P]),
+    "qk_quantize_per_token_asym": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P,
+                                                  _P]),
+    "qk_weight_row_sums": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, _P, _P]),
+    "qk_w8a8_gemm_asym": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P, _P,
+                                         ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "qk_w8a8_gemm_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "qk_w8a8_linear": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P,
                                       ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t,
@@ -131,6 +136,20 @@ def qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out,
 
 def qk_fp8_gemm(m, n, k, a, b, scale_a, scale_b, output_scale, out, out_dtype, stream) -> int:
     return lib().qk_fp8_gemm(m, n, k, a, b, scale_a, scale_b, output_scale, out, out_dtype, stream)
+
+
+def qk_quantize_per_token_asym(m, k, x, x_dtype, q, scale, zero_point, stream) -> int:
+    return lib().qk_quantize_per_token_asym(m, k, x, x_dtype, q, scale, zero_point, stream)
+
+
+def qk_weight_row_sums(n, k, w, wsum, stream) -> int:
+    return lib().qk_weight_row_sums(n, k, w, wsum, stream)
+
+
+def qk_w8a8_gemm_asym(m, n, k, a, zero_point_a, b, wsum_b, scale_a, scale_b, output_scale, c, out,
+                      out_dtype, workspace, workspace_bytes, stream) -> int:
+    return lib().qk_w8a8_gemm_asym(m, n, k, a, zero_point_a, b, wsum_b, scale_a, scale_b, output_scale,
+                                   c, out, out_dtype, workspace, workspace_bytes, stream)
 
 
 def qk_w8a8_gemm_workspace_size(m, n, k, group_k) -> int:
@@ -301,6 +320,52 @@ def fp8_gemm(a, b, scale_a, scale_b, output_scale: float = 1.0, out_dtype=None, 
     _check(qk_fp8_gemm(m, n, k, _ptr(a), _ptr(b), _ptr(scale_a), _ptr(scale_b), float(output_scale),
                        _ptr(out), _dtype_code(out), _stream(stream)), "qk_fp8_gemm")
     return out
+
+
+def quantize_per_token_asym(x, stream=None):
+    """x [m, k] bf16/fp32 -> (q int8 [m, k], scale fp32 [m], zero_point int32 [m])."""
+    torch = _torch()
+    _need_cuda(x)
+    assert x.dim() == 2 and x.is_contiguous()
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    scale = torch.empty((m,), dtype=torch.float32, device=x.device)
+    zp = torch.empty((m,), dtype=torch.int32, device=x.device)
+    _check(qk_quantize_per_token_asym(m, k, _ptr(x), _dtype_code(x), _ptr(q), _ptr(scale), _ptr(zp),
+                                      _stream(stream)), "qk_quantize_per_token_asym")
+    return q, scale, zp
+
+
+def weight_row_sums(w, stream=None):
+    """w [n, k] int8 -> wsum int32 [n] (sum over k of each row)."""
+    torch = _torch()
+    _need_cuda(w)
+    n, k = w.shape
+    out = torch.empty((n,), dtype=torch.int32, device=w.device)
+    _check(qk_weight_row_sums(n, k, _ptr(w), _ptr(out), _stream(stream)), "qk_weight_row_sums")
+    return out
+
+
+def w8a8_gemm_asym(a, zero_point_a, b, wsum_b, scale_a, scale_b, output_scale: float = 1.0,
+                   out_dtype=None, want_out: bool = True, want_c: bool = False, workspace=None,
+                   stream=None):
+    """Asymmetric activations: (out [m, n] or None, c int32 [m, n] or None)."""
+    torch = _torch()
+    _need_cuda(a, b, zero_point_a, wsum_b)
+    m, k = a.shape
+    n = b.shape[0]
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = torch.empty((m, n), dtype=out_dtype, device=a.device) if want_out else None
+    c = torch.empty((m, n), dtype=torch.int32, device=a.device) if want_c else None
+    need = qk_w8a8_gemm_workspace_size(m, n, k, 0)
+    if need and workspace is None:
+        workspace = cached_workspace(need, a.device)
+    code = _dtype_code(out) if out is not None else QK_BF16
+    _check(qk_w8a8_gemm_asym(m, n, k, _ptr(a), _ptr(zero_point_a), _ptr(b), _ptr(wsum_b), _ptr(scale_a),
+                             _ptr(scale_b), float(output_scale), _ptr(c), _ptr(out), code, _ptr(workspace),
+                             0 if workspace is None else workspace.numel(), _stream(stream)),
+           "qk_w8a8_gemm_asym")
+    return out, c
 
 
 _workspaces: dict = {}
