@@ -29,6 +29,8 @@ Which page each function follows:
   per-token INT8 ("write-int8-quantized-kernel", Inputs: asymmetric maps
   [-128, 127] to an arbitrary range with a non-zero zero-point) and the
   GEMM with the zero-point correction.
+* :func:`quantize_static` -- static per-tensor INT8 ("write-int8-quantized-
+  kernel", Inputs: per-tensor granularity, scales computed offline).
 * :func:`gemm_fp8` -- the FP8 x FP8 product with the exact accumulator
   (every e4m3 value is an integer multiple of 2^-9) and the per-channel
   epilogue.
@@ -116,6 +118,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.qko_weight_row_sums.restype = i32
     lib.qko_gemm_s32_asym.argtypes = [i32, i32, i32, P, P, P, P]
     lib.qko_gemm_s32_asym.restype = i32
+    lib.qko_quantize_static.argtypes = [i32, i32, P, i32, f32, P]
+    lib.qko_quantize_static.restype = i32
     return lib
 
 
@@ -376,3 +380,13 @@ class Oracle:
         acc = self.gemm_s32_asym(q, zp, w_q)
         out = self.epilogue_per_channel(acc, sa, sw, alpha)
         return {"acc": acc, "out_f32": out, "out_bf16": self.f32_to_bf16(out)}
+
+    # -- static per-tensor INT8 -----------------------------------------------
+    def quantize_static(self, x: np.ndarray, scale: float) -> np.ndarray:
+        """x [m, k] -> q int8 [m, k] = clamp(rne(x / scale), -127, 127) (via 1 / scale)."""
+        x = np.ascontiguousarray(x)
+        m, k = x.shape
+        q = np.empty((m, k), np.int8)
+        _check(self.lib.qko_quantize_static(m, k, _ptr(x), _dtype_code(x), ctypes.c_float(scale),
+                                            _ptr(q)), "quantize_static")
+        return q

@@ -62,6 +62,9 @@
  *  - the GEMM's accumulator is sum_k (q - zp) * w = acc - zp * wsum[n],
  *    wsum[n] = sum_k w[n][k]; the epilogue is the per-channel one.
  *
+ * Static per-tensor INT8 (same page: per-tensor granularity, scales computed
+ * offline): inv = 1 / scale, q = clamp(rne(x * inv), -127, 127).
+ *
  * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread (no fast-math),
  * so every float operation below is a single IEEE binary32 RN operation.
  *
@@ -606,4 +609,24 @@ int qko_gemm_s32_asym(int m, int n, int k, const int8_t* a, const int32_t* zp, c
     }
   }
   return overflow ? QKO_ERR_OVERFLOW : QKO_OK;
+}
+
+/* ----------------------------------------------------------------------- */
+/* Static per-tensor INT8 ("write-int8-quantized-kernel", Inputs: per-     */
+/* tensor granularity, one scale for the entire tensor, computed offline).  */
+/* ----------------------------------------------------------------------- */
+
+/* inv = 1 / scale (fp32 RN); q = clamp(round_half_even(x * inv), -127, 127);
+ * values beyond 127 * scale saturate. */
+int qko_quantize_static(int m, int k, const void* x, int dtype, float scale, int8_t* q) {
+  if (m < 0 || k <= 0 || (dtype != QKO_F32 && dtype != QKO_BF16) || !(scale > 0.0f))
+    return QKO_ERR_ARG;
+  const float inv = 1.0f / scale;
+  for (int64_t i = 0; i < (int64_t)m * k; ++i) {
+    float r = nearbyintf(qko_load(x, dtype, i) * inv);
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    q[i] = (int8_t)(int)r;
+  }
+  return QKO_OK;
 }

@@ -446,7 +446,25 @@ def pin_asym_gemm(O) -> None:
     assert np.array_equal(O.weight_row_sums(w), w.astype(np.int64).sum(axis=1))
 
 
+def pin_static_quant(O) -> None:
+    # scale 1: q = clamp(rne(x)); ties to even; saturation at +-127
+    x = np.float32([[0.5, 1.5, 2.5, -0.5, -2.5, 126.6, 127.4, 300.0, -1e6, 3.49]])
+    assert O.quantize_static(x, 1.0).tolist() == [[0, 2, 2, 0, -2, 127, 127, 127, -127, 3]]
+    # scale 0.25: inv 4 exactly
+    y = np.float32([[0.125, 0.375, -0.1, 31.75, 40.0]])
+    assert O.quantize_static(y, 0.25).tolist() == [[0, 2, 0, 127, 127]]
+    # random values: the round trip within half a step inside the range
+    rng = np.random.default_rng(23)
+    z = rng.standard_normal((4, 200)).astype(np.float32) * 3
+    s = 0.02
+    q = O.quantize_static(z, s)
+    inside = np.abs(z.astype(np.float64) / s) <= 126.5
+    err = np.abs(q.astype(np.float64) * s - z.astype(np.float64))
+    assert float(err[inside].max()) <= s * (0.5 + 2.0 ** -16)
+    assert np.all(np.abs(q[~inside]) == 127)
+
+
 ALL_PINS = [pin_exp, pin_silu, pin_bf16_rounding, pin_quant_golden, pin_quant_invariants,
             pin_quant_bf16_path, pin_silu_quant, pin_gemm_bruteforce, pin_gemm_closed_forms,
             pin_epilogue_per_channel, pin_group, pin_linear_golden, pin_e4m3_codec, pin_fp8_quant,
-            pin_fp8_silu_quant, pin_fp8_gemm, pin_asym_quant, pin_asym_gemm]
+            pin_fp8_silu_quant, pin_fp8_gemm, pin_asym_quant, pin_asym_gemm, pin_static_quant]

@@ -66,6 +66,10 @@ MUTANTS = [
      "s += ((int64_t)a[(int64_t)r * k + i]) * (int64_t)w[(int64_t)c * k + i];"),
     ("asym_wsum_dropped", "for (int i = 0; i < k; ++i) t += w[(int64_t)c * k + i];",
      "for (int i = 1; i < k; ++i) t += w[(int64_t)c * k + i];"),
+    ("static_ties_away", "float r = nearbyintf(qko_load(x, dtype, i) * inv);",
+     "float r = roundf(qko_load(x, dtype, i) * inv);"),
+    ("static_no_saturation", "    if (r > 127.0f) r = 127.0f;\n    if (r < -127.0f) r = -127.0f;\n    q[i] = (int8_t)(int)r;\n  }\n  return QKO_OK;",
+     "    q[i] = (int8_t)(int)r;\n  }\n  return QKO_OK;"),
     ("fp8_gemm_units", ": (int64_t)(8 + m) << (e - 1);", ": (int64_t)(8 + m) << e;"),
     ("fp8_gemm_dropped_term", "for (int i = 0; i < j->k; ++i) s += qko_e4m3_units(ar[i]) * qko_e4m3_units(wr[i]);",
      "for (int i = 1; i < j->k; ++i) s += qko_e4m3_units(ar[i]) * qko_e4m3_units(wr[i]);"),
