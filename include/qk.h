@@ -50,7 +50,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 4
+#define QK_ABI_VERSION 5
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -265,6 +265,18 @@ QK_API qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_
  *   qk_weight_row_sums.  k <= 66311, so that k * 255 * 127 < 2^31 (else
  *   QK_ERR_OVERFLOW_BOUND).  Workspace as qk_w8a8_gemm.
  */
+/*
+ * qk_quantize_static -- static per-tensor INT8 ("write-int8-quantized-
+ * kernel", Inputs the agent should gather first: per-tensor granularity, one
+ * scale for the entire tensor, computed offline): inv = 1 / *scale (fp32
+ * RN), q = clamp(rne(x * inv), -127, 127); values beyond 127 * scale
+ * saturate.  scale: device pointer to one fp32 (> 0), 4-byte aligned; x, q
+ * as qk_quantize_per_token.  The GEMM then takes scale_a as an [m] vector
+ * holding that one value.
+ */
+QK_API qk_status qk_quantize_static(int m, int k, const void* x, qk_dtype x_dtype,
+                                    const float* scale, int8_t* q, qk_stream stream);
+
 QK_API qk_status qk_quantize_per_token_asym(int m, int k, const void* x, qk_dtype x_dtype,
                                             int8_t* q, float* scale, int32_t* zero_point,
                                             qk_stream stream);

@@ -113,3 +113,32 @@ def test_asym_errors():
     st = qk.qk_w8a8_gemm_asym(4, 16, 64, qk._ptr(a), None, qk._ptr(w), qk._ptr(z), qk._ptr(s),
                               qk._ptr(s), 1.0, None, qk._ptr(out), qk.QK_BF16, None, 0, qk._stream())
     assert st == qk.QK_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- static per-tensor
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("m,k,scale", [(1, 16, 1.0), (7, 512, 0.02), (300, 4096, 0.05),
+                                       (4096, 4096, 0.03), (3, 14336, 0.25)])
+def test_static_quant(O, m, k, dtype, scale):
+    x = _rand(m, k, dtype, seed=7000 + m + k)
+    s = torch.tensor([scale], dtype=torch.float32, device="cuda")
+    q = qk.quantize_static(x_dev(x), s)
+    torch.cuda.synchronize()
+    assert_bits(host(q), O.quantize_static(x, scale), "q")
+
+
+def test_static_then_gemm(O):
+    # a static per-tensor scale feeds the GEMM as an [m] vector of one value
+    m, n, k, scale = 200, 264, 384, 0.04
+    r = synth.streams(71, ["x", "o", "w", "sw"])
+    x, _ = synth.activation(r["x"], r["o"], m, k, "bf16", 0.01, 20.0)
+    w = synth.int8_uniform(r["w"], (n, k))
+    sw = synth.scales_uniform(r["sw"], (n,))
+    q = qk.quantize_static(x_dev(x), torch.tensor([scale], dtype=torch.float32, device="cuda"))
+    sa = torch.full((m,), scale, dtype=torch.float32, device="cuda")
+    out, c = qk.w8a8_gemm(q, dev(w), sa, dev(sw), 0, 1.0, want_c=True)
+    torch.cuda.synchronize()
+    qr = O.quantize_static(x, scale)
+    ref = O.linear_from_q(qr, np.full((m,), scale, np.float32), w, sw, 0, 1.0)
+    assert_bits(host(c), ref["acc"], "acc")
+    assert_bits(host(out), ref["out_bf16"], "bf16 out")

@@ -286,6 +286,21 @@ qk_status qk_quantize_per_token_asym(int m, int k, const void* x, qk_dtype x_dty
                      "asymmetric quantize launch");
 }
 
+qk_status qk_quantize_static(int m, int k, const void* x, qk_dtype x_dtype, const float* scale,
+                             int8_t* q, qk_stream stream) {
+  if (m < 0 || k <= 0 || (k % 16) != 0) return QK_ERR_INVALID_ARG;
+  if (x_dtype != QK_F32 && x_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (m == 0) return QK_OK;
+  if (x == nullptr || scale == nullptr || q == nullptr) return QK_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale, 4)) return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  return cuda_status(quant::launch_static(static_cast<int64_t>(m) * k, x, x_dtype == QK_BF16, scale, q,
+                                          dev->sms, reinterpret_cast<cudaStream_t>(stream)),
+                     "static quantize launch");
+}
+
 qk_status qk_weight_row_sums(int n, int k, const int8_t* w, int32_t* wsum, qk_stream stream) {
   if (n < 0 || k <= 0 || (k % 16) != 0) return QK_ERR_INVALID_ARG;
   if (k > kMaxK) return QK_ERR_OVERFLOW_BOUND;

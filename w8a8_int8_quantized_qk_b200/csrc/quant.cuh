@@ -635,6 +635,54 @@ inline cudaError_t launch_asym(const AsymArgs& a, bool bf16, cudaStream_t stream
               : launch_pdl(quant_asym_kernel<false>, dim3(a.m), dim3(kAsymThreads), 0, stream, 1, a);
 }
 
+// ---------------------------------------------------------------------------
+// Static per-tensor INT8 ("write-int8-quantized-kernel", Inputs: per-tensor
+// granularity, scales computed offline): inv = 1 / scale (scale read from
+// device memory), q = clamp(rint(x * inv), -127, 127).  Elementwise:
+// persistent grid-stride over the tensor's 16-byte vectors.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t static_byte(float x, float inv) {
+  const float r = fminf(fmaxf(rintf(__fmul_rn(x, inv)), -127.0f), 127.0f);
+  return static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) quant_static_kernel(int64_t nvec, const void* x,
+                                                           const float* scale, int8_t* q) {
+  constexpr int E = BF16 ? 8 : 4;
+  griddep_wait();
+  griddep_launch_dependents();
+  const float inv = __fdiv_rn(1.0f, __ldg(scale));
+  const char* xb = static_cast<const char*>(x);
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float f[E];
+    widen<BF16>(ld_nc_v4(xb + v * 16), f);
+    uint32_t w[E / 4];
+#pragma unroll
+    for (int j = 0; j < E / 4; ++j)
+      w[j] = static_byte(f[4 * j], inv) | (static_byte(f[4 * j + 1], inv) << 8) |
+             (static_byte(f[4 * j + 2], inv) << 16) | (static_byte(f[4 * j + 3], inv) << 24);
+    if constexpr (E == 8)
+      *reinterpret_cast<uint2*>(q + v * E) = make_uint2(w[0], w[1]);
+    else
+      *reinterpret_cast<uint32_t*>(q + v * E) = w[0];
+  }
+}
+
+inline cudaError_t launch_static(int64_t count, const void* x, bool bf16, const float* scale,
+                                 int8_t* q, int num_sms, cudaStream_t stream) {
+  const int64_t nvec = count / (bf16 ? 8 : 4);
+  int64_t blocks = (nvec + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return bf16 ? launch_pdl(quant_static_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                           stream, 1, nvec, x, scale, q)
+              : launch_pdl(quant_static_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                           stream, 1, nvec, x, scale, q);
+}
+
 // wsum[r] = sum_k w[r][k] for the zero-point correction: one warp per row,
 // 16-byte loads, dp4a against bytes of 1 (exact int32 sums).
 __global__ void __launch_bounds__(256) weight_row_sums_kernel(int n, int k, const int8_t* w,

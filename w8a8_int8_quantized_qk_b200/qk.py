@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 4
+ABI_VERSION = 5
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -55,6 +55,7 @@ _SIGNATURES = {
                                    _P, ctypes.c_int, _P]),
     "qk_quantize_per_token_asym": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P,
                                                   _P]),
+    "qk_quantize_static": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P]),
     "qk_weight_row_sums": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, _P, _P]),
     "qk_w8a8_gemm_asym": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P, _P,
                                          ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
@@ -140,6 +141,10 @@ def qk_fp8_gemm(m, n, k, a, b, scale_a, scale_b, output_scale, out, out_dtype, s
 
 def qk_quantize_per_token_asym(m, k, x, x_dtype, q, scale, zero_point, stream) -> int:
     return lib().qk_quantize_per_token_asym(m, k, x, x_dtype, q, scale, zero_point, stream)
+
+
+def qk_quantize_static(m, k, x, x_dtype, scale, q, stream) -> int:
+    return lib().qk_quantize_static(m, k, x, x_dtype, scale, q, stream)
 
 
 def qk_weight_row_sums(n, k, w, wsum, stream) -> int:
@@ -334,6 +339,19 @@ def quantize_per_token_asym(x, stream=None):
     _check(qk_quantize_per_token_asym(m, k, _ptr(x), _dtype_code(x), _ptr(q), _ptr(scale), _ptr(zp),
                                       _stream(stream)), "qk_quantize_per_token_asym")
     return q, scale, zp
+
+
+def quantize_static(x, scale, stream=None):
+    """x [m, k] bf16/fp32 -> q int8 [m, k] with the per-tensor scale (a one-element
+    fp32 CUDA tensor)."""
+    torch = _torch()
+    _need_cuda(x, scale)
+    assert x.dim() == 2 and x.is_contiguous()
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    _check(qk_quantize_static(m, k, _ptr(x), _dtype_code(x), _ptr(scale), _ptr(q), _stream(stream)),
+           "qk_quantize_static")
+    return q
 
 
 def weight_row_sums(w, stream=None):
