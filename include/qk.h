@@ -50,7 +50,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 5
+#define QK_ABI_VERSION 6
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -265,6 +265,34 @@ QK_API qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_
  *   qk_weight_row_sums.  k <= 66311, so that k * 255 * 127 < 2^31 (else
  *   QK_ERR_OVERFLOW_BOUND).  Workspace as qk_w8a8_gemm.
  */
+/*
+ * qk_w8a8_moe_gemm -- the W8A8 GEMM of a mixture-of-experts layer in one
+ * launch (grouped GEMM): tokens already grouped by expert, expert e owning
+ * rows [expert_offsets[e], expert_offsets[e + 1]) of a; each group times
+ * its own expert's int8 weights, with the per-token x per-channel epilogue.
+ *
+ * num_experts    E >= 1
+ * total_m        rows of a and out (the tokens of all experts)
+ * n, k           per expert: b is [E, n, k] (row e * n + j is expert e's
+ *                output channel j), k % 16 == 0, n % 8 == 0, k <= 133144
+ * max_m_per_expert   an upper bound on every expert's token count: it sizes
+ *                the tile space (E x ceil(max / 128) x ceil(n / 256) tiles,
+ *                the empty ones skipped); rows of an expert beyond it are
+ *                not computed
+ * expert_offsets [E + 1] int32 device array, non-decreasing, offsets[0] = 0,
+ *                offsets[E] = total_m (rows outside [0, total_m) are never
+ *                written)
+ * a              [total_m, k] int8, 16-B aligned; scale_a [total_m] fp32
+ * b              [E * n, k] int8, 16-B aligned; scale_b [E, n] fp32, 16-B
+ *                aligned
+ * out            [total_m, n] bf16 or fp32, 16-B aligned
+ * Errors as qk_w8a8_gemm (per channel only, no workspace, no c).
+ */
+QK_API qk_status qk_w8a8_moe_gemm(int num_experts, int total_m, int n, int k, int max_m_per_expert,
+                                  const int32_t* expert_offsets, const int8_t* a, const int8_t* b,
+                                  const float* scale_a, const float* scale_b, float output_scale,
+                                  void* out, qk_dtype out_dtype, qk_stream stream);
+
 /*
  * qk_quantize_static -- static per-tensor INT8 ("write-int8-quantized-
  * kernel", Inputs the agent should gather first: per-tensor granularity, one

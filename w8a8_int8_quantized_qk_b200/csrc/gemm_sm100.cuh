@@ -81,7 +81,44 @@ struct Args {
   // [n] = sum_k b[n][k]; the epilogues use acc - zp[m] * wsum[n]
   const int32_t* zp;
   const int32_t* wsum;
+  // MoE grouped GEMM (1-SM kernel): tokens grouped by expert, expert e's rows
+  // [moe_off[e], moe_off[e + 1]) of a (m rows in all); b is [experts * n, k]
+  // and sw [experts, n]; tiles_m = experts * mt_max M tiles, those past an
+  // expert's tokens are skipped
+  int mt_max;
+  const int32_t* moe_off;
 };
+
+// One output tile of the 1-SM kernels: A rows from a_row0 (rows from row_end
+// on belong to another expert, or to none, and are masked), B rows from
+// b_row0, output columns from col0, channel scales from sw.  False for an
+// empty MoE tile; every role skips the same tiles.
+struct ChanTile {
+  int a_row0, b_row0, col0, row_end;
+  const float* sw;
+};
+
+template <int BN, bool MOE>
+__device__ __forceinline__ bool chan_tile(const Args& p, int tile, ChanTile& t) {
+  const int tmg = tile % p.tiles_m, tn = tile / p.tiles_m;
+  if constexpr (MOE) {
+    const int e = tmg / p.mt_max, tm = tmg % p.mt_max;
+    const int r0 = __ldg(p.moe_off + e), r1 = __ldg(p.moe_off + e + 1);
+    if (r0 + tm * BM >= r1) return false;
+    t.a_row0 = r0 + tm * BM;
+    t.row_end = r1 < p.m ? r1 : p.m;
+    t.b_row0 = e * p.n + tn * BN;
+    t.col0 = tn * BN;
+    t.sw = p.sw + static_cast<int64_t>(e) * p.n;
+  } else {
+    t.a_row0 = tmg * BM;
+    t.row_end = p.m;
+    t.b_row0 = tn * BN;
+    t.col0 = tn * BN;
+    t.sw = p.sw;
+  }
+  return true;
+}
 
 template <int BN, int STAGES, int NACC, int SCALE_FLOATS>
 struct alignas(1024) Storage {
@@ -114,15 +151,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // ---------------------------------------------------------------- producer
-template <int BN, int STAGES, class S>
+template <int BN, int STAGES, bool MOE = false, class S>
 __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, const Args& p) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const uint32_t bytes = static_cast<uint32_t>((BM + BN) * BK);
   uint32_t stage = 0, phase = 0, issued = 0;
   bool ok = true;
   for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
-    const int tile = unit / p.splits;
-    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    ChanTile t;
+    if (!chan_tile<BN, MOE>(p, unit / p.splits, t)) continue;
     const int kb0 = (unit % p.splits) * p.kb_per_split;
     const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
     for (int kb = kb0; kb < kb1; ++kb) {
@@ -132,8 +169,8 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
       }
       const uint32_t fb = smem_addr(&s.full[stage]);
       mbar_arrive_expect_tx(fb, bytes);
-      tma_load_2d(smem_addr(s.a[stage]), tmA, fb, kb * BK, tm * BM);
-      tma_load_2d(smem_addr(s.b[stage]), tmB, fb, kb * BK, tn * BN);
+      tma_load_2d(smem_addr(s.a[stage]), tmA, fb, kb * BK, t.a_row0);
+      tma_load_2d(smem_addr(s.b[stage]), tmB, fb, kb * BK, t.b_row0);
       ++issued;
       if (++stage == STAGES) {
         stage = 0;
@@ -151,13 +188,17 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
 // ---------------------------------------------------------------- MMA issuer
 // GROUP: one accumulator buffer per K block (each K block is one group);
 // otherwise one buffer per tile.
-template <int BN, int STAGES, int NACC, bool GROUP, bool F8 = false, class S>
+template <int BN, int STAGES, int NACC, bool GROUP, bool F8 = false, bool MOE = false, class S>
 __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   constexpr uint32_t idesc = F8 ? idesc_e4m3(BM, BN) : idesc_i8(BM, BN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
   for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
+    if constexpr (MOE) {
+      ChanTile t;
+      if (!chan_tile<BN, true>(p, unit, t)) continue;
+    }
     const int kb0 = (unit % p.splits) * p.kb_per_split;
     const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
     if (!GROUP) {
@@ -368,7 +409,7 @@ __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tm
 // row's token scale; the 32-column TMEM loads are double-buffered so the
 // next load is in flight while the current chunk is converted and stored.
 // bf16 output without c leaves through TMA stores (store32_tma).
-template <int BN, int NACC, bool F8 = false, class S>
+template <int BN, int NACC, bool F8 = false, bool MOE = false, class S>
 __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUtensorMap* tmO) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const int lane = threadIdx.x & 31;
@@ -378,18 +419,18 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
   uint8_t* box = s.out_stage[ew];
   uint32_t abuf = 0, aphase = 0;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
-    const int tile = unit / p.splits;
-    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    const int row0 = tm * BM + quad * 32, row = row0 + lane;
-    const bool rv = row < p.m;
+    ChanTile t;
+    if (!chan_tile<BN, MOE>(p, unit / p.splits, t)) continue;
+    const int row0 = t.a_row0 + quad * 32, row = row0 + lane;
+    const bool rv = row >= 0 && row < t.row_end;
     const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
-    const int colbase = tn * BN;
+    const int colbase = t.col0;
     if (p.out) {
 #pragma unroll
       for (int c4 = lane * 4; c4 < BN; c4 += 128) {  // n % 8 == 0: a group of 4 is all in or out
         const int col = colbase + c4;
         *reinterpret_cast<float4*>(sws + c4) =
-            col < p.n ? __ldg(reinterpret_cast<const float4*>(p.sw + col))
+            col < p.n ? __ldg(reinterpret_cast<const float4*>(t.sw + col))
                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       }
     }
@@ -776,7 +817,7 @@ struct alignas(1024) ChannelStorage {
   int abort;
 };
 
-template <bool F8>
+template <bool F8, bool MOE = false>
 __global__ void __launch_bounds__(kChannelThreads, 1)
     gemm_i8_channel_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
@@ -794,13 +835,13 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
   griddep_launch_dependents();
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
-    if (lane == 0) produce<kChannelBN, kChannelStages>(s, &tmA, &tmB, p);
+    if (lane == 0) produce<kChannelBN, kChannelStages, MOE>(s, &tmA, &tmB, p);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false, F8>(s, tmem, p);
+    if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false, F8, MOE>(s, tmem, p);
     __syncwarp();
   } else {
-    epilogue_channel<kChannelBN, 2, F8>(s, tmem, p, &tmO);
+    epilogue_channel<kChannelBN, 2, F8, MOE>(s, tmem, p, &tmO);
   }
   if (p.csplit) {
     cluster_sync_all();  // every CTA of the cluster has staged its partial
@@ -1471,7 +1512,7 @@ inline bool cached_tmap(CUtensorMap* map, const void* base, int rows, int k, int
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel).
 template <class K>
 inline cudaError_t set_smem_once(K kernel, int dev, int slot, size_t bytes) {
-  static std::atomic<unsigned long long> done[6] = {};
+  static std::atomic<unsigned long long> done[8] = {};
   const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
   if (bit && (done[slot].load(std::memory_order_acquire) & bit)) return cudaSuccess;
   const cudaError_t e =
@@ -1840,6 +1881,40 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
       }
     }
   }
+  *err = e;
+  return e == cudaSuccess ? 0 : 2;
+}
+
+// MoE grouped GEMM on the 1-SM kernel: `experts` groups of tokens (expert e
+// owns rows [off[e], off[e + 1]) of A, m rows in all), B stacked [experts *
+// n, k], per-channel scales [experts, n]; mt_max bounds every expert's M
+// tiles.  Whole tiles, per channel, direct stores (a TMA box could cross
+// into the next expert's rows).  0 ok, 1 tensor-map failure, 2 CUDA error.
+inline int launch_moe(Args a, const int8_t* A, const int8_t* B, int experts, int mt_max,
+                      const int32_t* off, int dev, int num_sms, cudaStream_t stream,
+                      cudaError_t* err) {
+  a.mt_max = mt_max;
+  a.moe_off = off;
+  a.tiles_m = experts * mt_max;
+  a.tiles_n = (a.n + kChannelBN - 1) / kChannelBN;
+  a.num_kb = (a.k + BK - 1) / BK;
+  a.groups = 0;
+  a.splits = 1;
+  a.kb_per_split = a.num_kb;
+  a.csplit = 0;
+  a.tail_splits = 1;
+  a.tma_out = 0;
+  a.c = nullptr;
+  CUtensorMap ta, tb;
+  if (!cached_tmap(&ta, A, a.m, a.k, BM) || !cached_tmap(&tb, B, experts * a.n, a.k, kChannelBN))
+    return 1;
+  const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
+  const int grid = ntiles < num_sms ? static_cast<int>(ntiles) : num_sms;
+  const size_t smem = channel_smem();
+  cudaError_t e = set_smem_once(gemm_i8_channel_kernel<false, true>, dev, 6, smem);
+  if (e == cudaSuccess)
+    e = launch_pdl(gemm_i8_channel_kernel<false, true>, dim3(grid), dim3(kChannelThreads), smem,
+                   stream, 1u, ta, tb, ta, a);
   *err = e;
   return e == cudaSuccess ? 0 : 2;
 }

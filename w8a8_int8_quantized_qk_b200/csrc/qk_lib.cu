@@ -286,6 +286,45 @@ qk_status qk_quantize_per_token_asym(int m, int k, const void* x, qk_dtype x_dty
                      "asymmetric quantize launch");
 }
 
+qk_status qk_w8a8_moe_gemm(int num_experts, int total_m, int n, int k, int max_m_per_expert,
+                           const int32_t* expert_offsets, const int8_t* a, const int8_t* b,
+                           const float* scale_a, const float* scale_b, float output_scale,
+                           void* out, qk_dtype out_dtype, qk_stream stream) {
+  if (num_experts < 1 || total_m < 0 || n < 0 || k <= 0 || max_m_per_expert < 0)
+    return QK_ERR_INVALID_ARG;
+  if ((k % 16) != 0 || (n % 8) != 0) return QK_ERR_INVALID_ARG;
+  if (k > kMaxK) return QK_ERR_OVERFLOW_BOUND;
+  if (out_dtype != QK_F32 && out_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (total_m == 0 || n == 0 || max_m_per_expert == 0) return QK_OK;
+  if (static_cast<int64_t>(num_experts) * n > INT32_MAX) return QK_ERR_INVALID_ARG;
+  if (expert_offsets == nullptr || a == nullptr || b == nullptr || scale_a == nullptr ||
+      scale_b == nullptr || out == nullptr)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(scale_a, 4) ||
+      !aligned(scale_b, 16) || !aligned(expert_offsets, 4))
+    return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  gemm::Args g = {};
+  g.m = total_m;
+  g.n = n;
+  g.k = k;
+  g.sa = scale_a;
+  g.sw = scale_b;
+  g.alpha = output_scale;
+  g.out = out;
+  g.out_bf16 = out_dtype == QK_BF16;
+  cudaError_t e = cudaSuccess;
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const int mt_max = (max_m_per_expert + 127) / 128;
+  const int r = gemm::launch_moe(g, a, b, num_experts, mt_max, expert_offsets, dev_id, dev->sms,
+                                 reinterpret_cast<cudaStream_t>(stream), &e);
+  if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
+  return r == 0 ? QK_OK : cuda_status(e, "moe gemm launch");
+}
+
 qk_status qk_quantize_static(int m, int k, const void* x, qk_dtype x_dtype, const float* scale,
                              int8_t* q, qk_stream stream) {
   if (m < 0 || k <= 0 || (k % 16) != 0) return QK_ERR_INVALID_ARG;

@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 5
+ABI_VERSION = 6
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -55,6 +55,8 @@ _SIGNATURES = {
                                    _P, ctypes.c_int, _P]),
     "qk_quantize_per_token_asym": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P,
                                                   _P]),
+    "qk_w8a8_moe_gemm": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        _P, _P, _P, _P, _P, ctypes.c_float, _P, ctypes.c_int, _P]),
     "qk_quantize_static": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P]),
     "qk_weight_row_sums": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, _P, _P]),
     "qk_w8a8_gemm_asym": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P, _P,
@@ -141,6 +143,12 @@ def qk_fp8_gemm(m, n, k, a, b, scale_a, scale_b, output_scale, out, out_dtype, s
 
 def qk_quantize_per_token_asym(m, k, x, x_dtype, q, scale, zero_point, stream) -> int:
     return lib().qk_quantize_per_token_asym(m, k, x, x_dtype, q, scale, zero_point, stream)
+
+
+def qk_w8a8_moe_gemm(num_experts, total_m, n, k, max_m_per_expert, expert_offsets, a, b, scale_a, scale_b,
+                     output_scale, out, out_dtype, stream) -> int:
+    return lib().qk_w8a8_moe_gemm(num_experts, total_m, n, k, max_m_per_expert, expert_offsets, a, b,
+                                  scale_a, scale_b, output_scale, out, out_dtype, stream)
 
 
 def qk_quantize_static(m, k, x, x_dtype, scale, q, stream) -> int:
@@ -339,6 +347,22 @@ def quantize_per_token_asym(x, stream=None):
     _check(qk_quantize_per_token_asym(m, k, _ptr(x), _dtype_code(x), _ptr(q), _ptr(scale), _ptr(zp),
                                       _stream(stream)), "qk_quantize_per_token_asym")
     return q, scale, zp
+
+
+def w8a8_moe_gemm(a, expert_offsets, b, scale_a, scale_b, max_m_per_expert: int, output_scale: float = 1.0,
+                  out_dtype=None, stream=None):
+    """a [total_m, k] int8 grouped by expert, expert_offsets int32 [E + 1] (CUDA),
+    b [E, n, k] int8, scale_a [total_m], scale_b [E, n] -> out [total_m, n]."""
+    torch = _torch()
+    _need_cuda(a, b, scale_a, scale_b, expert_offsets)
+    total_m, k = a.shape
+    e, n, _ = b.shape
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = torch.empty((total_m, n), dtype=out_dtype, device=a.device)
+    _check(qk_w8a8_moe_gemm(e, total_m, n, k, int(max_m_per_expert), _ptr(expert_offsets), _ptr(a), _ptr(b),
+                            _ptr(scale_a), _ptr(scale_b), float(output_scale), _ptr(out), _dtype_code(out),
+                            _stream(stream)), "qk_w8a8_moe_gemm")
+    return out
 
 
 def quantize_static(x, scale, stream=None):
