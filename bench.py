@@ -392,6 +392,56 @@ def measure_fp8(torch, qk, iters: int, pk: dict) -> dict:
     return res
 
 
+def measure_moe(torch, qk, iters: int, pk: dict) -> dict:
+    """The MoE grouped GEMM (qk_w8a8_moe_gemm) on a synthetic routing: 8
+    experts of 4096 x 4096 int8 weights, 4096 tokens routed with Zipf-like
+    expert frequencies (1/rank), activations already quantised."""
+    import ctypes
+
+    import numpy as np
+
+    from w8a8_int8_quantized_qk_b200 import synth
+
+    e, n, k, total = 8, 4096, 4096, 4096
+    r = synth.streams(41, ["route", "a", "w", "sa", "sw"])
+    probs = 1.0 / np.arange(1, e + 1)
+    counts = np.bincount(r["route"].choice(e, total, p=probs / probs.sum()), minlength=e)
+    off = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).cuda()
+    a = torch.from_numpy(synth.int8_uniform(r["a"], (total, k))).cuda()
+    w0 = torch.from_numpy(synth.int8_uniform(r["w"], (e, n, k))).cuda()
+    sa = torch.from_numpy(synth.scales_uniform(r["sa"], (total,), 0.001, 0.05)).cuda()
+    sw = torch.from_numpy(synth.scales_uniform(r["sw"], (e, n))).cuda()
+    R = _copies(w0.numel() + a.numel())
+    ws = [w0.clone() for _ in range(R)]
+    outs = [torch.empty((total, n), dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+
+    class _M:
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    M = _M()
+    mx = int(counts.max())
+
+    def call(i):
+        j = i % R
+        st = qk.qk_w8a8_moe_gemm(e, total, n, k, mx, P(off), P(a), P(ws[j]), P(sa), P(sw), 1.0, P(outs[j]),
+                                 qk.QK_BF16, M.stream)
+        if st != 0:
+            raise qk.QKError(st, "moe gemm")
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize()
+    us = _graph_us(torch, M, call, iters)
+    ops = 2.0 * total * n * k
+    wbytes = e * n * k
+    return {"experts": e, "n": n, "k": k, "tokens": total, "tokens_per_expert": counts.tolist(),
+            "copies": R, "timing": f"CUDA graph of {iters} iterations", "gemm_us": us,
+            "gemm_TOPS": ops / (us * 1e-6) / 1e12, "gemm_tensor_frac": ops / (us * 1e-6) / 1e12 / pk["int8_tops"],
+            "weight_GBs": wbytes / (us * 1e-6) / 1e9,
+            "note": "1-SM tcgen05 kernel over experts x M tiles x N tiles, empty tiles skipped"}
+
+
 def cpu_baseline(seconds: float = 10.0) -> dict:
     """The oracle, as it stands, on a bounded sample of rows of the prefill
     workload: quantise those rows, INT8 GEMM + per-channel epilogue."""
@@ -626,6 +676,7 @@ def run_ours(args):
         for name in ("decode", "prefill", "mlp_down", "group", "tiny"):
             stages[name] = measure_workload(torch, qk, name, args.stage_iters, pk)
         stages["prefill_fp8"] = measure_fp8(torch, qk, args.stage_iters, pk)
+        stages["moe"] = measure_moe(torch, qk, args.stage_iters, pk)
         d = stages["decode"]
         gbs = d["bytes"]["gemm"] / (d["gemm_us"] * 1e-6) / 1e9
         decode = {"value": gbs, "unit": "GB/s", "workload": "decode linear X bf16 [4,4096] x W int8 "
@@ -681,7 +732,7 @@ def main():
                     help="dram__bytes_read.sum + dram__bytes_write.sum of one prefill GEMM launch")
     ap.add_argument("--gemv-traffic", type=float, default=GEMV_TRAFFIC_BYTES,
                     help="the same for one decode GEMV launch")
-    ap.add_argument("--only", choices=["tiny", "decode", "prefill", "mlp_down", "group", "prefill_fp8"],
+    ap.add_argument("--only", choices=["tiny", "decode", "prefill", "mlp_down", "group", "prefill_fp8", "moe"],
                     help="profiling aid: time one workload's stages and print them")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
@@ -692,8 +743,12 @@ def main():
 
         from w8a8_int8_quantized_qk_b200 import qk
 
-        res = (measure_fp8(torch, qk, args.steps, peaks()) if args.only == "prefill_fp8"
-               else measure_workload(torch, qk, args.only, args.steps, peaks()))
+        if args.only == "prefill_fp8":
+            res = measure_fp8(torch, qk, args.steps, peaks())
+        elif args.only == "moe":
+            res = measure_moe(torch, qk, args.steps, peaks())
+        else:
+            res = measure_workload(torch, qk, args.only, args.steps, peaks())
         print(json.dumps({"only": args.only, **res}), flush=True)
         return 0
     return run_ours(args)

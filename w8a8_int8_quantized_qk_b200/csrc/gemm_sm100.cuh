@@ -100,17 +100,30 @@ struct ChanTile {
 
 template <int BN, bool MOE>
 __device__ __forceinline__ bool chan_tile(const Args& p, int tile, ChanTile& t) {
-  const int tmg = tile % p.tiles_m, tn = tile / p.tiles_m;
   if constexpr (MOE) {
-    const int e = tmg / p.mt_max, tm = tmg % p.mt_max;
-    const int r0 = __ldg(p.moe_off + e), r1 = __ldg(p.moe_off + e + 1);
-    if (r0 + tm * BM >= r1) return false;
-    t.a_row0 = r0 + tm * BM;
-    t.row_end = r1 < p.m ? r1 : p.m;
-    t.b_row0 = e * p.n + tn * BN;
-    t.col0 = tn * BN;
-    t.sw = p.sw + static_cast<int64_t>(e) * p.n;
+    // compact numbering of the non-empty tiles: expert by expert, M tiles
+    // fastest; tile numbers past the last one are empty
+    const int experts = p.tiles_m / p.mt_max;
+    int u = tile;
+    for (int e = 0; e < experts; ++e) {
+      const int r0 = __ldg(p.moe_off + e), r1 = __ldg(p.moe_off + e + 1);
+      int mt = r1 > r0 ? (r1 - r0 + BM - 1) / BM : 0;
+      mt = mt < p.mt_max ? mt : p.mt_max;
+      const int cnt = mt * p.tiles_n;
+      if (u < cnt) {
+        const int tm = u % mt, tn = u / mt;
+        t.a_row0 = r0 + tm * BM;
+        t.row_end = r1 < p.m ? r1 : p.m;
+        t.b_row0 = e * p.n + tn * BN;
+        t.col0 = tn * BN;
+        t.sw = p.sw + static_cast<int64_t>(e) * p.n;
+        return true;
+      }
+      u -= cnt;
+    }
+    return false;
   } else {
+    const int tmg = tile % p.tiles_m, tn = tile / p.tiles_m;
     t.a_row0 = tmg * BM;
     t.row_end = p.m;
     t.b_row0 = tn * BN;
