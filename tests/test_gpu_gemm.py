@@ -162,6 +162,28 @@ def test_gemm_group(O, m, n, k):
     assert_bits(out_nc, out, "group out without c")
 
 
+# group mode without the int32 sums runs the 128 x 256 kernel: more tiles
+# than SMs (several per CTA), group counts that are not a multiple of the
+# 16-group scale slice (3, 17), ragged M and N edges, bf16 and fp32 outputs
+GROUP_WIDE_SHAPES = [(1100, 4360, 2176), (300, 2056, 384), (129, 264, 128)]
+
+
+@pytest.mark.parametrize("m,n,k", GROUP_WIDE_SHAPES)
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gemm_group_without_c(O, m, n, k, out_dtype):
+    a, w, sa, sw = _problem(m, n, k, 128, seed=m * 5 + n * 3 + k)
+    alpha = 0.75
+    out, c = _run(a, w, sa, sw, 128, alpha, out_dtype=out_dtype, want_c=False)
+    assert c is None
+    rows = _sample_rows(m, 24, seed=m + n) if m > 256 else np.arange(m)
+    ref = O.linear_from_q(a[rows], sa[rows], w, sw, 128, alpha)
+    if out_dtype == torch.float32:
+        assert_bits(out[rows], ref["out_f32"], "fp32 out")
+    else:
+        exact = check_out(out[rows], ref["out_f32"], ref["out_bf16"])
+        assert exact == 1.0, exact
+
+
 def test_gemm_saturating_closed_form(O):
     # all operands 127: acc = 16129 k at the largest k the bound allows (multiple of 128)
     k = 133120
@@ -224,3 +246,9 @@ def test_workload_full_size(O, name):
     else:
         exact = check_out(out_h[rows], ref["out_f32"], ref["out_bf16"])
         assert exact == 1.0, exact
+    # the output-only launch (the form the benchmark times; for group mode a
+    # different kernel) gives the same bits
+    out_only, _ = qk.w8a8_gemm(q, w_q, sa, sw, w.group_k, w.alpha, out_dtype, want_c=False)
+    torch.cuda.synchronize()
+    assert qk.device_status() == qk.QK_OK
+    assert_bits(host(out_only), out_h, "output-only launch")

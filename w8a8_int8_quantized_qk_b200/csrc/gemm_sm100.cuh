@@ -17,11 +17,13 @@
 //    columns per instruction), apply the scales and store the outputs;
 //  - per-channel mode keeps two 128 x 256 accumulators in TMEM (all 512
 //    columns), so the epilogue of tile i overlaps the MMAs of tile i+1;
-//  - per-group mode (group = 128 = one stage of K) keeps four 128 x 128
-//    int32 partial buffers in TMEM: the MMA writes one group's partial per
-//    buffer and moves on while eight epilogue warps convert each partial
-//    exactly to fp32 and fold it in with fmaf(P_g, s[n, g], f), in
-//    ascending group order, in registers.
+//  - per-group mode (group = 128 = one stage of K) keeps int32 partial
+//    buffers in TMEM: the MMA writes one group's partial per buffer and moves
+//    on while 16 epilogue warps convert each partial exactly to fp32 and fold
+//    it in with fmaf(P_g, s[n, g], f), in ascending group order, in
+//    registers.  128 x 256 tiles with two buffers when only the output is
+//    wanted; 128 x 128 tiles with four buffers when the int32 sums are also
+//    written.
 //
 // Every wait is bounded (about one second): on expiry the kernel records
 // QK_ERR_TIMEOUT, every role leaves its loop, the producer waits (bounded)
@@ -523,7 +525,7 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
 // broadcast float4 loads and never wait on global memory.
 //
 // Accumulation per element, in ascending group order as the definition
-// states: pf = (float)P_g (exact: |P_g| < 2^22, via the bits of 1.5 * 2^23),
+// states: pf = (float)P_g (exact: |P_g| <= 128 * 127^2 < 2^24),
 // f = fma(pf, sw[n, g], f).
 constexpr int kScaleGroups = 16;
 
@@ -538,7 +540,9 @@ struct GroupCfg {
   static constexpr int threads = 64 + epi_warps * 32 + 32;
 };
 
-template <int BN, class S>
+// CH column chunks of 32 (CH x kScaleGroups loads) are in flight together;
+// CH = BN / 32 makes the slice one memory round trip.
+template <int BN, int CH, class S>
 __device__ void stage_group_scales(S& s, const Args& p) {
   const int ntiles = p.tiles_m * p.tiles_n;
   const int lane = threadIdx.x & 31;
@@ -549,21 +553,23 @@ __device__ void stage_group_scales(S& s, const Args& p) {
     for (int b = 0; b < batches; ++b) {
       if (!warp_wait(smem_addr(&s.aux_empty[buf]), phase ^ 1u, &s.abort)) return;
       float* dst = s.scales + buf * (kScaleGroups * BN);
-      // all BN / 32 x kScaleGroups loads of the slice in flight together:
-      // one memory round trip per slice
-      float v[BN / 32][kScaleGroups];
 #pragma unroll
-      for (int i = 0; i < BN / 32; ++i) {
-        const int col = col0 + lane + 32 * i;
-        const float* src = p.sw + static_cast<int64_t>(col) * p.groups + b * kScaleGroups;
+      for (int i0 = 0; i0 < BN / 32; i0 += CH) {
+        float v[CH][kScaleGroups];
 #pragma unroll
-        for (int gg = 0; gg < kScaleGroups; ++gg)
-          v[i][gg] = (col < p.n && b * kScaleGroups + gg < p.groups) ? __ldg(src + gg) : 0.0f;
+        for (int i = 0; i < CH; ++i) {
+          const int col = col0 + lane + 32 * (i0 + i);
+          const float* src = p.sw + static_cast<int64_t>(col) * p.groups + b * kScaleGroups;
+#pragma unroll
+          for (int gg = 0; gg < kScaleGroups; ++gg)
+            v[i][gg] = (col < p.n && b * kScaleGroups + gg < p.groups) ? __ldg(src + gg) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < CH; ++i)
+#pragma unroll
+          for (int gg = 0; gg < kScaleGroups; ++gg)
+            dst[gg * BN + lane + 32 * (i0 + i)] = v[i][gg];
       }
-#pragma unroll
-      for (int i = 0; i < BN / 32; ++i)
-#pragma unroll
-        for (int gg = 0; gg < kScaleGroups; ++gg) dst[gg * BN + lane + 32 * i] = v[i][gg];
       mbar_arrive(smem_addr(&s.aux_full[buf]));  // release: this lane's stores
       if (++buf == 2) {
         buf = 0;
@@ -586,8 +592,8 @@ __device__ __forceinline__ void group_fma32(float (&f)[COLS], int (&cs)[NC],
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int j = j4 * 4 + e;
-      // |P| < 2^22: the bits of 1.5 * 2^23 plus P, minus 1.5 * 2^23, is (float)P exactly
-      const float pf = __fsub_rn(__int_as_float(static_cast<int>(v[j]) + 0x4B400000), 12582912.0f);
+      // |P| < 2^24: the conversion is exact
+      const float pf = __int2float_rn(static_cast<int>(v[j]));
       f[C0 + j] = __fmaf_rn(pf, sv[e], f[C0 + j]);
       if constexpr (NC == COLS) cs[C0 + j] += static_cast<int>(v[j]);
     }
@@ -893,7 +899,157 @@ __global__ void __launch_bounds__(GroupCfg<WITH_C>::threads, 1)
   } else if (warp < 2 + kEpiWarps) {
     epilogue_group<kGroupBN, 4, WITH_C>(s, tmem, p);
   } else {
-    stage_group_scales<kGroupBN>(s, p);
+    stage_group_scales<kGroupBN, kGroupBN / 32>(s, p);
+  }
+  teardown(s, tmem);
+}
+
+// ---------------------------------------------------------------- group-128, 128 x 256 tiles
+// Wide form of the group kernel, for outputs without the int32 sums.  The
+// 128 x 256 MMA (N = 256) reads fewer operand bytes per multiply-add than
+// 128 x 128, so the tensor pipe accepts a group's four MMAs faster; TMEM
+// holds two 256-column partial buffers, shared memory four 48 KB stages and
+// a 32 KB scale slice.
+//
+// Warpgroup 0: TMA producer (warp 0), MMA issuer (warp 1), scale stager
+// (warp 2), warp 3 idle.  Warpgroups 1-4: 16 epilogue warps; warp w owns
+// TMEM lanes 32*(w%4) and columns [64 h, 64 h + 64), h = (w - 4) / 4, so
+// each epilogue thread keeps 64 fp32 running sums.  The registers follow the
+// work: warpgroup 0 drops to 64 per thread and the epilogue rises to 104
+// (128*64 + 512*104 = 61440 = 640*96, the launch allocation).
+//
+// Per element and group: one exact int-to-float conversion and one fused
+// multiply-add, in ascending group order.  (Packed f32x2 pairs with the
+// 1.5 * 2^23 bias trick issue more instructions here, because forming the
+// pairs costs moves: 318.6 against 273.8 us at 2048 x 8192 x 8192.)
+constexpr int kGroupWideBN = 256;
+constexpr int kGroupWideStages = 4;
+constexpr int kGroupWideEpiWarps = 16;
+constexpr int kGroupWideCols = 64;  // columns per epilogue warp
+constexpr int kGroupWideThreads = 128 + kGroupWideEpiWarps * 32;
+constexpr int kGroupWideCtrlRegs = 64;
+constexpr int kGroupWideEpiRegs = 104;
+constexpr int kGroupWideLaunchRegs =  // registers per thread the launch must provide
+    (128 * kGroupWideCtrlRegs + kGroupWideEpiWarps * 32 * kGroupWideEpiRegs + kGroupWideThreads - 1) /
+    kGroupWideThreads;
+using GroupWideStorage =
+    Storage<kGroupWideBN, kGroupWideStages, 2, 2 * kScaleGroups * kGroupWideBN>;
+
+template <class S>
+__device__ void epilogue_group_wide(S& s, uint32_t tmem, const Args& p) {
+  constexpr int BN = kGroupWideBN, COLS = kGroupWideCols;
+  const int ntiles = p.tiles_m * p.tiles_n;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int quad = warp & 3;
+  const int sub = (warp - 4) >> 2;  // column slice of the tile
+  uint32_t abuf = 0, aphase = 0, sbuf = 0, sphase = 0;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    const int colbase = tn * BN + sub * COLS;
+    float fs[COLS];
+#pragma unroll
+    for (int j = 0; j < COLS; ++j) fs[j] = 0.0f;
+    for (int g = 0; g < p.groups; ++g) {
+      const int gs = g % kScaleGroups;
+      if (gs == 0 && !warp_wait(smem_addr(&s.aux_full[sbuf]), sphase, &s.abort)) {
+        ok = false;
+        break;
+      }
+      if (!warp_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN +
+                          sub * COLS;
+      const float4* sc4 = reinterpret_cast<const float4*>(s.scales + sbuf * (kScaleGroups * BN) +
+                                                          gs * BN + sub * COLS);
+#pragma unroll
+      for (int c = 0; c < COLS / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tb + c * 16, v);
+        tmem_ld_wait();
+        if (c == COLS / 16 - 1) release_acc<2>(s, abuf, aphase, lane);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 s4 = sc4[c * 4 + q];
+          const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = c * 16 + q * 4 + e;
+            // |P| < 2^24: the conversion is exact
+            fs[j] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * q + e])), sv[e], fs[j]);
+          }
+        }
+      }
+      if (gs == kScaleGroups - 1 || g + 1 == p.groups) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&s.aux_empty[sbuf]));
+        if (++sbuf == 2) {
+          sbuf = 0;
+          sphase ^= 1u;
+        }
+      }
+    }
+    if (!ok) break;
+    const int row = tm * BM + quad * 32 + lane;
+    if (row < p.m) {
+      const float sa = __ldg(p.sa + row);
+#pragma unroll
+      for (int g8 = 0; g8 < COLS / 8; ++g8) {
+        const int col = colbase + g8 * 8;
+        if (col >= p.n) break;
+        const int64_t o = static_cast<int64_t>(row) * p.n + col;
+        float r[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = __fmul_rn(__fmul_rn(fs[g8 * 8 + e], sa), p.alpha);
+        if (p.out_bf16) {
+          uint4 pk;
+          pk.x = pack_bf16x2(r[0], r[1]);
+          pk.y = pack_bf16x2(r[2], r[3]);
+          pk.z = pack_bf16x2(r[4], r[5]);
+          pk.w = pack_bf16x2(r[6], r[7]);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o) = pk;
+        } else {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
+          dst[0] = make_float4(r[0], r[1], r[2], r[3]);
+          dst[1] = make_float4(r[4], r[5], r[6], r[7]);
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGroupWideThreads, 1)
+    gemm_i8_group_wide_kernel(const __grid_constant__ CUtensorMap tmA,
+                              const __grid_constant__ CUtensorMap tmB, const Args p) {
+  extern __shared__ uint8_t smem_raw[];
+  GroupWideStorage& s = storage<GroupWideStorage>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  setup<GroupWideStorage, kGroupWideStages, 2, kGroupWideEpiWarps>(s);
+  griddep_wait();  // set-up above overlapped the previous kernel
+  griddep_launch_dependents();
+  const uint32_t tmem = s.tmem_base;
+  if (warp < 4) {
+    regs_dec<kGroupWideCtrlRegs>();
+    if (warp == 0) {
+      if (lane == 0) produce<kGroupWideBN, kGroupWideStages>(s, &tmA, &tmB, p);
+      __syncwarp();
+    } else if (warp == 1) {
+      if (lane == 0) mma_issue<kGroupWideBN, kGroupWideStages, 2, true>(s, tmem, p);
+      __syncwarp();
+    } else if (warp == 2) {
+      stage_group_scales<kGroupWideBN, 1>(s, p);
+    }
+  } else {
+    regs_inc<kGroupWideEpiRegs>();
+    epilogue_group_wide(s, tmem, p);
   }
   teardown(s, tmem);
 }
@@ -1760,6 +1916,25 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
   return e == cudaSuccess ? 0 : 2;
 }
 inline size_t group_smem() { return sizeof(GroupStorage) + 1024; }
+inline size_t group_wide_smem() { return sizeof(GroupWideStorage) + 1024; }
+
+// The wide group kernel moves registers between warpgroups with setmaxnreg;
+// the budgets only add up if the compiled kernel launches with at least
+// kGroupWideLaunchRegs registers per thread (otherwise the increase would
+// wait for registers that never come back).  Checked once per device.
+inline bool group_wide_ok(int dev) {
+  static int cache[64] = {};
+  if (dev < 0 || dev >= 64) return false;
+  if (cache[dev] == 0) {
+    cudaFuncAttributes fa;
+    const bool ok = cudaFuncGetAttributes(&fa, gemm_i8_group_wide_kernel) == cudaSuccess &&
+                    fa.numRegs >= kGroupWideLaunchRegs &&
+                    fa.numRegs * kGroupWideThreads <= 65536;
+    if (!ok) cudaGetLastError();
+    cache[dev] = ok ? 1 : -1;
+  }
+  return cache[dev] > 0;
+}
 
 // 0 ok, 1 tensor-map failure, 2 CUDA error
 // Largest number of co-resident clusters of `cluster` CTAs of the 1-SM
@@ -1839,7 +2014,9 @@ inline bool prefer_channel_split(int m, int n, int k, int num_sms, int dev) {
 
 inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev, int num_sms,
                   cudaStream_t stream, cudaError_t* err) {
-  const int bn = group ? kGroupBN : kChannelBN;
+  // group mode without the int32 sums: the 128 x 256 kernel
+  const bool wide = group && a.c == nullptr && group_wide_ok(dev);
+  const int bn = group ? (wide ? kGroupWideBN : kGroupBN) : kChannelBN;
   a.tiles_m = (a.m + BM - 1) / BM;
   a.tiles_n = (a.n + bn - 1) / bn;
   a.num_kb = (a.k + BK - 1) / BK;
@@ -1879,6 +2056,16 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
                      a.csplit ? static_cast<unsigned>(a.splits) : 1u, ta, tb, to, a);
     }
   } else {
+    if (wide) {
+      const size_t smem = group_wide_smem();
+      e = set_smem_once(gemm_i8_group_wide_kernel, dev, 7, smem);
+      if (e == cudaSuccess) {
+        e = launch_pdl(gemm_i8_group_wide_kernel, dim3(grid), dim3(kGroupWideThreads), smem, stream,
+                       1, ta, tb, a);
+      }
+      *err = e;
+      return e == cudaSuccess ? 0 : 2;
+    }
     const size_t smem = group_smem();
     if (a.c) {
       e = set_smem_once(gemm_i8_group_kernel<true>, dev, 2, smem);
