@@ -233,7 +233,10 @@ QK_API qk_status qk_w8a8_gemm(int m, int n, int k, const int8_t* a, const int8_t
  * m, n, k        k % 16 == 0, n % 8 == 0 (either of m, n 0: no-op)
  * The accumulation order inside the tensor core is the hardware's, so the
  * results match the exact dot product to within fp32 summation error, not
- * bit for bit.  No workspace (whole tiles, no split-K).
+ * bit for bit.  No workspace.  When the output tiles are too few to fill
+ * the GPU, each tile's K range is split over the CTAs of one cluster and
+ * the fp32 partials are added in ascending slice order through distributed
+ * shared memory, so the result does not depend on which CTA finishes first.
  * Errors: QK_ERR_INVALID_ARG, QK_ERR_MISALIGNED, QK_ERR_UNSUPPORTED,
  *         QK_ERR_CUDA.
  */

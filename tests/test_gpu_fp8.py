@@ -146,7 +146,14 @@ def _check_fp8(O, got, acc_exact, bound, sa, sw, alpha, bf16):
 
 
 FP8_GEMM_SHAPES = [(1, 64, 32), (4, 136, 272), (9, 256, 128), (100, 1032, 3008), (128, 256, 4096),
-                   (130, 264, 272), (257, 520, 1040), (300, 1000, 1552), (1024, 2048, 512)]
+                   (130, 264, 272), (257, 520, 1040), (300, 1000, 1552), (1024, 2048, 512),
+                   # K split over the CTAs of a cluster, fp32 partials added in
+                   # slice order: 1-SM kernel, clusters of 4 (few tiles, m <= 128)
+                   (64, 512, 8192),
+                   # CTA-pair kernel, cluster split-K (few tiles)
+                   (256, 1024, 8192),
+                   # CTA-pair kernel, more tiles than pairs (whole tiles)
+                   (2560, 2048, 2048)]
 
 
 @pytest.mark.parametrize("m,n,k", FP8_GEMM_SHAPES)
@@ -161,6 +168,20 @@ def test_fp8_gemm(O, m, n, k):
         torch.cuda.synchronize()
         assert qk.device_status() == qk.QK_OK
         _check_fp8(O, host(out), acc, bound, sa, sw, alpha, dt == torch.bfloat16)
+
+
+def test_fp8_gemm_split_deterministic():
+    # the cluster split-K adds the fp32 partials in slice order, whichever CTA
+    # finishes first: repeated launches give the same bits
+    need_gpu()
+    for m, n, k in ((256, 1024, 8192), (64, 512, 8192)):
+        a, w, sa, sw = (torch.from_numpy(t).cuda() for t in _fp8_problem(m, n, k, seed=m + n + k))
+        ref = qk.fp8_gemm(a, w, sa, sw, 1.0, torch.float32)
+        for _ in range(3):
+            again = qk.fp8_gemm(a, w, sa, sw, 1.0, torch.float32)
+            torch.cuda.synchronize()
+            assert torch.equal(again.view(torch.int32), ref.view(torch.int32))
+        assert qk.device_status() == qk.QK_OK
 
 
 def test_fp8_linear_chain(O):

@@ -319,6 +319,23 @@ __device__ __forceinline__ float acc_value(uint32_t v) {
   return __int2float_rn(static_cast<int>(v));
 }
 
+// Sum of two split-K partials: int32 (exact in any order) for the INT8 kind;
+// for the FP8 kind binary32, rounded to nearest.  The reductions add the
+// slices in ascending slice order, so that an FP8 result does not depend on
+// which CTA finishes first.
+template <bool F8>
+__device__ __forceinline__ uint32_t acc_add(uint32_t x, uint32_t y) {
+  if constexpr (F8) return __float_as_uint(__fadd_rn(__uint_as_float(x), __uint_as_float(y)));
+  return x + y;
+}
+template <bool F8>
+__device__ __forceinline__ void acc_add4(uint32_t* v, const int4& t) {
+  v[0] = acc_add<F8>(v[0], static_cast<uint32_t>(t.x));
+  v[1] = acc_add<F8>(v[1], static_cast<uint32_t>(t.y));
+  v[2] = acc_add<F8>(v[2], static_cast<uint32_t>(t.z));
+  v[3] = acc_add<F8>(v[3], static_cast<uint32_t>(t.w));
+}
+
 // Zero-point correction of 32 int32 accumulators of one row (columns col0 ..
 // col0 + 31): v -= zp[row] * wsum[col], in two's-complement arithmetic
 // (exact whenever the corrected sum fits in int32, which the host's bound
@@ -763,7 +780,7 @@ __device__ __forceinline__ void teardown(S& s, uint32_t tmem) {
 // loads in flight together; integer adds, exact), then dequantises and
 // stores.  The scales of the whole tile were staged in the warp's slot
 // before the accumulator was ready.
-template <int BN, class S>
+template <int BN, bool F8, class S>
 __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* tmO) {
   const int lane = threadIdx.x & 31;
   const int ew = (threadIdx.x >> 5) - 2;
@@ -780,8 +797,6 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
   for (int c = j; c < BN / 32; c += p.splits) {
     const int col0 = tn * BN + c * 32;
     uint32_t va[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) va[i] = 0;
     // every source's part of the chunk requested at once (32 loads in
     // flight per lane: one cluster round trip per chunk)
     int4 t4[4][8];
@@ -798,20 +813,25 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
     for (int o = 0; o < 4; ++o)
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) order_after_loads(t4[o][q4]);
+    // slice 0, then the others in ascending order
 #pragma unroll
-    for (int o = 0; o < 4; ++o)
+    for (int q4 = 0; q4 < 8; ++q4) {
+      va[q4 * 4] = static_cast<uint32_t>(t4[0][q4].x);
+      va[q4 * 4 + 1] = static_cast<uint32_t>(t4[0][q4].y);
+      va[q4 * 4 + 2] = static_cast<uint32_t>(t4[0][q4].z);
+      va[q4 * 4 + 3] = static_cast<uint32_t>(t4[0][q4].w);
+    }
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        va[q4 * 4] += t4[o][q4].x;
-        va[q4 * 4 + 1] += t4[o][q4].y;
-        va[q4 * 4 + 2] += t4[o][q4].z;
-        va[q4 * 4 + 3] += t4[o][q4].w;
+    for (int o = 1; o < 4; ++o)
+      if (o < p.splits) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[o][q4]);
       }
-    if (p.zp) apply_zp(p, row, col0, va);
+    if (!F8 && p.zp) apply_zp(p, row, col0, va);
     if (p.tma_out)
-      store32_tma(p, tmO, box, row0, col0, sa, sws + c * 32, va);
+      store32_tma<F8>(p, tmO, box, row0, col0, sa, sws + c * 32, va);
     else if (rv && col0 < p.n)
-      store32_channel(p, row, col0, sa, sws + c * 32, va);
+      store32_channel<F8>(p, row, col0, sa, sws + c * 32, va);
   }
   if (p.tma_out && lane == 0) bulk_wait_all();  // the output stores are complete
   __syncwarp();
@@ -864,7 +884,7 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
   }
   if (p.csplit) {
     cluster_sync_all();  // every CTA of the cluster has staged its partial
-    if (warp >= 2) channel_cluster_reduce<kChannelBN>(s, p, &tmO);
+    if (warp >= 2) channel_cluster_reduce<kChannelBN, F8>(s, p, &tmO);
     cluster_sync_all();  // the peers are done reading this CTA's slots
   }
   teardown(s, tmem);
@@ -1222,6 +1242,7 @@ __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uin
 // adds them to its own accumulator, still in TMEM (integer adds, exact in
 // any order), runs the per-channel epilogue and resets the counter.  No
 // slice waits for another.
+template <bool F8>
 __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region, uint32_t tb,
                                     int row, bool rv, float sa, int colbase, const float* sws,
                                     const CUtensorMap* tmO, uint8_t* box) {
@@ -1251,31 +1272,44 @@ __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region
   last = __shfl_sync(0xFFFFFFFFu, last, 0);
   if (!last) return;
   __threadfence();
+  // the slices in ascending order, this CTA's own from TMEM
 #pragma unroll 1
   for (int ch = 0; ch < 4; ++ch) {
-    tmem_ld_32x32b_x32(tb + ch * 32, va);
+    uint32_t own[32];
+    tmem_ld_32x32b_x32(tb + ch * 32, own);
 #pragma unroll 1
     for (int o = 0; o < S; ++o) {
-      if (o == u.slice) continue;
-      const int4* src =
-          reinterpret_cast<const int4*>(slots + (static_cast<int64_t>(o) * 16 + region) * kRegionInts);
       int4 t4[8];
+      if (o != u.slice) {
+        const int4* src = reinterpret_cast<const int4*>(
+            slots + (static_cast<int64_t>(o) * 16 + region) * kRegionInts);
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) t4[q4] = __ldcg(src + (ch * 8 + q4) * 32 + lane);
-      tmem_ld_wait();
+        for (int q4 = 0; q4 < 8; ++q4) t4[q4] = __ldcg(src + (ch * 8 + q4) * 32 + lane);
+      } else {
+        tmem_ld_wait();
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        va[q4 * 4] += t4[q4].x;
-        va[q4 * 4 + 1] += t4[q4].y;
-        va[q4 * 4 + 2] += t4[q4].z;
-        va[q4 * 4 + 3] += t4[q4].w;
+        for (int q4 = 0; q4 < 8; ++q4)
+          t4[q4] = make_int4(static_cast<int>(own[q4 * 4]), static_cast<int>(own[q4 * 4 + 1]),
+                             static_cast<int>(own[q4 * 4 + 2]), static_cast<int>(own[q4 * 4 + 3]));
+      }
+      if (o == 0) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          va[q4 * 4] = static_cast<uint32_t>(t4[q4].x);
+          va[q4 * 4 + 1] = static_cast<uint32_t>(t4[q4].y);
+          va[q4 * 4 + 2] = static_cast<uint32_t>(t4[q4].z);
+          va[q4 * 4 + 3] = static_cast<uint32_t>(t4[q4].w);
+        }
+      } else {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[q4]);
       }
     }
-    if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
+    if (!F8 && p.zp) apply_zp(p, row, colbase + ch * 32, va);
     if (p.tma_out)
-      store32_tma(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
+      store32_tma<F8>(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
     else if (rv)
-      store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
+      store32_channel<F8>(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
   }
   __syncwarp();
   if (lane == 0) *cnt = 0;  // ready for the next call
@@ -1321,9 +1355,9 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
                         half * (kPairBN / 2);
     uint32_t va[32], vb[32];
     if (tail) {
-      tail_slice_epilogue(p, u, region, tb, row, rv, sa, colbase, sws, tmO, box);
-    } else if constexpr (F8) {
-      // FP8 kind (fp32 accumulator; whole tiles only)
+      tail_slice_epilogue<F8>(p, u, region, tb, row, rv, sa, colbase, sws, tmO, box);
+    } else if (F8 && !p.csplit) {
+      // FP8 kind, whole tile (fp32 accumulator)
       auto emit = [&](int ch, const uint32_t(&v)[32]) {
         if (p.tma_out)
           store32_tma<true>(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, v);
@@ -1479,6 +1513,7 @@ __device__ void cluster_reduce_scales(PairStorage& s, const Args& p, uint32_t cr
   }
 }
 
+template <bool F8>
 __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t crank) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -1499,8 +1534,6 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
     const uint32_t slot = static_cast<uint32_t>(hh * 4 + ((quad + 2) & 3));  // staging warp of (quad, hh)
     const uint32_t off = base + slot * kSlotBytes + static_cast<uint32_t>((ch * 8 * 32 + lane) * 16);
     uint32_t va[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) va[i] = 0;
     // all sources' loads of this chunk in flight together (splits <= 4):
     // one round trip through the cluster per chunk
     int4 t4[4][8];
@@ -1516,18 +1549,23 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
     for (int o = 0; o < 4; ++o)
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) order_after_loads(t4[o][q4]);
+    // slice 0, then the others in ascending order
 #pragma unroll
-    for (int o = 0; o < 4; ++o)
+    for (int q4 = 0; q4 < 8; ++q4) {
+      va[q4 * 4] = static_cast<uint32_t>(t4[0][q4].x);
+      va[q4 * 4 + 1] = static_cast<uint32_t>(t4[0][q4].y);
+      va[q4 * 4 + 2] = static_cast<uint32_t>(t4[0][q4].z);
+      va[q4 * 4 + 3] = static_cast<uint32_t>(t4[0][q4].w);
+    }
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        va[q4 * 4] += t4[o][q4].x;
-        va[q4 * 4 + 1] += t4[o][q4].y;
-        va[q4 * 4 + 2] += t4[o][q4].z;
-        va[q4 * 4 + 3] += t4[o][q4].w;
+    for (int o = 1; o < 4; ++o)
+      if (o < p.splits) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[o][q4]);
       }
     const int col0 = tn * kPairBN + c * 32;
-    if (p.zp) apply_zp(p, row, col0, va);
-    if (rv && col0 < p.n) store32_channel(p, row, col0, sa, sws + t * 32, va);
+    if (!F8 && p.zp) apply_zp(p, row, col0, va);
+    if (rv && col0 < p.n) store32_channel<F8>(p, row, col0, sa, sws + t * 32, va);
   }
 }
 
@@ -1582,7 +1620,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (p.csplit) {
     if (warp >= 2) cluster_reduce_scales(s, p, crank);
     cluster_sync_all();  // every CTA of the cluster has staged its partial
-    if (warp >= 2) cluster_reduce_pair(s, p, crank);
+    if (warp >= 2) cluster_reduce_pair<F8>(s, p, crank);
   }
   tc_fence_before();
   __syncthreads();
@@ -1778,7 +1816,11 @@ struct PairPlan {
   int dp_tiles, tail_splits, tail_kbps;
 };
 
-inline PairPlan pair_plan(int m, int n, int k, int pairs, int dev) {
+// f8: the FP8 kind.  Its fp32 partials are summed in a fixed order, which
+// the cluster split-K gives; the workspace split-K adds them in arrival
+// order and is left to the INT8 kind, and the tail split measured slower
+// than whole tiles for FP8 (56.5 against 55.7 us at 4096^3).
+inline PairPlan pair_plan(int m, int n, int k, int pairs, int dev, bool f8 = false) {
   PairPlan pl;
   pl.tiles = ((m + kPairBM - 1) / kPairBM) * ((n + kPairBN - 1) / kPairBN);
   pl.csplit = 0;
@@ -1786,6 +1828,11 @@ inline PairPlan pair_plan(int m, int n, int k, int pairs, int dev) {
   pl.tail_splits = 1;
   pl.tail_kbps = 0;
   const int num_kb = (k + BK - 1) / BK;
+  if (pl.tiles > pairs && pairs > 0 && f8) {
+    pl.splits = 1;
+    pl.kb_per_split = num_kb;
+    return pl;
+  }
   if (pl.tiles > pairs && pairs > 0) {
     const int r = pl.tiles % pairs;
     int ts = r > 0 ? pairs / r : 1;
@@ -1823,12 +1870,16 @@ inline PairPlan pair_plan(int m, int n, int k, int pairs, int dev) {
       if (max_pair_clusters(dev, 2 * cs) < pl.tiles) continue;
       const int kbps = (num_kb + cs - 1) / cs;
       if ((num_kb + kbps - 1) / kbps != cs) continue;
-      if (kbps + 3.0 < cost_ws) {
+      if (kbps + 3.0 < cost_ws || f8) {
         pl.splits = cs;
         pl.kb_per_split = kbps;
         pl.csplit = 1;
       }
       break;
+    }
+    if (f8 && !pl.csplit) {
+      pl.splits = 1;
+      pl.kb_per_split = num_kb;
     }
   }
   return pl;
@@ -1864,15 +1915,13 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
   a.num_kb = (a.k + BK - 1) / BK;
   a.groups = 0;
   const int pairs = max_pairs(dev, num_sms);
-  PairPlan pl = pair_plan(a.m, a.n, a.k, pairs, dev);
+  PairPlan pl = pair_plan(a.m, a.n, a.k, pairs, dev, a.f8 != 0);
   if (!allow_split || static_cast<int64_t>(pl.tiles) * pl.splits > pairs) {
     // (split-K stages partials in the operand ring: one unit per pair)
     pl.splits = 1;
     pl.kb_per_split = a.num_kb;
   }
-  if (!allow_split || a.f8) {  // (the FP8 kind runs whole tiles only)
-    pl.splits = 1;
-    pl.kb_per_split = a.num_kb;
+  if (!allow_split) {
     pl.tail_splits = 1;
     pl.dp_tiles = pl.tiles;
   }
@@ -2025,7 +2074,7 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   a.kb_per_split = a.num_kb;
   a.csplit = 0;
   a.tail_splits = 1;
-  if (!group && !a.f8) {  // (the FP8 kind runs whole tiles only)
+  if (!group) {
     const ChannelPlan pl = channel_plan(a.m, a.n, a.k, num_sms, dev);
     if (pl.splits > 1) {
       a.splits = pl.splits;

@@ -457,7 +457,8 @@ qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
   const int8_t* ai = reinterpret_cast<const int8_t*>(a);
   const int8_t* bi = reinterpret_cast<const int8_t*>(b);
   // m <= 128: the 1-SM kernel (rows beyond m read as zero); otherwise the
-  // CTA-pair kernel; whole tiles only
+  // CTA-pair kernel.  Few tiles: split-K over the CTAs of a cluster (no
+  // workspace); otherwise whole tiles.
   const int r = m <= 128 ? gemm::launch(g, ai, bi, false, dev_id, dev->sms, s, &e)
                          : gemm::launch_pair(g, ai, bi, dev_id, dev->sms, nullptr, s, &e);
   if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
