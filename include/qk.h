@@ -201,10 +201,18 @@ QK_API qk_status qk_silu_mul_quant_per_token_fp8(int m, int k, const void* gate,
  *                are cut into 2 to 4 K slices that run first; every slice
  *                stores its INT32 partial in the workspace and the last to
  *                finish adds them up (the same 4 KB header, 16 MB left for
- *                the split-K accumulators, then 256 KB per partial).  It
+ *                the split-K accumulators, then 256 KB per partial).  In
+ *                group mode (the output-only form) the last partial wave's
+ *                tiles are instead cut at their middle K group: the first
+ *                part runs early on one CTA and leaves its fp32 running sums
+ *                in the workspace, the second runs last on another CTA and
+ *                continues them in the same group order, so the result is
+ *                unchanged (16 flags per cut tile, padded to 256 B, then
+ *                128 KB of sums per cut tile).  The workspace
  *                must be zero-filled before its first use; every completed
- *                call leaves the header and the split-K accumulators zero
- *                again (the partials past them need no initialisation), so
+ *                call leaves the header, the flags and the split-K
+ *                accumulators zero again (the partials and sums need no
+ *                initialisation), so
  *                one workspace (sized for the largest problem) can be
  *                reused across calls and shapes.  The call
  *                owns it until the work on `stream` completes: calls that

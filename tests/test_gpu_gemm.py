@@ -164,8 +164,11 @@ def test_gemm_group(O, m, n, k):
 
 # group mode without the int32 sums runs the 128 x 256 kernel: more tiles
 # than SMs (several per CTA), group counts that are not a multiple of the
-# 16-group scale slice (3, 17), ragged M and N edges, bf16 and fp32 outputs
-GROUP_WIDE_SHAPES = [(1100, 4360, 2176), (300, 2056, 384), (129, 264, 128)]
+# 16-group scale slice (3, 17), ragged M and N edges, bf16 and fp32 outputs.
+# With 148 SMs, 1100 x 4360 (162 tiles) and 1280 x 4096 (160 tiles) cut
+# their last wave's tiles at the middle group (17 groups: 8 + 9; 2 groups:
+# 1 + 1), one CTA continuing another's running sums.
+GROUP_WIDE_SHAPES = [(1100, 4360, 2176), (1280, 4096, 256), (300, 2056, 384), (129, 264, 128)]
 
 
 @pytest.mark.parametrize("m,n,k", GROUP_WIDE_SHAPES)

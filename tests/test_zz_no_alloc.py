@@ -85,3 +85,36 @@ def test_noalloc_without_split_k_and_scratch_bound():
     for m, n, k in [(200, 256, 131072), (256, 4096, 14336), (1024, 3072, 8192), (2000, 1800, 4096),
                     (4096, 4096, 4096), (4096, 14336, 4096), (2560, 2048, 4096), (9000, 2304, 8192)]:
         assert qk.qk_w8a8_gemm_workspace_size(m, n, k, 0) <= NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_group_split():
+    # group mode, output only: on 148 SMs the 160 tiles of 128 x 256 cut the
+    # last wave's 12 tiles at their middle group, whose running sums pass
+    # through the scratch (one counter per tile, left zero for the next call)
+    need_gpu()
+    m, n, k = 1280, 4096, 1024
+    need = qk.qk_w8a8_gemm_workspace_size(m, n, k, 128)
+    assert need <= NOALLOC_SCRATCH_BYTES
+    r = synth.streams(11, ["a", "w", "sa", "sw"])
+    a = dev(synth.int8_uniform(r["a"], (m, k)))
+    w = dev(synth.int8_uniform(r["w"], (n, k)))
+    sa = dev(synth.scales_uniform(r["sa"], (m,), 0.001, 0.05))
+    sw = dev(synth.scales_uniform(r["sw"], (n, k // 128)))
+    ws = torch.zeros((max(need, 1),), dtype=torch.uint8, device="cuda")
+    ref = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    st = qk.qk_w8a8_gemm(m, n, k, qk._ptr(a), qk._ptr(w), qk._ptr(sa), qk._ptr(sw), 128, 1.0, None,
+                         qk._ptr(ref), qk.QK_BF16, qk._ptr(ws), ws.numel(), qk._stream())
+    assert st == qk.QK_OK, qk.qk_status_string(st)
+    for _ in range(2):
+        out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+        st = qk.qk_w8a8_gemm_noalloc(m, n, k, qk._ptr(a), qk._ptr(w), qk._ptr(sa), qk._ptr(sw), 128,
+                                     1.0, None, qk._ptr(out), qk.QK_BF16, qk._stream())
+        assert st == qk.QK_OK, qk.qk_status_string(st)
+        torch.cuda.synchronize()
+        assert qk.device_status() == qk.QK_OK
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    # the regular call left its counters zero: the workspace's first 256 bytes
+    assert int(ws[:256].count_nonzero()) == 0
+    # every group-mode split fits the built-in scratch (at most 74 cut tiles)
+    for m, n, k in [(2048, 8192, 8192), (4096, 14336, 4096), (9472, 4096, 1024), (640, 9472, 2048)]:
+        assert qk.qk_w8a8_gemm_workspace_size(m, n, k, 128) <= NOALLOC_SCRATCH_BYTES

@@ -77,7 +77,8 @@ struct Args {
   // tail paths
   int tma_out;
   // 1: a and b are float8 e4m3 codes, the MMA is kind::f8f6f4 and the
-  // accumulator fp32 (channel and pair kernels, whole tiles only, no c)
+  // accumulator fp32 (channel and pair kernels, whole tiles or the cluster
+  // split-K, no c)
   int f8;
   // asymmetric activations (per channel only): zp [m] zero-points and wsum
   // [n] = sum_k b[n][k]; the epilogues use acc - zp[m] * wsum[n]
@@ -89,7 +90,49 @@ struct Args {
   // expert's tokens are skipped
   int mt_max;
   const int32_t* moe_off;
+  // wide group kernel, the last wave split along K (gsplit > 0): tiles
+  // [0, tiles - gsplit) run whole; tail tile (tiles - gsplit + j) is cut at
+  // group gmid.  Its first part is CTA j's first unit: it leaves its fp32
+  // running sums in gstate and sets the tile's 16 region flags in gflag.
+  // Its second part is CTA (gsplit + j)'s last unit: it waits for the flags,
+  // continues the sums in the same group order and leaves the flags zero.
+  int gsplit, gmid;
+  float* gstate;
+  int* gflag;
 };
+
+// Work unit of the wide group kernel: groups [g0, g1) of output tile
+// `tile`; part 0 whole, 1 the first part of a split tile, 2 its second.
+struct GroupUnit {
+  int tile, g0, g1, part;
+};
+
+// The i-th unit of this CTA (false past its last); every role walks the
+// same list.  Without the split, tiles blockIdx.x, + gridDim.x, ...; with
+// it (gsplit = r tail tiles, 2 r <= gridDim.x, whole tiles a multiple of
+// the grid), CTA j < r first takes the first part of tail tile j, and CTA
+// r + j takes the second part of tail tile j after its whole tiles.
+__device__ __forceinline__ bool group_unit(const Args& p, int i, GroupUnit& u) {
+  const int c = static_cast<int>(blockIdx.x), P = static_cast<int>(gridDim.x), r = p.gsplit;
+  const int dp = p.tiles_m * p.tiles_n - r;
+  if (c < r) {
+    if (i == 0) {
+      u = {dp + c, 0, p.gmid, 1};
+      return true;
+    }
+    --i;
+  }
+  const int t = c + i * P;
+  if (t < dp) {
+    u = {t, 0, p.groups, 0};
+    return true;
+  }
+  if (c >= r && c < 2 * r && i == (dp - c + P - 1) / P) {
+    u = {dp + c - r, p.gmid, p.groups, 2};
+    return true;
+  }
+  return false;
+}
 
 // One output tile of the 1-SM kernels: A rows from a_row0 (rows from row_end
 // on belong to another expert, or to none, and are masked), B rows from
@@ -166,17 +209,31 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // ---------------------------------------------------------------- producer
-template <int BN, int STAGES, bool MOE = false, class S>
+// GUNITS: the wide group kernel's unit list (group_unit); otherwise units
+// blockIdx.x, + gridDim.x, ... of tiles x splits.
+template <int BN, int STAGES, bool MOE = false, bool GUNITS = false, class S>
 __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, const Args& p) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   const uint32_t bytes = static_cast<uint32_t>((BM + BN) * BK);
   uint32_t stage = 0, phase = 0, issued = 0;
   bool ok = true;
-  for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
+  for (int i = 0; ok; ++i) {
     ChanTile t;
-    if (!chan_tile<BN, MOE>(p, unit / p.splits, t)) continue;
-    const int kb0 = (unit % p.splits) * p.kb_per_split;
-    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+    int kb0, kb1;
+    if constexpr (GUNITS) {
+      GroupUnit gu;
+      if (!group_unit(p, i, gu)) break;
+      t.a_row0 = (gu.tile % p.tiles_m) * BM;
+      t.b_row0 = (gu.tile / p.tiles_m) * BN;
+      kb0 = gu.g0;
+      kb1 = gu.g1;
+    } else {
+      const int unit = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+      if (unit >= nunits) break;
+      if (!chan_tile<BN, MOE>(p, unit / p.splits, t)) continue;
+      kb0 = (unit % p.splits) * p.kb_per_split;
+      kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+    }
     for (int kb = kb0; kb < kb1; ++kb) {
       if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, &s.abort)) {
         ok = false;
@@ -203,19 +260,30 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
 // ---------------------------------------------------------------- MMA issuer
 // GROUP: one accumulator buffer per K block (each K block is one group);
 // otherwise one buffer per tile.
-template <int BN, int STAGES, int NACC, bool GROUP, bool F8 = false, bool MOE = false, class S>
+template <int BN, int STAGES, int NACC, bool GROUP, bool F8 = false, bool MOE = false,
+          bool GUNITS = false, class S>
 __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
   const int nunits = p.tiles_m * p.tiles_n * p.splits;
   constexpr uint32_t idesc = F8 ? idesc_e4m3(BM, BN) : idesc_i8(BM, BN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
-  for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x) {
-    if constexpr (MOE) {
-      ChanTile t;
-      if (!chan_tile<BN, true>(p, unit, t)) continue;
+  for (int i = 0; ok; ++i) {
+    int kb0, kb1;
+    if constexpr (GUNITS) {
+      GroupUnit gu;
+      if (!group_unit(p, i, gu)) break;
+      kb0 = gu.g0;
+      kb1 = gu.g1;
+    } else {
+      const int unit = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+      if (unit >= nunits) break;
+      if constexpr (MOE) {
+        ChanTile t;
+        if (!chan_tile<BN, true>(p, unit, t)) continue;
+      }
+      kb0 = (unit % p.splits) * p.kb_per_split;
+      kb1 = min(p.num_kb, kb0 + p.kb_per_split);
     }
-    const int kb0 = (unit % p.splits) * p.kb_per_split;
-    const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
     if (!GROUP) {
       if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) break;
       tc_fence_after();
@@ -559,33 +627,57 @@ struct GroupCfg {
 
 // CH column chunks of 32 (CH x kScaleGroups loads) are in flight together;
 // CH = BN / 32 makes the slice one memory round trip.
-template <int BN, int CH, class S>
+// A unit's groups [g0, g1) are staged in slices of kScaleGroups from g0 on
+// (GUNITS: the wide kernel's unit list; otherwise whole tiles).
+template <int BN, int CH, bool GUNITS, class S>
 __device__ void stage_group_scales(S& s, const Args& p) {
   const int ntiles = p.tiles_m * p.tiles_n;
   const int lane = threadIdx.x & 31;
-  const int batches = (p.groups + kScaleGroups - 1) / kScaleGroups;
   uint32_t buf = 0, phase = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int col0 = (tile / p.tiles_m) * BN;
+  for (int i = 0;; ++i) {
+    GroupUnit u;
+    if constexpr (GUNITS) {
+      if (!group_unit(p, i, u)) break;
+    } else {
+      u = {static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x), 0, p.groups, 0};
+      if (u.tile >= ntiles) break;
+    }
+    const int col0 = (u.tile / p.tiles_m) * BN;
+    const int batches = (u.g1 - u.g0 + kScaleGroups - 1) / kScaleGroups;
+    if (GUNITS && u.part == 2) {
+      // the first part's running sums (written by another CTA) must be
+      // complete before this unit's first slice is published
+      bool seen = true;
+      if (lane == 0) {
+        int* cnt = p.gflag + (u.tile - (ntiles - p.gsplit));
+        seen = flag_wait(cnt, 16, &s.abort);
+        if (seen) {
+          __threadfence();
+          *cnt = 0;  // ready for the next call
+        }
+      }
+      if (!__shfl_sync(0xFFFFFFFFu, seen ? 1 : 0, 0)) return;
+    }
     for (int b = 0; b < batches; ++b) {
       if (!warp_wait(smem_addr(&s.aux_empty[buf]), phase ^ 1u, &s.abort)) return;
       float* dst = s.scales + buf * (kScaleGroups * BN);
+      const int gb = u.g0 + b * kScaleGroups;  // first group of the slice
 #pragma unroll
       for (int i0 = 0; i0 < BN / 32; i0 += CH) {
         float v[CH][kScaleGroups];
 #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          const int col = col0 + lane + 32 * (i0 + i);
-          const float* src = p.sw + static_cast<int64_t>(col) * p.groups + b * kScaleGroups;
+        for (int c = 0; c < CH; ++c) {
+          const int col = col0 + lane + 32 * (i0 + c);
+          const float* src = p.sw + static_cast<int64_t>(col) * p.groups + gb;
 #pragma unroll
           for (int gg = 0; gg < kScaleGroups; ++gg)
-            v[i][gg] = (col < p.n && b * kScaleGroups + gg < p.groups) ? __ldg(src + gg) : 0.0f;
+            v[c][gg] = (col < p.n && gb + gg < u.g1) ? __ldg(src + gg) : 0.0f;
         }
 #pragma unroll
-        for (int i = 0; i < CH; ++i)
+        for (int c = 0; c < CH; ++c)
 #pragma unroll
           for (int gg = 0; gg < kScaleGroups; ++gg)
-            dst[gg * BN + lane + 32 * (i0 + i)] = v[i][gg];
+            dst[gg * BN + lane + 32 * (i0 + c)] = v[c][gg];
       }
       mbar_arrive(smem_addr(&s.aux_full[buf]));  // release: this lane's stores
       if (++buf == 2) {
@@ -919,7 +1011,7 @@ __global__ void __launch_bounds__(GroupCfg<WITH_C>::threads, 1)
   } else if (warp < 2 + kEpiWarps) {
     epilogue_group<kGroupBN, 4, WITH_C>(s, tmem, p);
   } else {
-    stage_group_scales<kGroupBN, kGroupBN / 32>(s, p);
+    stage_group_scales<kGroupBN, kGroupBN / 32, false>(s, p);
   }
   teardown(s, tmem);
 }
@@ -955,6 +1047,17 @@ constexpr int kGroupWideLaunchRegs =  // registers per thread the launch must pr
 using GroupWideStorage =
     Storage<kGroupWideBN, kGroupWideStages, 2, 2 * kScaleGroups * kGroupWideBN>;
 
+// A split tile's running sums in the workspace: [tail tile][region]
+// [column][lane], so each column's 32 rows are one 128-byte line.  Each of
+// the 16 epilogue warps of the first part adds 1 to the tile's counter
+// gflag[tail tile] once its region is written.  In the CTA running the
+// second part, the scale stager waits for 16 (bounded) before it publishes
+// the part's first scale slice, and leaves the counter zero for the next
+// call; the epilogue warps read the sums after that slice's barrier.
+__device__ __forceinline__ float* group_state(const Args& p, int tt, int region) {
+  return p.gstate + (static_cast<int64_t>(tt) * 16 + region) * (kGroupWideCols * 32);
+}
+
 template <class S>
 __device__ void epilogue_group_wide(S& s, uint32_t tmem, const Args& p) {
   constexpr int BN = kGroupWideBN, COLS = kGroupWideCols;
@@ -963,19 +1066,28 @@ __device__ void epilogue_group_wide(S& s, uint32_t tmem, const Args& p) {
   const int warp = threadIdx.x >> 5;
   const int quad = warp & 3;
   const int sub = (warp - 4) >> 2;  // column slice of the tile
+  const int region = warp - 4;  // 0..15
   uint32_t abuf = 0, aphase = 0, sbuf = 0, sphase = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+  GroupUnit u;
+  for (int i = 0; ok && group_unit(p, i, u); ++i) {
+    const int tm = u.tile % p.tiles_m, tn = u.tile / p.tiles_m;
     const int colbase = tn * BN + sub * COLS;
     float fs[COLS];
 #pragma unroll
     for (int j = 0; j < COLS; ++j) fs[j] = 0.0f;
-    for (int g = 0; g < p.groups; ++g) {
-      const int gs = g % kScaleGroups;
+    for (int g = u.g0; g < u.g1; ++g) {
+      const int gs = (g - u.g0) % kScaleGroups;
       if (gs == 0 && !warp_wait(smem_addr(&s.aux_full[sbuf]), sphase, &s.abort)) {
         ok = false;
         break;
+      }
+      if (u.part == 2 && g == u.g0) {
+        // continue from the first part's sums (another CTA's; the stager
+        // saw them complete before publishing this slice)
+        const float* st = group_state(p, u.tile - (ntiles - p.gsplit), region) + lane;
+#pragma unroll
+        for (int j = 0; j < COLS; ++j) fs[j] = __ldcg(st + j * 32);
       }
       if (!warp_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) {
         ok = false;
@@ -1004,7 +1116,7 @@ __device__ void epilogue_group_wide(S& s, uint32_t tmem, const Args& p) {
           }
         }
       }
-      if (gs == kScaleGroups - 1 || g + 1 == p.groups) {
+      if (gs == kScaleGroups - 1 || g + 1 == u.g1) {
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(&s.aux_empty[sbuf]));
         if (++sbuf == 2) {
@@ -1014,6 +1126,17 @@ __device__ void epilogue_group_wide(S& s, uint32_t tmem, const Args& p) {
       }
     }
     if (!ok) break;
+    if (u.part == 1) {
+      // hand the running sums to the CTA that finishes the tile
+      const int tt = u.tile - (ntiles - p.gsplit);
+      float* st = group_state(p, tt, region) + lane;
+#pragma unroll
+      for (int j = 0; j < COLS; ++j) __stcg(st + j * 32, fs[j]);
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicAdd(p.gflag + tt, 1);
+      continue;
+    }
     const int row = tm * BM + quad * 32 + lane;
     if (row < p.m) {
       const float sa = __ldg(p.sa + row);
@@ -1059,13 +1182,13 @@ __global__ void __launch_bounds__(kGroupWideThreads, 1)
   if (warp < 4) {
     regs_dec<kGroupWideCtrlRegs>();
     if (warp == 0) {
-      if (lane == 0) produce<kGroupWideBN, kGroupWideStages>(s, &tmA, &tmB, p);
+      if (lane == 0) produce<kGroupWideBN, kGroupWideStages, false, true>(s, &tmA, &tmB, p);
       __syncwarp();
     } else if (warp == 1) {
-      if (lane == 0) mma_issue<kGroupWideBN, kGroupWideStages, 2, true>(s, tmem, p);
+      if (lane == 0) mma_issue<kGroupWideBN, kGroupWideStages, 2, true, false, false, true>(s, tmem, p);
       __syncwarp();
     } else if (warp == 2) {
-      stage_group_scales<kGroupWideBN, 1>(s, p);
+      stage_group_scales<kGroupWideBN, 1, true>(s, p);
     }
   } else {
     regs_inc<kGroupWideEpiRegs>();
@@ -1967,6 +2090,28 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
 inline size_t group_smem() { return sizeof(GroupStorage) + 1024; }
 inline size_t group_wide_smem() { return sizeof(GroupWideStorage) + 1024; }
 
+// K split of the wide group kernel's last wave (Args::gsplit): with T tiles
+// on P = min(T, num_sms) CTAs and T = q P + r, the r tail tiles are cut in
+// two when 0 < 2 r <= P and there are at least two groups, so that CTAs
+// 0 .. 2r - 1 each run q tiles and one part (q + 1/2 tiles where whole tiles
+// would take q + 1).  Returns r, or 0 when the split is off.
+inline int group_split_tiles(int m, int n, int k, int num_sms) {
+  const int tiles = ((m + BM - 1) / BM) * ((n + kGroupWideBN - 1) / kGroupWideBN);
+  if (num_sms <= 0 || tiles <= num_sms || k / 128 < 2) return 0;
+  const int r = tiles % num_sms;
+  return (r > 0 && 2 * r <= num_sms) ? r : 0;
+}
+// Its workspace: one arrival counter per tail tile (zero before a call,
+// zero after it), padded to 256 bytes, then each tail tile's running sums,
+// 128 x 256 fp32.
+inline size_t group_flag_bytes(int r) {
+  return (static_cast<size_t>(r) * sizeof(int) + 255) & ~static_cast<size_t>(255);
+}
+inline size_t group_workspace_bytes(int r) {
+  return r > 0 ? group_flag_bytes(r) + static_cast<size_t>(r) * BM * kGroupWideBN * sizeof(float)
+               : 0;
+}
+
 // The wide group kernel moves registers between warpgroups with setmaxnreg;
 // the budgets only add up if the compiled kernel launches with at least
 // kGroupWideLaunchRegs registers per thread (otherwise the increase would
@@ -2061,8 +2206,10 @@ inline bool prefer_channel_split(int m, int n, int k, int num_sms, int dev) {
   return cp.kb_per_split < pair_kb;
 }
 
+// `workspace`: group_workspace_bytes(group_split_tiles(...)) bytes for the
+// wide group kernel's split (null: whole tiles only); unused otherwise.
 inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev, int num_sms,
-                  cudaStream_t stream, cudaError_t* err) {
+                  cudaStream_t stream, cudaError_t* err, void* workspace = nullptr) {
   // group mode without the int32 sums: the 128 x 256 kernel
   const bool wide = group && a.c == nullptr && group_wide_ok(dev);
   const int bn = group ? (wide ? kGroupWideBN : kGroupBN) : kChannelBN;
@@ -2106,6 +2253,12 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
     }
   } else {
     if (wide) {
+      a.gsplit = workspace ? group_split_tiles(a.m, a.n, a.k, num_sms) : 0;
+      a.gmid = a.groups / 2;
+      a.gflag = static_cast<int*>(workspace);
+      a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                     group_flag_bytes(a.gsplit))
+                          : nullptr;
       const size_t smem = group_wide_smem();
       e = set_smem_once(gemm_i8_group_wide_kernel, dev, 7, smem);
       if (e == cudaSuccess) {

@@ -104,6 +104,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Wait until the global counter `*flag` reaches `target` (other CTAs of the
+// same grid add to it after a __threadfence).  Gives up like mbar_wait: on
+// the shared `abort` flag, or after kWaitLimitNs (records QK_ERR_TIMEOUT and
+// sets `abort`).  Returns true when the target was seen.
+__device__ __forceinline__ bool flag_wait(const int* flag, int target, volatile int* abort) {
+  const volatile int* f = flag;
+  if (*f >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(256);
+    if (*f >= target) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_status(QK_ERR_TIMEOUT);
+      if (abort != nullptr) *abort = 1;
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (bulk tensor copy global -> shared, completion on an mbarrier)
 // ---------------------------------------------------------------------------
@@ -192,16 +212,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-// 32 lanes x 32 bits, 8 consecutive columns.
-__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
       : "r"(taddr)
       : "memory");
 }

@@ -228,7 +228,19 @@ bool pair_plan_for(int m, int n, int k, int group_k, gemm::PairPlan* pl) {
 }
 }  // namespace
 
+namespace {
+// Tail tiles of the group kernel's K split for this problem on the current
+// device (0: no split, or not group mode, or bad arguments).
+int group_split_for(int m, int n, int k, int group_k) {
+  if (group_k == 0 || gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return 0;
+  const DeviceInfo* dev = nullptr;
+  if (check_device(&dev) != QK_OK) return 0;
+  return gemm::group_split_tiles(m, n, k, dev->sms);
+}
+}  // namespace
+
 size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
+  if (group_k != 0) return gemm::group_workspace_bytes(group_split_for(m, n, k, group_k));
   gemm::PairPlan pl;
   return pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_bytes(pl) : 0;
 }
@@ -417,7 +429,8 @@ qk_status gemm_common(int m, int n, int k, const int8_t* a, const int8_t* b,
   if (path == GemmPath::kTensorPair) {
     r = gemm::launch_pair(g, a, b, dev_id, dev->sms, workspace, s, &e);
   } else {
-    r = gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev_id, dev->sms, s, &e);
+    r = gemm::launch(g, a, b, path == GemmPath::kTensorGroup, dev_id, dev->sms, s, &e,
+                     need > 0 ? workspace : nullptr);
   }
   if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
   return r == 0 ? QK_OK : cuda_status(e, "gemm launch");
@@ -526,10 +539,14 @@ qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_
   if (need > QK_NOALLOC_SCRATCH_BYTES) return QK_ERR_WORKSPACE;
   void* scratch = noalloc_scratch();
   if (scratch == nullptr) return QK_ERR_CUDA;
-  // The arrival counters and the split-K accumulators must start at zero
-  // (the tail split's partials need no initialisation).
+  // The arrival counters, the group split's flags and the split-K
+  // accumulators must start at zero (partials and running sums need no
+  // initialisation).
   gemm::PairPlan pl;
-  const size_t zero = pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_zero_bytes(pl) : need;
+  const int gsplit = group_split_for(m, n, k, group_k);
+  const size_t zero = gsplit > 0 ? gemm::group_flag_bytes(gsplit)
+                      : pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_zero_bytes(pl)
+                                                             : need;
   if (cudaMemsetAsync(scratch, 0, zero, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return QK_ERR_CUDA;
   return qk_w8a8_gemm(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
