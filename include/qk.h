@@ -207,8 +207,9 @@ QK_API qk_status qk_silu_mul_quant_per_token_fp8(int m, int k, const void* gate,
  *                part runs early on one CTA and leaves its fp32 running sums
  *                in the workspace, the second runs last on another CTA and
  *                continues them in the same group order, so the result is
- *                unchanged (16 flags per cut tile, padded to 256 B, then
- *                128 KB of sums per cut tile).  The workspace
+ *                unchanged (one counter per cut tile in the 4 KB header, the
+ *                sums, 128 KB per cut tile, past the 16 MB of split-K
+ *                accumulators).  The workspace
  *                must be zero-filled before its first use; every completed
  *                call leaves the header, the flags and the split-K
  *                accumulators zero again (the partials and sums need no

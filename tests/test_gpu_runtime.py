@@ -67,6 +67,38 @@ def test_split_k_workspace_left_zero():
         assert all(np.array_equal(outs[0], o) for o in outs[1:])
 
 
+def test_group_split_leaves_shared_workspace_usable():
+    # group mode's last-wave split passes running sums through the workspace;
+    # they must land past the counters and split-K accumulators, so that a
+    # per-channel split-K call can reuse the same workspace right after
+    need_gpu()
+    mg, ng, kg = 1280, 4096, 1024  # 160 group tiles on 148 SMs: 12 cut tiles
+    mc, nc, kc = 256, 8960, 4096   # per-channel split-K through the workspace
+    need = max(qk.qk_w8a8_gemm_workspace_size(mg, ng, kg, 128),
+               qk.qk_w8a8_gemm_workspace_size(mc, nc, kc, 0))
+    ws = torch.zeros((need,), dtype=torch.uint8, device="cuda")
+    r = synth.streams(21, ["a", "w", "sa", "sw", "a2", "w2", "sa2", "sw2"])
+    ag = dev(synth.int8_uniform(r["a"], (mg, kg)))
+    wg = dev(synth.int8_uniform(r["w"], (ng, kg)))
+    sag = dev(synth.scales_uniform(r["sa"], (mg,), 0.001, 0.05))
+    swg = dev(synth.scales_uniform(r["sw"], (ng, kg // 128)))
+    ac = dev(synth.int8_uniform(r["a2"], (mc, kc)))
+    wc = dev(synth.int8_uniform(r["w2"], (nc, kc)))
+    sac = dev(synth.scales_uniform(r["sa2"], (mc,), 0.001, 0.05))
+    swc = dev(synth.scales_uniform(r["sw2"], (nc,)))
+    ref_c, _ = qk.w8a8_gemm(ac, wc, sac, swc, workspace=torch.zeros_like(ws))
+    ref_g, _ = qk.w8a8_gemm(ag, wg, sag, swg, 128, workspace=torch.zeros_like(ws))
+    for _ in range(2):
+        out_g, _ = qk.w8a8_gemm(ag, wg, sag, swg, 128, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws[:4096 + (16 << 20)].count_nonzero()) == 0
+        out_c, _ = qk.w8a8_gemm(ac, wc, sac, swc, workspace=ws)
+        torch.cuda.synchronize()
+        assert qk.device_status() == qk.QK_OK
+        assert torch.equal(out_g.view(torch.int16), ref_g.view(torch.int16))
+        assert torch.equal(out_c.view(torch.int16), ref_c.view(torch.int16))
+
+
 def test_graph_capture_of_the_layer():
     # the same quantise + GEMM calls captured into a CUDA graph and replayed
     # (as the benchmark runs them) give the eager results, including the

@@ -905,20 +905,30 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
     for (int o = 0; o < 4; ++o)
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) order_after_loads(t4[o][q4]);
-    // slice 0, then the others in ascending order
+    if constexpr (F8) {
+      // slice 0, then the others in ascending order (fp32: order matters)
 #pragma unroll
-    for (int q4 = 0; q4 < 8; ++q4) {
-      va[q4 * 4] = static_cast<uint32_t>(t4[0][q4].x);
-      va[q4 * 4 + 1] = static_cast<uint32_t>(t4[0][q4].y);
-      va[q4 * 4 + 2] = static_cast<uint32_t>(t4[0][q4].z);
-      va[q4 * 4 + 3] = static_cast<uint32_t>(t4[0][q4].w);
-    }
-#pragma unroll
-    for (int o = 1; o < 4; ++o)
-      if (o < p.splits) {
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[o][q4]);
+      for (int q4 = 0; q4 < 8; ++q4) {
+        va[q4 * 4] = static_cast<uint32_t>(t4[0][q4].x);
+        va[q4 * 4 + 1] = static_cast<uint32_t>(t4[0][q4].y);
+        va[q4 * 4 + 2] = static_cast<uint32_t>(t4[0][q4].z);
+        va[q4 * 4 + 3] = static_cast<uint32_t>(t4[0][q4].w);
       }
+#pragma unroll
+      for (int o = 1; o < 4; ++o)
+        if (o < p.splits) {
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) acc_add4<true>(va + q4 * 4, t4[o][q4]);
+        }
+    } else {
+      // int32: any order (sources past `splits` were loaded as zero)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) va[i] = 0;
+#pragma unroll
+      for (int o = 0; o < 4; ++o)
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) acc_add4<false>(va + q4 * 4, t4[o][q4]);
+    }
     if (!F8 && p.zp) apply_zp(p, row, col0, va);
     if (p.tma_out)
       store32_tma<F8>(p, tmO, box, row0, col0, sa, sws + c * 32, va);
@@ -1672,20 +1682,30 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
     for (int o = 0; o < 4; ++o)
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) order_after_loads(t4[o][q4]);
-    // slice 0, then the others in ascending order
+    if constexpr (F8) {
+      // slice 0, then the others in ascending order (fp32: order matters)
 #pragma unroll
-    for (int q4 = 0; q4 < 8; ++q4) {
-      va[q4 * 4] = static_cast<uint32_t>(t4[0][q4].x);
-      va[q4 * 4 + 1] = static_cast<uint32_t>(t4[0][q4].y);
-      va[q4 * 4 + 2] = static_cast<uint32_t>(t4[0][q4].z);
-      va[q4 * 4 + 3] = static_cast<uint32_t>(t4[0][q4].w);
-    }
-#pragma unroll
-    for (int o = 1; o < 4; ++o)
-      if (o < p.splits) {
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[o][q4]);
+      for (int q4 = 0; q4 < 8; ++q4) {
+        va[q4 * 4] = static_cast<uint32_t>(t4[0][q4].x);
+        va[q4 * 4 + 1] = static_cast<uint32_t>(t4[0][q4].y);
+        va[q4 * 4 + 2] = static_cast<uint32_t>(t4[0][q4].z);
+        va[q4 * 4 + 3] = static_cast<uint32_t>(t4[0][q4].w);
       }
+#pragma unroll
+      for (int o = 1; o < 4; ++o)
+        if (o < p.splits) {
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) acc_add4<true>(va + q4 * 4, t4[o][q4]);
+        }
+    } else {
+      // int32: any order (sources past `splits` were loaded as zero)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) va[i] = 0;
+#pragma unroll
+      for (int o = 0; o < 4; ++o)
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) acc_add4<false>(va + q4 * 4, t4[o][q4]);
+    }
     const int col0 = tn * kPairBN + c * 32;
     if (!F8 && p.zp) apply_zp(p, row, col0, va);
     if (rv && col0 < p.n) store32_channel<F8>(p, row, col0, sa, sws + t * 32, va);
@@ -2095,22 +2115,27 @@ inline size_t group_wide_smem() { return sizeof(GroupWideStorage) + 1024; }
 // two when 0 < 2 r <= P and there are at least two groups, so that CTAs
 // 0 .. 2r - 1 each run q tiles and one part (q + 1/2 tiles where whole tiles
 // would take q + 1).  Returns r, or 0 when the split is off.
+constexpr int kGroupWideMaxSplit = 512;  // (2 r <= SMs per GPU)
 inline int group_split_tiles(int m, int n, int k, int num_sms) {
   const int tiles = ((m + BM - 1) / BM) * ((n + kGroupWideBN - 1) / kGroupWideBN);
-  if (num_sms <= 0 || tiles <= num_sms || k / 128 < 2) return 0;
+  if (num_sms <= 0 || num_sms > 2 * kGroupWideMaxSplit || tiles <= num_sms || k / 128 < 2) return 0;
   const int r = tiles % num_sms;
   return (r > 0 && 2 * r <= num_sms) ? r : 0;
 }
-// Its workspace: one arrival counter per tail tile (zero before a call,
-// zero after it), padded to 256 bytes, then each tail tile's running sums,
-// 128 x 256 fp32.
+// Its workspace follows the layout the pair kernel's splits use, so that one
+// workspace serves every call: one arrival counter per tail tile in the
+// counter header (zero before a call, zero after it; the first
+// group_flag_bytes must be zero), and each tail tile's running sums
+// (128 x 256 fp32, scratch) from kTailOffset on, past the split-K
+// accumulators that other calls need left zero.
 inline size_t group_flag_bytes(int r) {
   return (static_cast<size_t>(r) * sizeof(int) + 255) & ~static_cast<size_t>(255);
 }
 inline size_t group_workspace_bytes(int r) {
-  return r > 0 ? group_flag_bytes(r) + static_cast<size_t>(r) * BM * kGroupWideBN * sizeof(float)
-               : 0;
+  return r > 0 ? kTailOffset + static_cast<size_t>(r) * BM * kGroupWideBN * sizeof(float) : 0;
 }
+static_assert(kGroupWideMaxSplit * sizeof(int) <= kCounterHeaderBytes,
+              "group split counters fit the counter header");
 
 // The wide group kernel moves registers between warpgroups with setmaxnreg;
 // the budgets only add up if the compiled kernel launches with at least
@@ -2256,8 +2281,7 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
       a.gsplit = workspace ? group_split_tiles(a.m, a.n, a.k, num_sms) : 0;
       a.gmid = a.groups / 2;
       a.gflag = static_cast<int*>(workspace);
-      a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                                     group_flag_bytes(a.gsplit))
+      a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)
                           : nullptr;
       const size_t smem = group_wide_smem();
       e = set_smem_once(gemm_i8_group_wide_kernel, dev, 7, smem);
