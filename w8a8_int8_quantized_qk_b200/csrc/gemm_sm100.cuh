@@ -1369,15 +1369,18 @@ __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uin
 // Tail split, one epilogue warp's 32 x 128 region (TMEM columns from tb) of
 // K slice `u.slice` of tile `u.tile`.  Partial slots in `tail_ws` are
 // [tail tile][slice][region][column quad][lane][4] int32, so each group of
-// 32 lanes moves 512 contiguous bytes.  Every slice stores its partial and
-// then takes a ticket on the region's counter (release); the slice whose
-// ticket is the last one knows the others' partials are complete (acquire),
-// adds them to its own accumulator, still in TMEM (integer adds, exact in
-// any order), runs the per-channel epilogue and resets the counter.  No
-// slice waits for another.
+// 32 lanes moves 512 contiguous bytes.  Every slice stores its partial,
+// hands its TMEM buffer back to the MMA (acc_empty_lead: the lead CTA's
+// barrier) and then takes a ticket on the region's counter (release); the
+// slice whose ticket is the last one knows every partial is complete
+// (acquire), sums them from L2 in ascending slice order (exact for int32,
+// fixed order for fp32), runs the per-channel epilogue and resets the
+// counter.  No slice waits for another, and none holds its TMEM buffer
+// through the reduction.
 template <bool F8>
-__device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region, uint32_t tb,
-                                    int row, bool rv, float sa, int colbase, const float* sws,
+__device__ void tail_slice_epilogue(uint32_t acc_empty_lead, const Args& p,
+                                    const PairUnit& u, int region, uint32_t tb, int row, bool rv,
+                                    float sa, int colbase, const float* sws,
                                     const CUtensorMap* tmO, uint8_t* box) {
   constexpr int kRegionInts = 32 * (kPairBN / 2);
   const int lane = threadIdx.x & 31;
@@ -1398,6 +1401,11 @@ __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region
                make_int4(va[q4 * 4], va[q4 * 4 + 1], va[q4 * 4 + 2], va[q4 * 4 + 3]));
     }
   }
+  // the accumulator is in the workspace: hand the TMEM buffer back to the
+  // MMA before the (slower) reduction, so later units are not held up
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(acc_empty_lead);
   __threadfence();
   __syncwarp();
   int last = 0;
@@ -1405,39 +1413,32 @@ __device__ void tail_slice_epilogue(const Args& p, const PairUnit& u, int region
   last = __shfl_sync(0xFFFFFFFFu, last, 0);
   if (!last) return;
   __threadfence();
-  // the slices in ascending order, this CTA's own from TMEM
+  // every slice's part of a 32-column chunk requested at once (S <= 4),
+  // then added in ascending slice order
 #pragma unroll 1
   for (int ch = 0; ch < 4; ++ch) {
-    uint32_t own[32];
-    tmem_ld_32x32b_x32(tb + ch * 32, own);
-#pragma unroll 1
-    for (int o = 0; o < S; ++o) {
-      int4 t4[8];
-      if (o != u.slice) {
-        const int4* src = reinterpret_cast<const int4*>(
-            slots + (static_cast<int64_t>(o) * 16 + region) * kRegionInts);
+    int4 t4[4][8];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) t4[q4] = __ldcg(src + (ch * 8 + q4) * 32 + lane);
-      } else {
-        tmem_ld_wait();
+    for (int o = 0; o < 4; ++o) {
+      const int4* src = reinterpret_cast<const int4*>(
+          slots + (static_cast<int64_t>(o < S ? o : 0) * 16 + region) * kRegionInts);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          t4[q4] = make_int4(static_cast<int>(own[q4 * 4]), static_cast<int>(own[q4 * 4 + 1]),
-                             static_cast<int>(own[q4 * 4 + 2]), static_cast<int>(own[q4 * 4 + 3]));
-      }
-      if (o == 0) {
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          va[q4 * 4] = static_cast<uint32_t>(t4[q4].x);
-          va[q4 * 4 + 1] = static_cast<uint32_t>(t4[q4].y);
-          va[q4 * 4 + 2] = static_cast<uint32_t>(t4[q4].z);
-          va[q4 * 4 + 3] = static_cast<uint32_t>(t4[q4].w);
-        }
-      } else {
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[q4]);
-      }
+      for (int q4 = 0; q4 < 8; ++q4)
+        t4[o][q4] = o < S ? __ldcg(src + (ch * 8 + q4) * 32 + lane) : make_int4(0, 0, 0, 0);
     }
+#pragma unroll
+    for (int q4 = 0; q4 < 8; ++q4) {
+      va[q4 * 4] = static_cast<uint32_t>(t4[0][q4].x);
+      va[q4 * 4 + 1] = static_cast<uint32_t>(t4[0][q4].y);
+      va[q4 * 4 + 2] = static_cast<uint32_t>(t4[0][q4].z);
+      va[q4 * 4 + 3] = static_cast<uint32_t>(t4[0][q4].w);
+    }
+#pragma unroll
+    for (int o = 1; o < 4; ++o)
+      if (o < S) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[o][q4]);
+      }
     if (!F8 && p.zp) apply_zp(p, row, colbase + ch * 32, va);
     if (p.tma_out)
       store32_tma<F8>(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
@@ -1488,7 +1489,9 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
                         half * (kPairBN / 2);
     uint32_t va[32], vb[32];
     if (tail) {
-      tail_slice_epilogue<F8>(p, u, region, tb, row, rv, sa, colbase, sws, tmO, box);
+      // (releases the TMEM buffer itself, before its reduction)
+      tail_slice_epilogue<F8>(map_to_rank(smem_addr(&s.acc_empty[abuf]), lead), p, u, region,
+                              tb, row, rv, sa, colbase, sws, tmO, box);
     } else if (F8 && !p.csplit) {
       // FP8 kind, whole tile (fp32 accumulator)
       auto emit = [&](int ch, const uint32_t(&v)[32]) {
@@ -1609,9 +1612,11 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
         if (lane == 0) p.cnt[tile * 16 + region] = 0;  // ready for the next call
       }
     }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_addr(&s.acc_empty[abuf]), lead));
+    if (!tail) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_addr(&s.acc_empty[abuf]), lead));
+    }
     if (++abuf == 2) {
       abuf = 0;
       aphase ^= 1u;
