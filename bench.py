@@ -43,7 +43,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "prefill INT8 TOPS and decode weight-stream GB/s, % of B200 roofline"
 # ncu counters of the current kernels (see the --gemm-traffic help)
-GEMM_TRAFFIC_BYTES = 34.081024e6 + 15.462144e6
+GEMM_TRAFFIC_BYTES = 34.281216e6 + 14.385152e6
 GEMV_TRAFFIC_BYTES = 58.801920e6 + 0.029952e6
 L2_BYTES = 126 * 1024 * 1024
 
@@ -382,7 +382,7 @@ def measure_fp8(torch, qk, iters: int, pk: dict) -> dict:
            "quant_kernel": "quantize_per_token_fp8 (e4m3)", "quant_us": quant_us,
            "quant_GBs": qb / (quant_us * 1e-6) / 1e9,
            "quant_hbm_frac": qb / (quant_us * 1e-6) / 1e9 / pk["hbm_gbs"],
-           "gemm_kernel": "tcgen05 kind::f8f6f4 (e4m3, fp32 accumulate), CTA pair, whole tiles",
+           "gemm_kernel": "tcgen05 kind::f8f6f4 (e4m3, fp32 accumulate), CTA pair, whole tiles at this shape",
            "gemm_us": gemm_us, "gemm_TOPS": ops / (gemm_us * 1e-6) / 1e12,
            "gemm_tensor_frac": ops / (gemm_us * 1e-6) / 1e12 / pk["int8_tops"],
            "tensor_peak_note": "dense e4m3 peak taken equal to the int8 one (nominal 4.5 PFLOP/s both)",
