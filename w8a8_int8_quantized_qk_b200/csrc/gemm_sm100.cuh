@@ -1882,10 +1882,12 @@ inline size_t pair_smem() { return sizeof(PairStorage) + 1024; }
 // Largest number of co-resident clusters of `cluster` CTAs of the pair
 // kernel (queried once per device and size; 0 when the size cannot run).
 inline int max_pair_clusters(int dev, int cluster) {
-  static int cache[64][5] = {};  // cluster 2, 4, 6, 8 (index cluster / 2)
+  // (relaxed atomics: host threads may race to fill an entry, all with the same value)
+  static std::atomic<int> cache[64][5] = {};  // cluster 2, 4, 6, 8 (index cluster / 2)
   const int ci = cluster / 2;
   if (dev < 0 || dev >= 64 || ci < 1 || ci > 4 || cluster % 2) return 0;
-  if (cache[dev][ci] != 0) return cache[dev][ci] > 0 ? cache[dev][ci] : 0;
+  const int known = cache[dev][ci].load(std::memory_order_relaxed);
+  if (known != 0) return known > 0 ? known : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(cluster) * 16, 1, 1);
   cfg.blockDim = dim3(kPairThreads, 1, 1);
@@ -1904,14 +1906,17 @@ inline int max_pair_clusters(int dev, int cluster) {
     cudaGetLastError();
     n = 0;
   }
-  cache[dev][ci] = n > 0 ? n : -1;
+  cache[dev][ci].store(n > 0 ? n : -1, std::memory_order_relaxed);
   return n > 0 ? n : 0;
 }
 
 // Largest number of co-resident CTA pairs (queried once per device).
 inline int max_pairs(int dev, int num_sms) {
-  static int cache[64] = {0};
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  static std::atomic<int> cache[64] = {};
+  if (dev >= 0 && dev < 64) {
+    const int known = cache[dev].load(std::memory_order_relaxed);
+    if (known > 0) return known;
+  }
   int pairs = num_sms / 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
@@ -1931,7 +1936,7 @@ inline int max_pairs(int dev, int num_sms) {
     pairs = n < pairs ? n : pairs;
   else
     cudaGetLastError();
-  if (dev >= 0 && dev < 64) cache[dev] = pairs;
+  if (dev >= 0 && dev < 64) cache[dev].store(pairs, std::memory_order_relaxed);
   return pairs;
 }
 
@@ -2147,26 +2152,29 @@ static_assert(kGroupWideMaxSplit * sizeof(int) <= kCounterHeaderBytes,
 // kGroupWideLaunchRegs registers per thread (otherwise the increase would
 // wait for registers that never come back).  Checked once per device.
 inline bool group_wide_ok(int dev) {
-  static int cache[64] = {};
+  static std::atomic<int> cache[64] = {};
   if (dev < 0 || dev >= 64) return false;
-  if (cache[dev] == 0) {
+  int known = cache[dev].load(std::memory_order_relaxed);
+  if (known == 0) {
     cudaFuncAttributes fa;
     const bool ok = cudaFuncGetAttributes(&fa, gemm_i8_group_wide_kernel) == cudaSuccess &&
                     fa.numRegs >= kGroupWideLaunchRegs &&
                     fa.numRegs * kGroupWideThreads <= 65536;
     if (!ok) cudaGetLastError();
-    cache[dev] = ok ? 1 : -1;
+    known = ok ? 1 : -1;
+    cache[dev].store(known, std::memory_order_relaxed);
   }
-  return cache[dev] > 0;
+  return known > 0;
 }
 
 // 0 ok, 1 tensor-map failure, 2 CUDA error
 // Largest number of co-resident clusters of `cluster` CTAs of the 1-SM
 // channel kernel (queried once per device and size; 0 when it cannot run).
 inline int max_channel_clusters(int dev, int cluster) {
-  static int cache[64][5] = {};
+  static std::atomic<int> cache[64][5] = {};
   if (dev < 0 || dev >= 64 || cluster < 2 || cluster > 4) return 0;
-  if (cache[dev][cluster] != 0) return cache[dev][cluster] > 0 ? cache[dev][cluster] : 0;
+  const int known = cache[dev][cluster].load(std::memory_order_relaxed);
+  if (known != 0) return known > 0 ? known : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(cluster) * 16, 1, 1);
   cfg.blockDim = dim3(kChannelThreads, 1, 1);
@@ -2185,7 +2193,7 @@ inline int max_channel_clusters(int dev, int cluster) {
     cudaGetLastError();
     n = 0;
   }
-  cache[dev][cluster] = n > 0 ? n : -1;
+  cache[dev][cluster].store(n > 0 ? n : -1, std::memory_order_relaxed);
   return n > 0 ? n : 0;
 }
 

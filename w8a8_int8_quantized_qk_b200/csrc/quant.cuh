@@ -13,6 +13,8 @@
 // registers.  Rows too long to keep on chip fall back to the two-pass form.
 #pragma once
 
+#include <atomic>
+
 #include <cooperative_groups.h>
 
 #include "qk_common.cuh"
@@ -482,8 +484,9 @@ inline cudaError_t launch_rows(const Args& a, int num_sms, cudaStream_t stream);
 // and 9.97 us with all that fit.
 template <bool BF16, bool SILU, int V>
 inline int persistent_ctas_per_sm() {
-  static int cached = 0;
-  if (cached == 0) {
+  static std::atomic<int> cached{0};  // (host threads may race to fill it, with one value)
+  int known = cached.load(std::memory_order_relaxed);
+  if (known == 0) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
             &n, quant_rows_persistent_kernel<BF16, SILU, V>, kPersistThreads, 0) != cudaSuccess ||
@@ -491,9 +494,10 @@ inline int persistent_ctas_per_sm() {
       cudaGetLastError();
       n = 1;
     }
-    cached = n < 8 ? n : 8;
+    known = n < 8 ? n : 8;
+    cached.store(known, std::memory_order_relaxed);
   }
-  return cached;
+  return known;
 }
 
 template <bool BF16, bool SILU, int V>
