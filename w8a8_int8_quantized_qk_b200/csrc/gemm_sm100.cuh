@@ -1040,6 +1040,10 @@ __global__ void __launch_bounds__(GroupCfg<WITH_C>::threads, 1)
 // work: warpgroup 0 drops to 64 per thread and the epilogue rises to 104
 // (128*64 + 512*104 = 61440 = 640*96, the launch allocation).
 //
+// Work comes as units (group_unit): whole tiles, and, when the last wave
+// would be partial, the halves of its tiles cut at the middle group, the
+// running sums passing from one CTA to another through the workspace.
+//
 // Per element and group: one exact int-to-float conversion and one fused
 // multiply-add, in ascending group order.  (Packed f32x2 pairs with the
 // 1.5 * 2^23 bias trick issue more instructions here, because forming the
