@@ -39,7 +39,7 @@ def nvcc() -> str:
 
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(INCLUDE, "qk.h")])
+                  + glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(INCLUDE, "qk.h")])
 
 
 def up_to_date() -> bool:

@@ -34,6 +34,7 @@
 #include <atomic>
 #include <mutex>
 
+#include "group_plan.h"
 #include "qk_common.cuh"
 
 namespace qk {
@@ -101,37 +102,11 @@ struct Args {
   int* gflag;
 };
 
-// Work unit of the wide group kernel: groups [g0, g1) of output tile
-// `tile`; part 0 whole, 1 the first part of a split tile, 2 its second.
-struct GroupUnit {
-  int tile, g0, g1, part;
-};
-
-// The i-th unit of this CTA (false past its last); every role walks the
-// same list.  Without the split, tiles blockIdx.x, + gridDim.x, ...; with
-// it (gsplit = r tail tiles, 2 r <= gridDim.x, whole tiles a multiple of
-// the grid), CTA j < r first takes the first part of tail tile j, and CTA
-// r + j takes the second part of tail tile j after its whole tiles.
+// The i-th unit of this CTA in the wide group kernel's schedule (false past
+// its last); every role walks the same list (group_plan.h).
 __device__ __forceinline__ bool group_unit(const Args& p, int i, GroupUnit& u) {
-  const int c = static_cast<int>(blockIdx.x), P = static_cast<int>(gridDim.x), r = p.gsplit;
-  const int dp = p.tiles_m * p.tiles_n - r;
-  if (c < r) {
-    if (i == 0) {
-      u = {dp + c, 0, p.gmid, 1};
-      return true;
-    }
-    --i;
-  }
-  const int t = c + i * P;
-  if (t < dp) {
-    u = {t, 0, p.groups, 0};
-    return true;
-  }
-  if (c >= r && c < 2 * r && i == (dp - c + P - 1) / P) {
-    u = {dp + c - r, p.gmid, p.groups, 2};
-    return true;
-  }
-  return false;
+  return group_unit_at(static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x),
+                       p.tiles_m * p.tiles_n, p.gsplit, p.groups, p.gmid, i, u);
 }
 
 // One output tile of the 1-SM kernels: A rows from a_row0 (rows from row_end
@@ -2132,9 +2107,8 @@ inline size_t group_wide_smem() { return sizeof(GroupWideStorage) + 1024; }
 constexpr int kGroupWideMaxSplit = 512;  // (2 r <= SMs per GPU)
 inline int group_split_tiles(int m, int n, int k, int num_sms) {
   const int tiles = ((m + BM - 1) / BM) * ((n + kGroupWideBN - 1) / kGroupWideBN);
-  if (num_sms <= 0 || num_sms > 2 * kGroupWideMaxSplit || tiles <= num_sms || k / 128 < 2) return 0;
-  const int r = tiles % num_sms;
-  return (r > 0 && 2 * r <= num_sms) ? r : 0;
+  if (num_sms > 2 * kGroupWideMaxSplit) return 0;
+  return group_split_count(tiles, k / 128, num_sms);
 }
 // Its workspace follows the layout the pair kernel's splits use, so that one
 // workspace serves every call: one arrival counter per tail tile in the
