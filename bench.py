@@ -35,6 +35,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import threading
 import time
 
@@ -587,9 +588,12 @@ def run_ours(args):
     g_warm.replay()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                          if args.smi else None)
+    csv_path = None
+    if args.smi:
+        csv_dir = args.clocks_dir or tempfile.gettempdir()
+        os.makedirs(csv_dir, exist_ok=True)
+        csv_path = os.path.join(csv_dir, f"clocks_rank{rank}.csv")
+    clocks = ClockSampler(local, csv_path)
     barrier()
     with clocks:
         start.record(stream)
@@ -721,6 +725,9 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline only (for profiling runs)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-smi", dest="smi", action="store_false")
+    ap.add_argument("--clocks-dir", default=None,
+                    help="where the nvidia-smi clock log of the timed region goes "
+                         "(clocks_rank<r>.csv; default: the system temp directory)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="CPU time budget of the whole --impl reference run")
