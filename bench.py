@@ -50,7 +50,9 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 def peaks() -> dict:
-    """Roofline denominators: the driver's measured peaks when present."""
+    """Roofline denominators: the measured peaks of MEASURED_PEAKS.json when
+    present (a STREAM-style copy and a cuBLAS bf16 GEMM on this GPU model),
+    else fallback figures."""
     p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):

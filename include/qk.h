@@ -56,7 +56,7 @@ typedef enum qk_status {
   QK_OK = 0,
   QK_ERR_INVALID_ARG = 1,    /* bad size, dtype, group size or NULL pointer */
   QK_ERR_MISALIGNED = 2,     /* a pointer or row stride breaks its alignment rule */
-  QK_ERR_UNSUPPORTED = 3,    /* valid request this build does not implement
+  QK_ERR_UNSUPPORTED = 3,    /* valid request the library does not implement
                                 (e.g. no sm_100 device) */
   QK_ERR_OVERFLOW_BOUND = 4, /* k * 127^2 >= 2^31: the INT32 sum could overflow */
   QK_ERR_CUDA = 5,           /* a CUDA runtime/driver call or launch failed */
