@@ -390,7 +390,8 @@ QK_API size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k);
  *   results.  Serialise them.
  * - QK_NOALLOC_SCRATCH_BYTES covers every split-K problem (a 4 KB header,
  *   at most 64 split-K accumulator tiles and 128 tail-split partial tiles,
- *   each 256 KB); a problem
+ *   each 256 KB), and group mode's cut tiles (128 KB of running sums each
+ *   past the same 4 KB + 16 MB; at most half the SM count); a problem
  *   whose qk_w8a8_gemm_workspace_size exceeded it would be rejected with
  *   QK_ERR_WORKSPACE and nothing launched.  Other errors are those of
  *   qk_w8a8_gemm.
