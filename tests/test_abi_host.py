@@ -133,10 +133,37 @@ def test_selftest_arg_check(L):
 
 
 def test_no_cpu_fallback(L):
+    # every torch helper refuses host tensors before doing any work
     torch = pytest.importorskip("torch")
     x = torch.zeros((4, 16), dtype=torch.bfloat16)
-    with pytest.raises(ValueError):
-        qk.quantize_per_token(x)
+    a = torch.zeros((4, 16), dtype=torch.int8)
+    b = torch.zeros((8, 16), dtype=torch.int8)
+    s4 = torch.ones((4,), dtype=torch.float32)
+    s8 = torch.ones((8,), dtype=torch.float32)
+    u8a = torch.zeros((4, 16), dtype=torch.uint8)
+    u8b = torch.zeros((8, 16), dtype=torch.uint8)
+    zp = torch.zeros((4,), dtype=torch.int32)
+    ws = torch.zeros((8,), dtype=torch.int32)
+    off = torch.tensor([0, 4], dtype=torch.int32)
+    calls = [
+        lambda: qk.quantize_per_token(x),
+        lambda: qk.silu_mul_quant_per_token(x, x),
+        lambda: qk.quantize_per_token_fp8(x),
+        lambda: qk.silu_mul_quant_per_token_fp8(x, x),
+        lambda: qk.w8a8_gemm(a, b, s4, s8),
+        lambda: qk.fp8_gemm(u8a, u8b, s4, s8),
+        lambda: qk.quantize_per_token_asym(x),
+        lambda: qk.quantize_static(x, torch.ones((1,), dtype=torch.float32)),
+        lambda: qk.weight_row_sums(b),
+        lambda: qk.w8a8_gemm_asym(a, zp, b, ws, s4, s8),
+        lambda: qk.w8a8_moe_gemm(a, off, b, s4, s8, 4),
+        lambda: qk.w8a8_linear(x, b, s8),
+        lambda: qk.linear(x, b, s8),
+        lambda: qk.mlp_down(x, x, b, s8),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensors only"):
+            call()
 
 
 def test_product_never_touches_the_oracle():
