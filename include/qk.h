@@ -28,6 +28,11 @@
  * - Values of int8 operands are in [-127, 127] (what the quantisers
  *   produce); -128 and non-finite floating-point inputs are outside the
  *   contract and are not checked.
+ * - The library keeps per-device state for the life of the process: the
+ *   properties above, kernel attributes, cached tensor maps and the device
+ *   address of qk_w8a8_gemm_noalloc's scratch array.  A cudaDeviceReset
+ *   invalidates that state: do not call the library on a device after
+ *   resetting it in the same process.
  */
 #ifndef QK_H_
 #define QK_H_

@@ -20,7 +20,10 @@ What pins what:
                        the int32 bound K * 127^2 < 2^31.
 * epilogues         -- float64 value within the rounding bound of the
                        left-to-right fp32 chain; exact power-of-two cases;
-                       group mode against a float64 sum of per-group terms.
+                       group mode against a float64 sum of per-group terms;
+                       the operation order itself on hand-derived values
+                       that round differently under any reordering (golden
+                       ``epilogue_order.json``).
 * whole chain       -- hand-worked example (golden ``linear_hand.json``).
 * FP8 e4m3 codec    -- torch's float8_e4m3fn (decode of all 256 codes; the
                        float32 -> e4m3 cast on random values, every
@@ -268,6 +271,37 @@ def pin_group(O) -> None:
     assert acc.tolist() == [[70, -10]] and out.tolist() == [[8.75, -10.0]]
 
 
+def _hexf(v: str) -> np.float32:
+    return np.float32(float.fromhex(v))
+
+
+def pin_epilogue_order_golden(O) -> None:
+    """Hand-derived values (golden ``epilogue_order.json``) on which a
+    reordered epilogue rounds differently: (acc * sa) * sw before alpha, and
+    the fused group chain in ascending group order before sa and alpha."""
+    g = _golden("epilogue_order.json")
+    for case in g["per_channel"]:
+        out = O.epilogue_per_channel(np.int32([[case["acc"]]]), np.float32([_hexf(case["sa"])]),
+                                     np.float32([_hexf(case["sw"])]), float(_hexf(case["alpha"])))
+        want = _hexf(case["out"])
+        assert out.view(np.uint32)[0, 0] == np.float32(want).view(np.uint32), \
+            (float(out[0, 0]).hex(), case["out"])
+    for case in g["group"]:
+        gk = case["group_k"]
+        ng = len(case["partials"])
+        a = np.zeros((1, gk * ng), np.int8)
+        w = np.zeros((1, gk * ng), np.int8)
+        for i, (av, wv) in enumerate(case["partials"]):
+            a[0, i * gk] = av
+            w[0, i * gk] = wv
+        sw = np.float32([[_hexf(v) for v in case["sw"]]])
+        out, acc = O.gemm_group(a, w, np.float32([_hexf(case["sa"])]), sw, gk, float(_hexf(case["alpha"])))
+        assert int(acc[0, 0]) == case["acc"]
+        want = _hexf(case["out"])
+        assert out.view(np.uint32)[0, 0] == np.float32(want).view(np.uint32), \
+            (float(out[0, 0]).hex(), case["out"])
+
+
 # --------------------------------------------------------------------------- whole chain
 def pin_linear_golden(O) -> None:
     g = _golden("linear_hand.json")
@@ -466,5 +500,5 @@ def pin_static_quant(O) -> None:
 
 ALL_PINS = [pin_exp, pin_silu, pin_bf16_rounding, pin_quant_golden, pin_quant_invariants,
             pin_quant_bf16_path, pin_silu_quant, pin_gemm_bruteforce, pin_gemm_closed_forms,
-            pin_epilogue_per_channel, pin_group, pin_linear_golden, pin_e4m3_codec, pin_fp8_quant,
+            pin_epilogue_per_channel, pin_group, pin_epilogue_order_golden, pin_linear_golden, pin_e4m3_codec, pin_fp8_quant,
             pin_fp8_silu_quant, pin_fp8_gemm, pin_asym_quant, pin_asym_gemm, pin_static_quant]

@@ -51,6 +51,14 @@ def test_abi_version(L):
     assert qk.qk_abi_version() == qk.ABI_VERSION
 
 
+def test_noalloc_scratch_size_matches_header():
+    # the binding's constant (used by the tests) is the header's #define
+    hdr = open(HEADER).read()
+    expr = re.search(r"#define QK_NOALLOC_SCRATCH_BYTES \(([^)]*)\)", hdr).group(1)
+    assert re.fullmatch(r"[0-9u*+ ]+", expr), expr
+    assert eval(expr.replace("u", "")) == qk.NOALLOC_SCRATCH_BYTES  # integer arithmetic only
+
+
 def test_status_strings(L):
     for code in range(8):
         assert qk.qk_status_string(code)

@@ -70,11 +70,8 @@ def test_moe_synthetic_routing(O):
     torch.cuda.synchronize()
     for e in range(8):
         r0, r1 = int(off[e]), int(off[e + 1])
-        rows = np.arange(r0, r1)
-        if len(rows) > 64:  # sampled rows of the large experts
-            rows = np.concatenate([rows[:16], rows[-16:], np.random.default_rng(e).choice(rows, 32)])
-        ref = O.linear_from_q(a[rows], sa[rows], w[e], sw[e], 0, 1.0)
-        assert_bits(out[rows], ref["out_bf16"], f"expert {e}")
+        ref = O.linear_from_q(a[r0:r1], sa[r0:r1], w[e], sw[e], 0, 1.0)
+        assert_bits(out[r0:r1], ref["out_bf16"], f"expert {e}")
 
 
 def test_moe_errors():

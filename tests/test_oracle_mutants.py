@@ -33,6 +33,16 @@ MUTANTS = [
     ("epi_wrong_scale_index", "o = o * sw[c];", "o = o * sw[r % n];"),
     ("epi_wrong_sign", "o = o * sa[r];", "o = o * -sa[r];"),
     ("epi_dropped_alpha", "      o = o * alpha;\n      out[", "      out["),
+    ("epi_scales_multiplied_first", "      o = o * sa[r];\n      o = o * sw[c];",
+     "      o = o * (sa[r] * sw[c]);"),
+    ("epi_sw_before_sa", "      o = o * sa[r];\n      o = o * sw[c];", "      o = o * sw[c];\n      o = o * sa[r];"),
+    ("epi_alpha_first", "      o = o * sa[r];\n      o = o * sw[c];\n      o = o * alpha;",
+     "      o = o * alpha;\n      o = o * sa[r];\n      o = o * sw[c];"),
+    ("group_unfused", "f = fmaf((float)(int32_t)p, j->sw[(int64_t)c * ng + g], f);",
+     "f = f + (float)(int32_t)p * j->sw[(int64_t)c * ng + g];"),
+    ("group_descending", "for (int g = 0; g < ng; ++g) {", "for (int g = ng - 1; g >= 0; --g) {"),
+    ("group_sa_alpha_first", "float o = f * j->sa[r];\n        o = o * j->alpha;",
+     "float o = f * (j->sa[r] * j->alpha);"),
     ("group_scale_transposed", "f = fmaf((float)(int32_t)p, j->sw[(int64_t)c * ng + g], f);",
      "f = fmaf((float)(int32_t)p, j->sw[(int64_t)g * ng + c % ng], f);"),
     ("group_dropped_last", "for (int g = 0; g < ng; ++g) {", "for (int g = 0; g < ng - 1; ++g) {"),

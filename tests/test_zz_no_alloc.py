@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024 + 4096  # QK_NOALLOC_SCRATCH_BYTES in include/qk.h
+NOALLOC_SCRATCH_BYTES = qk.NOALLOC_SCRATCH_BYTES  # QK_NOALLOC_SCRATCH_BYTES of include/qk.h
 
 
 def _inputs(m, n, k, seed):

@@ -37,6 +37,11 @@ QK_ERR_WORKSPACE = 7
 QK_F32 = 0
 QK_BF16 = 1
 
+# QK_NOALLOC_SCRATCH_BYTES of include/qk.h: the size of the scratch array
+# built into the library for qk_w8a8_gemm_noalloc (a host test checks that
+# the two agree)
+NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024 + 4096
+
 # name -> (restype, argtypes), in include/qk.h order
 _P = ctypes.c_void_p
 _SIGNATURES = {
