@@ -1,0 +1,127 @@
+// mma_probe.cuh -- the INT8 tensor-core rate of this device, measured: a
+// diagnostic kernel that issues tcgen05.mma.kind::i8 back to back on fixed
+// shared-memory operands into one TMEM accumulator, with no global-memory
+// traffic, so that its duration is the tensor pipe's own time.  The roofline
+// of the library's GEMMs ("KV-cache kernels" section 01: the compute
+// ceiling against which a kernel's achieved rate is read) divides by the
+// rate this kernel reaches.
+//
+// Forms: cta_group::1 (one CTA per SM, M = 128) and cta_group::2 (a cluster
+// of two CTAs on the two SMs of a pair, M = 256, the leader issuing); N is
+// 32 .. 256 (a multiple of 16), K = 32 per instruction.  Every CTA's MMA
+// thread records the SM clock cycles from its first issue to the completion
+// of its last MMA, so the host can also form MACs per clock per SM.
+#pragma once
+
+#include "qk_common.cuh"
+
+namespace qk {
+namespace probe {
+
+constexpr int kThreads = 128;
+constexpr int kTileBytes = 128 * 128;  // one 128-row x 128-byte swizzled operand tile
+
+struct alignas(1024) ProbeStorage {
+  uint8_t a[kTileBytes];
+  uint8_t b[2 * kTileBytes];  // up to 256 rows of B
+  uint64_t done;
+  uint32_t tmem_base;
+};
+
+// `iters` instructions of shape (M = 128 * PAIR? 256 : 128) x n x 32.
+// cycles[cta] (optional): clock64 cycles between the first issue and the
+// last completion, on the issuing CTA (0 on a pair's second CTA).
+template <bool PAIR>
+__global__ void __launch_bounds__(kThreads, 1)
+    mma_rate_kernel(int n, int iters, unsigned long long* cycles) {
+  extern __shared__ uint8_t smem_raw[];
+  ProbeStorage& s = *reinterpret_cast<ProbeStorage*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const uint32_t crank = PAIR ? cluster_rank() : 0u;
+  // zero operands: the rate of an integer MMA does not depend on the values
+  for (int i = threadIdx.x; i < kTileBytes / 16; i += kThreads)
+    reinterpret_cast<int4*>(s.a)[i] = make_int4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < 2 * kTileBytes / 16; i += kThreads)
+    reinterpret_cast<int4*>(s.b)[i] = make_int4(0, 0, 0, 0);
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&s.done), 1);
+    fence_mbar_init();
+  }
+  fence_proxy_async_smem();  // the zeros are visible to the tensor core
+  if (warp == 0) {
+    if (PAIR) {
+      tmem_alloc_pair(smem_addr(&s.tmem_base), 256);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(&s.tmem_base), 256);
+      tmem_relinquish();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (PAIR) cluster_sync_all();  // both CTAs' operands, barriers and TMEM exist
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  if (threadIdx.x == 0 && crank == 0) {
+    const uint32_t idesc = idesc_i8(PAIR ? 256 : 128, n);
+    const uint32_t a0 = smem_addr(s.a), b0 = smem_addr(s.b);
+    const long long t0 = clock64();
+    for (int i = 0; i < iters; ++i) {
+      const uint32_t kk = static_cast<uint32_t>(i & 3) * 32u;  // walk the 128-byte row
+      if (PAIR)
+        mma_i8_pair(tmem, sdesc_k_sw128(a0 + kk), sdesc_k_sw128(b0 + kk), idesc, i > 0 ? 1u : 0u);
+      else
+        mma_i8(tmem, sdesc_k_sw128(a0 + kk), sdesc_k_sw128(b0 + kk), idesc, i > 0 ? 1u : 0u);
+    }
+    if (PAIR)
+      mma_commit_pair(smem_addr(&s.done), static_cast<uint16_t>(0x3u));
+    else
+      mma_commit(smem_addr(&s.done));
+    mbar_wait(smem_addr(&s.done), 0u, nullptr);
+    const long long t1 = clock64();
+    if (cycles) cycles[blockIdx.x] = static_cast<unsigned long long>(t1 - t0);
+  } else if (PAIR && threadIdx.x == 0) {
+    // the leader's commit also arrives here once the MMAs that wrote this
+    // CTA's TMEM are complete
+    mbar_wait(smem_addr(&s.done), 0u, nullptr);
+    if (cycles) cycles[blockIdx.x] = 0ull;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (PAIR) cluster_sync_all();
+  tc_fence_after();
+  if (warp == 0) {
+    if (PAIR)
+      tmem_dealloc_pair(tmem, 256);
+    else
+      tmem_dealloc(tmem, 256);
+  }
+}
+
+inline size_t smem_bytes() { return sizeof(ProbeStorage) + 1024; }
+
+// ctas: CTAs of the grid (a multiple of 2 for pairs).
+inline cudaError_t launch(bool pair, int n, int iters, int ctas, unsigned long long* cycles,
+                          cudaStream_t stream) {
+  auto k = pair ? mma_rate_kernel<true> : mma_rate_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem_bytes()));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_bytes();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pair ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pair ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, n, iters, cycles);
+}
+
+}  // namespace probe
+}  // namespace qk
