@@ -25,6 +25,16 @@
  *   launches nothing and writes nothing.
  * - The return value is a qk_status.  No entry point throws, aborts, traps
  *   or asserts on the device.
+ * - Kernels are launched with programmatic dependent launch: a kernel may
+ *   start while the kernel before it on the stream is finishing, if that one
+ *   allows it early (this library's kernels do; a kernel that does not is
+ *   waited for in full).  Each kernel waits for its predecessor before it
+ *   reads anything the predecessor may write or writes anything it may read,
+ *   with one exception: the GEMMs (qk_w8a8_gemm and its variants) and the
+ *   linear layer request their first weight tiles b (never scale_b or any
+ *   other input) before that wait.  So the kernel launched just before a GEMM
+ *   on the same stream must not write that GEMM's b if it triggers its
+ *   dependents early; the quantisers of this library never write weights.
  * - Values of int8 operands are in [-127, 127] (what the quantisers
  *   produce); -128 and non-finite floating-point inputs are outside the
  *   contract and are not checked.
@@ -55,7 +65,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 6
+#define QK_ABI_VERSION 8
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -209,12 +219,13 @@ QK_API qk_status qk_silu_mul_quant_per_token_fp8(int m, int k, const void* gate,
  *                the split-K accumulators, then 256 KB per partial).  In
  *                group mode (the output-only form) the last partial wave's
  *                tiles are instead cut at their middle K group: the first
- *                part runs early on one CTA and leaves its fp32 running sums
- *                in the workspace, the second runs last on another CTA and
- *                continues them in the same group order, so the result is
- *                unchanged (one counter per cut tile in the 4 KB header, the
- *                sums, 128 KB per cut tile, past the 16 MB of split-K
- *                accumulators).  The workspace
+ *                part runs early on one CTA pair (or CTA, for m <= 128) and
+ *                leaves its fp32 running sums in the workspace, the second
+ *                runs last on another and continues them in the same group
+ *                order, so the result is unchanged (one counter per cut tile
+ *                and CTA in the 4 KB header, then the sums, 256 KB per cut
+ *                256 x 256 tile or 128 KB per cut 128 x 256 tile, past the
+ *                16 MB of split-K accumulators).  The workspace
  *                must be zero-filled before its first use; every completed
  *                call leaves the header, the flags and the split-K
  *                accumulators zero again (the partials and sums need no
@@ -395,8 +406,10 @@ QK_API size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k);
  *   results.  Serialise them.
  * - QK_NOALLOC_SCRATCH_BYTES covers every split-K problem (a 4 KB header,
  *   at most 64 split-K accumulator tiles and 128 tail-split partial tiles,
- *   each 256 KB), and group mode's cut tiles (128 KB of running sums each
- *   past the same 4 KB + 16 MB; at most half the SM count); a problem
+ *   each 256 KB), and group mode's cut tiles (256 KB of running sums per cut
+ *   256 x 256 tile, at most a quarter of the SM count of them, or 128 KB per
+ *   cut 128 x 256 tile, at most half the SM count, past the same 4 KB +
+ *   16 MB); a problem
  *   whose qk_w8a8_gemm_workspace_size exceeded it would be rejected with
  *   QK_ERR_WORKSPACE and nothing launched.  Other errors are those of
  *   qk_w8a8_gemm.
@@ -426,6 +439,61 @@ QK_API qk_status qk_device_status(qk_stream stream);
  * that the bounded-wait path works on this device.
  */
 QK_API qk_status qk_selftest_bounded_wait(int timeout_us, qk_stream stream);
+
+/*
+ * qk_selftest_silu -- diagnostic: checks the fused SiLU arithmetic of the
+ * silu quantisers.  For every binary32 bit pattern g in [first, first +
+ * count) that is finite, it computes silu(g) * 1 the way the quantisers do
+ * (two values at a time, the exp's reduction, polynomial and the final
+ * multiply on packed binary32 pairs) and the way the definition reads (one
+ * value at a time, every step a scalar IEEE round-to-nearest operation), and
+ * counts the g whose two results differ in any bit.  g is the only input of that
+ * arithmetic, so first = 0, count = 2^32 covers every value it can see.
+ * Defined by the fused silu_and_mul quantisation of the vLLM PR "fused
+ * silu_and_mul + dynamic per-token FP8 quantization", Algorithm (silu(gate)
+ * computed in fp32 before the per-token absmax).
+ *
+ * first, count     the range of bit patterns; 1 <= count, first + count <= 2^32
+ * mismatches       device uint64 the kernel adds its count to (the caller
+ *                  zero-fills it), 8-byte aligned
+ * first_mismatch   optional device uint32 lowered (atomic minimum) to the
+ *                  smallest mismatching bit pattern; the caller sets it to
+ *                  0xFFFFFFFF first; NULL to skip
+ * Errors: QK_ERR_INVALID_ARG, QK_ERR_MISALIGNED, QK_ERR_UNSUPPORTED,
+ *         QK_ERR_CUDA.
+ */
+QK_API qk_status qk_selftest_silu(uint32_t first, uint64_t count, unsigned long long* mismatches,
+                                  uint32_t* first_mismatch, qk_stream stream);
+
+/*
+ * qk_selftest_mma_rate -- diagnostic: the INT8 tensor-core rate of the
+ * current device.  Launches `ctas` CTAs (cta_group 1: one per SM, M = 128;
+ * cta_group 2: clusters of two CTAs on an SM pair, M = 256, the pair's
+ * leader issuing tcgen05.mma.cta_group::2) that each issue `iters`
+ * tcgen05.mma.kind::i8 instructions of M x n x 32 back to back on fixed
+ * shared-memory operands into one TMEM accumulator: no global-memory traffic,
+ * so the kernel's duration is the tensor pipe's time.  Defined by the
+ * roofline reading of "KV-cache kernels" (day 26) section 01 (a kernel's
+ * achieved rate is read against the hardware's compute ceiling): the
+ * library's GEMM fractions divide by the rate this kernel reaches.
+ *
+ * Work per launch: (ctas / cta_group) * iters * M * n * 32 multiply-adds
+ * (2 int8 ops each); the caller times the launch with CUDA events.
+ * cta_group   1 or 2
+ * n           32 .. 256, a multiple of 16
+ * iters       1 .. 1048576 instructions per CTA (pair)
+ * ctas        1 .. 65535 CTAs, a multiple of cta_group; at most what the
+ *             device holds at once (one CTA per SM) for a meaningful rate
+ * cycles      optional device array [ctas] of uint64, 8-byte aligned: the
+ *             issuing CTA's SM clock cycles from its first issue to the
+ *             completion of its last MMA (0 for a pair's second CTA); NULL
+ *             to skip
+ * The completion wait is bounded like every other wait of the library.
+ * Errors: QK_ERR_INVALID_ARG, QK_ERR_MISALIGNED, QK_ERR_UNSUPPORTED,
+ *         QK_ERR_CUDA.
+ */
+QK_API qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas,
+                                      unsigned long long* cycles, qk_stream stream);
 
 #ifdef __cplusplus
 }

@@ -144,3 +144,21 @@ def test_workload_mlp_down_prologue(O):
     qr, sr = O.silu_mul_quant_per_token(w.gate, w.up)
     assert_bits(host(q), qr, "q")
     assert_bits(host(s), sr, "scale")
+
+
+def test_silu_arithmetic_every_binary32():
+    # The fused SiLU product as the quantisers compute it (partly on packed
+    # binary32 pairs) equals the definition's scalar chain on every finite
+    # binary32 gate value: the whole domain of that arithmetic, in four
+    # launches.
+    need_gpu()
+    import torch
+
+    bad = torch.zeros((1,), dtype=torch.int64, device="cuda")
+    low = torch.full((1,), -1, dtype=torch.int32, device="cuda")  # 0xFFFFFFFF
+    for first in range(0, 1 << 32, 1 << 30):
+        st = qk.qk_selftest_silu(first, 1 << 30, qk._ptr(bad), qk._ptr(low), qk._stream())
+        assert st == qk.QK_OK, qk.qk_status_string(st)
+    torch.cuda.synchronize()
+    n = int(bad.item())
+    assert n == 0, f"{n} mismatches, first at bits 0x{int(low.item()) & 0xFFFFFFFF:08x}"

@@ -42,7 +42,14 @@ def test_group128_workload_cuts_the_last_wave(checker):
     assert cut == 68 and longest == pytest.approx(3.5)
 
 
-@pytest.mark.parametrize("sms", [1, 2, 3, 7, 132, 148])
+def test_group128_workload_on_pairs_cuts_the_last_wave(checker):
+    # the CTA-pair kernel: 2048 x 8192 in 256 x 256 tiles = 256 tiles, 64
+    # groups, 74 pairs: 34 tail tiles cut, 3.5 tile-times instead of 4
+    cut, longest = _run(checker, 256, 64, 74)
+    assert cut == 34 and longest == pytest.approx(3.5)
+
+
+@pytest.mark.parametrize("sms", [1, 2, 3, 7, 74, 132, 148])
 @pytest.mark.parametrize("groups", [1, 2, 3, 17, 64])
 def test_schedule_invariants(checker, sms, groups):
     for tiles in list(range(1, 3 * sms + 4)) + [5 * sms + sms // 2, 9 * sms + 1]:

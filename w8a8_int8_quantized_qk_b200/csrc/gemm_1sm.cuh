@@ -161,11 +161,13 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
     if (p.tma_out) prefetch_tmap(&tmO);
   }
   setup<ChannelStorage, kChannelStages, 2, 4>(s);
-  griddep_wait();  // set-up above overlapped the previous kernel
-  griddep_launch_dependents();
+  if (warp != 0) {  // (the producer waits inside produce)
+    griddep_wait();  // set-up above overlapped the previous kernel
+    griddep_launch_dependents();
+  }
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
-    if (lane == 0) produce<kChannelBN, kChannelStages, MOE>(s, &tmA, &tmB, p);
+    if (lane == 0) produce<kChannelBN, kChannelStages, MOE, false, !MOE>(s, &tmA, &tmB, p);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false, F8, MOE>(s, tmem, p);
@@ -198,8 +200,10 @@ __global__ void __launch_bounds__(GroupCfg<WITH_C>::threads, 1)
   }
   constexpr int kEpiWarps = GroupCfg<WITH_C>::epi_warps;
   setup<GroupStorage, kGroupStages, 4, kEpiWarps>(s);
-  griddep_wait();  // set-up above overlapped the previous kernel
-  griddep_launch_dependents();
+  if (warp != 0) {  // (the producer waits inside produce)
+    griddep_wait();  // set-up above overlapped the previous kernel
+    griddep_launch_dependents();
+  }
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
     if (lane == 0) produce<kGroupBN, kGroupStages>(s, &tmA, &tmB, p);
@@ -379,8 +383,10 @@ __global__ void __launch_bounds__(kGroupWideThreads, 1)
     prefetch_tmap(&tmB);
   }
   setup<GroupWideStorage, kGroupWideStages, 2, kGroupWideEpiWarps>(s);
-  griddep_wait();  // set-up above overlapped the previous kernel
-  griddep_launch_dependents();
+  if (warp != 0) {  // (the producer waits inside produce)
+    griddep_wait();  // set-up above overlapped the previous kernel
+    griddep_launch_dependents();
+  }
   const uint32_t tmem = s.tmem_base;
   if (warp < 4) {
     regs_dec<kGroupWideCtrlRegs>();

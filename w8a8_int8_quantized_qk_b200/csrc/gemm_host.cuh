@@ -2,7 +2,7 @@
 // queries, the split plans and workspace sizes, and the launches.
 #pragma once
 
-#include "gemm_pair.cuh"
+#include "gemm_group_pair.cuh"
 
 namespace qk {
 namespace gemm {
@@ -97,7 +97,7 @@ inline bool cached_tmap(CUtensorMap* map, const void* base, int rows, int k, int
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel).
 template <class K>
 inline cudaError_t set_smem_once(K kernel, int dev, int slot, size_t bytes) {
-  static std::atomic<unsigned long long> done[8] = {};
+  static std::atomic<unsigned long long> done[16] = {};
   const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
   if (bit && (done[slot].load(std::memory_order_acquire) & bit)) return cudaSuccess;
   const cudaError_t e =
@@ -363,16 +363,9 @@ inline int group_split_tiles(int m, int n, int k, int num_sms) {
 }
 // Its workspace follows the layout the pair kernel's splits use, so that one
 // workspace serves every call: one arrival counter per tail tile in the
-// counter header (zero before a call, zero after it; the first
-// group_flag_bytes must be zero), and each tail tile's running sums
-// (128 x 256 fp32, scratch) from kTailOffset on, past the split-K
-// accumulators that other calls need left zero.
-inline size_t group_flag_bytes(int r) {
-  return (static_cast<size_t>(r) * sizeof(int) + 255) & ~static_cast<size_t>(255);
-}
-inline size_t group_workspace_bytes(int r) {
-  return r > 0 ? kTailOffset + static_cast<size_t>(r) * BM * kGroupWideBN * sizeof(float) : 0;
-}
+// counter header (zero before a call, zero after it), and each tail tile's
+// running sums (scratch) from kTailOffset on, past the split-K accumulators
+// that other calls need left zero (group_plan_workspace_bytes).
 static_assert(kGroupWideMaxSplit * sizeof(int) <= kCounterHeaderBytes,
               "group split counters fit the counter header");
 
@@ -395,6 +388,126 @@ inline bool group_wide_ok(int dev) {
   }
   return known > 0;
 }
+
+// ---------------------------------------------------------------- group-128 plans
+// The wide 1-SM kernel's K split relies on every CTA of its grid being
+// resident at once (a second part waits for a first part run by another
+// CTA): checked with the occupancy query, once per device.
+inline bool group_wide_resident(int dev, int grid) {
+  static std::atomic<int> cache[64] = {};  // CTAs per SM (-1: unknown / failed)
+  if (dev < 0 || dev >= 64) return false;
+  int per_sm = cache[dev].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaFuncSetAttribute(gemm_i8_group_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(group_wide_smem())) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemm_i8_group_wide_kernel, kGroupWideThreads,
+                                                      group_wide_smem()) != cudaSuccess) {
+      cudaGetLastError();
+      n = -1;
+    }
+    per_sm = n > 0 ? n : -1;
+    cache[dev].store(per_sm, std::memory_order_relaxed);
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+  return per_sm > 0 && static_cast<int64_t>(per_sm) * sms >= grid;
+}
+
+inline size_t group_pair_smem() { return sizeof(GroupPairStorage) + 1024; }
+
+// The group-128 pair kernel moves registers between warpgroups with
+// setmaxnreg; the budgets only add up if the compiled kernel launches with
+// at least kGpLaunchRegs registers per thread.  Checked once per device.
+inline bool group_pair_ok(int dev) {
+  static std::atomic<int> cache[64] = {};
+  if (dev < 0 || dev >= 64) return false;
+  int known = cache[dev].load(std::memory_order_relaxed);
+  if (known == 0) {
+    cudaFuncAttributes fa;
+    const bool ok = cudaFuncGetAttributes(&fa, gemm_i8_group_pair_kernel) == cudaSuccess &&
+                    fa.numRegs >= kGpLaunchRegs && fa.numRegs * kGpThreads <= 65536;
+    if (!ok) cudaGetLastError();
+    known = ok ? 1 : -1;
+    cache[dev].store(known, std::memory_order_relaxed);
+  }
+  return known > 0;
+}
+
+// Pairs of the group-128 pair kernel that are resident at once (queried once
+// per device; 0 when it cannot run).  The grid never exceeds it, so every
+// pair of a launch is resident together, which the K split's wait needs.
+inline int max_group_pairs(int dev, int num_sms) {
+  static std::atomic<int> cache[64] = {};
+  if (dev < 0 || dev >= 64) return 0;
+  const int known = cache[dev].load(std::memory_order_relaxed);
+  if (known != 0) return known > 0 ? known : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms - num_sms % 2), 1, 1);
+  cfg.blockDim = dim3(kGpThreads, 1, 1);
+  cfg.dynamicSmemBytes = group_pair_smem();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(gemm_i8_group_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(group_pair_smem())) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, gemm_i8_group_pair_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  n = n < num_sms / 2 ? n : num_sms / 2;
+  cache[dev].store(n > 0 ? n : -1, std::memory_order_relaxed);
+  return n > 0 ? n : 0;
+}
+
+// Which group-128 kernel runs an output-only problem, and how many tiles of
+// its last wave are cut at the middle group.  m > 128: the CTA-pair kernel
+// (256 x 256 tiles on the co-resident pairs); otherwise, or when the pair
+// kernel's register budget does not hold, the wide 1-SM kernel (128 x 256).
+struct GroupPlan {
+  bool pair;
+  int workers;  // pairs, or CTAs
+  int tiles;
+  int r;        // cut tail tiles (0: whole tiles only)
+};
+
+inline GroupPlan group_plan(int m, int n, int k, int dev, int num_sms) {
+  GroupPlan g;
+  const int groups = k / 128;
+  const int pairs = m > BM && group_pair_ok(dev) ? max_group_pairs(dev, num_sms) : 0;
+  if (pairs > 0) {
+    g.pair = true;
+    g.tiles = ((m + 255) / 256) * ((n + kGpBN - 1) / kGpBN);
+    g.workers = g.tiles < pairs ? g.tiles : pairs;
+    g.r = g.tiles <= 2 * kGroupWideMaxSplit ? group_split_count(g.tiles, groups, pairs) : 0;
+    return g;
+  }
+  g.pair = false;
+  g.tiles = ((m + BM - 1) / BM) * ((n + kGroupWideBN - 1) / kGroupWideBN);
+  g.workers = g.tiles < num_sms ? g.tiles : num_sms;
+  g.r = group_split_tiles(m, n, k, num_sms);
+  if (g.r > 0 && !group_wide_resident(dev, g.workers)) g.r = 0;
+  return g;
+}
+
+// Bytes of the group kernels' workspace: counters in the 4 KB header (one per
+// cut tile and CTA of a pair, or per cut tile), and the running sums past the
+// split-K accumulators (256 KB per cut pair tile, 128 KB per cut 1-SM tile).
+inline size_t group_plan_flag_bytes(const GroupPlan& g) {
+  const size_t n = static_cast<size_t>(g.r) * (g.pair ? 2 : 1) * sizeof(int);
+  return (n + 255) & ~static_cast<size_t>(255);
+}
+inline size_t group_plan_workspace_bytes(const GroupPlan& g) {
+  if (g.r <= 0) return 0;
+  return kTailOffset + static_cast<size_t>(g.r) * (g.pair ? 2u : 1u) * BM * kGroupWideBN * sizeof(float);
+}
+static_assert(2 * kGroupWideMaxSplit * sizeof(int) <= kCounterHeaderBytes,
+              "group split counters of the pair kernel fit the counter header");
 
 // 0 ok, 1 tensor-map failure, 2 CUDA error
 // Largest number of co-resident clusters of `cluster` CTAs of the 1-SM
@@ -473,7 +586,7 @@ inline bool prefer_channel_split(int m, int n, int k, int num_sms, int dev) {
   return cp.kb_per_split < pair_kb;
 }
 
-// `workspace`: group_workspace_bytes(group_split_tiles(...)) bytes for the
+// `workspace`: group_plan_workspace_bytes(group_plan(...)) bytes for the
 // wide group kernel's split (null: whole tiles only); unused otherwise.
 inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev, int num_sms,
                   cudaStream_t stream, cudaError_t* err, void* workspace = nullptr) {
@@ -520,7 +633,27 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
     }
   } else {
     if (wide) {
-      a.gsplit = workspace ? group_split_tiles(a.m, a.n, a.k, num_sms) : 0;
+      const GroupPlan gp = group_plan(a.m, a.n, a.k, dev, num_sms);
+      if (gp.pair) {
+        // 256 x 256 tiles on CTA pairs
+        a.tiles_m = (a.m + 255) / 256;
+        a.tiles_n = (a.n + kGpBN - 1) / kGpBN;
+        CUtensorMap tpa, tpb;
+        if (!cached_tmap(&tpa, A, a.m, a.k, 128) || !cached_tmap(&tpb, B, a.n, a.k, 128)) return 1;
+        a.gsplit = workspace ? gp.r : 0;
+        a.gmid = a.groups / 2;
+        a.gflag = static_cast<int*>(workspace);
+        a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)
+                            : nullptr;
+        const size_t smem = group_pair_smem();
+        e = set_smem_once(gemm_i8_group_pair_kernel, dev, 8, smem);
+        if (e == cudaSuccess)
+          e = launch_pdl(gemm_i8_group_pair_kernel, dim3(2 * gp.workers), dim3(kGpThreads), smem, stream,
+                         2, tpa, tpb, a);
+        *err = e;
+        return e == cudaSuccess ? 0 : 2;
+      }
+      a.gsplit = workspace ? gp.r : 0;
       a.gmid = a.groups / 2;
       a.gflag = static_cast<int*>(workspace);
       a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)

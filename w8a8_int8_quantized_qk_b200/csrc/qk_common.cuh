@@ -295,9 +295,15 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
+// Arrive on a barrier of any CTA of the cluster (address from mapa), with the
+// default release semantics at CTA scope.  Used to hand a TMEM accumulator
+// back to the pair's MMA thread: what must be ordered before the MMA
+// overwrites it are this thread's tcgen05.ld of that buffer, which are
+// complete (tcgen05.wait::ld) and ordered by tcgen05.fence::before_thread_sync
+// around this arrive; a cluster-scope release would additionally wait for the
+// thread's outstanding global stores, once per hand-off.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 // 16-byte load from another CTA's shared memory (address from mapa).

@@ -13,6 +13,7 @@
 
 #include "gemm_sm100.cuh"
 #include "gemv.cuh"
+#include "mma_probe.cuh"
 #include "qk_common.cuh"
 #include "quant.cuh"
 
@@ -143,6 +144,40 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   }
 }
 
+// Every finite binary32 g in [first, first + count): the fused SiLU product
+// as the quantisers compute it (quant::silu_mul2, partly on packed pairs)
+// against the scalar chain (quant::silu_mul), u = 1.  Counts the g whose results differ in any bit and keeps the
+// smallest such bit pattern.
+__global__ void __launch_bounds__(256) selftest_silu_kernel(uint32_t first, uint64_t count,
+                                                            unsigned long long* mismatches,
+                                                            uint32_t* first_mismatch) {
+  const uint64_t pairs = (count + 1) / 2;
+  unsigned long long local = 0;
+  uint32_t low = 0xFFFFFFFFu;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < pairs;
+       i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    const uint64_t o0 = 2 * i, o1 = 2 * i + 1;
+    const uint32_t b0 = first + static_cast<uint32_t>(o0);
+    const uint32_t b1 = first + static_cast<uint32_t>(o1 < count ? o1 : o0);
+    const float g0 = __uint_as_float(b0), g1 = __uint_as_float(b1);
+    float h0, h1;
+    quant::silu_mul2(g0, g1, 1.0f, 1.0f, h0, h1);
+    const float r0 = quant::silu_mul(g0, 1.0f), r1 = quant::silu_mul(g1, 1.0f);
+    if (isfinite(g0) && __float_as_uint(h0) != __float_as_uint(r0)) {
+      ++local;
+      low = b0 < low ? b0 : low;
+    }
+    if (o1 < count && isfinite(g1) && __float_as_uint(h1) != __float_as_uint(r1)) {
+      ++local;
+      low = b1 < low ? b1 : low;
+    }
+  }
+  if (local) {
+    atomicAdd(mismatches, local);
+    if (first_mismatch) atomicMin(first_mismatch, low);
+  }
+}
+
 // Scratch for qk_w8a8_gemm_noalloc: a split-K workspace that lives in the
 // library's own device memory (zero at module load).  Host code only ever sees
 // a stand-in for this symbol; its device address comes from
@@ -229,18 +264,24 @@ bool pair_plan_for(int m, int n, int k, int group_k, gemm::PairPlan* pl) {
 }  // namespace
 
 namespace {
-// Tail tiles of the group kernel's K split for this problem on the current
-// device (0: no split, or not group mode, or bad arguments).
-int group_split_for(int m, int n, int k, int group_k) {
-  if (group_k == 0 || gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return 0;
+// The output-only group kernel's plan for this problem on the current device
+// (false: not group mode, or bad arguments).
+bool group_plan_for(int m, int n, int k, int group_k, gemm::GroupPlan* g) {
+  if (group_k == 0 || gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return false;
   const DeviceInfo* dev = nullptr;
-  if (check_device(&dev) != QK_OK) return 0;
-  return gemm::group_split_tiles(m, n, k, dev->sms);
+  if (check_device(&dev) != QK_OK) return false;
+  int dev_id = 0;
+  if (cudaGetDevice(&dev_id) != cudaSuccess) return false;
+  *g = gemm::group_plan(m, n, k, dev_id, dev->sms);
+  return true;
 }
 }  // namespace
 
 size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k) {
-  if (group_k != 0) return gemm::group_workspace_bytes(group_split_for(m, n, k, group_k));
+  if (group_k != 0) {
+    gemm::GroupPlan g;
+    return group_plan_for(m, n, k, group_k, &g) ? gemm::group_plan_workspace_bytes(g) : 0;
+  }
   gemm::PairPlan pl;
   return pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_bytes(pl) : 0;
 }
@@ -543,8 +584,8 @@ qk_status qk_w8a8_gemm_noalloc(int m, int n, int k, const int8_t* a, const int8_
   // accumulators must start at zero (partials and running sums need no
   // initialisation).
   gemm::PairPlan pl;
-  const int gsplit = group_split_for(m, n, k, group_k);
-  const size_t zero = gsplit > 0 ? gemm::group_flag_bytes(gsplit)
+  gemm::GroupPlan gp;
+  const size_t zero = group_plan_for(m, n, k, group_k, &gp) ? gemm::group_plan_flag_bytes(gp)
                       : pair_plan_for(m, n, k, group_k, &pl) ? gemm::pair_workspace_zero_bytes(pl)
                                                              : need;
   if (cudaMemsetAsync(scratch, 0, zero, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -571,6 +612,39 @@ qk_status qk_selftest_bounded_wait(int timeout_us, qk_stream stream) {
   selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(timeout_us) * 1000ull);
   return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+}
+
+qk_status qk_selftest_silu(uint32_t first, uint64_t count, unsigned long long* mismatches,
+                           uint32_t* first_mismatch, qk_stream stream) {
+  if (count == 0 || count > (1ull << 32) || static_cast<uint64_t>(first) + count > (1ull << 32) ||
+      mismatches == nullptr)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(mismatches, 8) || !aligned(first_mismatch, 4)) return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  const uint64_t pairs = (count + 1) / 2;
+  uint64_t blocks = (pairs + 255) / 256;
+  const uint64_t cap = static_cast<uint64_t>(dev->sms) * 8;
+  if (blocks > cap) blocks = cap;
+  selftest_silu_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      first, count, mismatches, first_mismatch);
+  return cuda_status(cudaGetLastError(), "silu selftest launch");
+}
+
+qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas,
+                               unsigned long long* cycles, qk_stream stream) {
+  if ((cta_group != 1 && cta_group != 2) || n < 32 || n > 256 || (n % 16) != 0)
+    return QK_ERR_INVALID_ARG;
+  if (iters < 1 || iters > (1 << 20) || ctas < 1 || ctas > 65535 || (ctas % cta_group) != 0)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(cycles, 8)) return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  return cuda_status(probe::launch(cta_group == 2, n, iters, ctas, cycles,
+                                   reinterpret_cast<cudaStream_t>(stream)),
+                     "mma rate probe launch");
 }
 
 }  // extern "C"

@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 6
+ABI_VERSION = 8
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -75,6 +75,8 @@ _SIGNATURES = {
                                             ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P]),
     "qk_device_status": (ctypes.c_int, [_P]),
     "qk_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_int, _P]),
+    "qk_selftest_silu": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_uint64, _P, _P, _P]),
+    "qk_selftest_mma_rate": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -200,6 +202,14 @@ def qk_device_status(stream) -> int:
 
 def qk_selftest_bounded_wait(timeout_us, stream) -> int:
     return lib().qk_selftest_bounded_wait(timeout_us, stream)
+
+
+def qk_selftest_silu(first, count, mismatches, first_mismatch, stream) -> int:
+    return lib().qk_selftest_silu(first, count, mismatches, first_mismatch, stream)
+
+
+def qk_selftest_mma_rate(cta_group, n, iters, ctas, cycles, stream) -> int:
+    return lib().qk_selftest_mma_rate(cta_group, n, iters, ctas, cycles, stream)
 
 
 # ---------------------------------------------------------------- torch helpers
@@ -472,3 +482,34 @@ def mlp_down(gate, up, w_q, sw, output_scale: float = 1.0, out_dtype=None, strea
 
 def device_status(stream=None) -> int:
     return qk_device_status(_stream(stream))
+
+
+def mma_rate(cta_group: int = 2, n: int = 256, iters: int = 16384, ctas: int | None = None,
+             launches: int = 5, stream=None) -> dict:
+    """Time qk_selftest_mma_rate: `launches` back-to-back launches between
+    CUDA events on the current stream.  Returns the INT8 rate (TOPS, 2 ops
+    per multiply-add) and the issuing CTAs' median cycles per launch."""
+    torch = _torch()
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        ctas -= ctas % cta_group
+    cyc = torch.zeros((ctas,), dtype=torch.int64, device="cuda")
+    s = _stream(stream)
+    _check(qk_selftest_mma_rate(cta_group, n, iters, ctas, _ptr(cyc), s), "mma rate probe")  # warm-up
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for _ in range(launches):
+        _check(qk_selftest_mma_rate(cta_group, n, iters, ctas, _ptr(cyc), s), "mma rate probe")
+    e1.record(cur)
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) * 1e-3 / launches
+    macs = (ctas // cta_group) * iters * (128 * cta_group) * n * 32
+    issuing = cyc[::cta_group].double()
+    cycles = float(issuing.median().item())
+    return {"tops": 2.0 * macs / sec / 1e12, "seconds_per_launch": sec, "cycles": cycles,
+            "macs_per_clk_per_sm": macs / cta_group / (ctas // cta_group) / cycles if cycles > 0 else None,
+            "clock_mhz_from_cycles": cycles / sec / 1e6, "cta_group": cta_group, "n": n, "iters": iters,
+            "ctas": ctas}
+
