@@ -65,7 +65,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 8
+#define QK_ABI_VERSION 9
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -354,21 +354,21 @@ QK_API size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k);
  * qk_w8a8_linear -- the whole W8A8 linear layer in one call: dynamic
  * per-token quantisation of x (as qk_quantize_per_token) into the
  * workspace, then the INT8 GEMM and dequant epilogue (as qk_w8a8_gemm) on
- * the same stream.  The two kernels are launched with programmatic
- * dependent launch, so the GEMM's set-up overlaps the quantiser's tail.  The
- * int8 values, scales and outputs are bit-identical to the two-call form.
- * (A form with the quantiser inside every decode-GEMV CTA was built and
- * measured slower on this part -- 15.6 us against 13.2 us at 4 x 14336 x
- * 4096 -- because every CTA must read all of x to reduce the row maxima.)
+ * the same stream.  The int8 values, scales and outputs are bit-identical to
+ * the two-call form.  The two kernels are launched with programmatic
+ * dependent launch, so the GEMM's set-up overlaps the quantiser's tail.
  *
  * x              [m, k] activations, x_dtype QK_BF16 or QK_F32, 16-B aligned
  * b, scale_b, group_k, output_scale   as qk_w8a8_gemm
  * scale_a_out    optional [m] fp32: receives the per-token scales; NULL to skip
  * out            [m, n] output in out_dtype, 16-B aligned (required)
  * workspace      qk_w8a8_linear_workspace_size() bytes, 256-B aligned: the
- *                GEMM's workspace (which must be zero-filled before its
- *                first use and is left zero by every call), then q and the
- *                scales.  Calls that may overlap need separate workspaces.
+ *                GEMM's workspace and 256 bytes of flags used by
+ *                qk_w8a8_linear_fused (both must be zero-filled before the
+ *                first use and are left zero by every completed call;
+ *                zero-fill again after a call that ended in QK_ERR_TIMEOUT),
+ *                then q and the scales.  Calls that may overlap need
+ *                separate workspaces.
  * Errors: those of qk_quantize_per_token and qk_w8a8_gemm.
  */
 QK_API qk_status qk_w8a8_linear(int m, int n, int k, const void* x, qk_dtype x_dtype,
@@ -379,6 +379,36 @@ QK_API qk_status qk_w8a8_linear(int m, int n, int k, const void* x, qk_dtype x_d
 
 /* Bytes of workspace qk_w8a8_linear needs (0 for arguments it would reject). */
 QK_API size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k);
+
+/*
+ * qk_w8a8_linear_fused -- the decode linear layer (per-channel scales) in ONE
+ * launch: the quantiser inside the GEMV's grid ("dynquant-kernels" 0.2.0,
+ * What is in here: the decode GEMV as the memory-bound serving case;
+ * "KV-cache kernels" section 04: the same fusion instincts).  The grid's first
+ * m CTAs quantise one token each (the rule of qk_quantize_per_token) into the
+ * workspace and count it in a flag word there; the other CTAs run the GEMV,
+ * start the weight stream at once and wait (bounded, about a second) for the
+ * count to reach m before they read the tokens.  The grid never exceeds what
+ * the device holds at once; other work running on the device at the same
+ * time can make the wait expire (QK_ERR_TIMEOUT in qk_device_status, outputs
+ * incomplete).  Results are bit-identical to qk_w8a8_linear.
+ *
+ * On a B200, at 4 x 14336 x 4096 in CUDA graphs of back-to-back calls, it
+ * takes 14.9 us against 13.0 us for qk_w8a8_linear's two overlapped kernels:
+ * the weight requests queue in DRAM ahead of the tokens' own loads.  It saves
+ * the host one kernel launch per layer, which matters when decode steps are
+ * launched eagerly.
+ *
+ * Arguments, layouts and the workspace are those of qk_w8a8_linear with
+ * group_k = 0; the workspace's flag words must be zero before the call and
+ * are zero again after it.  Shapes: m <= 8, k <= 16384 (k % 16 == 0, n % 8 ==
+ * 0); others give QK_ERR_UNSUPPORTED.
+ * Errors: those of qk_w8a8_linear, and QK_ERR_UNSUPPORTED.
+ */
+QK_API qk_status qk_w8a8_linear_fused(int m, int n, int k, const void* x, qk_dtype x_dtype,
+                                      const int8_t* b, const float* scale_b, float output_scale,
+                                      float* scale_a_out, void* out, qk_dtype out_dtype,
+                                      void* workspace, size_t workspace_bytes, qk_stream stream);
 
 /*
  * qk_w8a8_gemm_noalloc -- qk_w8a8_gemm without a caller-provided workspace.

@@ -52,6 +52,12 @@ def test_linear_decode(O, m, n, k, dtype):
         assert check_out(host(out), ref["out_f32"], ref["out_bf16"]) == 1.0
     out2, sa2 = _two_call(x, wq, sw, 0, alpha, out_dtype)
     assert_bits(host(out), host(out2), "one call vs two calls")
+    # the one-launch form (the quantiser inside the GEMV's grid)
+    out3, sa3 = qk.w8a8_linear_fused(x, wq, sw, alpha, out_dtype, want_scale=True)
+    torch.cuda.synchronize()
+    assert qk.device_status() == qk.QK_OK
+    assert_bits(host(sa3), ref["sa"], "scale (one launch)")
+    assert_bits(host(out3), host(out2), "one launch vs two calls")
 
 
 @pytest.mark.parametrize("m,n,k,group_k", [(9, 256, 512, 0), (300, 520, 2048, 0), (200, 264, 384, 128),
@@ -83,6 +89,18 @@ def test_linear_decode_workload_and_api(O):
     assert_bits(host(out), host(out_f), "qk.linear vs qk.w8a8_linear")
 
 
+def test_linear_fused_unsupported_shapes():
+    need_gpu()
+    x = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")  # m > 8: not the decode form
+    w = torch.zeros((16, 64), dtype=torch.int8, device="cuda")
+    sw = torch.ones((16,), dtype=torch.float32, device="cuda")
+    out = torch.empty((16, 16), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros((qk.qk_w8a8_linear_workspace_size(16, 16, 64, 0),), dtype=torch.uint8, device="cuda")
+    st = qk.qk_w8a8_linear_fused(16, 16, 64, qk._ptr(x), qk.QK_BF16, qk._ptr(w), qk._ptr(sw), 1.0, None,
+                                 qk._ptr(out), qk.QK_BF16, qk._ptr(ws), ws.numel(), qk._stream())
+    assert st == qk.QK_ERR_UNSUPPORTED
+
+
 def test_linear_errors():
     need_gpu()
     x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
@@ -95,3 +113,33 @@ def test_linear_errors():
     st = qk.qk_w8a8_linear(4, 16, 64, qk._ptr(x), qk.QK_BF16, qk._ptr(w), qk._ptr(sw), 0, 1.0, None,
                            qk._ptr(out), qk.QK_BF16, None, 0, qk._stream())
     assert st == qk.QK_ERR_WORKSPACE  # q and the scales live in the workspace
+
+
+@pytest.mark.parametrize("m,n,k,dtype", [(4, 14336, 4096, "bf16"), (1, 520, 4096, "bf16"), (8, 264, 16384, "f32"),
+                                         (3, 1032, 4112, "bf16")])
+def test_linear_decode_one_launch_reuses_workspace(O, m, n, k, dtype):
+    # qk_w8a8_linear_fused quantises the tokens inside the GEMV's launch and
+    # hands them over through flag words in the workspace: three calls with
+    # new tokens on one workspace, each bit-identical to the oracle and to the
+    # two-call form, and the flags back at zero after every call
+    need = qk.qk_w8a8_linear_workspace_size(m, n, k, 0)
+    ws = torch.zeros((need,), dtype=torch.uint8, device="cuda")
+    g_bytes = 0  # the GEMV takes no GEMM workspace: the flags come first
+    assert qk.qk_w8a8_gemm_workspace_size(m, n, k, 0) == 0
+    out_dtype = torch.float32 if dtype == "f32" else torch.bfloat16
+    for call in range(3):
+        w = synth.make_linear(m, n, k, seed=1000 * call + m + n + k, x_dtype=dtype, outlier_frac=0.01,
+                              outlier_scale=20.0)
+        x, wq, sw = x_dev(w.x), dev(w.w_q), dev(w.sw)
+        out, sa = qk.w8a8_linear_fused(x, wq, sw, 0.75, out_dtype, want_scale=True, workspace=ws)
+        torch.cuda.synchronize()
+        assert qk.device_status() == qk.QK_OK
+        assert int(ws[g_bytes:g_bytes + 256].count_nonzero()) == 0, "flags left set"
+        ref = O.linear(w.x, w.w_q, w.sw, 0, 0.75)
+        assert_bits(host(sa), ref["sa"], "scale")
+        if out_dtype == torch.float32:
+            assert_bits(host(out), ref["out_f32"], "fp32 out")
+        else:
+            assert check_out(host(out), ref["out_f32"], ref["out_bf16"]) == 1.0
+        out2, _ = _two_call(x, wq, sw, 0, 0.75, out_dtype)
+        assert_bits(host(out), host(out2), "one launch vs two calls")

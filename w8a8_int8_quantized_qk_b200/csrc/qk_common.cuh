@@ -30,8 +30,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Limit of every barrier wait in the library's kernels.  A healthy wait lasts
-// microseconds; one second means a peer never arrived.
+// microseconds; one second means a peer never arrived.  The waits count SM
+// clock cycles (clock64, a register read) rather than %globaltimer, whose
+// read is slow enough to show in a per-group hand-off; the cycle limit is one
+// second at 2 GHz, and longer at the lower clocks a B200 runs at.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint64_t kCyclesPerNs = 2;
+
+__device__ __forceinline__ uint64_t cycles_now() { return static_cast<uint64_t>(clock64()); }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -86,17 +92,17 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 }
 
 // Wait until the phase with the given parity has completed.  Gives up when
-// `abort` (a shared flag) is set by another role, or after `limit_ns`, in
-// which case it records QK_ERR_TIMEOUT and sets `abort`.  Returns true when
-// the phase completed.
+// `abort` (a shared flag) is set by another role, or after `limit_ns` (2
+// cycles per ns), in which case it records QK_ERR_TIMEOUT and sets `abort`.
+// Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = cycles_now();
   while (true) {
     if (mbar_try_wait_suspend(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if (cycles_now() - t0 > limit_ns * kCyclesPerNs) {
       record_status(QK_ERR_TIMEOUT);
       if (abort != nullptr) *abort = 1;
       return false;
@@ -111,12 +117,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ bool flag_wait(const int* flag, int target, volatile int* abort) {
   const volatile int* f = flag;
   if (*f >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = cycles_now();
   while (true) {
     __nanosleep(256);
     if (*f >= target) return true;
     if (abort != nullptr && *abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (cycles_now() - t0 > kWaitLimitNs * kCyclesPerNs) {
       record_status(QK_ERR_TIMEOUT);
       if (abort != nullptr) *abort = 1;
       return false;

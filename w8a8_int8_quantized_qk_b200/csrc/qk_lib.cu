@@ -520,15 +520,18 @@ qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
 }
 
 // The linear layer's workspace: the GEMM's own (offset 0, so its
-// zero-on-return contract covers it), then q [m, k] int8, then the scales.
+// zero-on-return contract covers it), then 256 bytes of flags for the fused
+// decode kernel (zero before and after every call, like the GEMM's part),
+// then q [m, k] int8, then the scales.
 namespace {
 inline size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+constexpr size_t kLinearFlagBytes = 256;  // m + 1 <= 64 ints (the fused form has m <= 8)
 }  // namespace
 
 size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k) {
   if (gemm_check(m, n, k, group_k) != QK_OK || m == 0 || n == 0) return 0;
   const size_t g = round256(qk_w8a8_gemm_workspace_size(m, n, k, group_k));
-  return g + round256(static_cast<size_t>(m) * static_cast<size_t>(k)) +
+  return g + kLinearFlagBytes + round256(static_cast<size_t>(m) * static_cast<size_t>(k)) +
          round256(static_cast<size_t>(m) * 4);
 }
 
@@ -554,13 +557,69 @@ qk_status qk_w8a8_linear(int m, int n, int k, const void* x, qk_dtype x_dtype, c
   if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
     return QK_ERR_WORKSPACE;
   const size_t g_bytes = round256(qk_w8a8_gemm_workspace_size(m, n, k, group_k));
-  int8_t* q = reinterpret_cast<int8_t*>(static_cast<char*>(workspace) + g_bytes);
-  float* sa = reinterpret_cast<float*>(static_cast<char*>(workspace) + g_bytes +
+  int* flags = reinterpret_cast<int*>(static_cast<char*>(workspace) + g_bytes);
+  int8_t* q = reinterpret_cast<int8_t*>(static_cast<char*>(workspace) + g_bytes + kLinearFlagBytes);
+  float* sa = reinterpret_cast<float*>(static_cast<char*>(workspace) + g_bytes + kLinearFlagBytes +
                                        round256(static_cast<size_t>(m) * static_cast<size_t>(k)));
   st = quant_common(m, k, x, nullptr, k, x_dtype, q, sa, stream, false);
   if (st != QK_OK) return st;
   st = qk_w8a8_gemm(m, n, k, q, b, sa, scale_b, group_k, output_scale, nullptr, out, out_dtype,
                     g_bytes > 0 ? workspace : nullptr, g_bytes, stream);
+  if (st != QK_OK || scale_a_out == nullptr) return st;
+  return cuda_status(cudaMemcpyAsync(scale_a_out, sa, static_cast<size_t>(m) * 4,
+                                     cudaMemcpyDeviceToDevice, s),
+                     "scale copy");
+}
+
+qk_status qk_w8a8_linear_fused(int m, int n, int k, const void* x, qk_dtype x_dtype, const int8_t* b,
+                               const float* scale_b, float output_scale, float* scale_a_out, void* out,
+                               qk_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                               qk_stream stream) {
+  qk_status st = gemm_check(m, n, k, 0);
+  if (st != QK_OK) return st;
+  if (x_dtype != QK_F32 && x_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (out_dtype != QK_F32 && out_dtype != QK_BF16) return QK_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return QK_OK;
+  if (x == nullptr || b == nullptr || scale_b == nullptr || out == nullptr)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(b, 16) || !aligned(scale_b, 16) || !aligned(out, 16) ||
+      !aligned(scale_a_out, 4))
+    return QK_ERR_MISALIGNED;
+  if (gemm_path(m, n, k, 0) != GemmPath::kGemv || !gemv::pref_supported(m, k))
+    return QK_ERR_UNSUPPORTED;
+  const DeviceInfo* dev = nullptr;
+  st = check_device(&dev);
+  if (st != QK_OK) return st;
+  const size_t need = qk_w8a8_linear_workspace_size(m, n, k, 0);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
+    return QK_ERR_WORKSPACE;
+  // the workspace layout of qk_w8a8_linear (the GEMV takes no GEMM workspace)
+  const size_t g_bytes = round256(qk_w8a8_gemm_workspace_size(m, n, k, 0));
+  int* flags = reinterpret_cast<int*>(static_cast<char*>(workspace) + g_bytes);
+  int8_t* q = reinterpret_cast<int8_t*>(static_cast<char*>(workspace) + g_bytes + kLinearFlagBytes);
+  float* sa = reinterpret_cast<float*>(static_cast<char*>(workspace) + g_bytes + kLinearFlagBytes +
+                                       round256(static_cast<size_t>(m) * static_cast<size_t>(k)));
+  gemv::FusedArgs fa = {};
+  fa.g.m = m;
+  fa.g.n = n;
+  fa.g.k = k;
+  fa.g.a = q;
+  fa.g.w = b;
+  fa.g.sa = sa;
+  fa.g.sw = scale_b;
+  fa.g.alpha = output_scale;
+  fa.g.out = out;
+  fa.g.out_bf16 = out_dtype == QK_BF16;
+  fa.x = x;
+  fa.flags = flags;
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  const bool launched = x_dtype == QK_BF16 ? gemv::launch_fused<true>(fa, dev_id, dev->sms, s, &e)
+                                           : gemv::launch_fused<false>(fa, dev_id, dev->sms, s, &e);
+  if (!launched) return QK_ERR_UNSUPPORTED;
+  st = cuda_status(e, "fused decode launch");
   if (st != QK_OK || scale_a_out == nullptr) return st;
   return cuda_status(cudaMemcpyAsync(scale_a_out, sa, static_cast<size_t>(m) * 4,
                                      cudaMemcpyDeviceToDevice, s),

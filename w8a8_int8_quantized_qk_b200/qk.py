@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 8
+ABI_VERSION = 9
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -71,6 +71,8 @@ _SIGNATURES = {
                                       ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t,
                                       _P]),
     "qk_w8a8_linear_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "qk_w8a8_linear_fused": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P,
+                                            ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "qk_w8a8_gemm_noalloc": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
                                             ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P]),
     "qk_device_status": (ctypes.c_int, [_P]),
@@ -186,6 +188,12 @@ def qk_w8a8_linear(m, n, k, x, x_dtype, b, scale_b, group_k, output_scale, scale
 
 def qk_w8a8_linear_workspace_size(m, n, k, group_k) -> int:
     return lib().qk_w8a8_linear_workspace_size(m, n, k, group_k)
+
+
+def qk_w8a8_linear_fused(m, n, k, x, x_dtype, b, scale_b, output_scale, scale_a_out, out, out_dtype,
+                         workspace, workspace_bytes, stream) -> int:
+    return lib().qk_w8a8_linear_fused(m, n, k, x, x_dtype, b, scale_b, output_scale, scale_a_out, out,
+                                      out_dtype, workspace, workspace_bytes, stream)
 
 
 def qk_w8a8_gemm_noalloc(m, n, k, a, b, scale_a, scale_b, group_k, output_scale, c, out, out_dtype,
@@ -461,6 +469,29 @@ def w8a8_linear(x, w_q, sw, group_k: int = 0, output_scale: float = 1.0, out_dty
                           float(output_scale), _ptr(sa), _ptr(out), _dtype_code(out), _ptr(workspace),
                           0 if workspace is None else workspace.numel(), _stream(stream)),
            "qk_w8a8_linear")
+    return out, sa
+
+
+def w8a8_linear_fused(x, w_q, sw, output_scale: float = 1.0, out_dtype=None, want_scale: bool = False,
+                      workspace=None, stream=None):
+    """qk_w8a8_linear_fused (decode shapes, one launch): x [m, k] -> (out [m, n],
+    per-token scales [m] or None).  `workspace` (or a fresh zero-filled one)
+    holds the flag words, q and the scales."""
+    torch = _torch()
+    _need_cuda(x, w_q, sw)
+    assert x.dim() == 2 and x.is_contiguous()
+    m, k = x.shape
+    n = w_q.shape[0]
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = torch.empty((m, n), dtype=out_dtype, device=x.device)
+    sa = torch.empty((m,), dtype=torch.float32, device=x.device) if want_scale else None
+    need = qk_w8a8_linear_workspace_size(m, n, k, 0)
+    if workspace is None:
+        workspace = torch.zeros((max(need, 1),), dtype=torch.uint8, device=x.device)
+    _check(qk_w8a8_linear_fused(m, n, k, _ptr(x), _dtype_code(x), _ptr(w_q), _ptr(sw), float(output_scale),
+                                _ptr(sa), _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(),
+                                _stream(stream)),
+           "qk_w8a8_linear_fused")
     return out, sa
 
 
