@@ -333,27 +333,34 @@ def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
     quant_us = _graph_us(torch, L, lambda i: L.quant(i % L.R), iters)
     gemm_us = _graph_us(torch, L, lambda i: L.gemm(i % L.R), iters)
     step_us = _graph_us(torch, L, lambda i: L.step(i), iters)
-    linear_us = None
+    linear_us = {}
     if w.gate is None and w.group_k == 0 and w.m <= 8:
-        # the layer in one call (qk_w8a8_linear: at decode shapes one launch,
-        # the quantiser inside the GEMV's grid), one zero-filled workspace per copy
+        # the layer through its one-call entry points: qk_w8a8_linear (the
+        # quantiser and the GEMV as two kernels) and qk_w8a8_linear_fused (one
+        # launch, the quantiser inside the GEMV's grid), one zero-filled
+        # workspace per copy
         import ctypes
 
         wsn = qk.qk_w8a8_linear_workspace_size(w.m, w.n, w.k, 0)
         wss = [torch.zeros((wsn,), dtype=torch.uint8, device="cuda") for _ in range(L.R)]
+        for name, fn in (("linear_call_us", None), ("linear_fused_us", qk.qk_w8a8_linear_fused)):
 
-        def linear_call(i):
-            j = i % L.R
-            (xp, _), wp, _, _, op = L.p[j]
-            st = qk.qk_w8a8_linear(w.m, w.n, w.k, xp, L.xdt, wp, L.swp, 0, w.alpha, None, op, L.odt,
-                                   ctypes.c_void_p(wss[j].data_ptr()), wsn, L.stream)
-            if st != 0:
-                raise qk.QKError(st, "linear")
+            def linear_call(i, fn=fn):
+                j = i % L.R
+                (xp, _), wp, _, _, op = L.p[j]
+                ws = ctypes.c_void_p(wss[j].data_ptr())
+                if fn is None:
+                    st = qk.qk_w8a8_linear(w.m, w.n, w.k, xp, L.xdt, wp, L.swp, 0, w.alpha, None, op, L.odt,
+                                           ws, wsn, L.stream)
+                else:
+                    st = fn(w.m, w.n, w.k, xp, L.xdt, wp, L.swp, w.alpha, None, op, L.odt, ws, wsn, L.stream)
+                if st != 0:
+                    raise qk.QKError(st, name)
 
-        for i in range(3):
-            linear_call(i)
-        torch.cuda.synchronize()
-        linear_us = _graph_us(torch, L, linear_call, iters)
+            for i in range(3):
+                linear_call(i)
+            torch.cuda.synchronize()
+            linear_us[name] = _graph_us(torch, L, linear_call, iters)
     by = _bytes(w)
     ops = 2.0 * w.m * w.n * w.k
     gemm_kernel = "gemv (CUDA cores)" if (w.m <= 8 and not w.group_k) else (
@@ -372,9 +379,7 @@ def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
            "gemm_hbm_frac": by["gemm"] / (gemm_us * 1e-6) / 1e9 / pk["hbm_gbs"],
            "gemm_hbm_frac_nominal": by["gemm"] / (gemm_us * 1e-6) / 1e9 / NOMINAL["hbm_gbs"],
            "step_us": step_us, "bytes": by}
-    if linear_us is not None:
-        res["linear_one_call_us"] = linear_us
-        res["linear_one_call_note"] = "qk_w8a8_linear: quantiser inside the GEMV launch (flag hand-off)"
+    res.update(linear_us)
     del L
     torch.cuda.empty_cache()
     return res
@@ -800,7 +805,7 @@ def run_ours(args):
                           "frac": decode["roofline"]["frac"],
                           "frac_nominal": decode["roofline"]["frac_nominal"],
                           "step_us": decode["step_us"],
-                          "one_launch_step_us": stages["decode"].get("linear_one_call_us")}
+                          "one_launch_step_us": stages["decode"].get("linear_fused_us")}
     # details first (every workload's stages, the probe, the decode roofline),
     # then the headline line last
     details = {"bench_details": {"stages": stages, "decode": decode, "int8_probe": probe, "peaks": pk}}

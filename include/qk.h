@@ -401,8 +401,8 @@ QK_API size_t qk_w8a8_linear_workspace_size(int m, int n, int k, int group_k);
  *
  * Arguments, layouts and the workspace are those of qk_w8a8_linear with
  * group_k = 0; the workspace's flag words must be zero before the call and
- * are zero again after it.  Shapes: m <= 8, k <= 16384 (k % 16 == 0, n % 8 ==
- * 0); others give QK_ERR_UNSUPPORTED.
+ * are zero again after it.  Shapes: m <= 4 with k <= 16384, or 4 < m <= 8
+ * with k <= 8192 (k % 16 == 0, n % 8 == 0); others give QK_ERR_UNSUPPORTED.
  * Errors: those of qk_w8a8_linear, and QK_ERR_UNSUPPORTED.
  */
 QK_API qk_status qk_w8a8_linear_fused(int m, int n, int k, const void* x, qk_dtype x_dtype,

@@ -89,14 +89,17 @@ def test_linear_decode_workload_and_api(O):
     assert_bits(host(out), host(out_f), "qk.linear vs qk.w8a8_linear")
 
 
-def test_linear_fused_unsupported_shapes():
+@pytest.mark.parametrize("m,k", [(16, 64), (9, 256), (8, 16384), (5, 8208)])
+def test_linear_fused_unsupported_shapes(m, k):
+    # beyond the decode shapes: m > 8, or m > 4 with k > 8192
     need_gpu()
-    x = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")  # m > 8: not the decode form
-    w = torch.zeros((16, 64), dtype=torch.int8, device="cuda")
-    sw = torch.ones((16,), dtype=torch.float32, device="cuda")
-    out = torch.empty((16, 16), dtype=torch.bfloat16, device="cuda")
-    ws = torch.zeros((qk.qk_w8a8_linear_workspace_size(16, 16, 64, 0),), dtype=torch.uint8, device="cuda")
-    st = qk.qk_w8a8_linear_fused(16, 16, 64, qk._ptr(x), qk.QK_BF16, qk._ptr(w), qk._ptr(sw), 1.0, None,
+    n = 16
+    x = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((n, k), dtype=torch.int8, device="cuda")
+    sw = torch.ones((n,), dtype=torch.float32, device="cuda")
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros((qk.qk_w8a8_linear_workspace_size(m, n, k, 0),), dtype=torch.uint8, device="cuda")
+    st = qk.qk_w8a8_linear_fused(m, n, k, qk._ptr(x), qk.QK_BF16, qk._ptr(w), qk._ptr(sw), 1.0, None,
                                  qk._ptr(out), qk.QK_BF16, qk._ptr(ws), ws.numel(), qk._stream())
     assert st == qk.QK_ERR_UNSUPPORTED
 
@@ -115,8 +118,8 @@ def test_linear_errors():
     assert st == qk.QK_ERR_WORKSPACE  # q and the scales live in the workspace
 
 
-@pytest.mark.parametrize("m,n,k,dtype", [(4, 14336, 4096, "bf16"), (1, 520, 4096, "bf16"), (8, 264, 16384, "f32"),
-                                         (3, 1032, 4112, "bf16")])
+@pytest.mark.parametrize("m,n,k,dtype", [(4, 14336, 4096, "bf16"), (1, 520, 4096, "bf16"), (8, 264, 8192, "f32"),
+                                         (4, 264, 16384, "f32"), (3, 1032, 4112, "bf16")])
 def test_linear_decode_one_launch_reuses_workspace(O, m, n, k, dtype):
     # qk_w8a8_linear_fused quantises the tokens inside the GEMV's launch and
     # hands them over through flag words in the workspace: three calls with
