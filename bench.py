@@ -70,6 +70,8 @@ def peaks(probe: dict | None = None) -> dict:
     if probe is not None:
         p["int8_tops"] = probe["burst"]["tops"]
         p["int8_tops_sustained"] = probe["sustained"]["tops"] if probe.get("sustained") else None
+        rnd = probe.get("burst_random_operands")
+        p["int8_tops_random_operands"] = rnd["tops"] if rnd else None
         p["int8_source"] = "probe"
     else:
         p["int8_tops"] = 2.0 * p["bf16_tflops"]
@@ -90,9 +92,15 @@ def probe_int8_peak(torch, qk, local: int, sustained_s: float = 3.0) -> dict:
     with ClockSampler(local) as cl:
         burst = qk.mma_rate(2, 256, iters, launches=5)
     burst["clocks"] = cl.summary()
+    # the same loop on uniformly random operand bytes: the tensor pipe's rate
+    # depends on the values, and the benchmark's operands are random
+    with ClockSampler(local) as cl:
+        burst_random = qk.mma_rate(2, 256, iters, launches=5, operand_seed=12345)
+    burst_random["clocks"] = cl.summary()
     one_sm = qk.mma_rate(1, 256, iters, launches=5)
     res = {"kernel": "qk_selftest_mma_rate: tcgen05.mma.cta_group::2.kind::i8 256x256x32, shared-memory operands",
-           "burst": burst, "one_sm_128x256": one_sm, "sustained": None}
+           "burst": burst, "burst_random_operands": burst_random, "one_sm_128x256": one_sm,
+           "sustained": None, "sustained_random_operands": None}
     if sustained_s > 0:
         n = max(5, int(sustained_s / burst["seconds_per_launch"]))
         with ClockSampler(local) as cl:
@@ -100,6 +108,12 @@ def probe_int8_peak(torch, qk, local: int, sustained_s: float = 3.0) -> dict:
         sus["clocks"] = cl.summary()
         sus["launches"] = n
         res["sustained"] = sus
+        n = max(5, int(sustained_s / burst_random["seconds_per_launch"]))
+        with ClockSampler(local) as cl:
+            sus = qk.mma_rate(2, 256, iters, launches=n, operand_seed=12345)
+        sus["clocks"] = cl.summary()
+        sus["launches"] = n
+        res["sustained_random_operands"] = sus
     return res
 
 
@@ -375,6 +389,8 @@ def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
            "gemm_TOPS": ops / (gemm_us * 1e-6) / 1e12,
            "gemm_GBs": by["gemm"] / (gemm_us * 1e-6) / 1e9,
            "gemm_tensor_frac": ops / (gemm_us * 1e-6) / 1e12 / pk["int8_tops"],
+           "gemm_tensor_frac_random_operands": (ops / (gemm_us * 1e-6) / 1e12 / pk["int8_tops_random_operands"]
+                                                if pk.get("int8_tops_random_operands") else None),
            "gemm_tensor_frac_nominal": ops / (gemm_us * 1e-6) / 1e12 / NOMINAL["int8_tops"],
            "gemm_hbm_frac": by["gemm"] / (gemm_us * 1e-6) / 1e9 / pk["hbm_gbs"],
            "gemm_hbm_frac_nominal": by["gemm"] / (gemm_us * 1e-6) / 1e9 / NOMINAL["hbm_gbs"],
@@ -511,6 +527,8 @@ def measure_moe(torch, qk, iters: int, pk: dict) -> dict:
     return {"experts": e, "n": n, "k": k, "tokens": total, "tokens_per_expert": counts.tolist(),
             "copies": R, "timing": f"CUDA graph of {iters} iterations", "gemm_us": us,
             "gemm_TOPS": ops / (us * 1e-6) / 1e12, "gemm_tensor_frac": ops / (us * 1e-6) / 1e12 / pk["int8_tops"],
+            "gemm_tensor_frac_random_operands": (ops / (us * 1e-6) / 1e12 / pk["int8_tops_random_operands"]
+                                                 if pk.get("int8_tops_random_operands") else None),
             "gemm_tensor_frac_nominal": ops / (us * 1e-6) / 1e12 / NOMINAL["int8_tops"],
             "weight_GBs": wbytes / (us * 1e-6) / 1e9,
             "note": "1-SM tcgen05 kernel over experts x M tiles x N tiles, empty tiles skipped"}
@@ -692,11 +710,17 @@ def run_ours(args):
     roof = {"kernel": "gemm_i8_pair_kernel (tcgen05.mma.cta_group::2, 256x256 tiles)", "bound": "tensor",
             "achieved": gemm_tops, "peak": pk["int8_tops"], "unit": "TFLOP/s",
             "frac": gemm_tops / pk["int8_tops"], "frac_nominal": gemm_tops / NOMINAL["int8_tops"],
+            "peak_random_operands": pk.get("int8_tops_random_operands"),
+            "frac_random_operands": (gemm_tops / pk["int8_tops_random_operands"]
+                                     if pk.get("int8_tops_random_operands") else None),
             "traffic": args.gemm_traffic or None,
             "peak_note": f"measured ({pk['int8_source']}): the burst rate of a tcgen05 kind::i8 CTA-pair "
                          f"MMA loop with no memory traffic, at a median SM clock of "
-                         f"{probe['burst']['clocks']['sm_mhz']} MHz; frac_nominal against the "
-                         "4500 TOPS datasheet dense INT8 peak; int8 ops counted as 2*M*N*K",
+                         f"{probe['burst']['clocks']['sm_mhz']} MHz on zero operands; "
+                         "frac_random_operands against the same loop on uniformly random operand bytes "
+                         "(the benchmark's operands are random, and the tensor pipe is slower on them); "
+                         "frac_nominal against the 4500 TOPS datasheet dense INT8 peak; int8 ops counted "
+                         "as 2*M*N*K",
             "timing": f"average of a CUDA graph of {iters} back-to-back GEMM launches on the "
                       "headline's rotating buffers",
             "algorithmic_bytes": by["gemm"],
@@ -774,9 +798,11 @@ def run_ours(args):
     # the sustained form of the INT8 peak (seconds of back-to-back probe
     # launches), after the timed work so that its heat does not reach it
     if not args.quick and args.sustained_seconds > 0:
-        sus = probe_int8_peak(torch, qk, local, sustained_s=args.sustained_seconds)["sustained"]
-        probe["sustained"] = sus
-        pk["int8_tops_sustained"] = sus["tops"]
+        later = probe_int8_peak(torch, qk, local, sustained_s=args.sustained_seconds)
+        probe["sustained"] = later["sustained"]
+        probe["sustained_random_operands"] = later["sustained_random_operands"]
+        pk["int8_tops_sustained"] = later["sustained"]["tops"]
+        pk["int8_tops_sustained_random_operands"] = later["sustained_random_operands"]["tops"]
     if dist is not None:
         torch.cuda.synchronize()
         dist.destroy_process_group()

@@ -65,7 +65,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 9
+#define QK_ABI_VERSION 10
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -514,6 +514,12 @@ QK_API qk_status qk_selftest_silu(uint32_t first, uint64_t count, unsigned long 
  * iters       1 .. 1048576 instructions per CTA (pair)
  * ctas        1 .. 65535 CTAs, a multiple of cta_group; at most what the
  *             device holds at once (one CTA per SM) for a meaningful rate
+ * operand_seed  0: the operand tiles are zero; otherwise every CTA fills
+ *             them with bytes from a counter-based hash of the seed (close to
+ *             uniform over the int8 range).  The rate depends on the values:
+ *             on a B200 random operands run measurably slower than zeros at
+ *             the same SM clock, so a GEMM on random data is also read
+ *             against the random-operand rate
  * cycles      optional device array [ctas] of uint64, 8-byte aligned: the
  *             issuing CTA's SM clock cycles from its first issue to the
  *             completion of its last MMA (0 for a pair's second CTA); NULL
@@ -523,7 +529,8 @@ QK_API qk_status qk_selftest_silu(uint32_t first, uint64_t count, unsigned long 
  *         QK_ERR_CUDA.
  */
 QK_API qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas,
-                                      unsigned long long* cycles, qk_stream stream);
+                                      uint32_t operand_seed, unsigned long long* cycles,
+                                      qk_stream stream);
 
 #ifdef __cplusplus
 }

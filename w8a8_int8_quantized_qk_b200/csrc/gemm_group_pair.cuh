@@ -22,7 +22,11 @@
 // issuer (the pair's leader only), warps 2-3 the scale stagers, warps 4-11
 // the epilogue (warp w reads TMEM lanes 32 * (w % 4) and columns [128 h,
 // 128 h + 128), h = (w - 4) / 4).  setmaxnreg moves registers from the
-// control warpgroup (80 each) to the epilogue (208 each).
+// control warpgroup (80 each) to the epilogue (208 each).  A bf16 output
+// leaves through TMA bulk tensor stores from each epilogue warp's 2 KB box
+// (per-lane global stores of 16 bytes, one row per lane, measured 14.5 us
+// slower at 2048 x 8192 x 8192: the tile's stores hold up the next tile's
+// first groups).
 //
 // Work units come from group_plan.h with the pairs as workers: whole tiles,
 // and, when the last wave would be partial, its tiles cut at the middle
@@ -44,12 +48,13 @@ constexpr int kGpCtrlRegs = 80;
 constexpr int kGpEpiRegs = 208;
 constexpr int kGpLaunchRegs =  // registers per thread the launch must provide
     (128 * kGpCtrlRegs + kGpEpiWarps * 32 * kGpEpiRegs + kGpThreads - 1) / kGpThreads;
-constexpr int kGpSlice = 16;  // groups per staged scale slice
+constexpr int kGpSlice = 8;  // groups per staged scale slice
 
 struct alignas(1024) GroupPairStorage {
   uint8_t a[kGpStages][128 * BK];  // this CTA's 128 rows of A
   uint8_t b[kGpStages][128 * BK];  // this CTA's 128 rows of B
   float scales[2][kGpSlice * kGpBN];  // [slice buffer][group][column]
+  uint8_t out_stage[kGpEpiWarps][kOutBoxBytes];  // each epilogue warp's bf16 output box
   uint64_t full[kGpStages];
   uint64_t empty[kGpStages];
   uint64_t acc_full[2];
@@ -185,34 +190,31 @@ __device__ void gp_stage_scales(GroupPairStorage& s, const Args& p, uint32_t pr)
     }
     for (int gb = u.g0; gb < u.g1; gb += kGpSlice) {
       if (!mbar_wait(smem_addr(&s.aux_empty[buf]), phase ^ 1u, &s.abort)) return;
-      // two columns at a time (32 loads in flight per lane)
+      // the lane's four columns at once (32 values in flight)
+      float v[4][kGpSlice];
 #pragma unroll
-      for (int c2 = 0; c2 < 4; c2 += 2) {
-        float v[2][kGpSlice];
+      for (int c = 0; c < 4; ++c) {
+        const int col = col0 + c;
+        const float* src = p.sw + static_cast<int64_t>(col) * p.groups + gb;
+        if (vec_rows && (gb & 3) == 0 && col < p.n && gb + kGpSlice <= u.g1) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int col = col0 + c2 + c;
-          const float* src = p.sw + static_cast<int64_t>(col) * p.groups + gb;
-          if (vec_rows && (gb & 3) == 0 && col < p.n && gb + kGpSlice <= u.g1) {
-#pragma unroll
-            for (int q = 0; q < kGpSlice / 4; ++q) {
-              const float4 t = __ldg(reinterpret_cast<const float4*>(src) + q);
-              v[c][4 * q] = t.x;
-              v[c][4 * q + 1] = t.y;
-              v[c][4 * q + 2] = t.z;
-              v[c][4 * q + 3] = t.w;
-            }
-          } else {
-#pragma unroll
-            for (int gg = 0; gg < kGpSlice; ++gg)
-              v[c][gg] = (col < p.n && gb + gg < u.g1) ? __ldg(src + gg) : 0.0f;
+          for (int q = 0; q < kGpSlice / 4; ++q) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(src) + q);
+            v[c][4 * q] = t.x;
+            v[c][4 * q + 1] = t.y;
+            v[c][4 * q + 2] = t.z;
+            v[c][4 * q + 3] = t.w;
           }
-        }
-        float* dst = s.scales[buf] + c_lo + c2;
+        } else {
 #pragma unroll
-        for (int gg = 0; gg < kGpSlice; ++gg)
-          *reinterpret_cast<float2*>(dst + gg * kGpBN) = make_float2(v[0][gg], v[1][gg]);
+          for (int gg = 0; gg < kGpSlice; ++gg)
+            v[c][gg] = (col < p.n && gb + gg < u.g1) ? __ldg(src + gg) : 0.0f;
+        }
       }
+      float* dst = s.scales[buf] + c_lo;
+#pragma unroll
+      for (int gg = 0; gg < kGpSlice; ++gg)
+        *reinterpret_cast<float4*>(dst + gg * kGpBN) = make_float4(v[0][gg], v[1][gg], v[2][gg], v[3][gg]);
       mbar_arrive(smem_addr(&s.aux_full[buf]));  // release: this lane's stores
       if (++buf == 2) {
         buf = 0;
@@ -250,8 +252,8 @@ __device__ __forceinline__ void gp_fold16(float* f, const uint32_t (&v)[16], uin
   }
 }
 
-__device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, uint32_t pr,
-                            uint32_t lead) {
+__device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, const CUtensorMap* tmO,
+                            uint32_t pr, uint32_t lead) {
   const int np = gridDim.x >> 1, pi = blockIdx.x >> 1;
   const int ntiles = p.tiles_m * p.tiles_n;
   const int lane = threadIdx.x & 31;
@@ -343,12 +345,45 @@ __device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, u
       if (lane == 0) atomicAdd(p.gflag + 2 * tt + static_cast<int>(pr), 1);
       continue;
     }
-    const int row = tm * 256 + static_cast<int>(pr) * 128 + quad * 32 + lane;
+    const int row0 = tm * 256 + static_cast<int>(pr) * 128 + quad * 32;
+    const int row = row0 + lane;
+    const int colbase = tn * kGpBN + half * kGpCols;
+    const float sa = row < p.m ? __ldg(p.sa + row) : 0.0f;
+    const uint64_t sa2 = pack2(__float_as_uint(sa), __float_as_uint(sa));
+    const uint64_t al2 = pack2(__float_as_uint(p.alpha), __float_as_uint(p.alpha));
+    if (p.tma_out) {
+      // bf16: 32 x 32 boxes through this warp's shared-memory slot and TMA
+      // bulk tensor stores (clipped to the output's bounds)
+      if (row0 >= p.m) continue;  // warp-uniform
+      uint8_t* box = s.out_stage[ew];
+      const uint32_t rowaddr = smem_addr(box) + static_cast<uint32_t>(lane) * 64u;
+      const uint32_t sx = (static_cast<uint32_t>(lane) >> 1) & 3u;
+#pragma unroll
+      for (int b = 0; b < kGpCols / 32; ++b) {
+        if (colbase + b * 32 >= p.n) break;
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const uint64_t r2 = f32x2_mul(
+              f32x2_mul(pack2(__float_as_uint(f[b * 32 + 2 * e]), __float_as_uint(f[b * 32 + 2 * e + 1])), sa2),
+              al2);
+          w[e] = pack_bf16x2(lo_of(r2), hi_of(r2));
+        }
+        if (lane == 0) bulk_wait_read_all();  // the previous box has been read
+        __syncwarp();
+#pragma unroll
+        for (uint32_t j = 0; j < 4; ++j)
+          st_shared_v4(rowaddr + ((j ^ sx) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tmO, smem_addr(box), colbase + b * 32, row0);
+          bulk_commit();
+        }
+      }
+      continue;
+    }
     if (row < p.m) {
-      const float sa = __ldg(p.sa + row);
-      const uint64_t sa2 = pack2(__float_as_uint(sa), __float_as_uint(sa));
-      const uint64_t al2 = pack2(__float_as_uint(p.alpha), __float_as_uint(p.alpha));
-      const int colbase = tn * kGpBN + half * kGpCols;
 #pragma unroll
       for (int g8 = 0; g8 < kGpCols / 8; ++g8) {
         const int col = colbase + g8 * 8;
@@ -373,11 +408,14 @@ __device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, u
       }
     }
   }
+  if (p.tma_out && lane == 0) bulk_wait_all();  // the output stores are complete
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(kGpThreads, 1)
     gemm_i8_group_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                              const __grid_constant__ CUtensorMap tmB, const Args p) {
+                              const __grid_constant__ CUtensorMap tmB,
+                              const __grid_constant__ CUtensorMap tmO, const Args p) {
   extern __shared__ uint8_t smem_raw[];
   GroupPairStorage& s = storage<GroupPairStorage>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -386,6 +424,7 @@ __global__ void __launch_bounds__(kGpThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (p.tma_out) prefetch_tmap(&tmO);
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGpStages; ++i) {
@@ -426,7 +465,7 @@ __global__ void __launch_bounds__(kGpThreads, 1)
     }
   } else {
     regs_inc<kGpEpiRegs>();
-    gp_epilogue(s, tmem, p, pr, lead);
+    gp_epilogue(s, tmem, p, &tmO, pr, lead);
   }
   tc_fence_before();
   __syncthreads();

@@ -645,11 +645,15 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
         a.gflag = static_cast<int*>(workspace);
         a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)
                             : nullptr;
+        // bf16 out without c: TMA stores from shared memory
+        a.tma_out = (a.out != nullptr && a.out_bf16 && a.c == nullptr) ? 1 : 0;
+        CUtensorMap tpo = tpa;  // unused unless tma_out
+        if (a.tma_out && !cached_tmap(&tpo, a.out, a.m, a.n, 32, 1)) return 1;
         const size_t smem = group_pair_smem();
         e = set_smem_once(gemm_i8_group_pair_kernel, dev, 8, smem);
         if (e == cudaSuccess)
           e = launch_pdl(gemm_i8_group_pair_kernel, dim3(2 * gp.workers), dim3(kGpThreads), smem, stream,
-                         2, tpa, tpb, a);
+                         2, tpa, tpb, tpo, a);
         *err = e;
         return e == cudaSuccess ? 0 : 2;
       }

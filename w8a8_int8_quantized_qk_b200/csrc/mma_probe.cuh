@@ -11,6 +11,12 @@
 // 32 .. 256 (a multiple of 16), K = 32 per instruction.  Every CTA's MMA
 // thread records the SM clock cycles from its first issue to the completion
 // of its last MMA, so the host can also form MACs per clock per SM.
+//
+// Operands: all zero, or bytes from a counter-based hash of a seed.  The
+// rate depends on the values: on a B200 the pair form reaches about 8190
+// multiply-adds per clock per SM on zeros and measurably less on uniformly
+// random bytes at the same SM clock, so a GEMM on random operands is read
+// against the random-operand rate as well.
 #pragma once
 
 #include "qk_common.cuh"
@@ -28,27 +34,49 @@ struct alignas(1024) ProbeStorage {
   uint32_t tmem_base;
 };
 
+// Word w of a seeded operand tile: a 32-bit finaliser (multiply-xorshift) of
+// the word's index and the seed, so every byte is close to uniform.
+__device__ __forceinline__ uint32_t operand_word(uint32_t seed, uint32_t w) {
+  uint32_t x = w * 0x9E3779B1u ^ seed * 0x85EBCA77u;
+  x ^= x >> 16;
+  x *= 0x7FEB352Du;
+  x ^= x >> 15;
+  x *= 0x846CA68Bu;
+  x ^= x >> 16;
+  return x;
+}
+
 // `iters` instructions of shape (M = 128 * PAIR? 256 : 128) x n x 32.
 // cycles[cta] (optional): clock64 cycles between the first issue and the
 // last completion, on the issuing CTA (0 on a pair's second CTA).
 template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
-    mma_rate_kernel(int n, int iters, unsigned long long* cycles) {
+    mma_rate_kernel(int n, int iters, uint32_t seed, unsigned long long* cycles) {
   extern __shared__ uint8_t smem_raw[];
   ProbeStorage& s = *reinterpret_cast<ProbeStorage*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const uint32_t crank = PAIR ? cluster_rank() : 0u;
-  // zero operands: the rate of an integer MMA does not depend on the values
-  for (int i = threadIdx.x; i < kTileBytes / 16; i += kThreads)
-    reinterpret_cast<int4*>(s.a)[i] = make_int4(0, 0, 0, 0);
-  for (int i = threadIdx.x; i < 2 * kTileBytes / 16; i += kThreads)
-    reinterpret_cast<int4*>(s.b)[i] = make_int4(0, 0, 0, 0);
+  // operands: zeros (seed 0) or hashed bytes, different in every CTA
+  const uint32_t cseed = seed == 0 ? 0u : seed + 0x632BE5ABu * blockIdx.x;
+  auto fill = [&](uint8_t* dst, int bytes, uint32_t salt) {
+    for (int i = threadIdx.x; i < bytes / 16; i += kThreads) {
+      int4 v = make_int4(0, 0, 0, 0);
+      if (seed != 0) {
+        const uint32_t w = (salt + static_cast<uint32_t>(i)) * 4u;
+        v = make_int4(static_cast<int>(operand_word(cseed, w)), static_cast<int>(operand_word(cseed, w + 1)),
+                      static_cast<int>(operand_word(cseed, w + 2)), static_cast<int>(operand_word(cseed, w + 3)));
+      }
+      reinterpret_cast<int4*>(dst)[i] = v;
+    }
+  };
+  fill(s.a, kTileBytes, 0u);
+  fill(s.b, 2 * kTileBytes, static_cast<uint32_t>(kTileBytes / 16));
   if (threadIdx.x == 0) {
     mbar_init(smem_addr(&s.done), 1);
     fence_mbar_init();
   }
-  fence_proxy_async_smem();  // the zeros are visible to the tensor core
+  fence_proxy_async_smem();  // the operands are visible to the tensor core
   if (warp == 0) {
     if (PAIR) {
       tmem_alloc_pair(smem_addr(&s.tmem_base), 256);
@@ -102,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 inline size_t smem_bytes() { return sizeof(ProbeStorage) + 1024; }
 
 // ctas: CTAs of the grid (a multiple of 2 for pairs).
-inline cudaError_t launch(bool pair, int n, int iters, int ctas, unsigned long long* cycles,
+inline cudaError_t launch(bool pair, int n, int iters, int ctas, uint32_t seed, unsigned long long* cycles,
                           cudaStream_t stream) {
   auto k = pair ? mma_rate_kernel<true> : mma_rate_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -120,7 +148,7 @@ inline cudaError_t launch(bool pair, int n, int iters, int ctas, unsigned long l
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pair ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k, n, iters, cycles);
+  return cudaLaunchKernelEx(&cfg, k, n, iters, seed, cycles);
 }
 
 }  // namespace probe

@@ -691,7 +691,7 @@ qk_status qk_selftest_silu(uint32_t first, uint64_t count, unsigned long long* m
   return cuda_status(cudaGetLastError(), "silu selftest launch");
 }
 
-qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas,
+qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas, uint32_t operand_seed,
                                unsigned long long* cycles, qk_stream stream) {
   if ((cta_group != 1 && cta_group != 2) || n < 32 || n > 256 || (n % 16) != 0)
     return QK_ERR_INVALID_ARG;
@@ -701,7 +701,7 @@ qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas,
   const DeviceInfo* dev = nullptr;
   const qk_status st = check_device(&dev);
   if (st != QK_OK) return st;
-  return cuda_status(probe::launch(cta_group == 2, n, iters, ctas, cycles,
+  return cuda_status(probe::launch(cta_group == 2, n, iters, ctas, operand_seed, cycles,
                                    reinterpret_cast<cudaStream_t>(stream)),
                      "mma rate probe launch");
 }

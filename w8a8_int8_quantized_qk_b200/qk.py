@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 9
+ABI_VERSION = 10
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -78,7 +78,8 @@ _SIGNATURES = {
     "qk_device_status": (ctypes.c_int, [_P]),
     "qk_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_int, _P]),
     "qk_selftest_silu": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_uint64, _P, _P, _P]),
-    "qk_selftest_mma_rate": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P]),
+    "qk_selftest_mma_rate": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_uint32,
+                                            _P, _P]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -216,8 +217,8 @@ def qk_selftest_silu(first, count, mismatches, first_mismatch, stream) -> int:
     return lib().qk_selftest_silu(first, count, mismatches, first_mismatch, stream)
 
 
-def qk_selftest_mma_rate(cta_group, n, iters, ctas, cycles, stream) -> int:
-    return lib().qk_selftest_mma_rate(cta_group, n, iters, ctas, cycles, stream)
+def qk_selftest_mma_rate(cta_group, n, iters, ctas, operand_seed, cycles, stream) -> int:
+    return lib().qk_selftest_mma_rate(cta_group, n, iters, ctas, operand_seed, cycles, stream)
 
 
 # ---------------------------------------------------------------- torch helpers
@@ -516,23 +517,24 @@ def device_status(stream=None) -> int:
 
 
 def mma_rate(cta_group: int = 2, n: int = 256, iters: int = 16384, ctas: int | None = None,
-             launches: int = 5, stream=None) -> dict:
+             launches: int = 5, operand_seed: int = 0, stream=None) -> dict:
     """Time qk_selftest_mma_rate: `launches` back-to-back launches between
-    CUDA events on the current stream.  Returns the INT8 rate (TOPS, 2 ops
-    per multiply-add) and the issuing CTAs' median cycles per launch."""
+    CUDA events on the current stream, on zero operands (seed 0) or seeded
+    random bytes.  Returns the INT8 rate (TOPS, 2 ops per multiply-add) and
+    the issuing CTAs' median cycles per launch."""
     torch = _torch()
     if ctas is None:
         ctas = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
         ctas -= ctas % cta_group
     cyc = torch.zeros((ctas,), dtype=torch.int64, device="cuda")
     s = _stream(stream)
-    _check(qk_selftest_mma_rate(cta_group, n, iters, ctas, _ptr(cyc), s), "mma rate probe")  # warm-up
+    _check(qk_selftest_mma_rate(cta_group, n, iters, ctas, operand_seed, _ptr(cyc), s), "mma rate probe")  # warm-up
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     cur = torch.cuda.current_stream()
     e0.record(cur)
     for _ in range(launches):
-        _check(qk_selftest_mma_rate(cta_group, n, iters, ctas, _ptr(cyc), s), "mma rate probe")
+        _check(qk_selftest_mma_rate(cta_group, n, iters, ctas, operand_seed, _ptr(cyc), s), "mma rate probe")
     e1.record(cur)
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) * 1e-3 / launches
@@ -542,5 +544,5 @@ def mma_rate(cta_group: int = 2, n: int = 256, iters: int = 16384, ctas: int | N
     return {"tops": 2.0 * macs / sec / 1e12, "seconds_per_launch": sec, "cycles": cycles,
             "macs_per_clk_per_sm": macs / cta_group / (ctas // cta_group) / cycles if cycles > 0 else None,
             "clock_mhz_from_cycles": cycles / sec / 1e6, "cta_group": cta_group, "n": n, "iters": iters,
-            "ctas": ctas}
+            "ctas": ctas, "operands": "zero" if operand_seed == 0 else f"random (seed {operand_seed})"}
 
