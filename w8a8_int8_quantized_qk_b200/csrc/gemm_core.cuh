@@ -456,6 +456,10 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
 // at (col0, row0), which clips rows >= m and columns >= n.  Lane 0 issues
 // the copies; before rewriting the box it waits until the previous copy has
 // read it.  Every lane of the warp must call this.
+// The three multiplies run on binary32 pairs (mul.rn.f32x2: each lane an
+// IEEE round-to-nearest multiply, so the values are those of the scalar
+// form): half the FMA-pipe instructions, which compete with the tensor
+// core's MMAs on the same SM (0.6 us of a 52 us prefill GEMM).
 template <bool F8 = false>
 __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tmO, uint8_t* box,
                                             int row0, int col0, float sa, const float* sw,
@@ -463,14 +467,20 @@ __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tm
   if (col0 >= p.n || row0 >= p.m) return;  // the box lies wholly outside (warp-uniform)
   const int lane = threadIdx.x & 31;
   uint32_t w[16];
+  const uint64_t sa2 = pack2(__float_as_uint(sa), __float_as_uint(sa));
+  const uint64_t al2 = pack2(__float_as_uint(p.alpha), __float_as_uint(p.alpha));
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const float2 s2 = *reinterpret_cast<const float2*>(sw + 2 * j);
-    float t0 = acc_value<F8>(v[2 * j]);
-    float t1 = acc_value<F8>(v[2 * j + 1]);
-    t0 = __fmul_rn(__fmul_rn(__fmul_rn(t0, sa), s2.x), p.alpha);
-    t1 = __fmul_rn(__fmul_rn(__fmul_rn(t1, sa), s2.y), p.alpha);
-    w[j] = pack_bf16x2(t0, t1);
+    const uint64_t s2 = *reinterpret_cast<const unsigned long long*>(sw + 2 * j);
+    uint64_t t;
+    if constexpr (F8) {
+      t = pack2(v[2 * j], v[2 * j + 1]);
+    } else {
+      asm("{\n\t.reg .f32 x, y;\n\tcvt.rn.f32.s32 x, %1;\n\tcvt.rn.f32.s32 y, %2;\n\tmov.b64 %0, {x, y};\n\t}"
+          : "=l"(t) : "r"(v[2 * j]), "r"(v[2 * j + 1]));
+    }
+    t = f32x2_mul(f32x2_mul(f32x2_mul(t, sa2), s2), al2);
+    w[j] = pack_bf16x2(lo_of(t), hi_of(t));
   }
   if (lane == 0) bulk_wait_read_all();
   __syncwarp();

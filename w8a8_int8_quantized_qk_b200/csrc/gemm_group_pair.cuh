@@ -286,7 +286,7 @@ __device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, c
           f[2 * j + 1] = hi_of(w);
         }
       }
-      if (!mbar_wait(smem_addr(&s.acc_full[abuf]), aphase, &s.abort)) {
+      if (!mbar_wait_poll(smem_addr(&s.acc_full[abuf]), aphase, &s.abort, 20)) {
         ok = false;
         break;
       }

@@ -110,6 +110,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// mbar_wait for a waiter whose phases complete every few hundred cycles:
+// it polls with try_wait (no suspend-time hint) and sleeps `ns` between
+// polls.
+// Gives up like mbar_wait (`abort` must be non-null).  On the group-128
+// epilogue's per-group wait this measured 1.5 % faster than the suspending
+// form (177 against 180 us at 2048 x 8192 x 8192).
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               uint32_t ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = cycles_now();
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (cycles_now() - t0 > kWaitLimitNs * kCyclesPerNs) {
+      record_status(QK_ERR_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // Wait until the global counter `*flag` reaches `target` (other CTAs of the
 // same grid add to it after a __threadfence).  Gives up like mbar_wait: on
 // the shared `abort` flag, or after kWaitLimitNs (records QK_ERR_TIMEOUT and
