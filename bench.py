@@ -44,7 +44,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "prefill INT8 TOPS and decode weight-stream GB/s, % of B200 roofline"
 # ncu counters of the current kernels (see the --gemm-traffic help)
-GEMM_TRAFFIC_BYTES = 34.281216e6 + 14.385152e6
+GEMM_TRAFFIC_BYTES = 34.401792e6 + 15.697920e6
 GEMV_TRAFFIC_BYTES = 58.801920e6 + 0.029952e6
 L2_BYTES = 126 * 1024 * 1024
 
