@@ -98,9 +98,12 @@ def probe_int8_peak(torch, qk, local: int, sustained_s: float = 3.0) -> dict:
         burst_random = qk.mma_rate(2, 256, iters, launches=5, operand_seed=12345)
     burst_random["clocks"] = cl.summary()
     one_sm = qk.mma_rate(1, 256, iters, launches=5)
+    # the same pair MMA loop while the SM's other warps run arithmetic
+    # loops: cycles per group of four 256x256x32 MMAs (512 alone)
+    interference = qk.mma_interference(groups=4096)
     res = {"kernel": "qk_selftest_mma_rate: tcgen05.mma.cta_group::2.kind::i8 256x256x32, shared-memory operands",
            "burst": burst, "burst_random_operands": burst_random, "one_sm_128x256": one_sm,
-           "sustained": None, "sustained_random_operands": None}
+           "interference": interference, "sustained": None, "sustained_random_operands": None}
     if sustained_s > 0:
         n = max(5, int(sustained_s / burst["seconds_per_launch"]))
         with ClockSampler(local) as cl:

@@ -65,7 +65,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 10
+#define QK_ABI_VERSION 11
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -531,6 +531,35 @@ QK_API qk_status qk_selftest_silu(uint32_t first, uint64_t count, unsigned long 
 QK_API qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas,
                                       uint32_t operand_seed, unsigned long long* cycles,
                                       qk_stream stream);
+
+/*
+ * qk_selftest_mma_interference -- diagnostic: how much arithmetic on the
+ * CUDA cores slows the tensor core of the same SM.  Launches `ctas` CTAs of
+ * 384 threads in clusters of two (one pair per SM pair).  In each pair the
+ * leader issues `groups` groups of four tcgen05.mma.cta_group::2.kind::i8
+ * 256 x 256 x 32 (the group-128 GEMM's unit of work, 512 SM cycles at the
+ * full rate) on fixed pseudo-random shared-memory operands into alternating
+ * TMEM buffers.  Meanwhile warps 4..11 of both CTAs run a companion loop
+ * until the MMAs are done:
+ *   0 none; 1 fp32 fused multiply-add; 2 fp32 multiply; 3 int32 -> fp32
+ *   conversion and a logic op; 4 int32 multiply-add; 5 conversion and fused
+ *   multiply-add (the group-128 epilogue's arithmetic).
+ * Defined, like qk_selftest_mma_rate, by the roofline reading of
+ * "KV-cache kernels" (day 26) section 01: it tells whether an epilogue that
+ * overlaps the MMAs can be hidden under them.
+ *
+ * groups      1 .. 262144 groups of four MMAs per pair
+ * ctas        2 .. 65535, even; at most what the device holds at once
+ * cycles      optional device array [ctas] of uint64, 8-byte aligned: the
+ *             leader's SM clock cycles from its first MMA to the completion
+ *             of its last (0 on the second CTA of a pair); cycles / groups is
+ *             the time of one group
+ * The companion loops and the completion wait are bounded.
+ * Errors: QK_ERR_INVALID_ARG, QK_ERR_MISALIGNED, QK_ERR_UNSUPPORTED,
+ *         QK_ERR_CUDA.
+ */
+QK_API qk_status qk_selftest_mma_interference(int companion, int groups, int ctas,
+                                              unsigned long long* cycles, qk_stream stream);
 
 #ifdef __cplusplus
 }

@@ -126,3 +126,36 @@ def test_graph_capture_of_the_layer():
         assert qk.device_status() == qk.QK_OK
         assert np.array_equal(host(out), ref)
         assert np.array_equal(host(q), q_ref) and np.array_equal(host(s), s_ref)
+
+
+def test_mma_rate_probe_runs():
+    # the INT8 peak probe on zero and on random operands: every pair MMA loop
+    # completes, and the rate per clock is the same for both
+    need_gpu()
+    zero = qk.mma_rate(2, 256, 2048, launches=1)
+    rnd = qk.mma_rate(2, 256, 2048, launches=1, operand_seed=7)
+    assert qk.device_status() == qk.QK_OK
+    for r in (zero, rnd):
+        assert r["tops"] > 0 and r["cycles"] > 0
+    # 8192 multiply-adds per clock per SM at the full rate; allow slack
+    assert abs(zero["macs_per_clk_per_sm"] - rnd["macs_per_clk_per_sm"]) < 0.05 * zero["macs_per_clk_per_sm"]
+
+
+def test_mma_interference_probe_runs():
+    # every companion loop stops when the MMAs are done, and the MMA-only
+    # form reports about 512 cycles per group of four MMAs
+    need_gpu()
+    res = qk.mma_interference(groups=512)
+    assert qk.device_status() == qk.QK_OK
+    assert set(res) == set(qk.MMA_COMPANIONS.values())
+    for name, r in res.items():
+        assert r["cycles_per_group"] >= 500, (name, r)
+    assert res["none"]["cycles_per_group"] < 600
+
+
+def test_mma_interference_rejects_bad_arguments():
+    need_gpu()
+    s = qk._stream(torch.cuda.current_stream())
+    assert qk.qk_selftest_mma_interference(6, 16, 2, None, s) == qk.QK_ERR_INVALID_ARG
+    assert qk.qk_selftest_mma_interference(0, 16, 3, None, s) == qk.QK_ERR_INVALID_ARG
+    assert qk.qk_selftest_mma_interference(0, 0, 2, None, s) == qk.QK_ERR_INVALID_ARG

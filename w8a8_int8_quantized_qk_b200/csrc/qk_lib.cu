@@ -556,8 +556,8 @@ qk_status qk_w8a8_linear(int m, int n, int k, const void* x, qk_dtype x_dtype, c
   const size_t need = qk_w8a8_linear_workspace_size(m, n, k, group_k);
   if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
     return QK_ERR_WORKSPACE;
+  // workspace: [GEMM workspace | flag words of qk_w8a8_linear_fused | q | scales]
   const size_t g_bytes = round256(qk_w8a8_gemm_workspace_size(m, n, k, group_k));
-  int* flags = reinterpret_cast<int*>(static_cast<char*>(workspace) + g_bytes);
   int8_t* q = reinterpret_cast<int8_t*>(static_cast<char*>(workspace) + g_bytes + kLinearFlagBytes);
   float* sa = reinterpret_cast<float*>(static_cast<char*>(workspace) + g_bytes + kLinearFlagBytes +
                                        round256(static_cast<size_t>(m) * static_cast<size_t>(k)));
@@ -704,6 +704,19 @@ qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas, uint32
   return cuda_status(probe::launch(cta_group == 2, n, iters, ctas, operand_seed, cycles,
                                    reinterpret_cast<cudaStream_t>(stream)),
                      "mma rate probe launch");
+}
+
+qk_status qk_selftest_mma_interference(int companion, int groups, int ctas, unsigned long long* cycles,
+                                       qk_stream stream) {
+  if (companion < 0 || companion > 5 || groups < 1 || groups > (1 << 18) || ctas < 2 || ctas > 65535 ||
+      (ctas % 2) != 0)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned(cycles, 8)) return QK_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  const qk_status st = check_device(&dev);
+  if (st != QK_OK) return st;
+  return cuda_status(probe::launch_mix(companion, groups, ctas, cycles, reinterpret_cast<cudaStream_t>(stream)),
+                     "mma interference probe launch");
 }
 
 }  // extern "C"

@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 10
+ABI_VERSION = 11
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -80,6 +80,7 @@ _SIGNATURES = {
     "qk_selftest_silu": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_uint64, _P, _P, _P]),
     "qk_selftest_mma_rate": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_uint32,
                                             _P, _P]),
+    "qk_selftest_mma_interference": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P]),
 }
 
 _lib: ctypes.CDLL | None = None
@@ -219,6 +220,10 @@ def qk_selftest_silu(first, count, mismatches, first_mismatch, stream) -> int:
 
 def qk_selftest_mma_rate(cta_group, n, iters, ctas, operand_seed, cycles, stream) -> int:
     return lib().qk_selftest_mma_rate(cta_group, n, iters, ctas, operand_seed, cycles, stream)
+
+
+def qk_selftest_mma_interference(companion, groups, ctas, cycles, stream) -> int:
+    return lib().qk_selftest_mma_interference(companion, groups, ctas, cycles, stream)
 
 
 # ---------------------------------------------------------------- torch helpers
@@ -514,6 +519,36 @@ def mlp_down(gate, up, w_q, sw, output_scale: float = 1.0, out_dtype=None, strea
 
 def device_status(stream=None) -> int:
     return qk_device_status(_stream(stream))
+
+
+MMA_COMPANIONS = {0: "none", 1: "fp32 fma", 2: "fp32 mul", 3: "int32->fp32 cvt + logic", 4: "int32 mad",
+                  5: "cvt + fp32 fma (group-128 epilogue mix)"}
+
+
+def mma_interference(groups: int = 4096, ctas: int | None = None, stream=None) -> dict:
+    """qk_selftest_mma_interference for every companion loop: SM cycles per
+    group of four 256x256x32 pair MMAs (512 at the full rate) while the other
+    warps of the SM run that loop, and the clock the cycles imply."""
+    torch = _torch()
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        ctas -= ctas % 2
+    cyc = torch.zeros((ctas,), dtype=torch.int64, device="cuda")
+    s = _stream(stream)
+    out = {}
+    for c, name in MMA_COMPANIONS.items():
+        _check(qk_selftest_mma_interference(c, groups, ctas, _ptr(cyc), s), "mma interference probe")
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        cur = torch.cuda.current_stream()
+        e0.record(cur)
+        _check(qk_selftest_mma_interference(c, groups, ctas, _ptr(cyc), s), "mma interference probe")
+        e1.record(cur)
+        torch.cuda.synchronize()
+        cycles = float(cyc[::2].double().median().item())
+        sec = e0.elapsed_time(e1) * 1e-3
+        out[name] = {"cycles_per_group": cycles / groups, "clock_mhz_from_cycles": cycles / sec / 1e6}
+    return out
 
 
 def mma_rate(cta_group: int = 2, n: int = 256, iters: int = 16384, ctas: int | None = None,
