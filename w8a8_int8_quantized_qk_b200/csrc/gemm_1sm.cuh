@@ -67,7 +67,7 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
   const int ew = (threadIdx.x >> 5) - 2;
   const int quad = (threadIdx.x >> 5) & 3;
   const int j = static_cast<int>(cluster_rank());
-  const int tile = static_cast<int>(blockIdx.x) / p.splits;
+  const int tile = static_cast<int>(blockIdx.x) / p.sk.splits;
   const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
   const float* sws = s.sw_tile[ew];
   uint8_t* box = s.out_stage[ew];
@@ -75,7 +75,7 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
   const bool rv = row < p.m;
   const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
   const uint32_t slot = smem_addr(&s.a[0][0]) + static_cast<uint32_t>(quad * (32 * BN * 4));
-  for (int c = j; c < BN / 32; c += p.splits) {
+  for (int c = j; c < BN / 32; c += p.sk.splits) {
     const int col0 = tn * BN + c * 32;
     uint32_t va[32];
     // every source's part of the chunk requested at once (32 loads in
@@ -85,7 +85,7 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
     for (int o = 0; o < 4; ++o)
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4)
-        t4[o][q4] = o < p.splits
+        t4[o][q4] = o < p.sk.splits
                         ? ld_dsmem_v4(map_to_rank(
                               slot + static_cast<uint32_t>(((c * 8 + q4) * 32 + lane) * 16),
                               static_cast<uint32_t>(o)))
@@ -105,7 +105,7 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
       }
 #pragma unroll
       for (int o = 1; o < 4; ++o)
-        if (o < p.splits) {
+        if (o < p.sk.splits) {
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) acc_add4<true>(va + q4 * 4, t4[o][q4]);
         }
@@ -118,7 +118,7 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) acc_add4<false>(va + q4 * 4, t4[o][q4]);
     }
-    if (!F8 && p.zp) apply_zp(p, row, col0, va);
+    if (!F8 && p.asym.zp) apply_zp(p, row, col0, va);
     if (p.tma_out)
       store32_tma<F8>(p, tmO, box, row0, col0, sa, sws + c * 32, va);
     else if (rv && col0 < p.n)
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kChannelThreads, 1)
   } else {
     epilogue_channel<kChannelBN, 2, F8, MOE>(s, tmem, p, &tmO);
   }
-  if (p.csplit) {
+  if (p.sk.csplit) {
     cluster_sync_all();  // every CTA of the cluster has staged its partial
     if (warp >= 2) channel_cluster_reduce<kChannelBN, F8>(s, p, &tmO);
     cluster_sync_all();  // the peers are done reading this CTA's slots
@@ -262,7 +262,7 @@ using GroupWideStorage =
 // the part's first scale slice, and leaves the counter zero for the next
 // call; the epilogue warps read the sums after that slice's barrier.
 __device__ __forceinline__ float* group_state(const Args& p, int tt, int region) {
-  return p.gstate + (static_cast<int64_t>(tt) * 16 + region) * (kGroupWideCols * 32);
+  return p.gcut.gstate + (static_cast<int64_t>(tt) * 16 + region) * (kGroupWideCols * 32);
 }
 
 template <class S>
@@ -292,7 +292,7 @@ __device__ void epilogue_group_wide(S& s, uint32_t tmem, const Args& p) {
       if (u.part == 2 && g == u.g0) {
         // continue from the first part's sums (another CTA's; the stager
         // saw them complete before publishing this slice)
-        const float* st = group_state(p, u.tile - (ntiles - p.gsplit), region) + lane;
+        const float* st = group_state(p, u.tile - (ntiles - p.gcut.gsplit), region) + lane;
 #pragma unroll
         for (int j = 0; j < COLS; ++j) fs[j] = __ldcg(st + j * 32);
       }
@@ -335,13 +335,13 @@ __device__ void epilogue_group_wide(S& s, uint32_t tmem, const Args& p) {
     if (!ok) break;
     if (u.part == 1) {
       // hand the running sums to the CTA that finishes the tile
-      const int tt = u.tile - (ntiles - p.gsplit);
+      const int tt = u.tile - (ntiles - p.gcut.gsplit);
       float* st = group_state(p, tt, region) + lane;
 #pragma unroll
       for (int j = 0; j < COLS; ++j) __stcg(st + j * 32, fs[j]);
       __threadfence();
       __syncwarp();
-      if (lane == 0) atomicAdd(p.gflag + tt, 1);
+      if (lane == 0) atomicAdd(p.gcut.gflag + tt, 1);
       continue;
     }
     const int row = tm * BM + quad * 32 + lane;

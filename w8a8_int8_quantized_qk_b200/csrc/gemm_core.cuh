@@ -20,6 +20,64 @@ constexpr int BK = 128;     // K bytes per stage: one 128-byte swizzle row
 constexpr int UMMA_K = 32;  // K of one kind::i8 MMA instruction
 constexpr int kTmemCols = 512;
 
+// Args: the problem and its output form, which every GEMM kernel reads,
+// then one group of fields per mode.  A mode's group is all zero when the
+// mode is off; each kernel reads only the groups of the modes it has.
+//
+// split-K of a tile's K range (pair and 1-SM per-channel kernels): each
+// tile's K blocks are cut into `splits` slices of `kb_per_split`.  The
+// partial sums meet in the workspace `ws`, with per-region arrival counters
+// in the header (`cnt`: zero before the call, zero again after it), or,
+// when `csplit` is 1, in distributed shared memory: the slices are the CTAs
+// (pairs) of one cluster, and no workspace is needed.
+struct SplitK {
+  int splits, kb_per_split;
+  int32_t* ws;
+  int csplit;
+};
+
+// Tail split of a partial last wave (pair kernel; tail_splits > 1 and
+// splits == 1).  Tiles [0, dp_tiles) are computed whole.  Each remaining
+// tile is cut into `tail_splits` K slices of `tail_kbps` K blocks, and those
+// slices are the first unit of pairs 0 .. (tiles - dp_tiles) * tail_splits -
+// 1.  Every slice stores its partial in `tail_ws` and counts itself in
+// `cnt`.  The slice that arrives last adds the others' partials to its own,
+// runs the epilogue and leaves the counter zero (the partials are scratch).
+struct TailSplit {
+  int dp_tiles, tail_splits, tail_kbps;
+  int32_t* tail_ws;
+};
+
+// Asymmetric activations (per channel only): zp [m] zero-points and wsum [n]
+// = sum_k b[n][k]; the epilogues use acc - zp[m] * wsum[n].
+struct ZeroPoints {
+  const int32_t* zp;
+  const int32_t* wsum;
+};
+
+// MoE grouped GEMM (1-SM kernel).  Tokens are grouped by expert: expert e's
+// rows are [moe_off[e], moe_off[e + 1]) of a (m rows in all).  b is
+// [experts * n, k] and sw [experts, n].  tiles_m = experts * mt_max M tiles,
+// and those past an expert's tokens are skipped.
+struct MoeTiles {
+  int mt_max;
+  const int32_t* moe_off;
+};
+
+// The group-128 kernels' last wave, cut along K (gsplit > 0).  Tiles
+// [0, tiles - gsplit) run whole.  Tail tile (tiles - gsplit + j) is cut at
+// group gmid:
+// - its first part is worker j's first unit, which leaves its fp32 running
+//   sums in gstate and counts itself in gflag;
+// - its second part is worker (gsplit + j)'s last unit, which waits for the
+//   count, continues the sums in the same group order and leaves the count
+//   zero.
+struct GroupCut {
+  int gsplit, gmid;
+  float* gstate;
+  int* gflag;
+};
+
 struct Args {
   int m, n, k;
   const float* sa;  // [m]
@@ -29,59 +87,26 @@ struct Args {
   void* out;        // [m, n] or null
   int out_bf16;
   int tiles_m, tiles_n, num_kb, groups;
-  // split-K (pair kernel): each tile's K range is cut into `splits` pieces of
-  // `kb_per_split` K blocks; partial sums meet in `ws` with per-region
-  // arrival counters `cnt` (zero before the call, zero again after it).
-  int splits, kb_per_split;
-  int32_t* ws;
-  int* cnt;
-  // pair kernel: 1 when the `splits` K slices of a tile are the CTA pairs of
-  // one cluster and are summed through distributed shared memory (no
-  // workspace); 0 for the workspace form above
-  int csplit;
-  // pair kernel, tail split (tail_splits > 1, splits == 1): tiles
-  // [0, dp_tiles) are computed whole; each remaining tile is cut into
-  // `tail_splits` K slices of `tail_kbps` K blocks, and those slices are the
-  // first unit of pairs 0 .. (tiles - dp_tiles) * tail_splits - 1.  Every
-  // slice stores its partial in `tail_ws` and then counts itself in `cnt`;
-  // the slice that arrives last adds the others' partials to its own, runs
-  // the epilogue and leaves the counter zero (the partials are scratch).
-  int dp_tiles, tail_splits, tail_kbps;
-  int32_t* tail_ws;
-  // pair kernel: 1 when bf16 `out` (and no `c`) is written by TMA bulk
-  // tensor stores from shared memory (tensor map tmO) on the whole-tile and
-  // tail paths
+  // 1 when bf16 `out` (and no `c`) is written by TMA bulk tensor stores
+  // from shared memory (tensor map tmO)
   int tma_out;
   // 1: a and b are float8 e4m3 codes, the MMA is kind::f8f6f4 and the
   // accumulator fp32 (channel and pair kernels, whole tiles or the cluster
   // split-K, no c)
   int f8;
-  // asymmetric activations (per channel only): zp [m] zero-points and wsum
-  // [n] = sum_k b[n][k]; the epilogues use acc - zp[m] * wsum[n]
-  const int32_t* zp;
-  const int32_t* wsum;
-  // MoE grouped GEMM (1-SM kernel): tokens grouped by expert, expert e's rows
-  // [moe_off[e], moe_off[e + 1]) of a (m rows in all); b is [experts * n, k]
-  // and sw [experts, n]; tiles_m = experts * mt_max M tiles, those past an
-  // expert's tokens are skipped
-  int mt_max;
-  const int32_t* moe_off;
-  // wide group kernel, the last wave split along K (gsplit > 0): tiles
-  // [0, tiles - gsplit) run whole; tail tile (tiles - gsplit + j) is cut at
-  // group gmid.  Its first part is CTA j's first unit: it leaves its fp32
-  // running sums in gstate and sets the tile's 16 region flags in gflag.
-  // Its second part is CTA (gsplit + j)'s last unit: it waits for the flags,
-  // continues the sums in the same group order and leaves the flags zero.
-  int gsplit, gmid;
-  float* gstate;
-  int* gflag;
+  int* cnt;  // the workspace's arrival counters (split-K and tail split)
+  SplitK sk;
+  TailSplit tail;
+  ZeroPoints asym;
+  MoeTiles moe;
+  GroupCut gcut;
 };
 
 // The i-th unit of this CTA in the wide group kernel's schedule (false past
 // its last); every role walks the same list (group_plan.h).
 __device__ __forceinline__ bool group_unit(const Args& p, int i, GroupUnit& u) {
   return group_unit_at(static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x),
-                       p.tiles_m * p.tiles_n, p.gsplit, p.groups, p.gmid, i, u);
+                       p.tiles_m * p.tiles_n, p.gcut.gsplit, p.groups, p.gcut.gmid, i, u);
 }
 
 // One output tile of the 1-SM kernels: A rows from a_row0 (rows from row_end
@@ -98,12 +123,12 @@ __device__ __forceinline__ bool chan_tile(const Args& p, int tile, ChanTile& t) 
   if constexpr (MOE) {
     // compact numbering of the non-empty tiles: expert by expert, M tiles
     // fastest; tile numbers past the last one are empty
-    const int experts = p.tiles_m / p.mt_max;
+    const int experts = p.tiles_m / p.moe.mt_max;
     int u = tile;
     for (int e = 0; e < experts; ++e) {
-      const int r0 = __ldg(p.moe_off + e), r1 = __ldg(p.moe_off + e + 1);
+      const int r0 = __ldg(p.moe.moe_off + e), r1 = __ldg(p.moe.moe_off + e + 1);
       int mt = r1 > r0 ? (r1 - r0 + BM - 1) / BM : 0;
-      mt = mt < p.mt_max ? mt : p.mt_max;
+      mt = mt < p.moe.mt_max ? mt : p.moe.mt_max;
       const int cnt = mt * p.tiles_n;
       if (u < cnt) {
         const int tm = u % mt, tn = u / mt;
@@ -174,7 +199,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // CTA-pair prefill and the decode GEMV), so the other kernels wait first.
 template <int BN, int STAGES, bool MOE = false, bool GUNITS = false, bool EARLY_B = false, class S>
 __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, const Args& p) {
-  const int nunits = p.tiles_m * p.tiles_n * p.splits;
+  const int nunits = p.tiles_m * p.tiles_n * p.sk.splits;
   const uint32_t bytes = static_cast<uint32_t>((BM + BN) * BK);
   uint32_t stage = 0, phase = 0, issued = 0;
   bool ok = true;
@@ -204,9 +229,9 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
     } else {
       const int unit = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
       if (unit >= nunits) break;
-      if (!chan_tile<BN, MOE>(p, unit / p.splits, t)) continue;
-      kb0 = (unit % p.splits) * p.kb_per_split;
-      kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      if (!chan_tile<BN, MOE>(p, unit / p.sk.splits, t)) continue;
+      kb0 = (unit % p.sk.splits) * p.sk.kb_per_split;
+      kb1 = min(p.num_kb, kb0 + p.sk.kb_per_split);
     }
     for (int kb = kb0; kb < kb1; ++kb) {
       if (!waited && (pre_n == STAGES || (pre_n > 0 && kb != pre_kb0 + pre_n))) release_deferred();
@@ -247,7 +272,7 @@ __device__ void produce(S& s, const CUtensorMap* tmA, const CUtensorMap* tmB, co
 template <int BN, int STAGES, int NACC, bool GROUP, bool F8 = false, bool MOE = false,
           bool GUNITS = false, class S>
 __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
-  const int nunits = p.tiles_m * p.tiles_n * p.splits;
+  const int nunits = p.tiles_m * p.tiles_n * p.sk.splits;
   constexpr uint32_t idesc = F8 ? idesc_e4m3(BM, BN) : idesc_i8(BM, BN);
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
@@ -265,8 +290,8 @@ __device__ void mma_issue(S& s, uint32_t tmem, const Args& p) {
         ChanTile t;
         if (!chan_tile<BN, true>(p, unit, t)) continue;
       }
-      kb0 = (unit % p.splits) * p.kb_per_split;
-      kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      kb0 = (unit % p.sk.splits) * p.sk.kb_per_split;
+      kb1 = min(p.num_kb, kb0 + p.sk.kb_per_split);
     }
     if (!GROUP) {
       if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) break;
@@ -393,11 +418,11 @@ __device__ __forceinline__ void acc_add4(uint32_t* v, const int4& t) {
 // (exact whenever the corrected sum fits in int32, which the host's bound
 // on k guarantees).  Rows >= m and columns >= n (n % 8 == 0) take 0.
 __device__ __forceinline__ void apply_zp(const Args& p, int row, int col0, uint32_t (&v)[32]) {
-  const uint32_t z = row < p.m ? static_cast<uint32_t>(__ldg(p.zp + row)) : 0u;
+  const uint32_t z = row < p.m ? static_cast<uint32_t>(__ldg(p.asym.zp + row)) : 0u;
 #pragma unroll
   for (int g = 0; g < 8; ++g) {
     const int col = col0 + g * 4;
-    const int4 w4 = col < p.n ? __ldg(reinterpret_cast<const int4*>(p.wsum + col))
+    const int4 w4 = col < p.n ? __ldg(reinterpret_cast<const int4*>(p.asym.wsum + col))
                               : make_int4(0, 0, 0, 0);
     v[g * 4 + 0] -= z * static_cast<uint32_t>(w4.x);
     v[g * 4 + 1] -= z * static_cast<uint32_t>(w4.y);
@@ -459,7 +484,8 @@ __device__ __forceinline__ void store32_channel(const Args& p, int row, int col0
 // The three multiplies run on binary32 pairs (mul.rn.f32x2: each lane an
 // IEEE round-to-nearest multiply, so the values are those of the scalar
 // form): half the FMA-pipe instructions, which compete with the tensor
-// core's MMAs on the same SM (0.6 us of a 52 us prefill GEMM).
+// core's MMAs on the same SM (0.6 us of a 52 us prefill GEMM).  (Leaving
+// out the exact multiply by an output_scale of 1 measured no faster.)
 template <bool F8 = false>
 __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tmO, uint8_t* box,
                                             int row0, int col0, float sa, const float* sw,
@@ -505,7 +531,7 @@ __device__ __forceinline__ void store32_tma(const Args& p, const CUtensorMap* tm
 // bf16 output without c leaves through TMA stores (store32_tma).
 template <int BN, int NACC, bool F8 = false, bool MOE = false, class S>
 __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUtensorMap* tmO) {
-  const int nunits = p.tiles_m * p.tiles_n * p.splits;
+  const int nunits = p.tiles_m * p.tiles_n * p.sk.splits;
   const int lane = threadIdx.x & 31;
   const int ew = (threadIdx.x >> 5) - 2;  // epilogue warp 0..3
   const int quad = (threadIdx.x >> 5) & 3;
@@ -514,7 +540,7 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
   uint32_t abuf = 0, aphase = 0;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
     ChanTile t;
-    if (!chan_tile<BN, MOE>(p, unit / p.splits, t)) continue;
+    if (!chan_tile<BN, MOE>(p, unit / p.sk.splits, t)) continue;
     const int row0 = t.a_row0 + quad * 32, row = row0 + lane;
     const bool rv = row >= 0 && row < t.row_end;
     const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
@@ -533,7 +559,7 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
     tc_fence_after();
     const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + abuf * BN;
     uint32_t va[32], vb[32];
-    if (p.csplit) {
+    if (p.sk.csplit) {
       // Split-K inside the cluster (one unit per CTA, so the operand ring is
       // idle once acc_full has fired): stage this warp's 32 x BN partial in
       // its 32 KB slot of the ring, laid out [chunk][column quad][lane][4];
@@ -561,7 +587,7 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
         else if (rv)
           store32_channel<true>(p, row, colbase + ch * 32, sa, sws + ch * 32, v);
       } else {
-        if (p.zp) apply_zp(p, row, colbase + ch * 32, v);
+        if (p.asym.zp) apply_zp(p, row, colbase + ch * 32, v);
         if (p.tma_out)
           store32_tma(p, tmO, box, row0, colbase + ch * 32, sa, sws + ch * 32, v);
         else if (rv)
@@ -643,7 +669,7 @@ __device__ void stage_group_scales(S& s, const Args& p) {
       // complete before this unit's first slice is published
       bool seen = true;
       if (lane == 0) {
-        int* cnt = p.gflag + (u.tile - (ntiles - p.gsplit));
+        int* cnt = p.gcut.gflag + (u.tile - (ntiles - p.gcut.gsplit));
         seen = flag_wait(cnt, 16, &s.abort);
         if (seen) {
           __threadfence();

@@ -68,7 +68,7 @@ struct alignas(1024) GroupPairStorage {
 
 // The i-th unit of pair `pi` of `np` (false past its last).
 __device__ __forceinline__ bool gp_unit(const Args& p, int pi, int np, int i, GroupUnit& u) {
-  return group_unit_at(pi, np, p.tiles_m * p.tiles_n, p.gsplit, p.groups, p.gmid, i, u);
+  return group_unit_at(pi, np, p.tiles_m * p.tiles_n, p.gcut.gsplit, p.groups, p.gcut.gmid, i, u);
 }
 
 // A cut tile's running sums in the workspace: [tail tile][CTA of the pair]
@@ -79,7 +79,7 @@ __device__ __forceinline__ bool gp_unit(const Args& p, int pi, int np, int i, Gr
 // before it publishes the part's first scale slice and leaves the counter
 // zero for the next call.
 __device__ __forceinline__ uint64_t* gp_state(const Args& p, int tt, int rank, int ew) {
-  return reinterpret_cast<uint64_t*>(p.gstate) +
+  return reinterpret_cast<uint64_t*>(p.gcut.gstate) +
          ((static_cast<int64_t>(tt) * 2 + rank) * kGpEpiWarps + ew) * (kGpCols / 2) * 32;
 }
 
@@ -179,7 +179,7 @@ __device__ void gp_stage_scales(GroupPairStorage& s, const Args& p, uint32_t pr)
       // before this unit's first slice is published
       bool seen = true;
       if (lane == 0) {
-        int* cnt = p.gflag + 2 * (u.tile - (ntiles - p.gsplit)) + static_cast<int>(pr);
+        int* cnt = p.gcut.gflag + 2 * (u.tile - (ntiles - p.gcut.gsplit)) + static_cast<int>(pr);
         seen = flag_wait(cnt, kGpEpiWarps, &s.abort);
         if (seen) {
           __threadfence();
@@ -278,7 +278,7 @@ __device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, c
       if (u.part == 2 && g == u.g0) {
         // continue from the first part's sums (another pair's; the stager saw
         // them complete before publishing this slice)
-        const uint64_t* st = gp_state(p, u.tile - (ntiles - p.gsplit), static_cast<int>(pr), ew) + lane;
+        const uint64_t* st = gp_state(p, u.tile - (ntiles - p.gcut.gsplit), static_cast<int>(pr), ew) + lane;
 #pragma unroll
         for (int j = 0; j < kGpCols / 2; ++j) {
           const unsigned long long w = __ldcg(reinterpret_cast<const unsigned long long*>(st + j * 32));
@@ -334,7 +334,7 @@ __device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, c
     if (!ok) break;
     if (u.part == 1) {
       // hand the running sums to the pair that finishes the tile
-      const int tt = u.tile - (ntiles - p.gsplit);
+      const int tt = u.tile - (ntiles - p.gcut.gsplit);
       uint64_t* st = gp_state(p, tt, static_cast<int>(pr), ew) + lane;
 #pragma unroll
       for (int j = 0; j < kGpCols / 2; ++j)
@@ -342,7 +342,7 @@ __device__ void gp_epilogue(GroupPairStorage& s, uint32_t tmem, const Args& p, c
                pack2(__float_as_uint(f[2 * j]), __float_as_uint(f[2 * j + 1])));
       __threadfence();
       __syncwarp();
-      if (lane == 0) atomicAdd(p.gflag + 2 * tt + static_cast<int>(pr), 1);
+      if (lane == 0) atomicAdd(p.gcut.gflag + 2 * tt + static_cast<int>(pr), 1);
       continue;
     }
     const int row0 = tm * 256 + static_cast<int>(pr) * 128 + quad * 32;

@@ -309,30 +309,30 @@ inline int launch_pair(Args a, const int8_t* A, const int8_t* B, int dev, int nu
     pl.dp_tiles = pl.tiles;
   }
   if (pl.splits == 1) pl.csplit = 0;
-  a.splits = pl.splits;
-  a.kb_per_split = pl.kb_per_split;
-  a.csplit = pl.csplit;
-  a.dp_tiles = pl.dp_tiles;
-  a.tail_splits = pl.tail_splits;
-  a.tail_kbps = pl.tail_kbps;
-  a.ws = nullptr;
+  a.sk.splits = pl.splits;
+  a.sk.kb_per_split = pl.kb_per_split;
+  a.sk.csplit = pl.csplit;
+  a.tail.dp_tiles = pl.dp_tiles;
+  a.tail.tail_splits = pl.tail_splits;
+  a.tail.tail_kbps = pl.tail_kbps;
+  a.sk.ws = nullptr;
   a.cnt = nullptr;
-  a.tail_ws = nullptr;
+  a.tail.tail_ws = nullptr;
   if ((pl.splits > 1 && !pl.csplit) || pl.tail_splits > 1) {
     a.cnt = static_cast<int*>(workspace);
-    a.ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kCounterHeaderBytes);
-    a.tail_ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kTailOffset);
+    a.sk.ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kCounterHeaderBytes);
+    a.tail.tail_ws = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kTailOffset);
   }
   CUtensorMap ta, tb, to;
   if (!cached_tmap(&ta, A, a.m, a.k, 128) || !cached_tmap(&tb, B, a.n, a.k, 128)) return 1;
   // bf16 out without c, outside split-K: TMA stores from shared memory
-  a.tma_out = (a.out != nullptr && a.out_bf16 && a.c == nullptr && a.splits == 1) ? 1 : 0;
+  a.tma_out = (a.out != nullptr && a.out_bf16 && a.c == nullptr && a.sk.splits == 1) ? 1 : 0;
   if (a.tma_out) {
     if (!cached_tmap(&to, a.out, a.m, a.n, 32, 1)) return 1;
   } else {
     to = ta;  // unused
   }
-  const int ntiles = a.tiles_m * a.tiles_n * a.splits;  // > pairs whenever the tail split is on
+  const int ntiles = a.tiles_m * a.tiles_n * a.sk.splits;  // > pairs whenever the tail split is on
   const int grid_pairs = ntiles < pairs ? ntiles : pairs;
   cudaError_t e = a.f8 ? set_smem_once(gemm_i8_pair_kernel<true>, dev, 4, pair_smem())
                        : set_smem_once(gemm_i8_pair_kernel<false>, dev, 0, pair_smem());
@@ -597,16 +597,16 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   a.tiles_n = (a.n + bn - 1) / bn;
   a.num_kb = (a.k + BK - 1) / BK;
   a.groups = group ? a.k / 128 : 0;
-  a.splits = 1;
-  a.kb_per_split = a.num_kb;
-  a.csplit = 0;
-  a.tail_splits = 1;
+  a.sk.splits = 1;
+  a.sk.kb_per_split = a.num_kb;
+  a.sk.csplit = 0;
+  a.tail.tail_splits = 1;
   if (!group) {
     const ChannelPlan pl = channel_plan(a.m, a.n, a.k, num_sms, dev);
     if (pl.splits > 1) {
-      a.splits = pl.splits;
-      a.kb_per_split = pl.kb_per_split;
-      a.csplit = 1;
+      a.sk.splits = pl.splits;
+      a.sk.kb_per_split = pl.kb_per_split;
+      a.sk.csplit = 1;
     }
   }
   CUtensorMap ta, tb, to;
@@ -620,7 +620,7 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   }
   const int ntiles = a.tiles_m * a.tiles_n;
   // split-K: exactly one CTA per (tile, K slice), in clusters of `splits`
-  const int grid = a.csplit ? ntiles * a.splits : (ntiles < num_sms ? ntiles : num_sms);
+  const int grid = a.sk.csplit ? ntiles * a.sk.splits : (ntiles < num_sms ? ntiles : num_sms);
   cudaError_t e;
   if (!group) {
     const size_t smem = channel_smem();
@@ -629,7 +629,7 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
     if (e == cudaSuccess) {
       e = launch_pdl(a.f8 ? gemm_i8_channel_kernel<true> : gemm_i8_channel_kernel<false>, dim3(grid),
                      dim3(kChannelThreads), smem, stream,
-                     a.csplit ? static_cast<unsigned>(a.splits) : 1u, ta, tb, to, a);
+                     a.sk.csplit ? static_cast<unsigned>(a.sk.splits) : 1u, ta, tb, to, a);
     }
   } else {
     if (wide) {
@@ -640,10 +640,10 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
         a.tiles_n = (a.n + kGpBN - 1) / kGpBN;
         CUtensorMap tpa, tpb;
         if (!cached_tmap(&tpa, A, a.m, a.k, 128) || !cached_tmap(&tpb, B, a.n, a.k, 128)) return 1;
-        a.gsplit = workspace ? gp.r : 0;
-        a.gmid = a.groups / 2;
-        a.gflag = static_cast<int*>(workspace);
-        a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)
+        a.gcut.gsplit = workspace ? gp.r : 0;
+        a.gcut.gmid = a.groups / 2;
+        a.gcut.gflag = static_cast<int*>(workspace);
+        a.gcut.gstate = a.gcut.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)
                             : nullptr;
         // bf16 out without c: TMA stores from shared memory
         a.tma_out = (a.out != nullptr && a.out_bf16 && a.c == nullptr) ? 1 : 0;
@@ -657,10 +657,10 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
         *err = e;
         return e == cudaSuccess ? 0 : 2;
       }
-      a.gsplit = workspace ? gp.r : 0;
-      a.gmid = a.groups / 2;
-      a.gflag = static_cast<int*>(workspace);
-      a.gstate = a.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)
+      a.gcut.gsplit = workspace ? gp.r : 0;
+      a.gcut.gmid = a.groups / 2;
+      a.gcut.gflag = static_cast<int*>(workspace);
+      a.gcut.gstate = a.gcut.gsplit ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kTailOffset)
                           : nullptr;
       const size_t smem = group_wide_smem();
       e = set_smem_once(gemm_i8_group_wide_kernel, dev, 7, smem);
@@ -698,16 +698,16 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
 inline int launch_moe(Args a, const int8_t* A, const int8_t* B, int experts, int mt_max,
                       const int32_t* off, int dev, int num_sms, cudaStream_t stream,
                       cudaError_t* err) {
-  a.mt_max = mt_max;
-  a.moe_off = off;
+  a.moe.mt_max = mt_max;
+  a.moe.moe_off = off;
   a.tiles_m = experts * mt_max;
   a.tiles_n = (a.n + kChannelBN - 1) / kChannelBN;
   a.num_kb = (a.k + BK - 1) / BK;
   a.groups = 0;
-  a.splits = 1;
-  a.kb_per_split = a.num_kb;
-  a.csplit = 0;
-  a.tail_splits = 1;
+  a.sk.splits = 1;
+  a.sk.kb_per_split = a.num_kb;
+  a.sk.csplit = 0;
+  a.tail.tail_splits = 1;
   a.tma_out = 0;
   a.c = nullptr;
   CUtensorMap ta, tb;

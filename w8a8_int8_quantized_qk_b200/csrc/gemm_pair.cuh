@@ -53,20 +53,20 @@ struct PairUnit {
 // tail slice first (if it has one), then data-parallel tiles pi,
 // pi + npairs, ... below dp_tiles.
 __device__ __forceinline__ bool pair_unit(const Args& p, int pi, int npairs, int i, PairUnit& u) {
-  if (p.tail_splits > 1) {
-    const int tail_units = (p.tiles_m * p.tiles_n - p.dp_tiles) * p.tail_splits;
+  if (p.tail.tail_splits > 1) {
+    const int tail_units = (p.tiles_m * p.tiles_n - p.tail.dp_tiles) * p.tail.tail_splits;
     if (pi < tail_units) {
       if (i == 0) {
-        u.tile = p.dp_tiles + pi / p.tail_splits;
-        u.slice = pi % p.tail_splits;
-        u.kb0 = u.slice * p.tail_kbps;
-        u.kb1 = min(p.num_kb, u.kb0 + p.tail_kbps);
+        u.tile = p.tail.dp_tiles + pi / p.tail.tail_splits;
+        u.slice = pi % p.tail.tail_splits;
+        u.kb0 = u.slice * p.tail.tail_kbps;
+        u.kb1 = min(p.num_kb, u.kb0 + p.tail.tail_kbps);
         return true;
       }
       --i;
     }
     const int t = pi + i * npairs;
-    if (t >= p.dp_tiles) return false;
+    if (t >= p.tail.dp_tiles) return false;
     u.tile = t;
     u.slice = 0;
     u.kb0 = 0;
@@ -74,11 +74,11 @@ __device__ __forceinline__ bool pair_unit(const Args& p, int pi, int npairs, int
     return true;
   }
   const int unit = pi + i * npairs;
-  if (unit >= p.tiles_m * p.tiles_n * p.splits) return false;
-  u.tile = unit / p.splits;
-  u.slice = unit % p.splits;
-  u.kb0 = u.slice * p.kb_per_split;
-  u.kb1 = min(p.num_kb, u.kb0 + p.kb_per_split);
+  if (unit >= p.tiles_m * p.tiles_n * p.sk.splits) return false;
+  u.tile = unit / p.sk.splits;
+  u.slice = unit % p.sk.splits;
+  u.kb0 = u.slice * p.sk.kb_per_split;
+  u.kb1 = min(p.num_kb, u.kb0 + p.sk.kb_per_split);
   return true;
 }
 
@@ -185,10 +185,10 @@ __device__ void tail_slice_epilogue(uint32_t acc_empty_lead, const Args& p,
                                     const CUtensorMap* tmO, uint8_t* box) {
   constexpr int kRegionInts = 32 * (kPairBN / 2);
   const int lane = threadIdx.x & 31;
-  const int S = p.tail_splits;
-  const int tt = u.tile - p.dp_tiles;
+  const int S = p.tail.tail_splits;
+  const int tt = u.tile - p.tail.dp_tiles;
   int* cnt = p.cnt + tt * 16 + region;
-  int32_t* slots = p.tail_ws + static_cast<int64_t>(tt) * S * 16 * kRegionInts;
+  int32_t* slots = p.tail.tail_ws + static_cast<int64_t>(tt) * S * 16 * kRegionInts;
   uint32_t va[32];
   {
     int4* dst = reinterpret_cast<int4*>(slots + (static_cast<int64_t>(u.slice) * 16 + region) * kRegionInts);
@@ -240,7 +240,7 @@ __device__ void tail_slice_epilogue(uint32_t acc_empty_lead, const Args& p,
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) acc_add4<F8>(va + q4 * 4, t4[o][q4]);
       }
-    if (!F8 && p.zp) apply_zp(p, row, colbase + ch * 32, va);
+    if (!F8 && p.asym.zp) apply_zp(p, row, colbase + ch * 32, va);
     if (p.tma_out)
       store32_tma<F8>(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
     else if (rv)
@@ -271,7 +271,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
   PairUnit u;
   for (int i = 0; pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
     const int tile = u.tile;
-    const bool tail = p.tail_splits > 1 && tile >= p.dp_tiles;
+    const bool tail = p.tail.tail_splits > 1 && tile >= p.tail.dp_tiles;
     const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
     const int row = tm * kPairBM + static_cast<int>(pr) * 128 + quad * 32 + lane;
     const bool rv = row < p.m;
@@ -293,7 +293,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
       // (releases the TMEM buffer itself, before its reduction)
       tail_slice_epilogue<F8>(map_to_rank(smem_addr(&s.acc_empty[abuf]), lead), p, u, region,
                               tb, row, rv, sa, colbase, sws, tmO, box);
-    } else if (F8 && !p.csplit) {
+    } else if (F8 && !p.sk.csplit) {
       // FP8 kind, whole tile (fp32 accumulator)
       auto emit = [&](int ch, const uint32_t(&v)[32]) {
         if (p.tma_out)
@@ -318,29 +318,29 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
 #pragma unroll
       for (int ch = 0; ch < 4; ch += 2) {
         tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
-        if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
+        if (p.asym.zp) apply_zp(p, row, colbase + ch * 32, va);
         store32_tma(p, tmO, box, row - lane, colbase + ch * 32, sa, sws + ch * 32, va);
         tmem_ld_wait();
         if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
-        if (p.zp) apply_zp(p, row, colbase + (ch + 1) * 32, vb);
+        if (p.asym.zp) apply_zp(p, row, colbase + (ch + 1) * 32, vb);
         store32_tma(p, tmO, box, row - lane, colbase + (ch + 1) * 32, sa, sws + (ch + 1) * 32, vb);
         tmem_ld_wait();
       }
-    } else if (p.splits == 1) {
+    } else if (p.sk.splits == 1) {
       tmem_ld_32x32b_x32(tb, va);
       tmem_ld_wait();
 #pragma unroll
       for (int ch = 0; ch < 4; ch += 2) {
         tmem_ld_32x32b_x32(tb + (ch + 1) * 32, vb);
-        if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
+        if (p.asym.zp) apply_zp(p, row, colbase + ch * 32, va);
         if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
         tmem_ld_wait();
         if (ch + 2 < 4) tmem_ld_32x32b_x32(tb + (ch + 2) * 32, va);
-        if (p.zp) apply_zp(p, row, colbase + (ch + 1) * 32, vb);
+        if (p.asym.zp) apply_zp(p, row, colbase + (ch + 1) * 32, vb);
         if (rv) store32_channel(p, row, colbase + (ch + 1) * 32, sa, sws + (ch + 1) * 32, vb);
         tmem_ld_wait();
       }
-    } else if (p.csplit) {
+    } else if (p.sk.csplit) {
       // Split-K inside the cluster: stage this warp's 32 x 128 partial in its
       // 16 KB slot of the (idle) operand ring, [column quad][lane][4]; the
       // sum over the cluster's pairs is taken after the cluster barrier
@@ -367,7 +367,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
       // its counter zero for the next call.
       constexpr int kRegionInts = 32 * (kPairBN / 2);
       constexpr uint32_t kRegionBytes = kRegionInts * 4;
-      int32_t* acc_region = p.ws + (static_cast<int64_t>(tile) * 16 + region) * kRegionInts;
+      int32_t* acc_region = p.sk.ws + (static_cast<int64_t>(tile) * 16 + region) * kRegionInts;
       uint8_t* stg = &s.a[0][0] + (warp - 2) * kRegionBytes;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
@@ -387,7 +387,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
         bulk_wait_all();
         fence_proxy_async_global();
         __threadfence();
-        last = atomicAdd(p.cnt + tile * 16 + region, 1) == p.splits - 1;
+        last = atomicAdd(p.cnt + tile * 16 + region, 1) == p.sk.splits - 1;
       }
       last = __shfl_sync(0xFFFFFFFFu, last, 0);
       if (last) {
@@ -407,7 +407,7 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
             va[q4 * 4 + 3] = t4[q4].w;
             __stcg(reinterpret_cast<int4*>(acc_region + ((ch * 8 + q4) * 32 + lane) * 4), zero);
           }
-          if (p.zp) apply_zp(p, row, colbase + ch * 32, va);
+          if (p.asym.zp) apply_zp(p, row, colbase + ch * 32, va);
           if (rv) store32_channel(p, row, colbase + ch * 32, sa, sws + ch * 32, va);
         }
         if (lane == 0) p.cnt[tile * 16 + region] = 0;  // ready for the next call
@@ -443,10 +443,10 @@ __device__ void cluster_reduce_scales(PairStorage& s, const Args& p, uint32_t cr
   const int warp = threadIdx.x >> 5;
   const int w2 = (warp - 2) >> 2;
   const int j = static_cast<int>(crank >> 1);
-  const int tn = ((blockIdx.x >> 1) / p.splits) / p.tiles_m;
+  const int tn = ((blockIdx.x >> 1) / p.sk.splits) / p.tiles_m;
   float* sws = s.sw_tile[warp - 2];
   int t = 0;
-  for (int c = j + p.splits * w2; c < kPairBN / 32 && t < 2; c += 2 * p.splits, ++t) {
+  for (int c = j + p.sk.splits * w2; c < kPairBN / 32 && t < 2; c += 2 * p.sk.splits, ++t) {
     const int col = tn * kPairBN + c * 32 + lane;
     sws[t * 32 + lane] = (p.out && col < p.n) ? __ldg(p.sw + col) : 0.0f;
   }
@@ -459,7 +459,7 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
   const int quad = warp & 3;
   const int w2 = (warp - 2) >> 2;
   const int j = static_cast<int>(crank >> 1), h = static_cast<int>(crank & 1u);
-  const int tile = (blockIdx.x >> 1) / p.splits;
+  const int tile = (blockIdx.x >> 1) / p.sk.splits;
   const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
   const float* sws = s.sw_tile[warp - 2];
   int t = 0;
@@ -468,7 +468,7 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
   const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
   const uint32_t base = smem_addr(&s.a[0][0]);
   constexpr uint32_t kSlotBytes = 32 * (kPairBN / 2) * 4;
-  for (int c = j + p.splits * w2; c < kPairBN / 32; c += 2 * p.splits, ++t) {
+  for (int c = j + p.sk.splits * w2; c < kPairBN / 32; c += 2 * p.sk.splits, ++t) {
     const int hh = c >> 2, ch = c & 3;
     const uint32_t slot = static_cast<uint32_t>(hh * 4 + ((quad + 2) & 3));  // staging warp of (quad, hh)
     const uint32_t off = base + slot * kSlotBytes + static_cast<uint32_t>((ch * 8 * 32 + lane) * 16);
@@ -481,7 +481,7 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
       const uint32_t peer = static_cast<uint32_t>(2 * o + h);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4)
-        t4[o][q4] = o < p.splits ? ld_dsmem_v4(map_to_rank(off + q4 * 32 * 16, peer))
+        t4[o][q4] = o < p.sk.splits ? ld_dsmem_v4(map_to_rank(off + q4 * 32 * 16, peer))
                                  : make_int4(0, 0, 0, 0);
     }
 #pragma unroll
@@ -499,7 +499,7 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
       }
 #pragma unroll
       for (int o = 1; o < 4; ++o)
-        if (o < p.splits) {
+        if (o < p.sk.splits) {
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) acc_add4<true>(va + q4 * 4, t4[o][q4]);
         }
@@ -513,7 +513,7 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
         for (int q4 = 0; q4 < 8; ++q4) acc_add4<false>(va + q4 * 4, t4[o][q4]);
     }
     const int col0 = tn * kPairBN + c * 32;
-    if (!F8 && p.zp) apply_zp(p, row, col0, va);
+    if (!F8 && p.asym.zp) apply_zp(p, row, col0, va);
     if (rv && col0 < p.n) store32_channel<F8>(p, row, col0, sa, sws + t * 32, va);
   }
 }
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   } else {
     epilogue_pair<F8>(s, tmem, p, pr, lead, &tmO);
   }
-  if (p.csplit) {
+  if (p.sk.csplit) {
     if (warp >= 2) cluster_reduce_scales(s, p, crank);
     cluster_sync_all();  // every CTA of the cluster has staged its partial
     if (warp >= 2) cluster_reduce_pair<F8>(s, p, crank);

@@ -456,13 +456,9 @@ qk_status gemm_common(int m, int n, int k, const int8_t* a, const int8_t* b,
   g.c = c;
   g.out = out;
   g.out_bf16 = out_dtype == QK_BF16;
-  g.splits = 1;
-  g.kb_per_split = 0;
-  g.ws = nullptr;
-  g.cnt = nullptr;
-  g.csplit = 0;
-  g.zp = zp;
-  g.wsum = wsum;
+  g.sk.splits = 1;  // the split-K plan is the launcher's
+  g.asym.zp = zp;
+  g.asym.wsum = wsum;
   cudaError_t e = cudaSuccess;
   int dev_id = 0;
   cudaGetDevice(&dev_id);
@@ -502,7 +498,7 @@ qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
   g.c = nullptr;
   g.out = out;
   g.out_bf16 = out_dtype == QK_BF16;
-  g.splits = 1;
+  g.sk.splits = 1;
   g.f8 = 1;
   cudaError_t e = cudaSuccess;
   int dev_id = 0;
