@@ -162,13 +162,17 @@ def test_gemm_group(O, m, n, k):
     assert_bits(out_nc, out, "group out without c")
 
 
-# group mode without the int32 sums runs the 128 x 256 kernel: more tiles
-# than SMs (several per CTA), group counts that are not a multiple of the
-# 16-group scale slice (3, 17), ragged M and N edges, bf16 and fp32 outputs.
-# With 148 SMs, 1100 x 4360 (162 tiles) and 1280 x 4096 (160 tiles) cut
-# their last wave's tiles at the middle group (17 groups: 8 + 9; 2 groups:
-# 1 + 1), one CTA continuing another's running sums.
-GROUP_WIDE_SHAPES = [(1100, 4360, 2176), (1280, 4096, 256), (300, 2056, 384), (129, 264, 128)]
+# group mode without the int32 sums runs the CTA-pair kernel for m > 128
+# (256 x 256 tiles): more tiles than pairs (several per pair), group counts
+# that are not a multiple of the 8-group scale slice (3, 17), ragged M and N
+# edges, bf16 (TMA-store) and fp32 outputs.  With 74 pairs, 1100 x 4360 (90
+# tiles) and 1280 x 4096 (80 tiles) cut their last wave's tiles at the
+# middle group (17 groups: 8 + 9; 2 groups: 1 + 1), one pair continuing
+# another's running sums.
+# (m <= 128 takes the 1-SM 128 x 256 kernel: 128 x 40448 is 158 tiles on
+# 148 SMs, so its last wave is cut too.)
+GROUP_WIDE_SHAPES = [(1100, 4360, 2176), (1280, 4096, 256), (300, 2056, 384), (129, 264, 128),
+                     (128, 40448, 384)]
 
 
 @pytest.mark.parametrize("m,n,k", GROUP_WIDE_SHAPES)
@@ -289,9 +293,10 @@ def test_epilogue_order_golden(O, m, n, k):
             assert_bits(out, want, f"per-channel order, case {case['out']}")
 
 
-# the group chain: the 128 x 128 kernel (with c), the 128 x 256 kernel, and
-# (1280 x 4096, 160 tiles on 148 SMs) the cut last wave, where one CTA
-# continues another's running sums between the two groups
+# the group chain: the 128 x 128 kernel (with c), the 128 x 256 kernel (m =
+# 1), the CTA-pair kernel, and (1280 x 4096, 80 pair tiles on 74 pairs) the
+# cut last wave, where one pair continues another's running sums between
+# the two groups
 @pytest.mark.parametrize("m,n", [(1, 128), (300, 2056), (1280, 4096)])
 def test_group_order_golden(O, m, n):
     for case in _golden("epilogue_order.json")["group"]:
