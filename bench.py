@@ -7,19 +7,28 @@ One STEP is one pass of the whole hot path over one batch: per-token INT8
 quantisation of the activation, then the INT8 GEMM with its fused dequant
 epilogue.  The headline workload is the prefill linear layer (X bf16
 [4096, 4096], W int8 [4096, 4096], per-channel scales, bf16 out); ``value``
-is INT8 TOPS of the whole step (2*M*N*K per step / step time).  The same JSON
-line carries:
+is INT8 TOPS of the whole step (2*M*N*K per step / step time).  The run
+prints two JSON lines.  The last is the headline; besides ``value`` it
+carries:
 
+* ``roofline`` -- the dominant kernel (the GEMM) against the INT8 peak that
+  qk_selftest_mma_rate measures at the start of the run (zero operands;
+  ``frac_random_operands`` against the same probe on random bytes;
+  ``frac_nominal`` against the 4.5 POPS datasheet figure);
 * ``decode``   -- the decode linear layer's weight-stream GB/s (X bf16
-  [4, 4096], W int8 [14336, 4096]) with its HBM roofline;
-* ``stages``   -- per-stage device time and roofline fraction of all five
-  workloads (quantiser, fused SiLU quantiser, GEMV, tcgen05 GEMM per channel
-  and per 128-group);
-* ``roofline`` -- the dominant kernel (the GEMM) against the tensor peak;
+  [4, 4096], W int8 [14336, 4096]) with its HBM fraction and step times;
 * ``e2e``      -- the same metric through the public API with host buffers
   (pinned host -> device copy of X and device -> host copy of the output
   inside the timed region);
-* ``cpu_baseline`` -- the CPU oracle on a bounded sample of rows.
+* ``cpu_baseline`` -- the CPU oracle on a bounded sample of rows;
+* ``clocks``   -- SM clocks and clock-event reasons sampled in the timed
+  region.
+
+The line before it, ``{"bench_details": ...}``, holds the per-stage device
+times and roofline fractions of all workloads (quantiser, fused SiLU
+quantiser, GEMV, tcgen05 GEMM per channel and per 128-group, FP8, MoE), the
+decode roofline, and every run of the INT8 peak probe (burst, sustained,
+random operands, and the tensor-core rate with arithmetic on the same SM).
 
 L2 (126 MB) is defeated by rotating several copies of every input and output
 (working set >= 3x L2), so steps run back to back.  Times are CUDA events on

@@ -14,6 +14,13 @@
 // and a quarter of a broadcast shared load for the scales; the running sums
 // live in registers (128 per thread), and per-group overhead is amortised
 // over 128 columns per warp.
+// What bounds the kernel: fp32 arithmetic on the CUDA cores slows the tensor
+// core of the same SM (qk_selftest_mma_interference: a group of four pair
+// MMAs takes 512 cycles alone, 512 beside conversion or integer loops, and
+// 1201-3948 beside fp32 FFMA or FMUL loops).  One FFMA per element per group
+// is the minimum this definition allows, so the MMAs run at about a third of
+// their rate while the epilogue folds (176 us at 2048 x 8192 x 8192).  Half
+// the FFMA instructions as packed fma.rn.f32x2 measured slower (198 us).
 // The CTA pair keeps the MMA at N = 256 per SM while each SM loads only its
 // own halves of A and B (the streaming rate of this tile is 0.93 of the
 // tensor peak, against 0.81 for a 1-SM 128 x 256 tile).
