@@ -543,7 +543,8 @@ QK_API qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas,
  * until the MMAs are done:
  *   0 none; 1 fp32 fused multiply-add; 2 fp32 multiply; 3 int32 -> fp32
  *   conversion and a logic op; 4 int32 multiply-add; 5 conversion and fused
- *   multiply-add (the group-128 epilogue's arithmetic).
+ *   multiply-add (the group-128 epilogue's arithmetic); 6 fp32 pair ->
+ *   bf16x2 conversion (the epilogues' output packing).
  * Defined, like qk_selftest_mma_rate, by the roofline reading of
  * "KV-cache kernels" (day 26) section 01: it tells whether an epilogue that
  * overlaps the MMAs can be hidden under them.

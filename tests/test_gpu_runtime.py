@@ -156,6 +156,6 @@ def test_mma_interference_probe_runs():
 def test_mma_interference_rejects_bad_arguments():
     need_gpu()
     s = qk._stream(torch.cuda.current_stream())
-    assert qk.qk_selftest_mma_interference(6, 16, 2, None, s) == qk.QK_ERR_INVALID_ARG
+    assert qk.qk_selftest_mma_interference(7, 16, 2, None, s) == qk.QK_ERR_INVALID_ARG
     assert qk.qk_selftest_mma_interference(0, 16, 3, None, s) == qk.QK_ERR_INVALID_ARG
     assert qk.qk_selftest_mma_interference(0, 0, 2, None, s) == qk.QK_ERR_INVALID_ARG

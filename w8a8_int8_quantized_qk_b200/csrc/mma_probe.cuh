@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // done (a flag in each CTA's shared memory, bounded by an iteration count):
 //   0 none, 1 fp32 fused multiply-add, 2 fp32 multiply, 3 int32 -> fp32
 //   conversion and a logic op (the ALU pipe), 4 int32 multiply-add,
-//   5 conversion + fused multiply-add (the group-128 epilogue's mix).
+//   5 conversion + fused multiply-add (the group-128 epilogue's mix),
+//   6 fp32 pair -> bf16x2 conversion (the epilogues' output packing).
 // cycles[cta]: the leader's clock64 cycles from the first MMA issue to the
 // completion of the last (0 on the second CTA of a pair).
 constexpr int kMixThreads = 384;
@@ -172,6 +173,12 @@ __device__ __forceinline__ void companion_loop(volatile int* stop) {
         if constexpr (MODE == 5) {
           f[j] = __fmaf_rn(__int2float_rn(v[j]), sc, f[j]);
           v[j] ^= 0x1357;
+        }
+        if constexpr (MODE == 6) {
+          // the packed pair feeds the next one's operands, so the loop
+          // cannot be folded away
+          const uint32_t b2 = pack_bf16x2(__int_as_float(v[j]), __int_as_float(v[j] ^ 0x40000000));
+          v[j] = static_cast<int>(b2 ^ 0x3F803F80u);
         }
       }
     }
@@ -284,7 +291,8 @@ inline cudaError_t launch_mix(int companion, int groups, int ctas, unsigned long
     case 2: k = mma_mix_kernel<2>; break;
     case 3: k = mma_mix_kernel<3>; break;
     case 4: k = mma_mix_kernel<4>; break;
-    default: k = mma_mix_kernel<5>; break;
+    case 5: k = mma_mix_kernel<5>; break;
+    default: k = mma_mix_kernel<6>; break;
   }
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(mix_smem_bytes()));

@@ -704,7 +704,7 @@ qk_status qk_selftest_mma_rate(int cta_group, int n, int iters, int ctas, uint32
 
 qk_status qk_selftest_mma_interference(int companion, int groups, int ctas, unsigned long long* cycles,
                                        qk_stream stream) {
-  if (companion < 0 || companion > 5 || groups < 1 || groups > (1 << 18) || ctas < 2 || ctas > 65535 ||
+  if (companion < 0 || companion > 6 || groups < 1 || groups > (1 << 18) || ctas < 2 || ctas > 65535 ||
       (ctas % 2) != 0)
     return QK_ERR_INVALID_ARG;
   if (!aligned(cycles, 8)) return QK_ERR_MISALIGNED;

@@ -522,7 +522,7 @@ def device_status(stream=None) -> int:
 
 
 MMA_COMPANIONS = {0: "none", 1: "fp32 fma", 2: "fp32 mul", 3: "int32->fp32 cvt + logic", 4: "int32 mad",
-                  5: "cvt + fp32 fma (group-128 epilogue mix)"}
+                  5: "cvt + fp32 fma (group-128 epilogue mix)", 6: "fp32 -> bf16x2 pack"}
 
 
 def mma_interference(groups: int = 4096, ctas: int | None = None, stream=None) -> dict:
