@@ -474,9 +474,10 @@ QK_API qk_status qk_selftest_bounded_wait(int timeout_us, qk_stream stream);
  * qk_selftest_silu -- diagnostic: checks the fused SiLU arithmetic of the
  * silu quantisers.  For every binary32 bit pattern g in [first, first +
  * count) that is finite, it computes silu(g) * 1 the way the quantisers do
- * (two values at a time, the exp's reduction, polynomial and the final
- * multiply on packed binary32 pairs) and the way the definition reads (one
- * value at a time, every step a scalar IEEE round-to-nearest operation), and
+ * (two values at a time: the exp's reduction, polynomial, the divide -- by
+ * Markstein's method -- and the final multiply on packed binary32 pairs) and
+ * the way the definition reads (one value at a time, every step a scalar
+ * IEEE round-to-nearest operation, the divide IEEE's), and
  * counts the g whose two results differ in any bit.  g is the only input of that
  * arithmetic, so first = 0, count = 2^32 covers every value it can see.
  * Defined by the fused silu_and_mul quantisation of the vLLM PR "fused

