@@ -127,7 +127,10 @@ __device__ __forceinline__ uint64_t div2_rn(uint64_t g, uint64_t d) {
 // packed multiply feeds a packed add (the pair could be fused), so the clamp,
 // the 2^n scaling and the 1 + e stay scalar.  The two divides are one packed
 // Markstein division (div2_rn), checked against the IEEE divide for every
-// binary32 gate value: 8.36 -> 7.78 us for the mlp_down activations.
+// binary32 gate value: 8.36 -> 7.78 us for the mlp_down activations.  1 + e
+// is one packed fused multiply-add: p * 2^n is exact (a normal number for
+// every clamped argument), so the fused form rounds as the separate
+// multiply and add do.
 __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1, float& h0,
                                           float& h1) {
   constexpr float kLog2e = static_cast<float>(1.4426950408889634074);
@@ -154,10 +157,8 @@ __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1
   p = f32x2_fma(p, r, splat2(1.0f));
   const float two0 = __uint_as_float((__float_as_uint(nb0) - kRoundMagicBits + 127u) << 23);
   const float two1 = __uint_as_float((__float_as_uint(nb1) - kRoundMagicBits + 127u) << 23);
-  const float d0 = __fadd_rn(1.0f, __fmul_rn(lo_of(p), two0));
-  const float d1 = __fadd_rn(1.0f, __fmul_rn(hi_of(p), two1));
-  const uint64_t sq = div2_rn(pack2(__float_as_uint(g0), __float_as_uint(g1)),
-                              pack2(__float_as_uint(d0), __float_as_uint(d1)));
+  const uint64_t dd = f32x2_fma(p, pack2(__float_as_uint(two0), __float_as_uint(two1)), splat2(1.0f));
+  const uint64_t sq = div2_rn(pack2(__float_as_uint(g0), __float_as_uint(g1)), dd);
   const uint64_t h = f32x2_mul(sq, pack2(__float_as_uint(u0), __float_as_uint(u1)));
   h0 = lo_of(h);
   h1 = hi_of(h);
@@ -201,6 +202,27 @@ __device__ __forceinline__ void widen(const uint4& v, float (&f)[BF16 ? 8 : 4]) 
   }
 }
 
+
+// Two binary32 values -> round_half_even(x * inv) as int32 each (x * inv
+// rounded to binary32 first, on a packed pair; cvt.rni rounds half to even,
+// as the 1.5 * 2^23 trick of quant_bits does, and |x * inv| <= 127 (1 +
+// 2^-23) keeps both in range).  With the bytes packed by cvt.pack.sat this is
+// 16 instructions per 8 values against 22 (7.67 -> 7.49 us for the SiLU
+// quantiser of the mlp_down activations).
+__device__ __forceinline__ void quant2(float a, float b, uint64_t inv2, int& qa, int& qb) {
+  const uint64_t y = f32x2_mul(pack2(__float_as_uint(a), __float_as_uint(b)), inv2);
+  asm("cvt.rni.s32.f32 %0, %1;" : "=r"(qa) : "f"(lo_of(y)));
+  asm("cvt.rni.s32.f32 %0, %1;" : "=r"(qb) : "f"(hi_of(y)));
+}
+
+// Four int32 values in [-127, 127] -> int8x4 (a in the low byte).
+__device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
+  uint32_t t, r;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(d), "r"(c), "r"(0));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(b), "r"(a), "r"(t));
+  return r;
+}
+
 // Quantise E values and store E int8 at dst.
 template <int E>
 __device__ __forceinline__ void store_q(const Args& p, int8_t* dst, const float (&f)[E], float inv) {
@@ -221,16 +243,17 @@ __device__ __forceinline__ void store_q(const Args& p, int8_t* dst, const float 
     }
     return;
   }
+  const uint64_t inv2 = pack2(__float_as_uint(inv), __float_as_uint(inv));
+  int q[E];
+#pragma unroll
+  for (int i = 0; i < E; i += 2) quant2(f[i], f[i + 1], inv2, q[i], q[i + 1]);
   if constexpr (E == 8) {
     uint2 o;
-    o.x = pack_q4(quant_bits(f[0], inv), quant_bits(f[1], inv), quant_bits(f[2], inv),
-                  quant_bits(f[3], inv));
-    o.y = pack_q4(quant_bits(f[4], inv), quant_bits(f[5], inv), quant_bits(f[6], inv),
-                  quant_bits(f[7], inv));
+    o.x = pack_s8x4(q[0], q[1], q[2], q[3]);
+    o.y = pack_s8x4(q[4], q[5], q[6], q[7]);
     *reinterpret_cast<uint2*>(dst) = o;
   } else {
-    *reinterpret_cast<uint32_t*>(dst) = pack_q4(quant_bits(f[0], inv), quant_bits(f[1], inv),
-                                                quant_bits(f[2], inv), quant_bits(f[3], inv));
+    *reinterpret_cast<uint32_t*>(dst) = pack_s8x4(q[0], q[1], q[2], q[3]);
   }
 }
 
