@@ -101,8 +101,12 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // Newton step, the quotient, its exact remainder by a fused multiply-add, and
 // one fused correction.  A divisor at or above 2^126 (whose reciprocal would
 // be subnormal) is scaled by 2^-32 first; its quotient is normal (|g| >= 87
-// when d >= 2^126), so scaling back is exact.  A zero remainder keeps the
-// first quotient (it is exact, and keeps the sign of a zero g).
+// when d >= 2^126), so scaling back is exact.  The remainder is formed with
+// the opposite sign (d q0 - g) and the correction negated, so that a zero g
+// keeps its sign (-0 + -0) without a select.  (A packed multiply feeding a
+// packed add may be fused by the assembler: packing the reduction's
+// t * log2e + 1.5 * 2^23 that way gave 7 wrong results in 2^32, so that step
+// stays scalar.)
 __device__ __forceinline__ uint64_t div2_rn(uint64_t g, uint64_t d) {
   const float s0 = lo_of(d) >= 0x1p126f ? 0x1p-32f : 1.0f;
   const float s1 = hi_of(d) >= 0x1p126f ? 0x1p-32f : 1.0f;
@@ -113,12 +117,9 @@ __device__ __forceinline__ uint64_t div2_rn(uint64_t g, uint64_t d) {
   const uint64_t e = f32x2_fma(nds, y, splat2(1.0f));
   y = f32x2_fma(y, e, y);
   const uint64_t q0 = f32x2_mul(g, y);
-  const uint64_t r = f32x2_fma(nds, q0, g);
-  const uint64_t q1 = f32x2_fma(r, y, q0);
-  const uint32_t a = static_cast<uint32_t>(r) << 1 == 0 ? static_cast<uint32_t>(q0) : static_cast<uint32_t>(q1);
-  const uint32_t b = static_cast<uint32_t>(r >> 32) << 1 == 0 ? static_cast<uint32_t>(q0 >> 32)
-                                                              : static_cast<uint32_t>(q1 >> 32);
-  return f32x2_mul(pack2(a, b), s);
+  const uint64_t rn = f32x2_fma(ds, q0, g ^ 0x8000000080000000ull);  // d q0 - g, exact
+  const uint64_t q1 = f32x2_fma(rn ^ 0x8000000080000000ull, y, q0);
+  return f32x2_mul(q1, s);
 }
 
 // Two silu_mul at once: the same operations in the same order, with the
