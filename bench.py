@@ -389,9 +389,7 @@ def measure_workload(torch, qk, name: str, iters: int, pk: dict) -> dict:
             linear_us[name] = _graph_us(torch, L, linear_call, iters)
     by = _bytes(w)
     ops = 2.0 * w.m * w.n * w.k
-    gemm_kernel = "gemv (CUDA cores)" if (w.m <= 8 and not w.group_k) else (
-        "tcgen05 group-128" if w.group_k else
-        ("tcgen05 per-channel, 1 SM" if w.m <= 128 else "tcgen05 per-channel, CTA pair"))
+    gemm_kernel = qk.qk_w8a8_gemm_kernel(w.m, w.n, w.k, w.group_k, False)
     res = {"m": w.m, "n": w.n, "k": w.k, "copies": L.R, "timing": f"CUDA graph of {iters} iterations",
            "quant_kernel": "silu_mul_quant" if w.gate is not None else "quantize_per_token",
            "quant_us": quant_us, "quant_GBs": by["quant"] / (quant_us * 1e-6) / 1e9,

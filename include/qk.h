@@ -65,7 +65,7 @@ extern "C" {
  * built with; a binding must refuse to use a library whose number differs
  * (an idea taken from the dynquant-kernels package page, "Variants": an ABI
  * number baked into the binary and checked at import). */
-#define QK_ABI_VERSION 11
+#define QK_ABI_VERSION 12
 
 typedef enum qk_status {
   QK_OK = 0,
@@ -349,6 +349,16 @@ QK_API qk_status qk_w8a8_gemm_asym(int m, int n, int k, const int8_t* a,
  * device (0 when none; the split depends on the device's SM count).
  * Returns 0 for arguments qk_w8a8_gemm would reject. */
 QK_API size_t qk_w8a8_gemm_workspace_size(int m, int n, int k, int group_k);
+
+/* qk_w8a8_gemm_kernel -- diagnostic: which kernel, tile shape and split form
+ * qk_w8a8_gemm launches for this problem on the current device (the choice
+ * depends on m, n, k, group_k, whether the int32 sums c are requested
+ * (with_c != 0), and the device's SM count).  Returns a NUL-terminated
+ * string, never null: "unsupported" for shapes qk_w8a8_gemm rejects, "no
+ * device" without a usable sm_100 device.  The string is owned by the
+ * library and stays valid until the next call of this function on the same
+ * host thread. */
+QK_API const char* qk_w8a8_gemm_kernel(int m, int n, int k, int group_k, int with_c);
 
 /*
  * qk_w8a8_linear -- the whole W8A8 linear layer in one call: dynamic

@@ -135,6 +135,16 @@ def test_workspace_query(L):
     assert qk.qk_w8a8_gemm_workspace_size(4096, 4096, 4096, 0) >= 0
 
 
+def test_kernel_query_host_answers(L):
+    # shape checks come before any device query
+    assert qk.qk_w8a8_gemm_kernel(16, 64, 20, 0, False) == "unsupported"  # k % 16 != 0
+    assert qk.qk_w8a8_gemm_kernel(16, 60, 32, 0, False) == "unsupported"  # n % 8 != 0
+    assert qk.qk_w8a8_gemm_kernel(16, 64, 256, 64, False) == "unsupported"  # group_k not 0 / 128
+    assert qk.qk_w8a8_gemm_kernel(0, 64, 32, 0, False) == "none (empty output)"
+    name = qk.qk_w8a8_gemm_kernel(4096, 4096, 4096, 0, False)
+    assert name == "no device" or name.startswith("gemm_i8_pair_kernel")
+
+
 def test_selftest_arg_check(L):
     assert qk.qk_selftest_bounded_wait(0, NULL) == qk.QK_ERR_INVALID_ARG
     assert qk.qk_selftest_bounded_wait(3000000, NULL) == qk.QK_ERR_INVALID_ARG

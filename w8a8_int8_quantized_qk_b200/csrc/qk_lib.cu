@@ -474,6 +474,59 @@ qk_status gemm_common(int m, int n, int k, const int8_t* a, const int8_t* b,
 }
 }  // namespace
 
+const char* qk_w8a8_gemm_kernel(int m, int n, int k, int group_k, int with_c) {
+  thread_local char text[160];
+  if (gemm_check(m, n, k, group_k) != QK_OK) return "unsupported";
+  if (m == 0 || n == 0) return "none (empty output)";
+  const DeviceInfo* dev = nullptr;
+  if (check_device(&dev) != QK_OK) return "no device";
+  int dev_id = 0;
+  if (cudaGetDevice(&dev_id) != cudaSuccess) return "no device";
+  switch (gemm_path(m, n, k, group_k)) {
+    case GemmPath::kGemv:
+      return gemv::pref_supported(m, k) ? "gemv_i8_prefetch_kernel (CUDA cores, dp4a)"
+                                        : "gemv_i8_kernel (CUDA cores, dp4a)";
+    case GemmPath::kTensorChannel: {
+      const gemm::ChannelPlan pl = gemm::channel_plan(m, n, k, dev->sms, dev_id);
+      if (pl.splits > 1)
+        snprintf(text, sizeof text,
+                 "gemm_i8_channel_kernel (1 SM, 128x256 tiles, cluster split-K in %d slices)",
+                 pl.splits);
+      else
+        snprintf(text, sizeof text, "gemm_i8_channel_kernel (1 SM, 128x256 tiles)");
+      return text;
+    }
+    case GemmPath::kTensorPair: {
+      const int pairs = gemm::max_pairs(dev_id, dev->sms);
+      const gemm::PairPlan pl = gemm::pair_plan(m, n, k, pairs, dev_id);
+      const bool split = pl.splits > 1 && static_cast<int64_t>(pl.tiles) * pl.splits <= pairs;
+      if (pl.tail_splits > 1)
+        snprintf(text, sizeof text,
+                 "gemm_i8_pair_kernel (CTA pair, 256x256 tiles, last wave cut into %d K slices)",
+                 pl.tail_splits);
+      else if (split && pl.csplit)
+        snprintf(text, sizeof text,
+                 "gemm_i8_pair_kernel (CTA pair, 256x256 tiles, cluster split-K in %d slices)",
+                 pl.splits);
+      else if (split)
+        snprintf(text, sizeof text,
+                 "gemm_i8_pair_kernel (CTA pair, 256x256 tiles, split-K in %d slices through the "
+                 "workspace)",
+                 pl.splits);
+      else
+        snprintf(text, sizeof text, "gemm_i8_pair_kernel (CTA pair, 256x256 tiles)");
+      return text;
+    }
+    case GemmPath::kTensorGroup:
+      break;
+  }
+  if (with_c || !gemm::group_wide_ok(dev_id))
+    return "gemm_i8_group_kernel (1 SM, 128x128 tiles)";
+  return gemm::group_plan(m, n, k, dev_id, dev->sms).pair
+             ? "gemm_i8_group_pair_kernel (CTA pair, 256x256 tiles)"
+             : "gemm_i8_group_wide_kernel (1 SM, 128x256 tiles)";
+}
+
 qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_t* b,
                       const float* scale_a, const float* scale_b, float output_scale, void* out,
                       qk_dtype out_dtype, qk_stream stream) {

@@ -23,7 +23,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libqk.so")
 
-ABI_VERSION = 11
+ABI_VERSION = 12
 
 QK_OK = 0
 QK_ERR_INVALID_ARG = 1
@@ -67,6 +67,8 @@ _SIGNATURES = {
     "qk_w8a8_gemm_asym": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P, _P,
                                          ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "qk_w8a8_gemm_workspace_size": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "qk_w8a8_gemm_kernel": (ctypes.c_char_p, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int]),
     "qk_w8a8_linear": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P,
                                       ctypes.c_int, ctypes.c_float, _P, _P, ctypes.c_int, _P, ctypes.c_size_t,
                                       _P]),
@@ -178,6 +180,12 @@ def qk_w8a8_gemm_asym(m, n, k, a, zero_point_a, b, wsum_b, scale_a, scale_b, out
 
 def qk_w8a8_gemm_workspace_size(m, n, k, group_k) -> int:
     return lib().qk_w8a8_gemm_workspace_size(m, n, k, group_k)
+
+
+def qk_w8a8_gemm_kernel(m, n, k, group_k, with_c) -> str:
+    """The kernel, tile shape and split form qk_w8a8_gemm launches for this
+    problem on the current device."""
+    return lib().qk_w8a8_gemm_kernel(m, n, k, group_k, 1 if with_c else 0).decode()
 
 
 def qk_w8a8_linear(m, n, k, x, x_dtype, b, scale_b, group_k, output_scale, scale_a_out, out, out_dtype,
