@@ -94,44 +94,41 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-// q = RN(g / d) in both lanes, for finite g and d in [1, 2^128) (d = 1 + e,
+// q = RN(g / d) in both lanes, for finite g and d in [1, 2^127] (d = 1 + e,
 // e >= 0, as silu forms it), by Markstein's method (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990): an approximate reciprocal, one
-// Newton step, the quotient, its exact remainder by a fused multiply-add, and
-// one fused correction.  A divisor at or above 2^126 (whose reciprocal would
-// be subnormal) is scaled by 2^-32 first; its quotient is normal (|g| >= 87
-// when d >= 2^126), so scaling back is exact.  The remainder is formed with
-// the opposite sign (d q0 - g) and the correction negated, so that a zero g
-// keeps its sign (-0 + -0) without a select.  (A packed multiply feeding a
-// packed add may be fused by the assembler: packing the reduction's
-// t * log2e + 1.5 * 2^23 that way gave 7 wrong results in 2^32, so that step
-// stays scalar.)
-__device__ __forceinline__ uint64_t div2_rn(uint64_t g, uint64_t d) {
-  const float s0 = lo_of(d) >= 0x1p126f ? 0x1p-32f : 1.0f;
-  const float s1 = hi_of(d) >= 0x1p126f ? 0x1p-32f : 1.0f;
-  const uint64_t s = pack2(__float_as_uint(s0), __float_as_uint(s1));
-  const uint64_t ds = f32x2_mul(d, s);
-  uint64_t y = pack2(__float_as_uint(rcp_approx(lo_of(ds))), __float_as_uint(rcp_approx(hi_of(ds))));
-  const uint64_t nds = ds ^ 0x8000000080000000ull;
-  const uint64_t e = f32x2_fma(nds, y, splat2(1.0f));
-  y = f32x2_fma(y, e, y);
-  const uint64_t q0 = f32x2_mul(g, y);
-  const uint64_t rn = f32x2_fma(ds, q0, g ^ 0x8000000080000000ull);  // d q0 - g, exact
-  const uint64_t q1 = f32x2_fma(rn ^ 0x8000000080000000ull, y, q0);
-  return f32x2_mul(q1, s);
+// processor", IBM J. Res. Dev. 34(1), 1990), applied to (g/2) / (d/2).  The
+// caller passes dh = d/2, whose reciprocal is normal for every d the clamp
+// allows (d/2 < 2^126).  g/2 is exact except for |g| < 2^-125, where d = 2
+// exactly and the rounded g/2 is itself the answer.  The steps: an
+// approximate reciprocal of -dh, one Newton step, the quotient, its exact
+// remainder by a fused multiply-add, and one fused correction.  Starting
+// from the negative reciprocal gives every step the sign it needs, so no
+// lane is negated or selected, and a zero g keeps its sign (+0 -> +0,
+// -0 -> -0).
+__device__ __forceinline__ uint64_t div2_rn(uint64_t g, uint64_t dh) {
+  const uint64_t ngh = f32x2_mul(g, splat2(-0.5f));  // -g/2
+  uint64_t y = pack2(__float_as_uint(rcp_approx(-lo_of(dh))), __float_as_uint(rcp_approx(-hi_of(dh))));
+  const uint64_t e = f32x2_fma(dh, y, splat2(1.0f));  // 1 - dh/dh~
+  y = f32x2_fma(y, e, y);                              // ~ -1/dh
+  const uint64_t q0 = f32x2_mul(ngh, y);               // ~ (g/2) / dh
+  const uint64_t rn = f32x2_fma(dh, q0, ngh);          // dh q0 - g/2, exact
+  return f32x2_fma(rn, y, q0);                         // q0 - rn / dh
 }
 
 // Two silu_mul at once: the same operations in the same order, with the
 // reduction, polynomial and final multiply as packed pairs (per-lane IEEE
 // round-to-nearest), so each result is bit-identical to silu_mul's.  No
-// packed multiply feeds a packed add (the pair could be fused), so the clamp,
-// the 2^n scaling and the 1 + e stay scalar.  The two divides are one packed
-// Markstein division (div2_rn), checked against the IEEE divide for every
-// binary32 gate value: 8.36 -> 7.78 us for the mlp_down activations.  1 + e
-// is one packed fused multiply-add: p * 2^n is exact (a normal number for
-// every clamped argument), so the fused form rounds as the separate
-// multiply and add do.
+// packed multiply feeds a packed add (the assembler may fuse such a pair:
+// packing the reduction's t * log2e + 1.5 * 2^23 that way gave 7 wrong
+// results in 2^32), so the clamp and that step stay scalar; -n * ln2 is
+// n * (-ln2).  The two divides are one packed Markstein division (div2_rn),
+// checked against the IEEE divide for every binary32 gate value.  Its
+// divisor d/2 = 0.5 + p 2^(n-1) is one packed fused multiply-add: p 2^(n-1)
+// is exact, so it rounds as 1 + p 2^n does, halved.  (At n = -126 the
+// exponent field of 2^(n-1) is zero and the term drops out; there 1 + e
+// rounds to 1 anyway.)  mlp_down activations: 8.36 us with the IEEE
+// divide, 7.5 us with a scaled division, 6.5 us in this form.
 __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1, float& h0,
                                           float& h1) {
   constexpr float kLog2e = static_cast<float>(1.4426950408889634074);
@@ -145,9 +142,8 @@ __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1
   const uint64_t t = pack2(__float_as_uint(t0), __float_as_uint(t1));
   const uint64_t n =
       f32x2_add(pack2(__float_as_uint(nb0), __float_as_uint(nb1)), splat2(-kRoundMagic));
-  const uint64_t mn = n ^ 0x8000000080000000ull;  // -n in both lanes
-  uint64_t r = f32x2_fma(mn, splat2(kLn2Hi), t);
-  r = f32x2_fma(mn, splat2(kLn2Lo), r);
+  uint64_t r = f32x2_fma(n, splat2(-kLn2Hi), t);
+  r = f32x2_fma(n, splat2(-kLn2Lo), r);
   uint64_t p = f32x2_fma(splat2(static_cast<float>(1.0 / 5040.0)), r,
                          splat2(static_cast<float>(1.0 / 720.0)));
   p = f32x2_fma(p, r, splat2(static_cast<float>(1.0 / 120.0)));
@@ -156,10 +152,11 @@ __device__ __forceinline__ void silu_mul2(float g0, float g1, float u0, float u1
   p = f32x2_fma(p, r, splat2(0.5f));
   p = f32x2_fma(p, r, splat2(1.0f));
   p = f32x2_fma(p, r, splat2(1.0f));
-  const float two0 = __uint_as_float((__float_as_uint(nb0) - kRoundMagicBits + 127u) << 23);
-  const float two1 = __uint_as_float((__float_as_uint(nb1) - kRoundMagicBits + 127u) << 23);
-  const uint64_t dd = f32x2_fma(p, pack2(__float_as_uint(two0), __float_as_uint(two1)), splat2(1.0f));
-  const uint64_t sq = div2_rn(pack2(__float_as_uint(g0), __float_as_uint(g1)), dd);
+  // 2^(n-1): exponent field n + 126
+  const float two0 = __uint_as_float((__float_as_uint(nb0) - kRoundMagicBits + 126u) << 23);
+  const float two1 = __uint_as_float((__float_as_uint(nb1) - kRoundMagicBits + 126u) << 23);
+  const uint64_t dh = f32x2_fma(p, pack2(__float_as_uint(two0), __float_as_uint(two1)), splat2(0.5f));
+  const uint64_t sq = div2_rn(pack2(__float_as_uint(g0), __float_as_uint(g1)), dh);
   const uint64_t h = f32x2_mul(sq, pack2(__float_as_uint(u0), __float_as_uint(u1)));
   h0 = lo_of(h);
   h1 = hi_of(h);
