@@ -96,10 +96,12 @@ def test_gemm_split_k(O, m, n, k):
         assert_bits(out, ref["out_bf16"], "bf16 out")
 
 
-# few 128 x 256 tiles on the 1-SM kernel (m <= 128, or m <= 256 when that
-# gives each CTA fewer K blocks than the CTA-pair plan): K is split across
-# the CTAs of a cluster and the partials meet in distributed shared memory
-CHANNEL_SPLIT_SHAPES = [(64, 4096, 4096), (100, 1032, 3008), (17, 520, 2048), (256, 4096, 14336)]
+# few 128 x 128 or 128 x 256 tiles on the 1-SM kernel (m <= 128, or m <= 256
+# when that gives each CTA fewer K blocks than the CTA-pair plan): K is split
+# across the CTAs of a cluster and the partials meet in distributed shared
+# memory
+CHANNEL_SPLIT_SHAPES = [(64, 4096, 4096), (100, 1032, 3008), (17, 520, 2048), (256, 4096, 14336),
+                        (100, 10240, 3072)]
 
 
 @pytest.mark.parametrize("m,n,k", CHANNEL_SPLIT_SHAPES)
@@ -115,6 +117,31 @@ def test_gemm_channel_cluster_split(O, m, n, k):
     assert_bits(out32, ref["out_f32"], "fp32 out")
     out16, _ = _run(a, w, sa, sw, 0, 0.75, want_c=False)  # bf16 through TMA stores
     assert_bits(out16, ref["out_bf16"], "bf16 out, no c")
+
+
+# the two tile widths of the 1-SM kernel: 128 x 128 where it puts more CTAs
+# to work (with 4 or 2 cluster K slices, or none), 128 x 256 otherwise
+WIDTH_SHAPES = [((128, 4096, 14336), "128x128 tiles, cluster split-K in 4 slices"),
+                ((96, 8192, 4096), "128x128 tiles, cluster split-K in 2 slices"),
+                ((120, 4104, 2064), "128x128 tiles, cluster split-K in 2 slices"),
+                ((100, 1000, 1024), "128x128 tiles)"),
+                ((100, 10240, 3072), "128x256 tiles, cluster split-K in "),
+                ((256, 4096, 14336), "128x256 tiles, cluster split-K in 4 slices")]
+
+
+@pytest.mark.parametrize("shape,form", WIDTH_SHAPES)
+def test_gemm_channel_tile_widths(O, shape, form):
+    m, n, k = shape
+    assert qk.qk_w8a8_gemm_kernel(m, n, k, 0, True).startswith("gemm_i8_channel_kernel (1 SM, " + form)
+    a, w, sa, sw = _problem(m, n, k, 0, seed=m + 3 * n + k)
+    ref = O.linear_from_q(a, sa, w, sw, 0, 1.25)
+    out, c = _run(a, w, sa, sw, 0, 1.25)
+    assert_bits(c, ref["acc"], "acc")
+    assert_bits(out, ref["out_bf16"], "bf16 out")
+    out16, _ = _run(a, w, sa, sw, 0, 1.25, want_c=False)  # bf16 through TMA stores
+    assert_bits(out16, ref["out_bf16"], "bf16 out, no c")
+    out32, _ = _run(a, w, sa, sw, 0, 1.25, out_dtype=torch.float32, want_c=False)
+    assert_bits(out32, ref["out_f32"], "fp32 out")
 
 
 # more output tiles than CTA pairs, not a whole number of waves: the tiles of

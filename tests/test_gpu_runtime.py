@@ -132,7 +132,8 @@ def test_kernel_query_names_the_planned_kernel():
     need_gpu()
     q = qk.qk_w8a8_gemm_kernel
     assert q(4, 14336, 4096, 0, False).startswith("gemv_i8_prefetch_kernel")
-    assert q(16, 256, 512, 0, False) == "gemm_i8_channel_kernel (1 SM, 128x256 tiles)"
+    assert q(16, 256, 512, 0, False) == "gemm_i8_channel_kernel (1 SM, 128x128 tiles)"
+    assert q(128, 4096, 14336, 0, False) == "gemm_i8_channel_kernel (1 SM, 128x128 tiles, cluster split-K in 4 slices)"
     assert q(256, 4096, 14336, 0, False).startswith("gemm_i8_channel_kernel (1 SM, 128x256 tiles, cluster split-K")
     assert q(4096, 4096, 4096, 0, False).startswith("gemm_i8_pair_kernel (CTA pair, 256x256 tiles, last wave cut")
     assert q(2048, 8192, 8192, 128, False) == "gemm_i8_group_pair_kernel (CTA pair, 256x256 tiles)"

@@ -54,8 +54,8 @@ __device__ __forceinline__ void teardown(S& s, uint32_t tmem) {
 // Split-K of the 1-SM kernel through distributed shared memory.  The
 // cluster is the `splits` CTAs of one tile (CTA j computed K slice j, and j
 // is its cluster rank); each has staged its 128 x BN int32 partial in its
-// operand ring as four 32 KB slots, one per TMEM lane quadrant (see
-// epilogue_channel).  After a cluster barrier, CTA j takes the 32-column
+// operand ring as four slots of 32 x BN int32 (32 KB at BN = 256), one per
+// TMEM lane quadrant (see epilogue_channel).  After a cluster barrier, CTA j takes the 32-column
 // chunks c = j, j + splits, ... of the tile; for each, epilogue warp q sums
 // the chunk's 32 rows of quadrant q over the cluster's CTAs (all sources'
 // loads in flight together; integer adds, exact), then dequantises and
@@ -128,16 +128,30 @@ __device__ void channel_cluster_reduce(S& s, const Args& p, const CUtensorMap* t
   __syncwarp();
 }
 
+// The per-channel 1-SM kernel comes in two tile widths: 128 x 256 (4
+// stages) and 128 x 128 (6 stages, about the same shared memory).  The
+// narrow one is taken when it puts more CTAs to work on a small-M problem,
+// e.g. 128 x 4096 x 14336: 32 tiles x 4 slices on 128 SMs instead of
+// 16 x 4 on 64 (17.6 against 22.3 us), or as many CTAs in fewer, short
+// K slices (channel_plan).  At an equal CTA count and long slices the wide
+// tile is faster (256 x 4096 x 14336: 22.7 us for 32 tiles x 4 slices,
+// 24.2 us for 64 narrow tiles x 2 slices: the narrow tile reads the
+// activations twice as often per weight byte).
 constexpr int kChannelBN = 256;
-constexpr int kChannelStages = 4;
 constexpr int kChannelThreads = 64 + 4 * 32;
-struct alignas(1024) ChannelStorage {
-  uint8_t a[kChannelStages][BM * BK];
-  uint8_t b[kChannelStages][kChannelBN * BK];
+template <int BN>
+constexpr int channel_stages() {
+  return BN == 256 ? 4 : 6;
+}
+template <int BN>
+struct alignas(1024) ChannelStorageT {
+  static constexpr int kStages = channel_stages<BN>();
+  uint8_t a[kStages][BM * BK];
+  uint8_t b[kStages][BN * BK];
   uint8_t out_stage[4][kOutBoxBytes];  // each epilogue warp's TMA store box
-  float sw_tile[4][kChannelBN];        // each epilogue warp's channel scales
-  uint64_t full[kChannelStages];
-  uint64_t empty[kChannelStages];
+  float sw_tile[4][BN];                // each epilogue warp's channel scales
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t aux_full[2];  // (unused by this kernel; set up with the others)
@@ -146,38 +160,41 @@ struct alignas(1024) ChannelStorage {
   uint32_t tmem_base;
   int abort;
 };
+using ChannelStorage = ChannelStorageT<kChannelBN>;
 
-template <bool F8, bool MOE = false>
+template <bool F8, bool MOE = false, int BN = kChannelBN>
 __global__ void __launch_bounds__(kChannelThreads, 1)
     gemm_i8_channel_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmO, const Args p) {
+  using S = ChannelStorageT<BN>;
+  constexpr int kStages = S::kStages;
   extern __shared__ uint8_t smem_raw[];
-  ChannelStorage& s = storage<ChannelStorage>(smem_raw);
+  S& s = storage<S>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     if (p.tma_out) prefetch_tmap(&tmO);
   }
-  setup<ChannelStorage, kChannelStages, 2, 4>(s);
+  setup<S, kStages, 2, 4>(s);
   if (warp != 0) {  // (the producer waits inside produce)
     griddep_wait();  // set-up above overlapped the previous kernel
     griddep_launch_dependents();
   }
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
-    if (lane == 0) produce<kChannelBN, kChannelStages, MOE, false, !MOE>(s, &tmA, &tmB, p);
+    if (lane == 0) produce<BN, kStages, MOE, false, !MOE>(s, &tmA, &tmB, p);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) mma_issue<kChannelBN, kChannelStages, 2, false, F8, MOE>(s, tmem, p);
+    if (lane == 0) mma_issue<BN, kStages, 2, false, F8, MOE>(s, tmem, p);
     __syncwarp();
   } else {
-    epilogue_channel<kChannelBN, 2, F8, MOE>(s, tmem, p, &tmO);
+    epilogue_channel<BN, 2, F8, MOE>(s, tmem, p, &tmO);
   }
   if (p.sk.csplit) {
     cluster_sync_all();  // every CTA of the cluster has staged its partial
-    if (warp >= 2) channel_cluster_reduce<kChannelBN, F8>(s, p, &tmO);
+    if (warp >= 2) channel_cluster_reduce<BN, F8>(s, p, &tmO);
     cluster_sync_all();  // the peers are done reading this CTA's slots
   }
   teardown(s, tmem);

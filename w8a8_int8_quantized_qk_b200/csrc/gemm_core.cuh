@@ -562,7 +562,8 @@ __device__ void epilogue_channel(S& s, uint32_t tmem, const Args& p, const CUten
     if (p.sk.csplit) {
       // Split-K inside the cluster (one unit per CTA, so the operand ring is
       // idle once acc_full has fired): stage this warp's 32 x BN partial in
-      // its 32 KB slot of the ring, laid out [chunk][column quad][lane][4];
+      // its slot of the ring (32 KB at BN = 256), laid out
+      // [chunk][column quad][lane][4];
       // channel_cluster_reduce sums the slots over the cluster after a
       // cluster barrier.
       uint8_t* stg = &s.a[0][0] + quad * (32 * BN * 4);

@@ -106,7 +106,10 @@ inline cudaError_t set_smem_once(K kernel, int dev, int slot, size_t bytes) {
   return e;
 }
 
-inline size_t channel_smem() { return sizeof(ChannelStorage) + 1024; }
+template <int BN = kChannelBN>
+inline size_t channel_smem() {
+  return sizeof(ChannelStorageT<BN>) + 1024;
+}
 inline size_t pair_smem() { return sizeof(PairStorage) + 1024; }
 
 // Largest number of co-resident clusters of `cluster` CTAs of the pair
@@ -511,7 +514,9 @@ static_assert(2 * kGroupWideMaxSplit * sizeof(int) <= kCounterHeaderBytes,
 
 // 0 ok, 1 tensor-map failure, 2 CUDA error
 // Largest number of co-resident clusters of `cluster` CTAs of the 1-SM
-// channel kernel (queried once per device and size; 0 when it cannot run).
+// channel kernel of tile width BN (queried once per device, width and size;
+// 0 when it cannot run).
+template <int BN>
 inline int max_channel_clusters(int dev, int cluster) {
   static std::atomic<int> cache[64][5] = {};
   if (dev < 0 || dev >= 64 || cluster < 2 || cluster > 4) return 0;
@@ -520,7 +525,7 @@ inline int max_channel_clusters(int dev, int cluster) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(cluster) * 16, 1, 1);
   cfg.blockDim = dim3(kChannelThreads, 1, 1);
-  cfg.dynamicSmemBytes = channel_smem();
+  cfg.dynamicSmemBytes = channel_smem<BN>();
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
@@ -529,9 +534,10 @@ inline int max_channel_clusters(int dev, int cluster) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(gemm_i8_channel_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(channel_smem())) != cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, gemm_i8_channel_kernel<false>, &cfg) != cudaSuccess) {
+  auto* kernel = gemm_i8_channel_kernel<false, false, BN>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(channel_smem<BN>())) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -539,18 +545,25 @@ inline int max_channel_clusters(int dev, int cluster) {
   return n > 0 ? n : 0;
 }
 
-// Split-K plan of the 1-SM channel kernel: with fewer 128 x 256 tiles than
+// Split-K plan of the 1-SM channel kernel: with fewer 128 x BN tiles than
 // half the SMs, cut K into S <= 4 slices (>= 8 K blocks each), one CTA per
 // slice, the S CTAs of a tile forming one cluster whose partials meet in
 // distributed shared memory.  S = 1 when the clusters would not all be
-// co-resident.
+// co-resident.  Of the two tile widths, 128 is taken when its plan puts
+// more CTAs to work than 256's, or as many with at most 16 K blocks per
+// slice, where the fewer slices' shorter reduction outweighs the narrow
+// tile's extra activation reads (96 x 8192 x 4096: 12.7 us as 64 narrow
+// tiles x 2 slices, 14.5 us as 32 wide tiles x 4; at 256 x 4096 x 14336,
+// 56 K blocks per narrow slice, the wide plan wins).
 struct ChannelPlan {
-  int tiles, splits, kb_per_split;
+  int tiles, splits, kb_per_split, bn;
 };
 
-inline ChannelPlan channel_plan(int m, int n, int k, int num_sms, int dev) {
+template <int BN>
+inline ChannelPlan channel_plan_bn(int m, int n, int k, int num_sms, int dev) {
   ChannelPlan pl;
-  pl.tiles = ((m + BM - 1) / BM) * ((n + kChannelBN - 1) / kChannelBN);
+  pl.bn = BN;
+  pl.tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
   const int num_kb = (k + BK - 1) / BK;
   int s = 1;
   if (2 * pl.tiles <= num_sms) {
@@ -561,7 +574,7 @@ inline ChannelPlan channel_plan(int m, int n, int k, int num_sms, int dev) {
   while (s > 1) {
     const int kbps = (num_kb + s - 1) / s;
     const int ns = (num_kb + kbps - 1) / kbps;
-    if (ns > 1 && max_channel_clusters(dev, ns) >= pl.tiles) {
+    if (ns > 1 && max_channel_clusters<BN>(dev, ns) >= pl.tiles) {
       s = ns;
       break;
     }
@@ -571,6 +584,16 @@ inline ChannelPlan channel_plan(int m, int n, int k, int num_sms, int dev) {
   pl.kb_per_split = (num_kb + s - 1) / s;
   pl.splits = (num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
   return pl;
+}
+
+inline ChannelPlan channel_plan(int m, int n, int k, int num_sms, int dev) {
+  const ChannelPlan wide = channel_plan_bn<256>(m, n, k, num_sms, dev);
+  const ChannelPlan narrow = channel_plan_bn<128>(m, n, k, num_sms, dev);
+  const int ctas_wide = wide.tiles * wide.splits, ctas_narrow = narrow.tiles * narrow.splits;
+  if (ctas_narrow > num_sms) return wide;
+  if (ctas_narrow > ctas_wide) return narrow;
+  if (ctas_narrow == ctas_wide && narrow.splits < wide.splits && narrow.kb_per_split <= 16) return narrow;
+  return wide;
 }
 
 // For 128 < m <= 256 (two 128-row tiles): the 1-SM kernel with cluster
@@ -592,7 +615,9 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
                   cudaStream_t stream, cudaError_t* err, void* workspace = nullptr) {
   // group mode without the int32 sums: the 128 x 256 kernel
   const bool wide = group && a.c == nullptr && group_wide_ok(dev);
-  const int bn = group ? (wide ? kGroupWideBN : kGroupBN) : kChannelBN;
+  ChannelPlan cpl = {};
+  if (!group) cpl = channel_plan(a.m, a.n, a.k, num_sms, dev);
+  const int bn = group ? (wide ? kGroupWideBN : kGroupBN) : cpl.bn;
   a.tiles_m = (a.m + BM - 1) / BM;
   a.tiles_n = (a.n + bn - 1) / bn;
   a.num_kb = (a.k + BK - 1) / BK;
@@ -601,13 +626,10 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   a.sk.kb_per_split = a.num_kb;
   a.sk.csplit = 0;
   a.tail.tail_splits = 1;
-  if (!group) {
-    const ChannelPlan pl = channel_plan(a.m, a.n, a.k, num_sms, dev);
-    if (pl.splits > 1) {
-      a.sk.splits = pl.splits;
-      a.sk.kb_per_split = pl.kb_per_split;
-      a.sk.csplit = 1;
-    }
+  if (!group && cpl.splits > 1) {
+    a.sk.splits = cpl.splits;
+    a.sk.kb_per_split = cpl.kb_per_split;
+    a.sk.csplit = 1;
   }
   CUtensorMap ta, tb, to;
   if (!cached_tmap(&ta, A, a.m, a.k, BM) || !cached_tmap(&tb, B, a.n, a.k, bn)) return 1;
@@ -623,13 +645,19 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   const int grid = a.sk.csplit ? ntiles * a.sk.splits : (ntiles < num_sms ? ntiles : num_sms);
   cudaError_t e;
   if (!group) {
-    const size_t smem = channel_smem();
-    e = a.f8 ? set_smem_once(gemm_i8_channel_kernel<true>, dev, 5, smem)
-             : set_smem_once(gemm_i8_channel_kernel<false>, dev, 1, smem);
-    if (e == cudaSuccess) {
-      e = launch_pdl(a.f8 ? gemm_i8_channel_kernel<true> : gemm_i8_channel_kernel<false>, dim3(grid),
-                     dim3(kChannelThreads), smem, stream,
-                     a.sk.csplit ? static_cast<unsigned>(a.sk.splits) : 1u, ta, tb, to, a);
+    const unsigned cluster = a.sk.csplit ? static_cast<unsigned>(a.sk.splits) : 1u;
+    if (bn == 128) {
+      const size_t smem = channel_smem<128>();
+      auto* kernel = a.f8 ? gemm_i8_channel_kernel<true, false, 128> : gemm_i8_channel_kernel<false, false, 128>;
+      e = set_smem_once(kernel, dev, a.f8 ? 10 : 9, smem);
+      if (e == cudaSuccess)
+        e = launch_pdl(kernel, dim3(grid), dim3(kChannelThreads), smem, stream, cluster, ta, tb, to, a);
+    } else {
+      const size_t smem = channel_smem();
+      auto* kernel = a.f8 ? gemm_i8_channel_kernel<true> : gemm_i8_channel_kernel<false>;
+      e = set_smem_once(kernel, dev, a.f8 ? 5 : 1, smem);
+      if (e == cudaSuccess)
+        e = launch_pdl(kernel, dim3(grid), dim3(kChannelThreads), smem, stream, cluster, ta, tb, to, a);
     }
   } else {
     if (wide) {

@@ -490,10 +490,10 @@ const char* qk_w8a8_gemm_kernel(int m, int n, int k, int group_k, int with_c) {
       const gemm::ChannelPlan pl = gemm::channel_plan(m, n, k, dev->sms, dev_id);
       if (pl.splits > 1)
         snprintf(text, sizeof text,
-                 "gemm_i8_channel_kernel (1 SM, 128x256 tiles, cluster split-K in %d slices)",
+                 "gemm_i8_channel_kernel (1 SM, 128x%d tiles, cluster split-K in %d slices)", pl.bn,
                  pl.splits);
       else
-        snprintf(text, sizeof text, "gemm_i8_channel_kernel (1 SM, 128x256 tiles)");
+        snprintf(text, sizeof text, "gemm_i8_channel_kernel (1 SM, 128x%d tiles)", pl.bn);
       return text;
     }
     case GemmPath::kTensorPair: {
