@@ -304,9 +304,10 @@ QK_API qk_status qk_fp8_gemm(int m, int n, int k, const uint8_t* a, const uint8_
  * n, k           per expert: b is [E, n, k] (row e * n + j is expert e's
  *                output channel j), k % 16 == 0, n % 8 == 0, k <= 133144
  * max_m_per_expert   an upper bound on every expert's token count: it sizes
- *                the tile space (E x ceil(max / 128) x ceil(n / 256) tiles,
- *                the empty ones skipped); rows of an expert beyond it are
- *                not computed
+ *                the tile space (E x ceil(max / T) x ceil(n / 256) tiles of
+ *                T rows, the empty ones skipped; T = 256 on CTA pairs when
+ *                total_m >= 128 E, else T = 128 on single SMs); rows of an
+ *                expert beyond it are not computed
  * expert_offsets [E + 1] int32 device array, non-decreasing, offsets[0] = 0,
  *                offsets[E] = total_m (rows outside [0, total_m) are never
  *                written)

@@ -34,11 +34,16 @@ def _moe(counts, n, k, seed):
     return a, w, sa, sw, off
 
 
+# Experts averaging fewer than 128 tokens run on the 1-SM kernel (128-row
+# tiles), the others on CTA pairs (256-row tiles): the first, second and
+# fourth cases take the 1-SM form, the third and fifth (and the synthetic
+# routing below) the pair form.
 @pytest.mark.parametrize("counts,n,k", [
     ([5, 0, 130, 1, 256, 77], 264, 512),
     ([0, 0, 3], 136, 272),
     ([1000, 24, 0, 300, 129, 128, 127, 2], 520, 1040),
     ([64] * 16, 2048, 1024),
+    ([256, 257, 511, 0, 128], 776, 2064),
 ])
 def test_moe_gemm(O, counts, n, k):
     a, w, sa, sw, off = _moe(counts, n, k, seed=sum(counts) + n + k)

@@ -718,6 +718,39 @@ inline int launch(Args a, const int8_t* A, const int8_t* B, bool group, int dev,
   return e == cudaSuccess ? 0 : 2;
 }
 
+// MoE grouped GEMM on the CTA-pair kernel (MOE form): 256-row pair tiles over
+// the compact list of each expert's tiles (moe_pair_unit), whole K, per
+// channel, direct stores (rows past an expert's last are not stored).
+// mt_max bounds every expert's 256-row tiles.  0 ok, 1 tensor-map failure,
+// 2 CUDA error.
+inline int launch_moe_pair(Args a, const int8_t* A, const int8_t* B, int experts, int mt_max,
+                           const int32_t* off, int dev, int num_sms, cudaStream_t stream,
+                           cudaError_t* err) {
+  a.moe.mt_max = mt_max;
+  a.moe.moe_off = off;
+  a.tiles_m = experts * mt_max;
+  a.tiles_n = (a.n + kPairBN - 1) / kPairBN;
+  a.num_kb = (a.k + BK - 1) / BK;
+  a.groups = 0;
+  a.sk.splits = 1;
+  a.sk.kb_per_split = a.num_kb;
+  a.sk.csplit = 0;
+  a.tail.tail_splits = 1;
+  a.tma_out = 0;
+  a.c = nullptr;
+  CUtensorMap ta, tb;
+  if (!cached_tmap(&ta, A, a.m, a.k, 128) || !cached_tmap(&tb, B, experts * a.n, a.k, 128)) return 1;
+  const int pairs = max_pairs(dev, num_sms);
+  const int64_t units = static_cast<int64_t>(a.tiles_m) * a.tiles_n;  // an upper bound
+  const int grid_pairs = units < pairs ? static_cast<int>(units) : pairs;
+  cudaError_t e = set_smem_once(gemm_i8_pair_kernel<false, true>, dev, 11, pair_smem());
+  if (e == cudaSuccess)
+    e = launch_pdl(gemm_i8_pair_kernel<false, true>, dim3(2 * grid_pairs), dim3(kPairThreads), pair_smem(),
+                   stream, 2u, ta, tb, ta, a);
+  *err = e;
+  return e == cudaSuccess ? 0 : 2;
+}
+
 // MoE grouped GEMM on the 1-SM kernel: `experts` groups of tokens (expert e
 // owns rows [off[e], off[e + 1]) of A, m rows in all), B stacked [experts *
 // n, k], per-channel scales [experts, n]; mt_max bounds every expert's M

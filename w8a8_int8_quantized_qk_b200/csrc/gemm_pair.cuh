@@ -46,6 +46,7 @@ struct alignas(1024) PairStorage {
 // slice is the K slice index (0 for a whole tile).
 struct PairUnit {
   int tile, kb0, kb1, slice;
+  int expert, row0, row_end, tn;  // the MoE form only (moe_pair_unit)
 };
 
 // The i-th unit of pair `pi` (false past its last).  Without the tail split,
@@ -82,18 +83,65 @@ __device__ __forceinline__ bool pair_unit(const Args& p, int pi, int npairs, int
   return true;
 }
 
+// The MoE form (grouped GEMM, whole K, no split): the i-th unit of pair pi
+// in the compact list of non-empty 256-row tiles, expert by expert and M
+// tiles fastest, so the pairs working at once share their expert's B tile.
+// Expert e owns A rows [off[e], off[e + 1]) and B rows [e n, e n + n);
+// p.moe.mt_max bounds every expert's M tiles and p.tiles_m = experts x
+// mt_max.  A tile's rows past its expert's last are computed (the TMA reads
+// the next expert's rows, or zeros past m) and never stored.
+__device__ __forceinline__ bool moe_pair_unit(const Args& p, int pi, int npairs, int i, PairUnit& u) {
+  int t = pi + i * npairs;
+  const int experts = p.tiles_m / p.moe.mt_max;
+  for (int e = 0; e < experts; ++e) {
+    const int r0 = __ldg(p.moe.moe_off + e), r1 = __ldg(p.moe.moe_off + e + 1);
+    int mt = r1 > r0 ? (r1 - r0 + kPairBM - 1) / kPairBM : 0;
+    mt = mt < p.moe.mt_max ? mt : p.moe.mt_max;
+    const int cnt = mt * p.tiles_n;
+    if (t < cnt) {
+      const int tm = t % mt;
+      u.tn = t / mt;
+      u.tile = 0;
+      u.slice = 0;
+      u.kb0 = 0;
+      u.kb1 = p.num_kb;
+      u.expert = e;
+      u.row0 = r0 + tm * kPairBM;
+      u.row_end = r1 < p.m ? r1 : p.m;
+      return true;
+    }
+    t -= cnt;
+  }
+  return false;
+}
+
+template <bool MOE>
+__device__ __forceinline__ bool next_unit(const Args& p, int pi, int npairs, int i, PairUnit& u) {
+  if constexpr (MOE)
+    return moe_pair_unit(p, pi, npairs, i, u);
+  else
+    return pair_unit(p, pi, npairs, i, u);
+}
+
 // pr: this CTA's rank within its pair; lead: the cluster rank of its pair's
 // leader (clusters hold one pair, or the `splits` pairs of one tile).
+template <bool MOE>
 __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUtensorMap* tmB,
                              const Args& p, uint32_t pr, uint32_t lead) {
   const int npairs = gridDim.x >> 1;
   uint32_t stage = 0, phase = 0, issued = 0;
   bool ok = true;
   PairUnit u;
-  for (int i = 0; ok && pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
-    const int tm = u.tile % p.tiles_m, tn = u.tile / p.tiles_m;
-    const int ya = tm * kPairBM + static_cast<int>(pr) * 128;
-    const int yb = tn * kPairBN + static_cast<int>(pr) * 128;
+  for (int i = 0; ok && next_unit<MOE>(p, blockIdx.x >> 1, npairs, i, u); ++i) {
+    int ya, yb;
+    if constexpr (MOE) {
+      ya = u.row0 + static_cast<int>(pr) * 128;
+      yb = u.expert * p.n + u.tn * kPairBN + static_cast<int>(pr) * 128;
+    } else {
+      const int tm = u.tile % p.tiles_m, tn = u.tile / p.tiles_m;
+      ya = tm * kPairBM + static_cast<int>(pr) * 128;
+      yb = tn * kPairBN + static_cast<int>(pr) * 128;
+    }
     for (int kb = u.kb0; kb < u.kb1; ++kb) {
       if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, &s.abort)) {
         ok = false;
@@ -120,7 +168,7 @@ __device__ void produce_pair(PairStorage& s, const CUtensorMap* tmA, const CUten
   }
 }
 
-template <bool F8>
+template <bool F8, bool MOE>
 __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t lead) {
   const uint16_t pair_mask = static_cast<uint16_t>(0x3u << lead);
   const int npairs = gridDim.x >> 1;
@@ -128,7 +176,7 @@ __device__ void mma_issue_pair(PairStorage& s, uint32_t tmem, const Args& p, uin
   uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
   bool ok = true;
   PairUnit u;
-  for (int i = 0; ok && pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
+  for (int i = 0; ok && next_unit<MOE>(p, blockIdx.x >> 1, npairs, i, u); ++i) {
     const int kb0 = u.kb0, kb1 = u.kb1;
     if (!mbar_wait(smem_addr(&s.acc_empty[abuf]), aphase ^ 1u, &s.abort)) break;
     tc_fence_after();
@@ -256,7 +304,7 @@ __device__ void tail_slice_epilogue(uint32_t acc_empty_lead, const Args& p,
 // token scale is fetched before the accumulator is ready, and the four
 // 32-column TMEM loads are double-buffered so the next load is in flight
 // while the current chunk is converted and stored.
-template <bool F8>
+template <bool F8, bool MOE>
 __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint32_t pr,
                               uint32_t lead, const CUtensorMap* tmO) {
   const int npairs = gridDim.x >> 1;
@@ -269,17 +317,27 @@ __device__ void epilogue_pair(PairStorage& s, uint32_t tmem, const Args& p, uint
   uint8_t* box = s.out_stage[warp - 2];
   uint32_t abuf = 0, aphase = 0;
   PairUnit u;
-  for (int i = 0; pair_unit(p, blockIdx.x >> 1, npairs, i, u); ++i) {
+  for (int i = 0; next_unit<MOE>(p, blockIdx.x >> 1, npairs, i, u); ++i) {
     const int tile = u.tile;
-    const bool tail = p.tail.tail_splits > 1 && tile >= p.tail.dp_tiles;
-    const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-    const int row = tm * kPairBM + static_cast<int>(pr) * 128 + quad * 32 + lane;
-    const bool rv = row < p.m;
+    const bool tail = !MOE && p.tail.tail_splits > 1 && tile >= p.tail.dp_tiles;
+    int row, colbase;
+    bool rv;
+    const float* swe = p.sw;  // this unit's channel scales (MoE: its expert's)
+    if constexpr (MOE) {
+      row = u.row0 + static_cast<int>(pr) * 128 + quad * 32 + lane;
+      rv = row < u.row_end;
+      colbase = u.tn * kPairBN + half * (kPairBN / 2);
+      swe = p.sw + static_cast<int64_t>(u.expert) * p.n;
+    } else {
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      row = tm * kPairBM + static_cast<int>(pr) * 128 + quad * 32 + lane;
+      rv = row < p.m;
+      colbase = tn * kPairBN + half * (kPairBN / 2);
+    }
     const float sa = (rv && p.out) ? __ldg(p.sa + row) : 0.0f;
-    const int colbase = tn * kPairBN + half * (kPairBN / 2);
     if (p.out) {
       const int c4 = colbase + lane * 4;  // n % 8 == 0: a group of 4 is all in or all out
-      const float4 v4 = c4 < p.n ? __ldg(reinterpret_cast<const float4*>(p.sw + c4))
+      const float4 v4 = c4 < p.n ? __ldg(reinterpret_cast<const float4*>(swe + c4))
                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       *reinterpret_cast<float4*>(sws + lane * 4) = v4;
     }
@@ -518,7 +576,7 @@ __device__ void cluster_reduce_pair(PairStorage& s, const Args& p, uint32_t cran
   }
 }
 
-template <bool F8>
+template <bool F8, bool MOE = false>
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -558,13 +616,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   griddep_launch_dependents();
   const uint32_t tmem = s.tmem_base;
   if (warp == 0) {
-    if (lane == 0) produce_pair(s, &tmA, &tmB, p, pr, lead);
+    if (lane == 0) produce_pair<MOE>(s, &tmA, &tmB, p, pr, lead);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && pr == 0) mma_issue_pair<F8>(s, tmem, p, lead);
+    if (lane == 0 && pr == 0) mma_issue_pair<F8, MOE>(s, tmem, p, lead);
     __syncwarp();
   } else {
-    epilogue_pair<F8>(s, tmem, p, pr, lead, &tmO);
+    epilogue_pair<F8, MOE>(s, tmem, p, pr, lead, &tmO);
   }
   if (p.sk.csplit) {
     if (warp >= 2) cluster_reduce_scales(s, p, crank);

@@ -339,6 +339,9 @@ qk_status qk_quantize_per_token_asym(int m, int k, const void* x, qk_dtype x_dty
                      "asymmetric quantize launch");
 }
 
+// tokens per expert, on average, from which the MoE GEMM runs on CTA pairs
+constexpr int kMoePairTokens = 128;
+
 qk_status qk_w8a8_moe_gemm(int num_experts, int total_m, int n, int k, int max_m_per_expert,
                            const int32_t* expert_offsets, const int8_t* a, const int8_t* b,
                            const float* scale_a, const float* scale_b, float output_scale,
@@ -371,9 +374,16 @@ qk_status qk_w8a8_moe_gemm(int num_experts, int total_m, int n, int k, int max_m
   cudaError_t e = cudaSuccess;
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  const int mt_max = (max_m_per_expert + 127) / 128;
-  const int r = gemm::launch_moe(g, a, b, num_experts, mt_max, expert_offsets, dev_id, dev->sms,
-                                 reinterpret_cast<cudaStream_t>(stream), &e);
+  // Experts averaging at least 128 tokens: 256-row tiles on CTA pairs (half
+  // the operand traffic per multiply-add of the 1-SM tile); fewer: 128-row
+  // tiles on single SMs, which pad small experts less.
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool pair = static_cast<int64_t>(total_m) >= static_cast<int64_t>(kMoePairTokens) * num_experts &&
+                    gemm::max_pairs(dev_id, dev->sms) > 0;
+  const int r = pair ? gemm::launch_moe_pair(g, a, b, num_experts, (max_m_per_expert + 255) / 256,
+                                             expert_offsets, dev_id, dev->sms, s, &e)
+                     : gemm::launch_moe(g, a, b, num_experts, (max_m_per_expert + 127) / 128,
+                                        expert_offsets, dev_id, dev->sms, s, &e);
   if (r == 1) return cuda_status(cudaErrorInvalidValue, "tensor map encoding");
   return r == 0 ? QK_OK : cuda_status(e, "moe gemm launch");
 }
