@@ -541,7 +541,8 @@ def measure_moe(torch, qk, iters: int, pk: dict) -> dict:
                                                  if pk.get("int8_tops_random_operands") else None),
             "gemm_tensor_frac_nominal": ops / (us * 1e-6) / 1e12 / NOMINAL["int8_tops"],
             "weight_GBs": wbytes / (us * 1e-6) / 1e9,
-            "note": "1-SM tcgen05 kernel over experts x M tiles x N tiles, empty tiles skipped"}
+            "note": ("CTA-pair tcgen05 kernel (256-row tiles; the experts average >= 128 tokens) over "
+                     "experts x M tiles x N tiles, empty tiles skipped")}
 
 
 def cpu_baseline(seconds: float = 10.0) -> dict:
