@@ -36,14 +36,16 @@ def _moe(counts, n, k, seed):
 
 # Experts averaging fewer than 128 tokens run on the 1-SM kernel (128-row
 # tiles), the others on CTA pairs (256-row tiles): the first, second and
-# fourth cases take the 1-SM form, the third and fifth (and the synthetic
-# routing below) the pair form.
+# fourth cases take the 1-SM form, the others (and the synthetic routing
+# below) the pair form.  The last has 11 x 9 = 99 pair tiles, more than one
+# wave on 74 pairs, and its last N tile holds 8 columns.
 @pytest.mark.parametrize("counts,n,k", [
     ([5, 0, 130, 1, 256, 77], 264, 512),
     ([0, 0, 3], 136, 272),
     ([1000, 24, 0, 300, 129, 128, 127, 2], 520, 1040),
     ([64] * 16, 2048, 1024),
     ([256, 257, 511, 0, 128], 776, 2064),
+    ([300, 300, 300, 100, 100, 0, 100, 100, 180], 2056, 1040),
 ])
 def test_moe_gemm(O, counts, n, k):
     a, w, sa, sw, off = _moe(counts, n, k, seed=sum(counts) + n + k)
