@@ -1,6 +1,7 @@
 // gemm_pair.cuh -- the CTA-pair tcgen05 GEMM kernel (cta_group::2, 256 x 256
 // tiles) with its split-K forms: through the workspace, through distributed
-// shared memory in a cluster, and the tail split of a partial last wave.
+// shared memory in a cluster, and the tail split of a partial last wave;
+// and its MoE form (grouped GEMM over per-expert tiles).
 #pragma once
 
 #include "gemm_1sm.cuh"
@@ -43,7 +44,9 @@ struct alignas(1024) PairStorage {
 };
 
 // One unit of a pair's work: K blocks [kb0, kb1) of output tile `tile`;
-// slice is the K slice index (0 for a whole tile).
+// slice is the K slice index (0 for a whole tile).  The MoE form describes
+// its tile by the expert, the tile's first A row, the end of the expert's
+// rows and the N tile instead.
 struct PairUnit {
   int tile, kb0, kb1, slice;
   int expert, row0, row_end, tn;  // the MoE form only (moe_pair_unit)
