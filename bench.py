@@ -837,7 +837,7 @@ def run_ours(args):
             "e2e": e2e, "decode": decode, "cpu_baseline": cpu,
             "peaks": {k: v for k, v in pk.items() if k != "nominal"},
             "gpu": torch.cuda.get_device_name(local)}
-    if decode is not None:  # the benchmark spec's second metric, compact
+    if decode is not None:  # the decode weight-stream GB/s (the second metric), compact
         line["decode"] = {"value": decode["value"], "unit": "GB/s", "gemv_us": decode["gemv_us"],
                           "frac": decode["roofline"]["frac"],
                           "frac_nominal": decode["roofline"]["frac_nominal"],
